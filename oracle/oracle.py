@@ -1,0 +1,278 @@
+"""LAPLEX oracle -- TEST INFRASTRUCTURE ONLY.
+
+A plain, slow, obviously-correct fp64 CPU statement of what the LAPLEX hot path
+computes.  Only tests/, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import it.  It shares no code with the CUDA library and never
+calls it; inputs are the same seeded arrays the GPU receives, promoted to fp64.
+
+Two independent routes are provided for every operator:
+
+* ``dense_*`` -- the definition written out with numpy: the matrix
+  K_ij = exp(-|a_i - b_j|) (times cos(phi_i - psi_j) when phased) is built and
+  multiplied ("LAPLEX - La FFT dei Nuclei di Laplace Apprendibili", technical
+  summary, §2.1 "L'Operatore").  Small sizes only.
+* sequential -- sort plus the prefix/suffix recurrences of the same summary's
+  §2.2 ("Algebra di Scansione Esatta"), in plain C (``laplex_oracle.c``), O(n).
+
+and ``rows_*`` evaluates chosen rows of the dense definition at any size.
+Parity of every function is pinned in tests/test_oracle_*.py against closed
+forms, invariants, brute force and hand-worked examples (see the test headers).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.c_int64
+
+#: fp64 exp underflows to exactly 0.0 below -745.14, so terms with |a_i - b_j|
+#: >= 746 are exactly zero in an fp64 evaluation of the definition.
+CUTOFF_F64 = 746.0
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(_build.build())
+        lib.orc_sym_sorted.argtypes = [_I64, _I64, _D, _D, _D]
+        lib.orc_general_sorted.argtypes = [_I64, _I64, _I64, _D, _D, _D, _D]
+        lib.orc_signed_sorted.argtypes = [_I64, _I64, _D, _D, _D]
+        lib.orc_rows_window.argtypes = [_I64, _D, _D, _I64, _I64, _D, _D, _D, ctypes.c_double,
+                                        _D, _D, _D]
+        for f in (lib.orc_sym_sorted, lib.orc_general_sorted, lib.orc_signed_sorted,
+                  lib.orc_rows_window):
+            f.restype = None
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(x):
+    return None if x is None else x.ctypes.data_as(_D)
+
+
+def _cols(x):
+    x = _f64(x)
+    return (x.reshape(-1, 1), True) if x.ndim == 1 else (x, False)
+
+
+# ---------------------------------------------------------------------------
+# sort (the O(n log n) step: "after sorting the anchors", summary §2.2)
+# ---------------------------------------------------------------------------
+
+def stable_sort(a):
+    """Ascending order of the anchors, ties by ascending index.
+
+    Returns (s, perm) with s = a[perm] (fp64) and perm int64.  A library stable
+    sort is the step; numeric comparison treats -0.0 and +0.0 as equal.
+    Non-finite anchors are rejected (the operator is undefined there).
+    """
+    a64 = _f64(a)
+    if a64.size and not np.all(np.isfinite(a64)):
+        raise ValueError("non-finite anchor")
+    perm = np.argsort(a64, kind="stable")
+    return a64[perm], perm
+
+
+# ---------------------------------------------------------------------------
+# dense definition (summary §2.1)
+# ---------------------------------------------------------------------------
+
+def dense_matrix(a, b=None, phi=None, psi=None):
+    """K_ij = exp(-|a_i - b_j|) [* cos(phi_i - psi_j)]; b = a, psi = phi when omitted."""
+    a = _f64(a)
+    b = a if b is None else _f64(b)
+    K = np.exp(-np.abs(a[:, None] - b[None, :]))
+    if phi is not None:
+        phi = _f64(phi)
+        psi = phi if psi is None else _f64(psi)
+        K = K * np.cos(phi[:, None] - psi[None, :])
+    return K
+
+
+def dense_matvec(a, x, b=None, phi=None, psi=None):
+    return dense_matrix(a, b, phi, psi) @ _f64(x)
+
+
+def dense_backward(a, x, g):
+    """For L = <g, K x>, K = K(a, a): dx = K^T g and
+    da_m = -sum_j sign(a_m - a_j) exp(-|a_m - a_j|) (g_m x_j + x_m g_j),
+    the derivative of the definition with d|t|/dt = sign(t), sign(0) = 0."""
+    a, x, g = _f64(a), _f64(x), _f64(g)
+    K = dense_matrix(a)
+    S = np.sign(a[:, None] - a[None, :]) * K
+    dx = K.T @ g
+    da = -(g * (S @ x) + x * (S @ g))
+    return dx, da
+
+
+# ---------------------------------------------------------------------------
+# sequential routes (summary §2.2)
+# ---------------------------------------------------------------------------
+
+def sym_sorted(s, x):
+    """y = K x for anchors s already ascending; x, y in that order (C recurrences)."""
+    s = _f64(s)
+    x2, flat = _cols(x)
+    n, B = x2.shape
+    y = np.empty_like(x2)
+    _L().orc_sym_sorted(n, B, _p(s), _p(x2), _p(y))
+    return y.ravel() if flat else y
+
+
+def sym(a, x):
+    """y = K x, K_ij = exp(-|a_i - a_j|), any anchor order (sort, recur, un-permute)."""
+    s, perm = stable_sort(a)
+    x2, flat = _cols(x)
+    ys = sym_sorted(s, x2[perm])
+    y = np.empty_like(ys)
+    y[perm] = ys
+    return y.ravel() if flat else y
+
+
+def general(a, b, x):
+    """y = K x with K_ij = exp(-|a_i - b_j|), a in R^n, b in R^k, x in R^k (or [k, B]).
+
+    The u/v interval aggregation of summary §2.2 "Caso Generale" (C code)."""
+    sa, pa = stable_sort(a)
+    sb, pb = stable_sort(b)
+    x2, flat = _cols(x)
+    xs = np.ascontiguousarray(x2[pb])
+    n, k, B = sa.size, sb.size, x2.shape[1]
+    ys = np.zeros((n, B))
+    if n and k:
+        _L().orc_general_sorted(n, k, B, _p(sa), _p(sb), _p(xs), _p(ys))
+    y = np.empty_like(ys)
+    y[pa] = ys
+    return y.ravel() if flat else y
+
+
+def general_T(a, b, w):
+    """z = K^T w for K = K(a, b): K^T_ji = exp(-|b_j - a_i|) = K(b, a)_ji."""
+    return general(b, a, w)
+
+
+def phased(a, phi, v, b=None, psi=None):
+    """y = K v with K_jk = exp(-|a_j - b_k|) cos(phi_j - psi_k) (summary §2.1),
+    through cos(p - q) = cos p cos q + sin p sin q: two unphased channels
+    cos(psi) v and sin(psi) v, recombined with cos(phi) and sin(phi)."""
+    phi = _f64(phi)
+    v = _f64(v)
+    sym_case = b is None
+    psi = phi if psi is None else _f64(psi)
+    ch = np.stack([np.cos(psi) * v, np.sin(psi) * v], axis=1)
+    u = sym(a, ch) if sym_case else general(a, b, ch)
+    return np.cos(phi) * u[:, 0] + np.sin(phi) * u[:, 1]
+
+
+def phased_T(a, phi, w, b, psi):
+    """K^T w for the phased K(a, phi; b, psi): the phased operator with roles swapped."""
+    return phased(b, psi, w, a, phi)
+
+
+def gram(a, v, phi=None, D=None, b=None, psi=None):
+    """z = K^T diag(D) K v (D = 1 when omitted), the Gram operator of summary §2.2
+    "Operatori di Gram" applied to a vector: two chained products."""
+    if phi is None:
+        u = sym(a, v) if b is None else general(a, b, v)
+    else:
+        u = phased(a, phi, v) if b is None else phased(a, phi, v, b, psi)
+    if D is not None:
+        u = u * _f64(D)
+    if phi is None:
+        return sym(a, u) if b is None else general_T(a, b, u)
+    return phased(a, phi, u) if b is None else phased_T(a, phi, u, b, psi)
+
+
+def signed_sorted(s, v):
+    """D_i = sum_j sign(s_i - s_j) exp(-|s_i - s_j|) v_j for ascending s (C code)."""
+    s = _f64(s)
+    v2, flat = _cols(v)
+    n, B = v2.shape
+    out = np.empty_like(v2)
+    _L().orc_signed_sorted(n, B, _p(s), _p(v2), _p(out))
+    return out.ravel() if flat else out
+
+
+def backward(a, x, g):
+    """Backward pass of L = <g, K x> w.r.t. x and the anchors (K = K(a, a)):
+    dx = K^T g = K g;  da = -(g * Dx + x * Dg) with D the signed sums above."""
+    s, perm = stable_sort(a)
+    x, g = _f64(x), _f64(g)
+    xs, gs = x[perm], g[perm]
+    dxs = sym_sorted(s, gs)
+    das = -(gs * signed_sorted(s, xs) + xs * signed_sorted(s, gs))
+    dx = np.empty_like(dxs)
+    da = np.empty_like(das)
+    dx[perm] = dxs
+    da[perm] = das
+    return dx, da
+
+
+# ---------------------------------------------------------------------------
+# rows of the dense definition at any size (sampled parity)
+# ---------------------------------------------------------------------------
+
+def rows(ra, sb, xs, rphi=None, spsi=None, cutoff=CUTOFF_F64):
+    """For chosen rows (anchors ra, phases rphi) against ascending b-anchors sb with
+    values xs ([k] or [k, B], phases spsi, all in sorted-b order) return
+    (K x, signed sums, K0 |x|) for those rows; see orc_rows_window."""
+    ra = _f64(ra)
+    sb = _f64(sb)
+    x2, flat = _cols(xs)
+    m, (k, B) = ra.size, x2.shape
+    out = np.empty((m, B))
+    sgn = np.empty((m, B))
+    absn = np.empty((m, B))
+    rphi = None if rphi is None else _f64(rphi)
+    spsi = None if spsi is None else _f64(spsi)
+    _L().orc_rows_window(m, _p(ra), _p(rphi), k, B, _p(sb), _p(spsi), _p(x2), float(cutoff),
+                         _p(out), _p(sgn), _p(absn))
+    if flat:
+        return out.ravel(), sgn.ravel(), absn.ravel()
+    return out, sgn, absn
+
+
+# ---------------------------------------------------------------------------
+# normalisers for the parity criterion max_i |y_i - y_ref_i| / norm_i
+# ---------------------------------------------------------------------------
+
+def norm_sym(a, x):
+    """K0 |x| with the unphased kernel: an upper bound of |K| |x| for every variant."""
+    return sym(a, np.abs(_f64(x)))
+
+
+def norm_general(a, b, x):
+    return general(a, b, np.abs(_f64(x)))
+
+
+def norm_gram(a, v, D=None, b=None):
+    u = norm_sym(a, v) if b is None else norm_general(a, b, v)
+    if D is not None:
+        u = u * np.abs(_f64(D))
+    return sym(a, u) if b is None else general_T(a, b, u)
+
+
+def norm_backward(a, x, g):
+    """(K0|g|, |g| K0|x| + |x| K0|g|): bounds of |dx| and |da| term by term."""
+    x, g = np.abs(_f64(x)), np.abs(_f64(g))
+    kx, kg = sym(a, x), sym(a, g)
+    return kg, g * kx + x * kg
+
+
+def max_norm_err(y, y_ref, norm):
+    """max_i |y_i - y_ref_i| / norm_i (norm_i = 0 only where y_ref_i = 0 exactly)."""
+    y = np.asarray(y, dtype=np.float64)
+    y_ref = _f64(y_ref)
+    norm = _f64(norm)
+    err = np.abs(y - y_ref)
+    safe = np.where(norm > 0, norm, 1.0)
+    return float(np.max(err / safe)) if err.size else 0.0

@@ -1,0 +1,395 @@
+"""Pins of the CPU oracle to facts other than itself (no GPU needed).
+
+Each test ties an oracle route to something it does not compute the same way:
+hand-worked examples (tests/golden/hand_examples.json), textbook closed forms
+(the Ornstein-Uhlenbeck tridiagonal inverse, the Kac-Murdock-Szego Toeplitz
+matrix through scipy), invariants of the definition, brute force on tiny inputs,
+and central finite differences.  The sources are the LAPLEX technical summaries
+("Riepilogo Tecnico: LAPLEX - La FFT dei Nuclei di Laplace Apprendibili" and its
+French twin), cited by section.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+import oracle as O
+from exact_laplace_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")
+NS = {"exp": math.exp, "cos": math.cos, "sin": math.sin, "pi": math.pi, "__builtins__": {}}
+
+
+def ev(e):
+    return float(eval(e, NS)) if isinstance(e, str) else float(e)
+
+
+def _examples():
+    with open(GOLDEN) as f:
+        return json.load(f)["examples"]
+
+
+@pytest.mark.parametrize("ex", _examples(), ids=lambda e: e["name"])
+def test_hand_examples(ex):
+    a = [ev(v) for v in ex["a"]]
+    op = ex["op"]
+    if op == "sort":
+        s, perm = O.stable_sort(np.array(a))
+        assert perm.tolist() == ex["expect_perm"]
+        return
+    x = [ev(v) for v in ex["x"]]
+    if op == "backward":
+        g = [ev(v) for v in ex["g"]]
+        dx, da = O.backward(a, x, g)
+        dxd, dad = O.dense_backward(a, x, g)
+        np.testing.assert_allclose(dx, [ev(e) for e in ex["expect_dx"]], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(da, [ev(e) for e in ex["expect_da"]], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(dxd, [ev(e) for e in ex["expect_dx"]], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(dad, [ev(e) for e in ex["expect_da"]], rtol=0, atol=1e-14)
+        return
+    exp = np.array([ev(e) for e in ex["expect"]])
+    if "decimal" in ex:  # the closed forms agree with the printed decimals
+        np.testing.assert_allclose(exp, ex["decimal"], rtol=0, atol=6e-9)
+    if op == "sym":
+        outs = [O.sym(a, x), O.dense_matvec(a, x)]
+    elif op == "phased":
+        phi = [ev(v) for v in ex["phi"]]
+        outs = [O.phased(a, phi, x), O.dense_matvec(a, x, phi=phi)]
+    elif op == "gram_phased":
+        phi = [ev(v) for v in ex["phi"]]
+        K = O.dense_matrix(a, phi=phi)
+        outs = [O.gram(a, x, phi=phi), K.T @ (K @ np.array(x))]
+    elif op == "general":
+        b = [ev(v) for v in ex["b"]]
+        outs = [O.general(a, b, x), O.dense_matvec(a, x, b=b)]
+    elif op == "general_T":
+        b = [ev(v) for v in ex["b"]]
+        outs = [O.general_T(a, b, x), O.dense_matrix(a, b).T @ np.array(x)]
+    else:
+        raise AssertionError(op)
+    for y in outs:
+        np.testing.assert_allclose(y, exp, rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# closed forms
+# ---------------------------------------------------------------------------
+
+def _ou_precision(s):
+    """Tridiagonal inverse of K_ij = exp(-|s_i - s_j|) for distinct ascending s: the
+    covariance of an Ornstein-Uhlenbeck process sampled at s is Markov, so its
+    precision matrix is tridiagonal with rho_i = exp(-(s_{i+1} - s_i)):
+    Q_{i,i+1} = -rho_i / (1 - rho_i^2),
+    Q_ii = 1 + rho_{i-1}^2 / (1 - rho_{i-1}^2) + rho_i^2 / (1 - rho_i^2)."""
+    n = len(s)
+    rho = np.exp(-np.diff(s))
+    off = -rho / (1 - rho ** 2)
+    t = rho ** 2 / (1 - rho ** 2)
+    diag = np.ones(n)
+    diag[1:] += t
+    diag[:-1] += t
+    return diag, off
+
+
+@pytest.mark.parametrize("n,seed", [(2, 0), (7, 1), (200, 2), (3000, 3)])
+def test_ou_tridiagonal_inverse(n, seed):
+    rng = np.random.default_rng(seed)
+    s = np.cumsum(rng.uniform(0.05, 2.0, size=n))
+    x = rng.normal(size=n)
+    y = O.sym_sorted(s, x)
+    diag, off = _ou_precision(s)
+    back = diag * y
+    back[:-1] += off * y[1:]
+    back[1:] += off * y[:-1]
+    np.testing.assert_allclose(back, x, rtol=0, atol=1e-10 * max(1.0, np.abs(x).max()))
+
+
+@pytest.mark.parametrize("n,h", [(1, 0.3), (64, 0.01), (512, 0.7)])
+def test_uniform_grid_is_kms_toeplitz(n, h):
+    """Anchors on a uniform grid make K the Toeplitz matrix rho^|i-j| (IT §2.3,
+    relation with the FFT); scipy builds it independently."""
+    rng = np.random.default_rng(n)
+    s = 5.0 + h * np.arange(n)
+    x = rng.normal(size=(n, 3))
+    T = scipy.linalg.toeplitz(np.exp(-h) ** np.arange(n))
+    np.testing.assert_allclose(O.sym_sorted(s, x), T @ x, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(O.sym(s[::-1].copy(), x[::-1]), (T @ x)[::-1], rtol=1e-12, atol=1e-12)
+
+
+def test_unit_vectors_give_columns():
+    rng = np.random.default_rng(5)
+    a = rng.normal(size=40) * 2
+    a[[3, 9]] = a[17]
+    for i in (0, 3, 17, 39):
+        e = np.zeros(40)
+        e[i] = 1
+        np.testing.assert_allclose(O.sym(a, e), np.exp(-np.abs(a - a[i])), rtol=0, atol=1e-15)
+
+
+def test_all_equal_anchors_sum():
+    x = np.random.default_rng(1).normal(size=(33, 2))
+    y = O.sym(np.full(33, 7.25), x)
+    np.testing.assert_allclose(y, np.broadcast_to(x.sum(0), y.shape), rtol=1e-13)
+
+
+def test_far_apart_anchors_identity():
+    rng = np.random.default_rng(2)
+    a = rng.permutation(np.arange(20) * 800.0)
+    x = rng.normal(size=20)
+    assert np.array_equal(O.sym(a, x), x)
+
+
+def test_temperature_zero_permutation_limit():
+    """IT §2.3 / §2.1: as t -> 0, exp(-|a_i - b_j| / t) tends to the equality routing
+    matrix; with b = a[pi] and distinct anchors, K x -> P x, (K x)_i = x_{pi^-1(i)}."""
+    rng = np.random.default_rng(3)
+    n = 50
+    a = rng.permutation(np.linspace(-3, 3, n))
+    pi = rng.permutation(n)
+    b = a[pi]
+    x = rng.normal(size=n)
+    t = (6 / (n - 1)) / 800  # every off-equality term is exp(-800): exactly 0 in fp64
+    y = O.general(a / t, b / t, x)
+    inv = np.empty(n, dtype=int)
+    inv[pi] = np.arange(n)
+    np.testing.assert_array_equal(y, x[inv])
+
+
+# ---------------------------------------------------------------------------
+# invariants
+# ---------------------------------------------------------------------------
+
+def test_symmetry_translation_reflection_permutation():
+    rng = np.random.default_rng(4)
+    a = rng.normal(size=300) * 10
+    a[::7] = a[1]
+    u, v = rng.normal(size=300), rng.normal(size=300)
+    Ku, Kv = O.sym(a, u), O.sym(a, v)
+    assert abs(u @ Kv - Ku @ v) < 1e-10 * np.abs(u).sum() * np.abs(Kv).max()
+    np.testing.assert_allclose(O.sym(a + 123.5, v), Kv, rtol=1e-9)
+    np.testing.assert_allclose(O.sym(-a, v), Kv, rtol=1e-12)
+    p = rng.permutation(300)
+    np.testing.assert_allclose(O.sym(a[p], v[p]), Kv[p], rtol=1e-12)
+
+
+def test_general_reduces_to_symmetric_and_transpose_identity():
+    rng = np.random.default_rng(6)
+    a = rng.uniform(-5, 5, size=120)
+    b = rng.uniform(-5, 5, size=77)
+    b[:10] = a[20:30]
+    x, w = rng.normal(size=77), rng.normal(size=120)
+    np.testing.assert_allclose(O.general(a, a, w), O.sym(a, w), rtol=1e-12, atol=1e-12)
+    assert abs(w @ O.general(a, b, x) - O.general_T(a, b, w) @ x) < 1e-10
+
+
+def test_phased_reduces_and_matches_definition():
+    rng = np.random.default_rng(7)
+    a = rng.uniform(0, 20, size=90)
+    b = rng.uniform(0, 20, size=60)
+    phi, psi = rng.uniform(0, 2 * np.pi, 90), rng.uniform(0, 2 * np.pi, 60)
+    v, x = rng.normal(size=90), rng.normal(size=60)
+    np.testing.assert_allclose(O.phased(a, np.zeros(90), v), O.sym(a, v), rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(O.phased(a, phi, v), O.dense_matvec(a, v, phi=phi), atol=1e-12)
+    np.testing.assert_allclose(O.phased(a, phi, x, b, psi),
+                               O.dense_matvec(a, x, b=b, phi=phi, psi=psi), atol=1e-12)
+    # a common phase shift cancels in cos(phi_j - phi_k)
+    np.testing.assert_allclose(O.phased(a, phi + 1.0, v), O.phased(a, phi, v), atol=1e-12)
+
+
+def test_gram_is_psd_and_composes():
+    rng = np.random.default_rng(8)
+    a = rng.uniform(0, 30, size=150)
+    phi = rng.uniform(0, 2 * np.pi, 150)
+    D = rng.uniform(0.5, 2, 150)
+    v = rng.normal(size=150)
+    K = O.dense_matrix(a, phi=phi)
+    z = O.gram(a, v, phi=phi, D=D)
+    np.testing.assert_allclose(z, K.T @ (D * (K @ v)), atol=1e-11)
+    assert v @ z >= 0
+    np.testing.assert_allclose(v @ z, np.sum(D * (K @ v) ** 2), rtol=1e-10)
+    b = rng.uniform(0, 30, size=70)
+    w = rng.normal(size=70)
+    Kg = O.dense_matrix(a, b)
+    np.testing.assert_allclose(O.gram(a, w, b=b), Kg.T @ (Kg @ w), atol=1e-10)
+
+
+def test_normaliser_bounds():
+    rng = np.random.default_rng(9)
+    a = rng.uniform(0, 10, size=80)
+    phi = rng.uniform(0, 6, 80)
+    x = rng.normal(size=80)
+    nrm = O.norm_sym(a, x)
+    assert np.all(np.abs(O.sym(a, x)) <= nrm + 1e-12)
+    assert np.all(np.abs(O.phased(a, phi, x)) <= nrm + 1e-12)
+
+
+# ---------------------------------------------------------------------------
+# brute force / dense agreement of the sequential routes
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n,B,ties", [(0, 1, False), (1, 1, False), (2, 3, True), (3, 1, True),
+                                      (17, 2, True), (257, 1, False), (1000, 4, True)])
+def test_sequential_matches_dense(n, B, ties):
+    rng = np.random.default_rng(n + B)
+    a = rng.normal(size=n) * (n ** 0.5 + 1)
+    if ties and n > 1:
+        a[rng.integers(0, n, n // 3 + 1)] = a[0]
+        a = np.round(a, 0)
+    x = rng.normal(size=(n, B))
+    np.testing.assert_allclose(O.sym(a, x), O.dense_matvec(a, x), rtol=1e-12, atol=1e-12)
+    k = max(1, n // 2 + 3)
+    b = np.round(rng.normal(size=k) * (n ** 0.5 + 1), 1)
+    if n:
+        b[: k // 4] = a[rng.integers(0, n, k // 4)]
+    xb = rng.normal(size=(k, B))
+    np.testing.assert_allclose(O.general(a, b, xb), O.dense_matvec(a, xb, b=b), rtol=1e-12, atol=1e-12)
+
+
+def test_rows_window_matches_dense_rows():
+    rng = np.random.default_rng(11)
+    n = 2000
+    a = rng.uniform(0, 3000, size=n)
+    a[::5] = np.round(a[::5])
+    phi = rng.uniform(0, 2 * np.pi, n)
+    x = rng.normal(size=(n, 2))
+    s, perm = O.stable_sort(a)
+    rowsel = rng.integers(0, n, 50)
+    out, sgn, absn = O.rows(a[rowsel], s, x[perm])
+    K = O.dense_matrix(a)
+    np.testing.assert_allclose(out, (K @ x)[rowsel], atol=1e-12)
+    np.testing.assert_allclose(absn, (K @ np.abs(x))[rowsel], atol=1e-12)
+    S = np.sign(a[:, None] - a[None, :]) * K
+    np.testing.assert_allclose(sgn, (S @ x)[rowsel], atol=1e-12)
+    outp, _, _ = O.rows(a[rowsel], s, x[perm, 0], rphi=phi[rowsel], spsi=phi[perm])
+    np.testing.assert_allclose(outp, O.dense_matvec(a, x[:, 0], phi=phi)[rowsel], atol=1e-12)
+
+
+def test_sort_matches_brute_force_comparator():
+    rng = np.random.default_rng(12)
+    specials = np.array([0.0, -0.0, 1e-45, -1e-45, 1e-40, 5e-324, -5e-324, 2.0, -2.0], dtype=np.float64)
+    for trial in range(20):
+        n = int(rng.integers(0, 40))
+        a = rng.choice(np.concatenate([specials, rng.normal(size=5)]), size=n)
+        a32 = a.astype(np.float32)
+        s, perm = O.stable_sort(a32)
+        brute = sorted(range(n), key=lambda i: (float(a32[i]), i))
+        assert perm.tolist() == brute
+        assert np.array_equal(s, a32[perm].astype(np.float64))
+    with pytest.raises(ValueError):
+        O.stable_sort(np.array([1.0, np.nan]))
+    with pytest.raises(ValueError):
+        O.stable_sort(np.array([np.inf, 1.0]))
+
+
+# ---------------------------------------------------------------------------
+# backward pass
+# ---------------------------------------------------------------------------
+
+def _loss(a, x, g):
+    return float(g @ O.dense_matvec(a, x))
+
+
+@pytest.mark.parametrize("tied", [False, True])
+def test_backward_central_differences(tied):
+    """Central differences of L = <g, K x>.  At a tie the two one-sided slopes of
+    exp(-|t|) are opposite, so the central difference is the sign(0) = 0 value."""
+    rng = np.random.default_rng(13 + tied)
+    n = 40
+    a = rng.uniform(0, 8, size=n)
+    if tied:
+        a[[4, 11, 30]] = a[2]
+    x, g = rng.normal(size=n), rng.normal(size=n)
+    dx, da = O.backward(a, x, g)
+    h = 1e-6
+    fd = np.empty(n)
+    for m in range(n):
+        ap, am = a.copy(), a.copy()
+        ap[m] += h
+        am[m] -= h
+        fd[m] = (_loss(ap, x, g) - _loss(am, x, g)) / (2 * h)
+    np.testing.assert_allclose(da, fd, rtol=0, atol=5e-8 * np.abs(fd).max())
+    for m in (0, 7):
+        e = np.zeros(n)
+        e[m] = 1
+        assert abs(dx[m] - (_loss(a, x + e, g) - _loss(a, x, g))) < 1e-10
+    assert abs(da.sum()) < 1e-9 * np.abs(da).sum()  # translation invariance of L
+    dxd, dad = O.dense_backward(a, x, g)
+    np.testing.assert_allclose(dx, dxd, atol=1e-12)
+    np.testing.assert_allclose(da, dad, atol=1e-12)
+
+
+def test_signed_sums_brute_force():
+    rng = np.random.default_rng(14)
+    s = np.sort(np.round(rng.uniform(0, 6, size=60), 0))
+    v = rng.normal(size=(60, 2))
+    brute = np.zeros_like(v)
+    for i in range(60):
+        for j in range(60):
+            brute[i] += np.sign(s[i] - s[j]) * math.exp(-abs(s[i] - s[j])) * v[j]
+    np.testing.assert_allclose(O.signed_sorted(s, v), brute, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# the pins catch planted mistakes (mutants built on the CPU from the oracle)
+# ---------------------------------------------------------------------------
+
+def _lower_only(s, x):
+    out, acc = np.empty_like(x), 0.0
+    for i in range(len(x)):
+        acc = x[i] + (math.exp(s[i - 1] - s[i]) * acc if i else 0.0)
+        out[i] = acc
+    return out
+
+
+def test_pins_reject_planted_mistakes():
+    rng = np.random.default_rng(15)
+    s = np.cumsum(rng.uniform(0.05, 2.0, size=64))
+    x = rng.normal(size=64)
+    diag, off = _ou_precision(s)
+
+    def ou_residual(y):
+        back = diag * y
+        back[:-1] += off * y[1:]
+        back[1:] += off * y[:-1]
+        return np.abs(back - x).max()
+
+    good = O.sym_sorted(s, x)
+    assert ou_residual(good) < 1e-10
+    mutants = {
+        "diagonal counted twice (dropped -x)": good + x,
+        "lower part only": _lower_only(s, x),
+        "reversed anchor order": O.sym_sorted(s[::-1].copy(), x),
+        "operand transposed (x reversed)": O.sym_sorted(s, x[::-1].copy()),
+    }
+    for name, y in mutants.items():
+        assert ou_residual(y) > 1e-3, name
+    # general case with a and b swapped is K^T, not K
+    a = rng.uniform(0, 5, 30)
+    b = rng.uniform(0, 5, 30)
+    xb = rng.normal(size=30)
+    assert np.abs(O.general(b, a, xb) - O.dense_matvec(a, xb, b=b)).max() > 1e-3
+    # backward with the sign of the signed sums flipped fails the finite differences
+    xx, gg = rng.normal(size=30), rng.normal(size=30)
+    _, da = O.backward(a, xx, gg)
+    h = 1e-6
+    ap, am = a.copy(), a.copy()
+    ap[3] += h
+    am[3] -= h
+    fd = (_loss(ap, xx, gg) - _loss(am, xx, gg)) / (2 * h)
+    assert abs(da[3] - fd) < 1e-6 and abs(-da[3] - fd) > 1e-3
+
+
+def test_generator_is_seeded_and_sorted():
+    a1 = synth.uniform(1000, 0, 64, seed=0)
+    assert np.array_equal(a1, synth.uniform(1000, 0, 64, seed=0))
+    assert not np.array_equal(a1, synth.uniform(1000, 0, 64, seed=1))
+    assert np.array_equal(synth.uniform(1000, 0, 64)[500:], synth.uniform(1000, 0, 64)[500:])
+    s = synth.sorted_uniform(100000, 0, 2.0 ** 30)
+    assert np.all(np.diff(s) >= 0) and s[0] >= 0 and s[-1] <= 2.0 ** 30
+    # sorted order statistics have the uniform distribution: compare quartiles
+    assert abs(np.median(s) / 2.0 ** 30 - 0.5) < 0.01
+    z = synth.normal(200000)
+    assert abs(z.mean()) < 0.01 and abs(z.std() - 1) < 0.01
