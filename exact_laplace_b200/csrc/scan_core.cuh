@@ -1,0 +1,310 @@
+// scan_core.cuh -- the first-order linear-recurrence scan of the LAPLEX products.
+//
+// With anchors ascending, the lower part L_i = sum_{j<=i} exp(s_j - s_i) x_j and
+// the upper part U_i = sum_{j>=i} exp(s_i - s_j) x_j obey
+//     L_i = x_i + exp(s_{i-1} - s_i) L_{i-1},   U_i = x_i + exp(s_i - s_{i+1}) U_{i+1}
+// ("LAPLEX - La FFT dei Nuclei di Laplace Apprendibili", technical summary, §2.2).
+// A run of elements is summarised by a pair: forward (e, V) = "V is L at the
+// element whose anchor is e, counting only that run"; backward (f, W) = "W is
+// U at the element whose anchor is f".  Runs combine associatively:
+//     forward   P (+) A  = (e_A, V_A + exp(e_P - e_A) V_P)      P left of A
+//     backward  A (+) S  = (f_A, W_A + exp(f_A - f_S) W_S)      A left of S
+// The decay across any number of elements is one exp of an anchor difference,
+// never a product of rounded per-step decays, so fp32 error does not grow with
+// the distance between tiles.  Elements past the end are padded with the last
+// anchor and value 0, which is neutral in both directions.
+#pragma once
+#include "common.cuh"
+
+namespace lx {
+
+// ---------------------------------------------------------------- warp level
+template <typename T, int C>
+__device__ __forceinline__ void warp_incl_fwd(const T e, T (&V)[C], const int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const T eo = __shfl_up_sync(FULL, e, off);
+        T Vo[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) Vo[c] = __shfl_up_sync(FULL, V[c], off);
+        if (lane >= off) {
+            const T d = dexp<T>(eo - e);
+#pragma unroll
+            for (int c = 0; c < C; ++c) V[c] = dfma<T>(d, Vo[c], V[c]);
+        }
+    }
+}
+
+template <typename T, int C>
+__device__ __forceinline__ void warp_incl_bwd(const T f, T (&W)[C], const int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const T fo = __shfl_down_sync(FULL, f, off);
+        T Wo[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) Wo[c] = __shfl_down_sync(FULL, W[c], off);
+        if (lane + off < 32) {
+            const T d = dexp<T>(f - fo);
+#pragma unroll
+            for (int c = 0; c < C; ++c) W[c] = dfma<T>(d, Wo[c], W[c]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- block level
+template <typename T, int C, int NT>
+struct BlockScanSmem {
+    static constexpr int NW = NT / 32;
+    T we[NW];
+    T wV[NW][C];
+    T pe[NW];      // exclusive prefix (forward) / suffix (backward) of each warp
+    T pV[NW][C];
+    T te;          // block total
+    T tV[C];
+};
+
+// Exclusive forward scan over the threads of the block, in thread order.
+// In: this thread's run summary (e, V).  Out: has (false for thread 0), the
+// summary (pe, pV) of all runs of lower threads, and the block total (te, tV).
+template <typename T, int C, int NT>
+__device__ __forceinline__ void block_excl_fwd(const T e, const T (&V)[C], bool& has, T& pe,
+                                               T (&pV)[C], T& te, T (&tV)[C],
+                                               BlockScanSmem<T, C, NT>& sm) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    T iV[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) iV[c] = V[c];
+    warp_incl_fwd<T, C>(e, iV, lane);
+    if (lane == 31) {
+        sm.we[w] = e;
+#pragma unroll
+        for (int c = 0; c < C; ++c) sm.wV[w][c] = iV[c];
+    }
+    __syncthreads();
+    if (w == 0) {
+        T ge = lane < NW ? sm.we[lane] : T(0);
+        T gV[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) gV[c] = lane < NW ? sm.wV[lane][c] : T(0);
+#pragma unroll
+        for (int off = 1; off < NW; off <<= 1) {
+            const T eo = __shfl_up_sync(FULL, ge, off);
+            T Vo[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) Vo[c] = __shfl_up_sync(FULL, gV[c], off);
+            if (lane >= off && lane < NW) {
+                const T d = dexp<T>(eo - ge);
+#pragma unroll
+                for (int c = 0; c < C; ++c) gV[c] = dfma<T>(d, Vo[c], gV[c]);
+            }
+        }
+        const T xe = __shfl_up_sync(FULL, ge, 1);
+        T xV[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) xV[c] = __shfl_up_sync(FULL, gV[c], 1);
+        if (lane > 0 && lane < NW) {
+            sm.pe[lane] = xe;
+#pragma unroll
+            for (int c = 0; c < C; ++c) sm.pV[lane][c] = xV[c];
+        }
+        if (lane == NW - 1) {
+            sm.te = ge;
+#pragma unroll
+            for (int c = 0; c < C; ++c) sm.tV[c] = gV[c];
+        }
+    }
+    __syncthreads();
+    const T le = __shfl_up_sync(FULL, e, 1);
+    T lV[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) lV[c] = __shfl_up_sync(FULL, iV[c], 1);
+    if (w > 0 && lane > 0) {
+        has = true;
+        pe = le;
+        const T d = dexp<T>(sm.pe[w] - le);
+#pragma unroll
+        for (int c = 0; c < C; ++c) pV[c] = dfma<T>(d, sm.pV[w][c], lV[c]);
+    } else if (w > 0) {
+        has = true;
+        pe = sm.pe[w];
+#pragma unroll
+        for (int c = 0; c < C; ++c) pV[c] = sm.pV[w][c];
+    } else if (lane > 0) {
+        has = true;
+        pe = le;
+#pragma unroll
+        for (int c = 0; c < C; ++c) pV[c] = lV[c];
+    } else {
+        has = false;
+        pe = T(0);
+#pragma unroll
+        for (int c = 0; c < C; ++c) pV[c] = T(0);
+    }
+    te = sm.te;
+#pragma unroll
+    for (int c = 0; c < C; ++c) tV[c] = sm.tV[c];
+}
+
+// Exclusive backward scan (suffix over higher threads), mirror of block_excl_fwd.
+template <typename T, int C, int NT>
+__device__ __forceinline__ void block_excl_bwd(const T f, const T (&W)[C], bool& has, T& nf,
+                                               T (&nW)[C], T& tf, T (&tW)[C],
+                                               BlockScanSmem<T, C, NT>& sm) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    T iW[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) iW[c] = W[c];
+    warp_incl_bwd<T, C>(f, iW, lane);
+    if (lane == 0) {
+        sm.we[w] = f;
+#pragma unroll
+        for (int c = 0; c < C; ++c) sm.wV[w][c] = iW[c];
+    }
+    __syncthreads();
+    if (w == 0) {
+        T gf = lane < NW ? sm.we[lane] : T(0);
+        T gW[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) gW[c] = lane < NW ? sm.wV[lane][c] : T(0);
+#pragma unroll
+        for (int off = 1; off < NW; off <<= 1) {
+            const T fo = __shfl_down_sync(FULL, gf, off);
+            T Wo[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) Wo[c] = __shfl_down_sync(FULL, gW[c], off);
+            if (lane + off < NW) {
+                const T d = dexp<T>(gf - fo);
+#pragma unroll
+                for (int c = 0; c < C; ++c) gW[c] = dfma<T>(d, Wo[c], gW[c]);
+            }
+        }
+        const T xf = __shfl_down_sync(FULL, gf, 1);
+        T xW[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) xW[c] = __shfl_down_sync(FULL, gW[c], 1);
+        if (lane < NW - 1) {
+            sm.pe[lane] = xf;
+#pragma unroll
+            for (int c = 0; c < C; ++c) sm.pV[lane][c] = xW[c];
+        }
+        if (lane == 0) {
+            sm.te = gf;
+#pragma unroll
+            for (int c = 0; c < C; ++c) sm.tV[c] = gW[c];
+        }
+    }
+    __syncthreads();
+    const T lf = __shfl_down_sync(FULL, f, 1);
+    T lW[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) lW[c] = __shfl_down_sync(FULL, iW[c], 1);
+    if (w < NW - 1 && lane < 31) {
+        has = true;
+        nf = lf;
+        const T d = dexp<T>(lf - sm.pe[w]);
+#pragma unroll
+        for (int c = 0; c < C; ++c) nW[c] = dfma<T>(d, sm.pV[w][c], lW[c]);
+    } else if (w < NW - 1) {
+        has = true;
+        nf = sm.pe[w];
+#pragma unroll
+        for (int c = 0; c < C; ++c) nW[c] = sm.pV[w][c];
+    } else if (lane < 31) {
+        has = true;
+        nf = lf;
+#pragma unroll
+        for (int c = 0; c < C; ++c) nW[c] = lW[c];
+    } else {
+        has = false;
+        nf = T(0);
+#pragma unroll
+        for (int c = 0; c < C; ++c) nW[c] = T(0);
+    }
+    tf = sm.te;
+#pragma unroll
+    for (int c = 0; c < C; ++c) tW[c] = sm.tV[c];
+}
+
+// ---------------------------------------------------------------- chunk level
+// A thread owns E consecutive elements: anchors s[E], values v[E][C].
+// dl[i] = exp(s[i-1] - s[i]) for i = 1..E-1 (dl[0] is set in chunk_final).
+template <typename T, int C, int E>
+__device__ __forceinline__ void chunk_aggregates(const T (&s)[E], const T (&v)[E][C], T (&dl)[E],
+                                                 T (&fV)[C], T (&bW)[C]) {
+#pragma unroll
+    for (int i = 1; i < E; ++i) dl[i] = dexp<T>(s[i - 1] - s[i]);
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        T a = v[0][c];
+#pragma unroll
+        for (int i = 1; i < E; ++i) a = dfma<T>(dl[i], a, v[i][c]);
+        fV[c] = a;
+        T b = v[E - 1][c];
+#pragma unroll
+        for (int i = E - 2; i >= 0; --i) b = dfma<T>(dl[i + 1], b, v[i][c]);
+        bW[c] = b;
+    }
+}
+
+// Given the state just before the chunk (anchor eprev, value Lprev) and just
+// after it (anchor enext, value Unext), out[i][c] = L_i + U_i - v_i.
+template <typename T, int C, int E>
+__device__ __forceinline__ void chunk_final(const T (&s)[E], const T (&v)[E][C], T (&dl)[E],
+                                            const T eprev, const T (&Lprev)[C], const T enext,
+                                            const T (&Unext)[C], T (&out)[E][C]) {
+    dl[0] = dexp<T>(eprev - s[0]);
+    const T dn = dexp<T>(s[E - 1] - enext);
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        T L = Lprev[c];
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            L = dfma<T>(dl[i], L, v[i][c]);
+            out[i][c] = L;
+        }
+        T U = dfma<T>(dn, Unext[c], v[E - 1][c]);
+        out[E - 1][c] += U - v[E - 1][c];
+#pragma unroll
+        for (int i = E - 2; i >= 0; --i) {
+            U = dfma<T>(dl[i + 1], U, v[i][c]);
+            out[i][c] += U - v[i][c];
+        }
+    }
+}
+
+// Combine a thread's in-tile exclusive prefix with the tile's carry-in.
+template <typename T, int C>
+__device__ __forceinline__ void apply_carry_fwd(const bool has, const T pe, const T (&pV)[C],
+                                                const T eT, const T (&VT)[C], T& eprev,
+                                                T (&Lprev)[C]) {
+    if (has) {
+        eprev = pe;
+        const T d = dexp<T>(eT - pe);
+#pragma unroll
+        for (int c = 0; c < C; ++c) Lprev[c] = dfma<T>(d, VT[c], pV[c]);
+    } else {
+        eprev = eT;
+#pragma unroll
+        for (int c = 0; c < C; ++c) Lprev[c] = VT[c];
+    }
+}
+
+template <typename T, int C>
+__device__ __forceinline__ void apply_carry_bwd(const bool has, const T nf, const T (&nW)[C],
+                                                const T fT, const T (&WT)[C], T& enext,
+                                                T (&Unext)[C]) {
+    if (has) {
+        enext = nf;
+        const T d = dexp<T>(nf - fT);
+#pragma unroll
+        for (int c = 0; c < C; ++c) Unext[c] = dfma<T>(d, WT[c], nW[c]);
+    } else {
+        enext = fT;
+#pragma unroll
+        for (int c = 0; c < C; ++c) Unext[c] = WT[c];
+    }
+}
+
+}  // namespace lx

@@ -1,0 +1,326 @@
+// sym.cu -- symmetric and phased-symmetric LAPLEX products on sorted anchors.
+//
+//   y = K x,   K_ij = exp(-|s_i - s_j|)                      (summary §2.1, §2.2)
+//   y = K x,   K_ij = exp(-|s_i - s_j|) cos(phi_i - phi_j)   (phased, §2.1)
+//
+// The phased product runs two unphased channels, cos(phi) x and sin(phi) x, and
+// recombines them with cos(phi_i) and sin(phi_i) (cos(p - q) = cos p cos q +
+// sin p sin q).  Each channel is the recurrence pair of scan_core.cuh.
+//
+// Three-phase reduce-then-scan over tiles of NT*E elements:
+//   1. k_sym_reduce   : per-tile forward/backward totals     (reads s, x)
+//   2. k_tile_carries : carries into every tile              (tiny)
+//   3. k_sym_final    : scans each tile again with its carries, writes y
+#include <algorithm>
+
+#include "laplex_impl.h"
+#include "scan_core.cuh"
+
+namespace lx {
+
+constexpr int SYM_NT = 256;
+
+template <typename T> __device__ __forceinline__ void dsincos(T a, T* s, T* c);
+template <> __device__ __forceinline__ void dsincos<float>(float a, float* s, float* c) { sincosf(a, s, c); }
+template <> __device__ __forceinline__ void dsincos<double>(double a, double* s, double* c) { sincos(a, s, c); }
+
+// Load the chunk [r0, r0 + E) : anchors, channel values, and (phased) cos/sin.
+template <typename T, int NCOL, bool PHASED, int E>
+__device__ __forceinline__ void sym_load(const SymArgs<T>& A, const int64_t r0, T (&s)[E],
+                                         T (&v)[E][PHASED ? 2 * NCOL : NCOL], T (&cph)[E],
+                                         T (&sph)[E]) {
+    constexpr int VN = V16<T>::N;
+    const int64_t n = A.n;
+    const bool full = r0 + E <= n;
+    if (full) {
+#pragma unroll
+        for (int i = 0; i < E; i += VN) ld16_stream<T>(A.s + r0 + i, &s[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < E; ++i) s[i] = A.s[min(r0 + i, n - 1)];
+    }
+    if (!PHASED && NCOL == 1 && full && A.pin == nullptr && A.D == nullptr && A.ldx == 1) {
+        T t[E];
+#pragma unroll
+        for (int i = 0; i < E; i += VN) ld16_stream<T>(A.x + r0 + i, &t[i]);
+#pragma unroll
+        for (int i = 0; i < E; ++i) v[i][0] = t[i];
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int64_t r = r0 + i;
+        if (r < n) {
+            const int64_t row = A.pin ? (int64_t)A.pin[r] : r;
+            const int64_t ar = A.paux ? (int64_t)A.paux[r] : r;
+            const T dsc = A.D ? A.D[ar] : T(1);
+            if (PHASED) dsincos<T>(A.phi[ar], &sph[i], &cph[i]);
+            const T* xr = A.x + row * A.ldx + A.col0;
+            T xv[NCOL];
+            if (NCOL >= VN && (NCOL % VN) == 0 && A.ncol == NCOL && (A.ldx % VN) == 0 &&
+                (A.col0 % VN) == 0) {
+#pragma unroll
+                for (int c = 0; c < NCOL; c += VN) ld16<T>(xr + c, &xv[c]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < NCOL; ++c) xv[c] = c < A.ncol ? xr[c] : T(0);
+            }
+#pragma unroll
+            for (int c = 0; c < NCOL; ++c) {
+                const T val = xv[c] * dsc;
+                if (PHASED) {
+                    v[i][2 * c] = cph[i] * val;
+                    v[i][2 * c + 1] = sph[i] * val;
+                } else {
+                    v[i][c] = val;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < (PHASED ? 2 * NCOL : NCOL); ++c) v[i][c] = T(0);
+            cph[i] = T(0);
+            sph[i] = T(0);
+        }
+    }
+}
+
+template <typename T, int NCOL, bool PHASED, int E>
+__device__ __forceinline__ void sym_store(const SymArgs<T>& A, const int64_t r0,
+                                          const T (&out)[E][PHASED ? 2 * NCOL : NCOL],
+                                          const T (&cph)[E], const T (&sph)[E]) {
+    constexpr int VN = V16<T>::N;
+    const int64_t n = A.n;
+    const bool full = r0 + E <= n;
+    if (!PHASED && NCOL == 1 && full && A.pout == nullptr && A.ldy == 1) {
+        T t[E];
+#pragma unroll
+        for (int i = 0; i < E; ++i) t[i] = out[i][0];
+#pragma unroll
+        for (int i = 0; i < E; i += VN) st16_stream<T>(A.y + r0 + i, &t[i]);
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        const int64_t r = r0 + i;
+        if (r < n) {
+            const int64_t row = A.pout ? (int64_t)A.pout[r] : r;
+            T* yr = A.y + row * A.ldy + A.col0;
+            T yv[NCOL];
+#pragma unroll
+            for (int c = 0; c < NCOL; ++c)
+                yv[c] = PHASED ? cph[i] * out[i][2 * c] + sph[i] * out[i][2 * c + 1] : out[i][c];
+            if (NCOL >= VN && (NCOL % VN) == 0 && A.ncol == NCOL && (A.ldy % VN) == 0 &&
+                (A.col0 % VN) == 0) {
+#pragma unroll
+                for (int c = 0; c < NCOL; c += VN) st16<T>(yr + c, &yv[c]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < NCOL; ++c)
+                    if (c < A.ncol) yr[c] = yv[c];
+            }
+        }
+    }
+}
+
+template <typename T, int NCOL, bool PHASED, int E, int NT>
+__global__ void __launch_bounds__(NT) k_sym_reduce(SymArgs<T> A, T* __restrict__ aggF,
+                                                   T* __restrict__ aggB) {
+    constexpr int C = PHASED ? 2 * NCOL : NCOL;
+    __shared__ BlockScanSmem<T, C, NT> smf, smb;
+    const int64_t r0 = (int64_t)blockIdx.x * (NT * E) + (int64_t)threadIdx.x * E;
+    T s[E], v[E][C], cph[E], sph[E], dl[E], fV[C], bW[C];
+    sym_load<T, NCOL, PHASED, E>(A, r0, s, v, cph, sph);
+    chunk_aggregates<T, C, E>(s, v, dl, fV, bW);
+    bool hf, hb;
+    T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
+    block_excl_fwd<T, C, NT>(s[E - 1], fV, hf, pe, pV, te, tV, smf);
+    block_excl_bwd<T, C, NT>(s[0], bW, hb, nf, nW, tf, tW, smb);
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            aggF[(int64_t)blockIdx.x * C + c] = tV[c];
+            aggB[(int64_t)blockIdx.x * C + c] = tW[c];
+        }
+    }
+}
+
+// Carries into each tile from the tile totals (one block; segments per thread).
+// carF[t] = L at the element before tile t (anchor = last anchor of tile t-1);
+// carB[t] = U at the element after tile t (anchor = first anchor of tile t+1).
+template <typename T, int C, int NT>
+__global__ void __launch_bounds__(NT) k_tile_carries(const T* __restrict__ s, int64_t n, int64_t tile,
+                                                     int64_t ntiles, const T* __restrict__ aggF,
+                                                     const T* __restrict__ aggB, T* __restrict__ carF,
+                                                     T* __restrict__ carB) {
+    __shared__ BlockScanSmem<T, C, NT> smf, smb;
+    const int64_t per = (ntiles + NT - 1) / NT;
+    const int64_t t0 = min((int64_t)threadIdx.x * per, ntiles);
+    const int64_t t1 = min(t0 + per, ntiles);
+    auto eL = [&](int64_t t) { return s[min((t + 1) * tile, n) - 1]; };
+    auto eF = [&](int64_t t) { return s[min(t * tile, n - 1)]; };
+    const T pad = s[n - 1];
+    // forward
+    T ae = pad, aV[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) aV[c] = T(0);
+    for (int64_t t = t0; t < t1; ++t) {
+        const T e = eL(t);
+        const T d = (t == t0) ? T(0) : dexp<T>(ae - e);
+#pragma unroll
+        for (int c = 0; c < C; ++c) aV[c] = dfma<T>(d, aV[c], aggF[t * C + c]);
+        ae = e;
+    }
+    bool has;
+    T pe, pV[C], te, tV[C];
+    block_excl_fwd<T, C, NT>(ae, aV, has, pe, pV, te, tV, smf);
+    T ce = has ? pe : s[0], cv[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) cv[c] = has ? pV[c] : T(0);
+    for (int64_t t = t0; t < t1; ++t) {
+#pragma unroll
+        for (int c = 0; c < C; ++c) carF[t * C + c] = cv[c];
+        const T e = eL(t);
+        const T d = dexp<T>(ce - e);
+#pragma unroll
+        for (int c = 0; c < C; ++c) cv[c] = dfma<T>(d, cv[c], aggF[t * C + c]);
+        ce = e;
+    }
+    // backward
+    T bf = pad, bW[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) bW[c] = T(0);
+    for (int64_t t = t1 - 1; t >= t0; --t) {
+        const T f = eF(t);
+        const T d = (t == t1 - 1) ? T(0) : dexp<T>(f - bf);
+#pragma unroll
+        for (int c = 0; c < C; ++c) bW[c] = dfma<T>(d, bW[c], aggB[t * C + c]);
+        bf = f;
+    }
+    T nf, nW[C], tf, tW[C];
+    block_excl_bwd<T, C, NT>(bf, bW, has, nf, nW, tf, tW, smb);
+    T cf = has ? nf : pad, cw[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) cw[c] = has ? nW[c] : T(0);
+    for (int64_t t = t1 - 1; t >= t0; --t) {
+#pragma unroll
+        for (int c = 0; c < C; ++c) carB[t * C + c] = cw[c];
+        const T f = eF(t);
+        const T d = dexp<T>(f - cf);
+#pragma unroll
+        for (int c = 0; c < C; ++c) cw[c] = dfma<T>(d, cw[c], aggB[t * C + c]);
+        cf = f;
+    }
+}
+
+template <typename T, int NCOL, bool PHASED, int E, int NT>
+__global__ void __launch_bounds__(NT) k_sym_final(SymArgs<T> A, const T* __restrict__ carF,
+                                                  const T* __restrict__ carB) {
+    constexpr int C = PHASED ? 2 * NCOL : NCOL;
+    __shared__ BlockScanSmem<T, C, NT> smf, smb;
+    const int64_t tile0 = (int64_t)blockIdx.x * (NT * E);
+    const int64_t r0 = tile0 + (int64_t)threadIdx.x * E;
+    T s[E], v[E][C], cph[E], sph[E], dl[E], fV[C], bW[C];
+    sym_load<T, NCOL, PHASED, E>(A, r0, s, v, cph, sph);
+    chunk_aggregates<T, C, E>(s, v, dl, fV, bW);
+    bool hf, hb;
+    T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
+    block_excl_fwd<T, C, NT>(s[E - 1], fV, hf, pe, pV, te, tV, smf);
+    block_excl_bwd<T, C, NT>(s[0], bW, hb, nf, nW, tf, tW, smb);
+    const int64_t n = A.n;
+    const T eT = tile0 > 0 ? A.s[tile0 - 1] : A.s[0];
+    const T fT = tile0 + NT * E < n ? A.s[tile0 + NT * E] : A.s[n - 1];
+    T VT[C], WT[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        VT[c] = carF[(int64_t)blockIdx.x * C + c];
+        WT[c] = carB[(int64_t)blockIdx.x * C + c];
+    }
+    T eprev, Lprev[C], enext, Unext[C], out[E][C];
+    apply_carry_fwd<T, C>(hf, pe, pV, eT, VT, eprev, Lprev);
+    apply_carry_bwd<T, C>(hb, nf, nW, fT, WT, enext, Unext);
+    chunk_final<T, C, E>(s, v, dl, eprev, Lprev, enext, Unext, out);
+    sym_store<T, NCOL, PHASED, E>(A, r0, out, cph, sph);
+}
+
+// ------------------------------------------------------------------ host side
+struct SymPlan {
+    int ncol;  // template columns per pass
+    int C;     // channels per pass
+    int E;     // elements per thread
+    int64_t tile;
+    int64_t ntiles;
+    int64_t groups;
+};
+
+static SymPlan sym_plan(int64_t n, int64_t B, bool phased, int f64) {
+    SymPlan p;
+    const int maxcol = phased ? 4 : 8;
+    int nc = 1;
+    while (nc < B && nc < maxcol) nc <<= 1;
+    p.ncol = nc;
+    p.C = phased ? 2 * nc : nc;
+    if (p.C == 1) p.E = f64 ? 8 : 16;
+    else if (p.C == 2) p.E = 8;
+    else p.E = 4;
+    p.tile = (int64_t)SYM_NT * p.E;
+    p.ntiles = (n + p.tile - 1) / p.tile;
+    p.groups = (B + nc - 1) / nc;
+    return p;
+}
+
+size_t sym_ws_bytes(int64_t n, int64_t B, bool phased, int f64) {
+    const SymPlan p = sym_plan(n, B, phased, f64);
+    const size_t es = f64 ? 8 : 4;
+    return 4 * Carve::need((size_t)(p.ntiles * p.C), es);
+}
+
+template <typename T, int NCOL, bool PHASED, int E>
+static cudaError_t sym_launch(const SymArgs<T>& A, int64_t ntiles, T* aggF, T* aggB, T* carF,
+                              T* carB, cudaStream_t st) {
+    constexpr int C = PHASED ? 2 * NCOL : NCOL;
+    k_sym_reduce<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, aggF, aggB);
+    k_tile_carries<T, C, 1024><<<1, 1024, 0, st>>>(A.s, A.n, (int64_t)SYM_NT * E, ntiles, aggF,
+                                                     aggB, carF, carB);
+    k_sym_final<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, carF, carB);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t sym_run(SymArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_bytes,
+                    cudaStream_t st) {
+    if (A.n == 0) return cudaSuccess;
+    const SymPlan p = sym_plan(A.n, B, phased, sizeof(T) == 8);
+    Carve cv(ws, ws_bytes);
+    T* aggF = cv.take<T>(p.ntiles * p.C);
+    T* aggB = cv.take<T>(p.ntiles * p.C);
+    T* carF = cv.take<T>(p.ntiles * p.C);
+    T* carB = cv.take<T>(p.ntiles * p.C);
+    if (!cv.ok) return cudaErrorInvalidValue;
+    for (int64_t g = 0; g < p.groups; ++g) {
+        A.col0 = g * p.ncol;
+        A.ncol = (int)std::min<int64_t>(p.ncol, B - A.col0);
+        cudaError_t e;
+        constexpr bool D = sizeof(T) == 8;
+        if (!phased) {
+            switch (p.ncol) {
+                case 1: e = sym_launch<T, 1, false, D ? 8 : 16>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
+                case 2: e = sym_launch<T, 2, false, 8>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
+                case 4: e = sym_launch<T, 4, false, 4>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
+                default: e = sym_launch<T, 8, false, 4>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
+            }
+        } else {
+            switch (p.ncol) {
+                case 1: e = sym_launch<T, 1, true, 8>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
+                case 2: e = sym_launch<T, 2, true, 4>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
+                default: e = sym_launch<T, 4, true, 4>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
+            }
+        }
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+template cudaError_t sym_run<float>(SymArgs<float>, int64_t, bool, void*, size_t, cudaStream_t);
+template cudaError_t sym_run<double>(SymArgs<double>, int64_t, bool, void*, size_t, cudaStream_t);
+
+}  // namespace lx

@@ -1,0 +1,186 @@
+/*
+ * laplex.h -- C ABI of liblaplex.so, the exact LAPLEX Laplace-kernel operator on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operator (page "Riepilogo Tecnico: LAPLEX - La FFT dei Nuclei di Laplace
+ * Apprendibili", gist.science technical summary of arXiv 2605.24584, §2.1
+ * "L'Operatore"; same text in the French summary, §2.1):
+ *
+ *     K_ij = exp(-|a_i - b_j|),      a in R^n, b in R^k (learnable 1-D anchors)
+ *     K_ij = exp(-|a_i - b_j|) * cos(phi_i - psi_j)     (phased variant)
+ *
+ * and its exact O(n log n) products (same page, §2.2 "Algebra di Scansione
+ * Esatta"): sort the anchors, then evaluate the lower and upper triangular
+ * parts as prefix and suffix recurrences, L_{i+1} = x_{i+1} + exp(a_i - a_{i+1}) L_i,
+ * never forming K.
+ *
+ * Common conventions
+ * ------------------
+ *  - Every pointer except `bytes` in laplex_workspace_size is a DEVICE pointer
+ *    on the current CUDA device, owned by the caller.  The library never
+ *    allocates, frees or retains memory; it keeps no state between calls.
+ *  - All work is enqueued asynchronously on `stream` (a cudaStream_t passed as
+ *    void*; NULL is the legacy default stream).  No call synchronises, except
+ *    laplex_get_device_status.
+ *  - dtype LAPLEX_F32: every floating array is float; LAPLEX_F64: double.
+ *    The kernels compute in that type.
+ *  - Vectors with B columns are row-major [len, B], contiguous.
+ *  - Every array must be 16-byte aligned; the workspace 256-byte aligned.
+ *  - Sizes: 0 <= n, k < 2^31; B >= 1.  Outputs must not overlap inputs.
+ *  - "sorted" anchors: ascending.  perm[r] (int32) is the caller-order index of
+ *    the r-th sorted anchor, as written by laplex_sort_anchors.  When a perm
+ *    pointer is non-NULL every per-anchor vector on that side (x, y, phi, ...)
+ *    is in the caller's original order and the kernels gather and scatter
+ *    through perm; when it is NULL those vectors are in sorted order.
+ *  - Workspace: `ws` of at least laplex_workspace_size(...) bytes.  Its first
+ *    256 bytes are a header holding a sticky device status word; zero the
+ *    header once before first use (laplex_workspace_init).  One workspace must
+ *    not be used by two calls that may run at the same time.
+ *  - Errors found on the host (bad argument, workspace too small, a failed CUDA
+ *    launch) return immediately with nothing enqueued, or, for a launch failure,
+ *    with earlier kernels of the call possibly enqueued; laplex_last_error()
+ *    then holds a message.  Errors found on the device (a non-finite anchor, an
+ *    inter-block wait that ran out) are recorded in the workspace header and
+ *    reported by laplex_get_device_status.  No call aborts or throws.
+ */
+#ifndef LAPLEX_H
+#define LAPLEX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LAPLEX_OK = 0,
+    LAPLEX_EINVAL = 1,      /* invalid argument (NULL, size, alignment, dtype) */
+    LAPLEX_ENONFINITE = 2,  /* an anchor was NaN or +-Inf (device-detected)    */
+    LAPLEX_EWORKSPACE = 3,  /* ws_bytes below laplex_workspace_size()           */
+    LAPLEX_ECUDA = 4,       /* a CUDA runtime call or launch failed             */
+    LAPLEX_ETIMEOUT = 5     /* a bounded inter-block wait expired (device)      */
+} laplex_status;
+
+typedef enum { LAPLEX_F32 = 0, LAPLEX_F64 = 1 } laplex_dtype;
+
+typedef enum {
+    LAPLEX_OP_SORT = 0,
+    LAPLEX_OP_MATVEC_SYM = 1,
+    LAPLEX_OP_MATVEC_GENERAL = 2,
+    LAPLEX_OP_MATVEC_PHASED = 3,
+    LAPLEX_OP_GRAM = 4,
+    LAPLEX_OP_BACKWARD = 5
+} laplex_op;
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+int laplex_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* laplex_status_string(laplex_status s);
+
+/* Message of the last host-side error on the calling thread ("" if none). */
+const char* laplex_last_error(void);
+
+/*
+ * Workspace bytes needed by `op` for these sizes (host only, no device work).
+ * n: anchors of a; k: anchors of b (0 for symmetric ops and the sort);
+ * B: columns of x (1 for the sort and the backward pass).
+ * For LAPLEX_OP_SORT, n is the number of keys.  The result covers every
+ * variant of the op (with or without perm, transposed or not) and includes
+ * the 256-byte header.  Errors: EINVAL for negative/oversized sizes or NULL bytes.
+ */
+laplex_status laplex_workspace_size(laplex_op op, int64_t n, int64_t k, int64_t B,
+                                    laplex_dtype dtype, size_t* bytes);
+
+/* Zero the workspace header (async on stream).  Call once per new workspace. */
+laplex_status laplex_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Wait for `stream`, read the sticky device status of `ws`, clear it, and
+ * return it: LAPLEX_OK, LAPLEX_ENONFINITE or LAPLEX_ETIMEOUT (ECUDA if the
+ * wait or the read fails).  The only call that synchronises.
+ */
+laplex_status laplex_get_device_status(void* ws, void* stream);
+
+/*
+ * Sort the anchors ("after sorting the anchors", summary §2.2; the O(n log n)
+ * term of the method, §2.2 and §3).
+ *   a      [n]   caller's anchors (read only).
+ *   sorted [n]   out: the anchors ascending.  -0.0 is stored as +0.0.
+ *   perm   [n]   out: int32, sorted[r] == a[perm[r]] (numerically); ties in
+ *                ascending caller index, so perm is unique.
+ * Stable LSD radix sort of the IEEE bit patterns.  A NaN or +-Inf anchor sets
+ * LAPLEX_ENONFINITE in the device status (outputs then unspecified).
+ * Workspace: laplex_workspace_size(LAPLEX_OP_SORT, n, 0, 1, dtype, ...).
+ */
+laplex_status laplex_sort_anchors(const void* a, int64_t n, laplex_dtype dtype,
+                                  void* sorted, int32_t* perm,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Symmetric product y = K x, K_ij = exp(-|a_i - a_j|) (summary §2.2, "Caso
+ * Simmetrico": lower part by the prefix recurrence, upper part by the suffix
+ * recurrence, y = L + U - x so that the diagonal counts once).
+ *   sorted [n]      anchors ascending (from laplex_sort_anchors, or already sorted).
+ *   perm   [n]|NULL see conventions: non-NULL -> x, y in caller order.
+ *   x      [n, B]   input;  y [n, B] output.
+ */
+laplex_status laplex_matvec_sym(const void* sorted, const int32_t* perm, int64_t n,
+                                const void* x, void* y, int64_t B, laplex_dtype dtype,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * General product, a != b (summary §2.2, "Caso Generale": the b-anchors'
+ * contributions are collected in the intervals cut by the sorted a-anchors and
+ * propagated by the symmetric recurrences; here done by one scan over the
+ * merged sorted sequence of a and b).
+ *   transpose = 0:  y = K x,    x [k, B] on the b side, y [n, B] on the a side.
+ *   transpose = 1:  y = K^T x,  x [n, B] on the a side, y [k, B] on the b side.
+ *   sa [n], pa|NULL: sorted a and its perm;  sb [k], pb|NULL: same for b.
+ */
+laplex_status laplex_matvec_general(const void* sa, const int32_t* pa, int64_t n,
+                                    const void* sb, const int32_t* pb, int64_t k,
+                                    const void* x, void* y, int64_t B, int transpose,
+                                    laplex_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Phased product with K_ij = exp(-|a_i - b_j|) cos(phi_i - psi_j) (summary §2.1),
+ * computed as two unphased channels through cos(p - q) = cos p cos q + sin p sin q.
+ *   sb == NULL: symmetric case (b = a, psi = phi); k, pb, psi ignored.
+ *   phi [n] on the a side, psi [k] on the b side (same order convention as x, y).
+ *   transpose = 0: y = K x (x on the b side, y on the a side); 1: y = K^T x.
+ *   x, y: [len, B].
+ */
+laplex_status laplex_matvec_phased(const void* sa, const int32_t* pa, const void* phi, int64_t n,
+                                   const void* sb, const int32_t* pb, const void* psi, int64_t k,
+                                   const void* x, void* y, int64_t B, int transpose,
+                                   laplex_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Gram operator z = K^T diag(D) K v (summary §2.2 "Operatori di Gram"; abstract:
+ * "an efficient Gram operator"), as two chained products through the workspace.
+ *   phi == NULL: unphased K; otherwise the phased K (psi used when sb != NULL).
+ *   sb == NULL: symmetric (b = a): v, z [n, B], D [n] or NULL (D = 1).
+ *   sb != NULL: v, z [k, B] on the b side, D [n] on the a side or NULL.
+ */
+laplex_status laplex_gram(const void* sa, const int32_t* pa, const void* phi, int64_t n,
+                          const void* sb, const int32_t* pb, const void* psi, int64_t k,
+                          const void* D, const void* v, void* z, int64_t B,
+                          laplex_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Backward pass of L = <g, K x>, K = K(a, a), w.r.t. x and the anchors
+ * (differentiability in the anchors: summary §2.3 and §4.1):
+ *   dx = K^T g = K g,
+ *   da_i = -g_i sum_j sign(a_i - a_j) K_ij x_j - x_i sum_j sign(a_i - a_j) K_ij g_j,
+ * with sign(0) = 0 for tied anchors.  x, g, dx, da: [n] (B = 1).
+ */
+laplex_status laplex_backward(const void* sorted, const int32_t* perm, int64_t n,
+                              const void* x, const void* g, void* dx, void* da,
+                              laplex_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LAPLEX_H */
