@@ -1,0 +1,344 @@
+#!/usr/bin/env python
+"""LAPLEX benchmark: symmetric matvec throughput at n = 2^30 (fp32) on B200.
+
+Workload (the headline): y = K x with K_ij = exp(-|a_i - a_j|), n = 2^30
+anchors a ~ U(0, 2^30) generated already ascending (pre-sorted path), x ~ N(0,1),
+B = 1, fp32.  One step = one laplex_matvec_sym call.  Inputs (12.9 GB moved per
+step) are far larger than the 126 MB L2, so no L2 flush is needed between steps.
+
+Printed (rank 0, one JSON line): metric/value (Gelem/s, whole job), roofline of
+the step against the measured HBM copy peak, the other hot-path rows measured on
+the same data (sort of the unsorted anchors, the permuted product, the backward
+pass), the end-to-end number through host buffers, the fp64 oracle timed on the
+host cores as a CPU baseline, SM clocks sampled during the timed region, and the
+number of this library's kernels launched in the timed region.
+
+--impl reference times the fp64 CPU oracle (the method's plain statement) on a
+bounded sample of the same workload on the host cores.
+Multi-GPU (torchrun): every rank runs an independent replica of the workload
+(weak scaling, no data-path collective); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LAPLEX sym matvec Gelem/s at n=2^30 fp32; achieved HBM GB/s vs B200 peak"
+BYTES_PER_ELEM_SYM = 12  # read s (4) + x (4), write y (4): the minimum the product moves
+KERNELS_PER_SYM_CALL = 3  # launches of this library per laplex_matvec_sym call (B <= 8)
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--n", type=int, default=1 << 30)
+    p.add_argument("--rows", default="sort,perm,backward",
+                   help="extra hot-path rows to time (comma list; empty for none)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def src_sha(*names):
+    h = hashlib.sha256()
+    for nm in names:
+        with open(os.path.join(ROOT, "exact_laplace_b200", "csrc", nm), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(kernel_key, sha, n):
+    """dram read+write bytes per launch from profiles/traffic.txt, if the record was
+    taken on the current kernel source (sha) at this n; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        kv = dict(tok.split("=", 1) for tok in line.split())
+        if kv.get("key") == kernel_key and kv.get("src_sha") == sha and int(kv.get("n", -1)) == n:
+            return float(kv["bytes_per_launch"])
+    return None
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons (background process)."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons, samples = [], [], set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f:
+            parts = [t.strip() for t in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                if int(parts[0]) != self.idx:
+                    continue
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            samples += 1
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.f.name)
+        # samples taken while the GPU was busy (the timed loop) sit near the top clock
+        busy = [c for c in sm if c > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": samples}
+
+
+def cpu_baseline(n_total, seed, budget_s=10.0, m=1 << 24):
+    """The fp64 oracle (sort-free sequential recurrences, plain C, one thread) on
+    contiguous m-element samples of the same pre-sorted workload."""
+    import oracle as O
+    from exact_laplace_b200 import synth
+    s, x = synth.sym_uniform(m, 0.0, float(1 << 30) * m / n_total, seed=seed, presorted=True)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        O.sym_sorted(s, x)
+        done += m
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": done / el / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done // m} x {m} contiguous anchors (same density as the n=2^30 "
+                      f"workload), fp64 sequential recurrences, {el:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle as O
+    from exact_laplace_b200 import synth
+    m = 1 << 22
+    s, x = synth.sym_uniform(m, 0.0, float(1 << 30) * m / args.n, seed=0, presorted=True)
+    for _ in range(args.warmup):
+        O.sym_sorted(s, x)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.sym_sorted(s, x)
+    el = time.perf_counter() - t0
+    val = args.steps * m / el / 1e9
+    line = {"metric": METRIC, "value": val, "unit": "Gelem/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "symmetric LAPLEX matvec, pre-sorted anchors U(0,2^30), "
+                                   "x~N(0,1), B=1; reference arm = fp64 CPU oracle on a "
+                                   f"{m}-anchor sample per step", "n": args.n, "B": 1},
+            "cpu_baseline": {"value": val, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{m} contiguous anchors per step, same density"},
+            "e2e": {"value": val, "unit": "Gelem/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from exact_laplace_b200 import laplex as X
+    from exact_laplace_b200 import synth
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    n = args.n
+    hi = float(1 << 30)
+    s_h, x_h = synth.sym_uniform(n, 0.0, hi * n / (1 << 30), seed=rank, presorted=True)
+    s_p = torch.from_numpy(s_h).pin_memory()
+    x_p = torch.from_numpy(x_h).pin_memory()
+    del s_h, x_h
+    s_d = s_p.to(dev)
+    x_d = x_p.to(dev)
+    y_d = torch.empty_like(x_d)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, steps, warmup):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        torch.cuda.synchronize(dev)
+        return max_over_ranks(e0.elapsed_time(e1))
+
+    # ---------------- headline: pre-sorted symmetric product
+    clk = Clocks(local)
+    ms = timed(lambda: X.matvec_sym(s_d, x_d, out=y_d), args.steps, args.warmup)
+    clocks = clk.stop()
+    X.device_status(dev)
+    ms_step = ms / args.steps
+    value = world * n / (ms_step * 1e-3) / 1e9
+    hbm, peak_kind = peaks()
+    achieved = BYTES_PER_ELEM_SYM * n / (ms_step * 1e-3) / 1e9
+    sha = src_sha("sym.cu", "scan_core.cuh", "common.cuh")
+    traffic = traffic_from_profile("matvec_sym_presorted_b1", sha, n)
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "traffic": traffic,
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback 6650 GB/s",
+            "kernel": "laplex_matvec_sym (whole call)",
+            "algorithmic_bytes_per_launch": BYTES_PER_ELEM_SYM * n}
+
+    # ---------------- other rows on the same data
+    rows = {}
+    wanted = [r for r in args.rows.split(",") if r]
+    rsteps = max(3, min(20, args.steps // 10))
+    if wanted:
+        a_h = synth.uniform(n, 0.0, hi * n / (1 << 30), seed=rank, stream="a")
+        a_d = torch.from_numpy(a_h).to(dev)
+        del a_h
+        s2 = torch.empty_like(a_d)
+        p2 = torch.empty(n, dtype=torch.int32, device=dev)
+        try:
+            if "sort" in wanted:
+                ms_s = timed(lambda: X.sort_anchors(a_d, s2, p2), rsteps, 1) / rsteps
+                X.device_status(dev)
+                rows["sort"] = {"ms": ms_s, "Gelem_s": world * n / ms_s / 1e6,
+                                "algorithmic_GB_s": 12 * n / ms_s / 1e6,
+                                "algorithmic_bytes_per_elem": 12}
+            if "perm" in wanted:
+                X.sort_anchors(a_d, s2, p2)
+                ms_p = timed(lambda: X.matvec_sym(s2, x_d, p2, out=y_d), rsteps, 1) / rsteps
+                X.device_status(dev)
+                rows["matvec_perm"] = {"ms": ms_p, "Gelem_s": world * n / ms_p / 1e6,
+                                       "algorithmic_GB_s": 16 * n / ms_p / 1e6,
+                                       "algorithmic_bytes_per_elem": 16}
+        except X.LaplexError as e:
+            rows["sort_error"] = str(e)
+        del a_d, s2, p2
+        if "backward" in wanted:
+            try:
+                g_d = torch.from_numpy(synth.normal(n, seed=rank, stream="g")).to(dev)
+                dx = torch.empty_like(x_d)
+                da = torch.empty_like(x_d)
+                ms_b = timed(lambda: X.backward(s_d, x_d, g_d, dx_out=dx, da_out=da), rsteps, 1) / rsteps
+                X.device_status(dev)
+                rows["backward"] = {"ms": ms_b, "Gelem_s": world * n / ms_b / 1e6,
+                                    "algorithmic_GB_s": 20 * n / ms_b / 1e6,
+                                    "algorithmic_bytes_per_elem": 20}
+                del g_d, dx, da
+            except X.LaplexError as e:
+                rows["backward_error"] = str(e)
+        torch.cuda.empty_cache()
+
+    # ---------------- end to end through host buffers (pinned)
+    e2e = None
+    if not args.no_e2e:
+        y_p = torch.empty(n, dtype=torch.float32).pin_memory()
+        esteps = max(2, min(5, args.steps))
+        ms_e = timed(lambda: X.matvec_sym_host(s_p, x_p, device=dev, out=y_p), esteps, 1)
+        e2e = {"value": world * n / (ms_e / esteps * 1e-3) / 1e9, "unit": "Gelem/s",
+               "h2d_bytes_per_step": s_p.numel() * 4 + x_p.numel() * 4,
+               "d2h_bytes_per_step": y_p.numel() * 4, "steps": esteps,
+               "path": "exact_laplace_b200.laplex.matvec_sym_host (pinned host -> device, "
+                       "laplex_matvec_sym, device -> pinned host)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(n, 0)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic",
+                "config": {"workload": "symmetric LAPLEX matvec y=Kx, K_ij=exp(-|a_i-a_j|), "
+                                       "n=2^30 anchors U(0,2^30) pre-sorted, x~N(0,1), B=1, fp32",
+                           "n": n, "B": 1, "seed": "rank", "parallelism": f"replicas x{world}",
+                           "l2": "inputs 12.9 GB per step >> 126 MB L2 (no flush needed)"},
+                "roofline": roof, "rows": rows, "e2e": e2e, "cpu_baseline": cpu,
+                "clocks": clocks, "gpu_launches": KERNELS_PER_SYM_CALL * args.steps}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
