@@ -151,7 +151,8 @@ template <typename T, int C, int NT>
 __global__ void __launch_bounds__(NT) k_tile_carries(const T* __restrict__ s, int64_t n, int64_t tile,
                                                      int64_t ntiles, const T* __restrict__ aggF,
                                                      const T* __restrict__ aggB, T* __restrict__ carF,
-                                                     T* __restrict__ carB) {
+                                                     T* __restrict__ carB, const uint32_t* gate) {
+    if (gate != nullptr && *gate == 0u) return;  // nothing to fix up
     __shared__ BlockScanSmem<T, C, NT> smf, smb;
     const int64_t per = (ntiles + NT - 1) / NT;
     const int64_t t0 = min((int64_t)threadIdx.x * per, ntiles);
@@ -242,6 +243,186 @@ __global__ void __launch_bounds__(NT) k_sym_final(SymArgs<T> A, const T* __restr
     sym_store<T, NCOL, PHASED, E>(A, r0, out, cph, sph);
 }
 
+
+// ------------------------------------------------------------------ single pass
+// One launch streams s and x once and writes y once (12 bytes per element for
+// B = 1).  Tiles are taken in order from an atomic ticket.  Each tile
+//   1. scans itself and publishes its forward and backward totals (flag 1),
+//   2. looks back over the tiles to its left for the prefix carry, using an
+//      inclusive prefix (flag 2) where one is published, and stopping as soon
+//      as the decay exp(e_j - e_T) is exactly 0 (then every term further left
+//      is exactly 0 as well), then publishes its own inclusive prefix,
+//   3. looks ahead over at most J tiles to its right for the suffix carry in
+//      the same way, then publishes its inclusive suffix,
+//   4. finishes its elements and writes them.
+// A tile publishes its totals before it waits for anything, and tiles are
+// started in ticket order, so a wait on a left neighbour always ends; a wait on
+// a right neighbour ends as long as J is below the number of co-resident
+// blocks.  Every wait is bounded: an expired look-back sets ST_TIMEOUT; a look-
+// ahead that is too deep or expires marks the tile, which is then completed by
+// k_tile_carries (exact suffix carries from the published totals) and
+// k_sym_fixup (adds exp(s_r - s_end) * carry to the marked tiles' outputs).
+template <typename T>
+struct OnePassWs {
+    uint32_t* ctrl;   // [0] ticket, [1] number of marked tiles, then the flags
+    uint32_t* fflag;  // [ntiles] forward: 1 totals, 2 inclusive
+    uint32_t* bflag;  // [ntiles] backward: 1 totals, 2 inclusive
+    uint32_t* fix;    // [ntiles] 1: suffix carry left to k_sym_fixup
+    T* fagg;
+    T* finc;
+    T* bagg;
+    T* binc;
+    T* carF;          // scratch of k_tile_carries
+    T* carB;          // exact suffix carries (marked tiles only)
+};
+
+constexpr uint32_t LOOKBACK_POLLS = 1u << 25;
+constexpr uint32_t LOOKAHEAD_POLLS = 1u << 16;
+constexpr int LOOKAHEAD_TILES = 64;
+
+template <typename T, int NCOL, bool PHASED, int E, int NT>
+__global__ void __launch_bounds__(NT) k_sym_onepass(SymArgs<T> A, OnePassWs<T> W, int64_t ntiles) {
+    constexpr int C = PHASED ? 2 * NCOL : NCOL;
+    constexpr int64_t TILE = (int64_t)NT * E;
+    __shared__ BlockScanSmem<T, C, NT> smf, smb;
+    __shared__ int64_t sh_tile;
+    __shared__ T sh_e[2];
+    __shared__ T sh_c[2][C];
+    if (threadIdx.x == 0) sh_tile = (int64_t)atomicAdd(&W.ctrl[0], 1u);
+    __syncthreads();
+    const int64_t t = sh_tile;
+    const int64_t n = A.n;
+    const int64_t tile0 = t * TILE;
+    const int64_t r0 = tile0 + (int64_t)threadIdx.x * E;
+    T s[E], v[E][C], cph[E], sph[E], dl[E], fV[C], bW[C];
+    sym_load<T, NCOL, PHASED, E>(A, r0, s, v, cph, sph);
+    chunk_aggregates<T, C, E>(s, v, dl, fV, bW);
+    bool hf, hb;
+    T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
+    block_excl_fwd<T, C, NT>(s[E - 1], fV, hf, pe, pV, te, tV, smf);
+    block_excl_bwd<T, C, NT>(s[0], bW, hb, nf, nW, tf, tW, smb);
+    if (threadIdx.x == 0) {
+        const bool first = t == 0, last = t == ntiles - 1;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            W.fagg[t * C + c] = tV[c];
+            W.bagg[t * C + c] = tW[c];
+            if (first) W.finc[c] = tV[c];
+            if (last) W.binc[t * C + c] = tW[c];
+        }
+        st_release(&W.fflag[t], first ? 2u : 1u);
+        st_release(&W.bflag[t], last ? 2u : 1u);
+        // ---- look-back: L at the element before this tile (anchor eT)
+        const T eT = first ? A.s[0] : A.s[tile0 - 1];
+        T acc[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) acc[c] = T(0);
+        for (int64_t j = t - 1; j >= 0; --j) {
+            const T f = dexp<T>(A.s[(j + 1) * TILE - 1] - eT);
+            if (f == T(0)) break;
+            const uint32_t fl = wait_flag(&W.fflag[j], 1u, LOOKBACK_POLLS);
+            if (fl == 0u) {
+                set_status(A.status, ST_TIMEOUT);
+                break;
+            }
+            const T* src = (fl == 2u ? W.finc : W.fagg) + j * C;
+#pragma unroll
+            for (int c = 0; c < C; ++c) acc[c] = dfma<T>(f, __ldcg(src + c), acc[c]);
+            if (fl == 2u) break;
+        }
+        if (!first) {
+            const T d = dexp<T>(eT - te);
+#pragma unroll
+            for (int c = 0; c < C; ++c) W.finc[t * C + c] = dfma<T>(d, acc[c], tV[c]);
+            st_release(&W.fflag[t], 2u);
+        }
+        sh_e[0] = eT;
+#pragma unroll
+        for (int c = 0; c < C; ++c) sh_c[0][c] = acc[c];
+        // ---- look-ahead: U at the element after this tile (anchor fT)
+        const T fT = last ? A.s[n - 1] : A.s[tile0 + TILE];
+        T accb[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) accb[c] = T(0);
+        bool defer = false;
+        int depth = 0;
+        for (int64_t j = t + 1; j < ntiles; ++j) {
+            const T f = dexp<T>(fT - A.s[j * TILE]);
+            if (f == T(0)) break;
+            if (++depth > LOOKAHEAD_TILES) {
+                defer = true;
+                break;
+            }
+            const uint32_t fl = wait_flag(&W.bflag[j], 1u, LOOKAHEAD_POLLS);
+            if (fl == 0u) {
+                defer = true;
+                break;
+            }
+            const T* src = (fl == 2u ? W.binc : W.bagg) + j * C;
+#pragma unroll
+            for (int c = 0; c < C; ++c) accb[c] = dfma<T>(f, __ldcg(src + c), accb[c]);
+            if (fl == 2u) break;
+        }
+        if (defer) {
+#pragma unroll
+            for (int c = 0; c < C; ++c) accb[c] = T(0);
+            W.fix[t] = 1u;
+            atomicAdd(&W.ctrl[1], 1u);
+        } else if (!last) {
+            const T d = dexp<T>(tf - fT);
+#pragma unroll
+            for (int c = 0; c < C; ++c) W.binc[t * C + c] = dfma<T>(d, accb[c], tW[c]);
+            st_release(&W.bflag[t], 2u);
+        }
+        sh_e[1] = fT;
+#pragma unroll
+        for (int c = 0; c < C; ++c) sh_c[1][c] = accb[c];
+    }
+    __syncthreads();
+    T VT[C], WT[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        VT[c] = sh_c[0][c];
+        WT[c] = sh_c[1][c];
+    }
+    T eprev, Lprev[C], enext, Unext[C], out[E][C];
+    apply_carry_fwd<T, C>(hf, pe, pV, sh_e[0], VT, eprev, Lprev);
+    apply_carry_bwd<T, C>(hb, nf, nW, sh_e[1], WT, enext, Unext);
+    chunk_final<T, C, E>(s, v, dl, eprev, Lprev, enext, Unext, out);
+    sym_store<T, NCOL, PHASED, E>(A, r0, out, cph, sph);
+}
+
+// Adds the suffix carry to the tiles k_sym_onepass marked (exits at once when
+// none is marked).  y_r += exp(s_r - s_end) * carB[t] (phased: recombined).
+template <typename T, int NCOL, bool PHASED, int NT>
+__global__ void __launch_bounds__(NT) k_sym_fixup(SymArgs<T> A, OnePassWs<T> W, int64_t tile) {
+    constexpr int C = PHASED ? 2 * NCOL : NCOL;
+    if (W.ctrl[1] == 0u) return;
+    const int64_t t = blockIdx.x;
+    if (W.fix[t] == 0u) return;
+    const int64_t n = A.n;
+    const int64_t b = t * tile, e = min(b + tile, n);
+    if (e >= n) return;
+    const T fT = A.s[e];
+    T cr[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) cr[c] = W.carB[t * C + c];
+    for (int64_t r = b + threadIdx.x; r < e; r += NT) {
+        const T f = dexp<T>(A.s[r] - fT);
+        if (f == T(0)) continue;
+        const int64_t row = A.pout ? (int64_t)A.pout[r] : r;
+        T* yr = A.y + row * A.ldy + A.col0;
+        if (PHASED) {
+            const int64_t ar = A.paux ? (int64_t)A.paux[r] : r;
+            T sp, cp;
+            dsincos<T>(A.phi[ar], &sp, &cp);
+            for (int c = 0; c < A.ncol; ++c) yr[c] += f * (cp * cr[2 * c] + sp * cr[2 * c + 1]);
+        } else {
+            for (int c = 0; c < A.ncol; ++c) yr[c] += f * cr[c];
+        }
+    }
+}
+
 // ------------------------------------------------------------------ host side
 struct SymPlan {
     int ncol;  // template columns per pass
@@ -271,7 +452,7 @@ static SymPlan sym_plan(int64_t n, int64_t B, bool phased, int f64) {
 size_t sym_ws_bytes(int64_t n, int64_t B, bool phased, int f64) {
     const SymPlan p = sym_plan(n, B, phased, f64);
     const size_t es = f64 ? 8 : 4;
-    return 4 * Carve::need((size_t)(p.ntiles * p.C), es);
+    return Carve::need((size_t)(2 + 3 * p.ntiles), 4) + 6 * Carve::need((size_t)(p.ntiles * p.C), es);
 }
 
 template <typename T, int NCOL, bool PHASED, int E>
@@ -280,8 +461,22 @@ static cudaError_t sym_launch(const SymArgs<T>& A, int64_t ntiles, T* aggF, T* a
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
     k_sym_reduce<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, aggF, aggB);
     k_tile_carries<T, C, 1024><<<1, 1024, 0, st>>>(A.s, A.n, (int64_t)SYM_NT * E, ntiles, aggF,
-                                                     aggB, carF, carB);
+                                                     aggB, carF, carB, nullptr);
     k_sym_final<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, carF, carB);
+    return cudaGetLastError();
+}
+
+template <typename T, int NCOL, bool PHASED, int E>
+static cudaError_t onepass_launch(const SymArgs<T>& A, int64_t ntiles, const OnePassWs<T>& W,
+                                  cudaStream_t st) {
+    constexpr int C = PHASED ? 2 * NCOL : NCOL;
+    constexpr int64_t TILE = (int64_t)SYM_NT * E;
+    cudaError_t e = cudaMemsetAsync(W.ctrl, 0, sizeof(uint32_t) * (2 + 3 * ntiles), st);
+    if (e != cudaSuccess) return e;
+    k_sym_onepass<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, W, ntiles);
+    k_tile_carries<T, C, 1024><<<1, 1024, 0, st>>>(A.s, A.n, TILE, ntiles, W.fagg, W.bagg, W.carF,
+                                                     W.carB, W.ctrl + 1);
+    k_sym_fixup<T, NCOL, PHASED, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, W, TILE);
     return cudaGetLastError();
 }
 
@@ -291,10 +486,17 @@ cudaError_t sym_run(SymArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_by
     if (A.n == 0) return cudaSuccess;
     const SymPlan p = sym_plan(A.n, B, phased, sizeof(T) == 8);
     Carve cv(ws, ws_bytes);
-    T* aggF = cv.take<T>(p.ntiles * p.C);
-    T* aggB = cv.take<T>(p.ntiles * p.C);
-    T* carF = cv.take<T>(p.ntiles * p.C);
-    T* carB = cv.take<T>(p.ntiles * p.C);
+    OnePassWs<T> W;
+    W.ctrl = cv.take<uint32_t>(2 + 3 * p.ntiles);
+    W.fflag = W.ctrl + 2;
+    W.bflag = W.fflag + p.ntiles;
+    W.fix = W.bflag + p.ntiles;
+    W.fagg = cv.take<T>(p.ntiles * p.C);
+    W.finc = cv.take<T>(p.ntiles * p.C);
+    W.bagg = cv.take<T>(p.ntiles * p.C);
+    W.binc = cv.take<T>(p.ntiles * p.C);
+    W.carF = cv.take<T>(p.ntiles * p.C);
+    W.carB = cv.take<T>(p.ntiles * p.C);
     if (!cv.ok) return cudaErrorInvalidValue;
     for (int64_t g = 0; g < p.groups; ++g) {
         A.col0 = g * p.ncol;
@@ -303,16 +505,16 @@ cudaError_t sym_run(SymArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_by
         constexpr bool D = sizeof(T) == 8;
         if (!phased) {
             switch (p.ncol) {
-                case 1: e = sym_launch<T, 1, false, D ? 8 : 16>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
-                case 2: e = sym_launch<T, 2, false, 8>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
-                case 4: e = sym_launch<T, 4, false, 4>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
-                default: e = sym_launch<T, 8, false, 4>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
+                case 1: e = onepass_launch<T, 1, false, D ? 8 : 16>(A, p.ntiles, W, st); break;
+                case 2: e = onepass_launch<T, 2, false, 8>(A, p.ntiles, W, st); break;
+                case 4: e = onepass_launch<T, 4, false, 4>(A, p.ntiles, W, st); break;
+                default: e = onepass_launch<T, 8, false, 4>(A, p.ntiles, W, st); break;
             }
         } else {
             switch (p.ncol) {
-                case 1: e = sym_launch<T, 1, true, 8>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
-                case 2: e = sym_launch<T, 2, true, 4>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
-                default: e = sym_launch<T, 4, true, 4>(A, p.ntiles, aggF, aggB, carF, carB, st); break;
+                case 1: e = onepass_launch<T, 1, true, 8>(A, p.ntiles, W, st); break;
+                case 2: e = onepass_launch<T, 2, true, 4>(A, p.ntiles, W, st); break;
+                default: e = onepass_launch<T, 4, true, 4>(A, p.ntiles, W, st); break;
             }
         }
         if (e != cudaSuccess) return e;

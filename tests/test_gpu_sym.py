@@ -107,3 +107,19 @@ def test_c5_full_size_presorted_sampled():
         sub = np.arange(lo, hi)
         out, _, absn = rows_local(s, x, sub)
         assert_close(y[sub], out, absn, np.float32, f"C5 rows {lo}..{hi}")
+
+
+@pytest.mark.parametrize("dtype", [np.float32, np.float64])
+def test_deep_lookahead_fixup(dtype):
+    """Dependencies that span more tiles than the look-ahead may wait for: all
+    anchors equal (every output is sum(x)) and 10^6 anchors inside one unit.
+    Exercises the deferred suffix-carry fix-up."""
+    n = 1_000_003
+    rng = np.random.default_rng(11)
+    x = rng.normal(size=n).astype(dtype)
+    a = np.full(n, -7.0, dtype=dtype)
+    assert_close(run_sym(a, x, False), O.sym(a, x), O.norm_sym(a, x), dtype, "all equal")
+    a = rng.uniform(0, 1, n).astype(dtype)
+    assert_close(run_sym(a, x, True), O.sym(a, x), O.norm_sym(a, x), dtype, "dense")
+    xb = rng.normal(size=(n, 3)).astype(dtype)
+    assert_close(run_sym(a, xb, True), O.sym(a, xb), O.norm_sym(a, xb), dtype, "dense B=3")
