@@ -104,6 +104,13 @@ uint32_t* ws_status(void* ws) { return static_cast<uint32_t*>(ws); }
 
 }  // namespace
 
+void lx::set_last_error(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+}
+
 extern "C" {
 
 int laplex_version(void) { return 10000; }

@@ -12,6 +12,9 @@ constexpr uint32_t ST_NONFINITE = 1u;
 constexpr uint32_t ST_TIMEOUT = 2u;
 constexpr size_t HEADER_BYTES = 256;
 
+// Sets the calling thread's message returned by laplex_last_error() (capi.cu).
+void set_last_error(const char* fmt, ...);
+
 // Bump allocator over the caller's workspace (256-byte granules).
 struct Carve {
     char* base;

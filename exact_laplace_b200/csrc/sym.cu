@@ -526,3 +526,99 @@ template cudaError_t sym_run<float>(SymArgs<float>, int64_t, bool, void*, size_t
 template cudaError_t sym_run<double>(SymArgs<double>, int64_t, bool, void*, size_t, cudaStream_t);
 
 }  // namespace lx
+
+// ------------------------------------------------------------------ no-alloc variant
+// laplex_matvec_sym_noalloc: the three-phase symmetric product (fp32, B = 1)
+// with its per-tile scratch in a fixed device array instead of a caller
+// workspace, for callers that cannot allocate device memory.
+#include <mutex>
+
+#include "laplex.h"
+
+namespace lx {
+
+constexpr int64_t NOALLOC_TILE = (int64_t)SYM_NT * 16;           // elements per tile (fp32, B = 1)
+constexpr int64_t NOALLOC_MAX_TILES = (int64_t)1 << 18;          // n <= 2^30
+constexpr size_t NOALLOC_BYTES = 4 * NOALLOC_MAX_TILES * sizeof(float);  // 4 MiB
+
+// Four float arrays of NOALLOC_MAX_TILES entries (tile totals and tile carries).
+// Every call writes each entry it reads, so nothing here needs clearing.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_BYTES];
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[NOALLOC_MAX_DEVICES];
+
+// Device address of g_noalloc_scratch on the current device (looked up once per
+// device; in host code the array's name is only a host-side handle).
+static cudaError_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace lx
+
+extern "C" laplex_status laplex_matvec_sym_noalloc(const float* sorted, const int32_t* perm,
+                                                   int64_t n, const float* x, float* y,
+                                                   void* stream) {
+    using namespace lx;
+    if (n < 0 || n > NOALLOC_MAX_TILES * NOALLOC_TILE) {
+        set_last_error("laplex_matvec_sym_noalloc: n = %lld outside [0, 2^30] (the fixed "
+                                 "scratch holds 2^18 tiles of 4096 anchors)", (long long)n);
+        return LAPLEX_EINVAL;
+    }
+    auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (n > 0 && (!sorted || !x || !y || !al(sorted) || !al(x) || !al(y) || (perm && !al(perm)))) {
+        set_last_error("laplex_matvec_sym_noalloc: sorted, x and y must be non-NULL and "
+                                 "16-byte aligned (perm too, when given)");
+        return LAPLEX_EINVAL;
+    }
+    void* scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) {
+        set_last_error("laplex_matvec_sym_noalloc: scratch set-up: %s", cudaGetErrorString(e));
+        return LAPLEX_ECUDA;
+    }
+    if (n == 0) {
+        set_last_error("");
+        return LAPLEX_OK;
+    }
+    const int64_t ntiles = (n + NOALLOC_TILE - 1) / NOALLOC_TILE;
+    float* aggF = static_cast<float*>(scratch);
+    float* aggB = aggF + NOALLOC_MAX_TILES;
+    float* carF = aggB + NOALLOC_MAX_TILES;
+    float* carB = carF + NOALLOC_MAX_TILES;
+    SymArgs<float> A;
+    A.s = sorted;
+    A.n = n;
+    A.x = x;
+    A.pin = perm;
+    A.ldx = 1;
+    A.y = y;
+    A.pout = perm;
+    A.ldy = 1;
+    A.phi = nullptr;
+    A.D = nullptr;
+    A.paux = perm;
+    A.col0 = 0;
+    A.ncol = 1;
+    A.status = nullptr;
+    e = sym_launch<float, 1, false, 16>(A, ntiles, aggF, aggB, carF, carB, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        set_last_error("laplex_matvec_sym_noalloc: %s", cudaGetErrorString(e));
+        return LAPLEX_ECUDA;
+    }
+    set_last_error("");
+    return LAPLEX_OK;
+}

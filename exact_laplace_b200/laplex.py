@@ -61,6 +61,7 @@ SIGNATURES = {
                      ctypes.c_size_t, _P], ctypes.c_int),
     "laplex_backward": ([_P, _P, _I64, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P],
                         ctypes.c_int),
+    "laplex_matvec_sym_noalloc": ([_P, _P, _I64, _P, _P, _P], ctypes.c_int),
 }
 
 
@@ -256,6 +257,22 @@ def backward(sorted_anchors, x, g, perm=None, dx_out=None, da_out=None):
     _check(lib().laplex_backward(_ptr(sorted_anchors), _ptr(perm), n, _ptr(x), _ptr(g), _ptr(dx),
                                  _ptr(da), _dt(x), _ptr(ws), nb, _stream(dev)))
     return dx, da
+
+
+def matvec_sym_noalloc(sorted_anchors: torch.Tensor, x: torch.Tensor, perm=None, out=None):
+    """y = K x through laplex_matvec_sym_noalloc: fp32, x of shape [n], n <= 2^30.
+
+    For callers that cannot give the library a workspace: the scratch is a fixed
+    array inside the library (shared by all calls on a device, so calls that may
+    overlap on the GPU must be serialised by the caller)."""
+    dev = _dev(sorted_anchors, x, _perm(perm), out)
+    if x.dtype != torch.float32 or x.dim() != 1:
+        raise LaplexError(EINVAL, "matvec_sym_noalloc takes fp32 x of shape [n]")
+    n = sorted_anchors.numel()
+    y = torch.empty_like(x) if out is None else out
+    _check(lib().laplex_matvec_sym_noalloc(_ptr(sorted_anchors), _ptr(perm), n, _ptr(x), _ptr(y),
+                                           _stream(dev)))
+    return y
 
 
 # ----------------------------------------------------------------------------- host buffers

@@ -180,6 +180,31 @@ laplex_status laplex_backward(const void* sorted, const int32_t* perm, int64_t n
                               const void* x, const void* g, void* dx, void* da,
                               laplex_dtype dtype, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Allocation-free symmetric product, y = K x (fp32, B = 1).  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate device
+ * memory -- code running where cudaMalloc is unavailable or forbidden (inside
+ * another library's allocator-free hot path, a real-time loop that must not
+ * allocate, or a host that owns a fixed memory budget) -- and so cannot
+ * provide the workspace laplex_matvec_sym needs.
+ *   sorted [n], perm [n]|NULL, x [n], y [n]: as in laplex_matvec_sym (fp32, B = 1).
+ *   stream: as elsewhere.
+ * Scratch: a fixed 4 MiB array compiled into the library as a __device__
+ * variable; every GPU that loads the library holds it until the process exits.
+ * It bounds n to 2^30 (2^18 tiles of 4096 anchors); larger n returns
+ * LAPLEX_EINVAL with a message.  The call allocates and frees nothing.
+ * The first call on each device looks up the array's device address (with that
+ * device current), so make that first call before any stream capture.
+ * Every call shares the one array per device and leaves its last contents
+ * there; each call writes every scratch entry before reading it, so nothing
+ * needs clearing, but calls that overlap on the GPU (several streams or host
+ * threads on one device) race on it and must be serialised by the caller.
+ * Errors: LAPLEX_EINVAL (sizes, NULL or misaligned pointers), LAPLEX_ECUDA
+ * (set-up or launch failure); laplex_last_error() holds the message.
+ */
+laplex_status laplex_matvec_sym_noalloc(const float* sorted, const int32_t* perm, int64_t n,
+                                        const float* x, float* y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
