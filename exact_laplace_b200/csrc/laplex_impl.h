@@ -57,6 +57,12 @@ template <typename T>
 cudaError_t sym_run(SymArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_bytes,
                     cudaStream_t st);
 
+// streaming path of the symmetric product (x in sorted order, one column)
+size_t stream_ws_bytes(int64_t n, int f64);
+template <typename T>
+cudaError_t stream_run(const T* s, const T* x, T* y, const int32_t* pout, int64_t n, void* ws,
+                       size_t ws_bytes, uint32_t* status, cudaStream_t st);
+
 // -------------------------------------------------------------- sort
 size_t sort_ws_bytes(int64_t n, int f64);
 template <typename T>

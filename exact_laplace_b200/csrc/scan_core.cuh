@@ -13,13 +13,30 @@
 // never a product of rounded per-step decays, so fp32 error does not grow with
 // the distance between tiles.  Elements past the end are padded with the last
 // anchor and value 0, which is neutral in both directions.
+//
+// The last CT channels ("tie channels") use the decay [e_P == e_A] instead of
+// exp(e_P - e_A): with sorted anchors that is the product of the per-step
+// indicators, so those channels sum over runs of equal anchors only (used by
+// the backward pass for the sign(0) = 0 terms).
 #pragma once
 #include "common.cuh"
 
 namespace lx {
 
+// decay applied to channel c of a combine across anchors p <= q
+template <typename T, int C, int CT>
+struct Decay {
+    T e;   // exp(p - q)
+    T t;   // [p == q]
+    __device__ __forceinline__ Decay(const T p, const T q) {
+        e = dexp<T>(p - q);
+        if (CT > 0) t = (p == q) ? T(1) : T(0);
+    }
+    __device__ __forceinline__ T operator[](int c) const { return (CT > 0 && c >= C - CT) ? t : e; }
+};
+
 // ---------------------------------------------------------------- warp level
-template <typename T, int C>
+template <typename T, int C, int CT = 0>
 __device__ __forceinline__ void warp_incl_fwd(const T e, T (&V)[C], const int lane) {
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -28,14 +45,14 @@ __device__ __forceinline__ void warp_incl_fwd(const T e, T (&V)[C], const int la
 #pragma unroll
         for (int c = 0; c < C; ++c) Vo[c] = __shfl_up_sync(FULL, V[c], off);
         if (lane >= off) {
-            const T d = dexp<T>(eo - e);
+            const Decay<T, C, CT> d(eo, e);
 #pragma unroll
-            for (int c = 0; c < C; ++c) V[c] = dfma<T>(d, Vo[c], V[c]);
+            for (int c = 0; c < C; ++c) V[c] = dfma<T>(d[c], Vo[c], V[c]);
         }
     }
 }
 
-template <typename T, int C>
+template <typename T, int C, int CT = 0>
 __device__ __forceinline__ void warp_incl_bwd(const T f, T (&W)[C], const int lane) {
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -44,9 +61,9 @@ __device__ __forceinline__ void warp_incl_bwd(const T f, T (&W)[C], const int la
 #pragma unroll
         for (int c = 0; c < C; ++c) Wo[c] = __shfl_down_sync(FULL, W[c], off);
         if (lane + off < 32) {
-            const T d = dexp<T>(f - fo);
+            const Decay<T, C, CT> d(f, fo);
 #pragma unroll
-            for (int c = 0; c < C; ++c) W[c] = dfma<T>(d, Wo[c], W[c]);
+            for (int c = 0; c < C; ++c) W[c] = dfma<T>(d[c], Wo[c], W[c]);
         }
     }
 }
@@ -66,7 +83,7 @@ struct BlockScanSmem {
 // Exclusive forward scan over the threads of the block, in thread order.
 // In: this thread's run summary (e, V).  Out: has (false for thread 0), the
 // summary (pe, pV) of all runs of lower threads, and the block total (te, tV).
-template <typename T, int C, int NT>
+template <typename T, int C, int NT, int CT = 0>
 __device__ __forceinline__ void block_excl_fwd(const T e, const T (&V)[C], bool& has, T& pe,
                                                T (&pV)[C], T& te, T (&tV)[C],
                                                BlockScanSmem<T, C, NT>& sm) {
@@ -75,7 +92,7 @@ __device__ __forceinline__ void block_excl_fwd(const T e, const T (&V)[C], bool&
     T iV[C];
 #pragma unroll
     for (int c = 0; c < C; ++c) iV[c] = V[c];
-    warp_incl_fwd<T, C>(e, iV, lane);
+    warp_incl_fwd<T, C, CT>(e, iV, lane);
     if (lane == 31) {
         sm.we[w] = e;
 #pragma unroll
@@ -94,9 +111,9 @@ __device__ __forceinline__ void block_excl_fwd(const T e, const T (&V)[C], bool&
 #pragma unroll
             for (int c = 0; c < C; ++c) Vo[c] = __shfl_up_sync(FULL, gV[c], off);
             if (lane >= off && lane < NW) {
-                const T d = dexp<T>(eo - ge);
+                const Decay<T, C, CT> d(eo, ge);
 #pragma unroll
-                for (int c = 0; c < C; ++c) gV[c] = dfma<T>(d, Vo[c], gV[c]);
+                for (int c = 0; c < C; ++c) gV[c] = dfma<T>(d[c], Vo[c], gV[c]);
             }
         }
         const T xe = __shfl_up_sync(FULL, ge, 1);
@@ -122,9 +139,9 @@ __device__ __forceinline__ void block_excl_fwd(const T e, const T (&V)[C], bool&
     if (w > 0 && lane > 0) {
         has = true;
         pe = le;
-        const T d = dexp<T>(sm.pe[w] - le);
+        const Decay<T, C, CT> d(sm.pe[w], le);
 #pragma unroll
-        for (int c = 0; c < C; ++c) pV[c] = dfma<T>(d, sm.pV[w][c], lV[c]);
+        for (int c = 0; c < C; ++c) pV[c] = dfma<T>(d[c], sm.pV[w][c], lV[c]);
     } else if (w > 0) {
         has = true;
         pe = sm.pe[w];
@@ -147,7 +164,7 @@ __device__ __forceinline__ void block_excl_fwd(const T e, const T (&V)[C], bool&
 }
 
 // Exclusive backward scan (suffix over higher threads), mirror of block_excl_fwd.
-template <typename T, int C, int NT>
+template <typename T, int C, int NT, int CT = 0>
 __device__ __forceinline__ void block_excl_bwd(const T f, const T (&W)[C], bool& has, T& nf,
                                                T (&nW)[C], T& tf, T (&tW)[C],
                                                BlockScanSmem<T, C, NT>& sm) {
@@ -156,7 +173,7 @@ __device__ __forceinline__ void block_excl_bwd(const T f, const T (&W)[C], bool&
     T iW[C];
 #pragma unroll
     for (int c = 0; c < C; ++c) iW[c] = W[c];
-    warp_incl_bwd<T, C>(f, iW, lane);
+    warp_incl_bwd<T, C, CT>(f, iW, lane);
     if (lane == 0) {
         sm.we[w] = f;
 #pragma unroll
@@ -175,9 +192,9 @@ __device__ __forceinline__ void block_excl_bwd(const T f, const T (&W)[C], bool&
 #pragma unroll
             for (int c = 0; c < C; ++c) Wo[c] = __shfl_down_sync(FULL, gW[c], off);
             if (lane + off < NW) {
-                const T d = dexp<T>(gf - fo);
+                const Decay<T, C, CT> d(gf, fo);
 #pragma unroll
-                for (int c = 0; c < C; ++c) gW[c] = dfma<T>(d, Wo[c], gW[c]);
+                for (int c = 0; c < C; ++c) gW[c] = dfma<T>(d[c], Wo[c], gW[c]);
             }
         }
         const T xf = __shfl_down_sync(FULL, gf, 1);
@@ -203,9 +220,9 @@ __device__ __forceinline__ void block_excl_bwd(const T f, const T (&W)[C], bool&
     if (w < NW - 1 && lane < 31) {
         has = true;
         nf = lf;
-        const T d = dexp<T>(lf - sm.pe[w]);
+        const Decay<T, C, CT> d(lf, sm.pe[w]);
 #pragma unroll
-        for (int c = 0; c < C; ++c) nW[c] = dfma<T>(d, sm.pV[w][c], lW[c]);
+        for (int c = 0; c < C; ++c) nW[c] = dfma<T>(d[c], sm.pV[w][c], lW[c]);
     } else if (w < NW - 1) {
         has = true;
         nf = sm.pe[w];
@@ -230,20 +247,27 @@ __device__ __forceinline__ void block_excl_bwd(const T f, const T (&W)[C], bool&
 // ---------------------------------------------------------------- chunk level
 // A thread owns E consecutive elements: anchors s[E], values v[E][C].
 // dl[i] = exp(s[i-1] - s[i]) for i = 1..E-1 (dl[0] is set in chunk_final).
-template <typename T, int C, int E>
+template <typename T, int C, int E, int CT = 0>
 __device__ __forceinline__ void chunk_aggregates(const T (&s)[E], const T (&v)[E][C], T (&dl)[E],
                                                  T (&fV)[C], T (&bW)[C]) {
 #pragma unroll
     for (int i = 1; i < E; ++i) dl[i] = dexp<T>(s[i - 1] - s[i]);
 #pragma unroll
     for (int c = 0; c < C; ++c) {
+        const bool tie = CT > 0 && c >= C - CT;
         T a = v[0][c];
 #pragma unroll
-        for (int i = 1; i < E; ++i) a = dfma<T>(dl[i], a, v[i][c]);
+        for (int i = 1; i < E; ++i) {
+            const T d = tie ? (s[i - 1] == s[i] ? T(1) : T(0)) : dl[i];
+            a = dfma<T>(d, a, v[i][c]);
+        }
         fV[c] = a;
         T b = v[E - 1][c];
 #pragma unroll
-        for (int i = E - 2; i >= 0; --i) b = dfma<T>(dl[i + 1], b, v[i][c]);
+        for (int i = E - 2; i >= 0; --i) {
+            const T d = tie ? (s[i] == s[i + 1] ? T(1) : T(0)) : dl[i + 1];
+            b = dfma<T>(d, b, v[i][c]);
+        }
         bW[c] = b;
     }
 }
@@ -275,15 +299,15 @@ __device__ __forceinline__ void chunk_final(const T (&s)[E], const T (&v)[E][C],
 }
 
 // Combine a thread's in-tile exclusive prefix with the tile's carry-in.
-template <typename T, int C>
+template <typename T, int C, int CT = 0>
 __device__ __forceinline__ void apply_carry_fwd(const bool has, const T pe, const T (&pV)[C],
                                                 const T eT, const T (&VT)[C], T& eprev,
                                                 T (&Lprev)[C]) {
     if (has) {
         eprev = pe;
-        const T d = dexp<T>(eT - pe);
+        const Decay<T, C, CT> d(eT, pe);
 #pragma unroll
-        for (int c = 0; c < C; ++c) Lprev[c] = dfma<T>(d, VT[c], pV[c]);
+        for (int c = 0; c < C; ++c) Lprev[c] = dfma<T>(d[c], VT[c], pV[c]);
     } else {
         eprev = eT;
 #pragma unroll
@@ -291,15 +315,15 @@ __device__ __forceinline__ void apply_carry_fwd(const bool has, const T pe, cons
     }
 }
 
-template <typename T, int C>
+template <typename T, int C, int CT = 0>
 __device__ __forceinline__ void apply_carry_bwd(const bool has, const T nf, const T (&nW)[C],
                                                 const T fT, const T (&WT)[C], T& enext,
                                                 T (&Unext)[C]) {
     if (has) {
         enext = nf;
-        const T d = dexp<T>(nf - fT);
+        const Decay<T, C, CT> d(nf, fT);
 #pragma unroll
-        for (int c = 0; c < C; ++c) Unext[c] = dfma<T>(d, WT[c], nW[c]);
+        for (int c = 0; c < C; ++c) Unext[c] = dfma<T>(d[c], WT[c], nW[c]);
     } else {
         enext = fT;
 #pragma unroll

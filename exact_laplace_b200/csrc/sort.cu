@@ -9,15 +9,18 @@
 // and is stable, so equal anchors keep ascending index order and the output
 // permutation is unique.  A NaN or Inf anchor sets ST_NONFINITE.
 //
-// One pass = three kernels:
-//   k_radix_upsweep   : digit counts of each contiguous segment of keys
-//   k_radix_scan      : exclusive scan of the counts, digit-major -> start of
-//                       every (digit, segment) run in the output
-//   k_radix_downsweep : each block walks its segment tile by tile in order,
-//                       ranks keys stably inside the tile (warp match + per-warp
-//                       counters), stages them in shared memory in digit order
-//                       and writes them to their runs (runs are contiguous, so
-//                       the writes coalesce).
+// Onesweep (Adinets & Merrill, "Onesweep: A Faster Least Significant Digit
+// Radix Sort for GPUs", 2022):
+//   k_radix_hist    : one read of the keys counts every digit of every pass
+//   k_radix_offsets : exclusive scan of each pass's 256 counts
+//   k_onesweep      : one kernel per pass.  Tiles are taken in ticket order;
+//                     each ranks its keys stably (warp match + per-warp
+//                     counters), publishes its 256 digit counts, and finds how
+//                     many keys of each digit lie in earlier tiles by a
+//                     decoupled look-back over 64-bit records (pass tag in the
+//                     high word, so one memset per call serves every pass).
+//                     Keys are staged in shared memory in digit order, so the
+//                     writes to each digit's run coalesce.
 // Pass 0 reads the anchors and generates the index payload; the last pass
 // writes the anchors back as values and the payload as perm.
 #include <algorithm>
@@ -90,157 +93,177 @@ __device__ __forceinline__ uint32_t block_excl_sum(uint32_t v, uint32_t* sm /*NT
     return r;
 }
 
+__device__ __forceinline__ void st_release64(uint64_t* p, uint64_t v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_acquire64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Counts of every digit of every pass in one read of the keys.
 template <typename T>
-__global__ void __launch_bounds__(SORT_NT) k_radix_upsweep(const T* __restrict__ a,
-                                                           const typename KeyOf<T>::K* __restrict__ ksrc,
-                                                           int64_t n, int shift, int64_t seg, int G,
-                                                           uint32_t* __restrict__ counts,
-                                                           uint32_t* status, int first) {
+__global__ void __launch_bounds__(SORT_NT) k_radix_hist(const T* __restrict__ a, int64_t n,
+                                                        uint32_t* __restrict__ hist,
+                                                        uint32_t* status) {
     using K = typename KeyOf<T>::K;
-    __shared__ uint32_t hist[RADIX];
-    hist[threadIdx.x] = 0;
+    constexpr int P = sizeof(K);
+    __shared__ uint32_t h[P][RADIX];
+    for (int j = threadIdx.x; j < P * RADIX; j += SORT_NT) (&h[0][0])[j] = 0u;
     __syncthreads();
-    const int64_t beg = (int64_t)blockIdx.x * seg;
-    const int64_t end = min(beg + seg, n);
     bool bad = false;
-    for (int64_t i = beg + threadIdx.x; i < end; i += SORT_NT) {
-        const K k = first ? to_key(a[i], bad) : ksrc[i];
-        atomicAdd(&hist[(unsigned)(k >> shift) & (RADIX - 1)], 1u);
+    const int64_t stride = (int64_t)gridDim.x * SORT_NT;
+    for (int64_t i = (int64_t)blockIdx.x * SORT_NT + threadIdx.x; i < n; i += stride) {
+        const K k = to_key(a[i], bad);
+#pragma unroll
+        for (int p = 0; p < P; ++p) atomicAdd(&h[p][(unsigned)(k >> (8 * p)) & (RADIX - 1)], 1u);
     }
     if (bad) set_status(status, ST_NONFINITE);
     __syncthreads();
-    counts[(int64_t)threadIdx.x * G + blockIdx.x] = hist[threadIdx.x];
-}
-
-// in-place exclusive scan of counts[0 .. total) (one block of 1024 threads)
-__global__ void __launch_bounds__(1024) k_radix_scan(uint32_t* __restrict__ counts, int64_t total) {
-    __shared__ uint32_t sm[1024 / 32 + 1];
-    const int64_t per = (total + 1023) / 1024;
-    const int64_t b = min((int64_t)threadIdx.x * per, total);
-    const int64_t e = min(b + per, total);
-    uint32_t s = 0;
-    for (int64_t i = b; i < e; ++i) s += counts[i];
-    uint32_t tot;
-    uint32_t run = block_excl_sum<1024>(s, sm, tot);
-    for (int64_t i = b; i < e; ++i) {
-        const uint32_t c = counts[i];
-        counts[i] = run;
-        run += c;
+    for (int j = threadIdx.x; j < P * RADIX; j += SORT_NT) {
+        const uint32_t c = (&h[0][0])[j];
+        if (c) atomicAdd(&hist[j], c);
     }
 }
 
+// hist[p][d] <- number of keys with a smaller digit d in pass p (one block per pass)
+__global__ void __launch_bounds__(SORT_NT) k_radix_offsets(uint32_t* __restrict__ hist) {
+    __shared__ uint32_t sm[SORT_NT / 32 + 1];
+    uint32_t* h = hist + (int64_t)blockIdx.x * RADIX;
+    uint32_t tot;
+    const uint32_t ex = block_excl_sum<SORT_NT>(h[threadIdx.x], sm, tot);
+    h[threadIdx.x] = ex;
+}
+
+constexpr uint32_t SORT_POLLS = 1u << 25;
+
 template <typename T, int KPT>
-__global__ void __launch_bounds__(SORT_NT) k_radix_downsweep(
+__global__ void __launch_bounds__(SORT_NT) k_onesweep(
     const T* __restrict__ a, const typename KeyOf<T>::K* __restrict__ ksrc,
-    const int32_t* __restrict__ vsrc, int64_t n, int shift, int64_t seg, int G,
-    const uint32_t* __restrict__ offsets, typename KeyOf<T>::K* __restrict__ kdst,
-    int32_t* __restrict__ vdst, int first, int last) {
+    const int32_t* __restrict__ vsrc, int64_t n, int pass, const uint32_t* __restrict__ offsets,
+    uint64_t* __restrict__ rec, uint32_t* __restrict__ ticket, typename KeyOf<T>::K* __restrict__ kdst,
+    int32_t* __restrict__ vdst, int last, uint32_t* status) {
     using K = typename KeyOf<T>::K;
     constexpr int NT = SORT_NT, NW = NT / 32, TILE = NT * KPT;
     __shared__ K skey[TILE];
     __shared__ int32_t sval[TILE];
     __shared__ uint32_t wcnt[NW][RADIX];
-    __shared__ uint32_t dstart[RADIX], dcount[RADIX], run[RADIX];
+    __shared__ uint32_t dstart[RADIX];
+    __shared__ int64_t gbase[RADIX];
     __shared__ uint32_t scan_sm[NT / 32 + 1];
+    __shared__ int64_t sh_tile;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int64_t beg = (int64_t)blockIdx.x * seg;
-    const int64_t end = min(beg + seg, n);
-    run[threadIdx.x] = offsets[(int64_t)threadIdx.x * G + blockIdx.x];
+    const int shift = 8 * pass;
+    const bool first = pass == 0;
+    if (threadIdx.x == 0) sh_tile = (int64_t)atomicAdd(ticket, 1u);
+    for (int j = threadIdx.x; j < NW * RADIX; j += NT) (&wcnt[0][0])[j] = 0u;
+    __syncthreads();
+    const int64_t t = sh_tile;
+    const int64_t tb = t * TILE;
+    const int64_t end = min(tb + TILE, n);
     const unsigned ltmask = lanemask_lt();
-    for (int64_t tb = beg; tb < end; tb += TILE) {
-        for (int j = threadIdx.x; j < NW * RADIX; j += NT) (&wcnt[0][0])[j] = 0u;
-        __syncthreads();
-        K k[KPT];
-        int32_t v[KPT];
-        int dg[KPT];
-        uint32_t rk[KPT];
-        bool bad = false;
+    K k[KPT];
+    int32_t v[KPT];
+    int dg[KPT];
+    uint32_t rk[KPT];
+    bool bad = false;
 #pragma unroll
-        for (int i = 0; i < KPT; ++i) {
-            const int64_t idx = tb + (int64_t)w * 32 * KPT + i * 32 + lane;
-            if (idx < end) {
-                k[i] = first ? to_key(a[idx], bad) : ksrc[idx];
-                v[i] = first ? (int32_t)idx : vsrc[idx];
-                dg[i] = (int)((unsigned)(k[i] >> shift) & (RADIX - 1));
-            } else {
-                k[i] = 0;
-                v[i] = 0;
-                dg[i] = RADIX;  // padding: never placed
+    for (int i = 0; i < KPT; ++i) {
+        const int64_t idx = tb + (int64_t)w * 32 * KPT + i * 32 + lane;
+        if (idx < end) {
+            k[i] = first ? to_key(a[idx], bad) : ksrc[idx];
+            v[i] = first ? (int32_t)idx : vsrc[idx];
+            dg[i] = (int)((unsigned)(k[i] >> shift) & (RADIX - 1));
+        } else {
+            k[i] = 0;
+            v[i] = 0;
+            dg[i] = RADIX;  // padding: never placed
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        const int d = dg[i];
+        const unsigned peers = __match_any_sync(FULL, d);
+        const uint32_t lower = __popc(peers & ltmask);
+        rk[i] = d < RADIX ? wcnt[w][d] + lower : 0u;
+        __syncwarp();
+        if (d < RADIX && lower == 0) wcnt[w][d] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    {
+        const int d = threadIdx.x;  // NT == RADIX: one digit per thread
+        uint32_t c = 0;
+#pragma unroll
+        for (int ww = 0; ww < NW; ++ww) {
+            const uint32_t x = wcnt[ww][d];
+            wcnt[ww][d] = c;
+            c += x;
+        }
+        // publish this tile's count of digit d, then look back for the keys of
+        // digit d in all earlier tiles
+        const uint64_t tagA = (uint64_t)(2 * pass + 2) << 32, tagI = (uint64_t)(2 * pass + 3) << 32;
+        uint64_t* my = rec + t * RADIX + d;
+        uint64_t excl = 0;
+        if (t == 0) {
+            st_release64(my, tagI | c);
+        } else {
+            st_release64(my, tagA | c);
+            for (int64_t j = t - 1; j >= 0; --j) {
+                const uint64_t* r = rec + j * RADIX + d;
+                uint64_t val = ld_acquire64(r);
+                uint32_t it = 0;
+                while ((val & 0xFFFFFFFF00000000ull) < tagA) {
+                    if (++it > SORT_POLLS) break;
+                    __nanosleep(32);
+                    val = ld_acquire64(r);
+                }
+                if ((val & 0xFFFFFFFF00000000ull) < tagA) {
+                    set_status(status, ST_TIMEOUT);
+                    break;
+                }
+                excl += val & 0xFFFFFFFFull;
+                if ((val & 0xFFFFFFFF00000000ull) == tagI) break;
             }
+            st_release64(my, tagI | (excl + c));
         }
+        gbase[d] = (int64_t)offsets[d] + (int64_t)excl;
+        uint32_t tot;
+        dstart[d] = block_excl_sum<NT>(c, scan_sm, tot);
+    }
+    __syncthreads();
 #pragma unroll
-        for (int i = 0; i < KPT; ++i) {
-            const int d = dg[i];
-            const unsigned peers = __match_any_sync(FULL, d);
-            const uint32_t lower = __popc(peers & ltmask);
-            rk[i] = d < RADIX ? wcnt[w][d] + lower : 0u;
-            __syncwarp();
-            if (d < RADIX && lower == 0) wcnt[w][d] += __popc(peers);
-            __syncwarp();
+    for (int i = 0; i < KPT; ++i) {
+        const int d = dg[i];
+        if (d < RADIX) {
+            const uint32_t pos = dstart[d] + wcnt[w][d] + rk[i];
+            skey[pos] = k[i];
+            sval[pos] = v[i];
         }
-        __syncthreads();
-        {
-            const int d = threadIdx.x;  // NT == RADIX
-            uint32_t c = 0;
-#pragma unroll
-            for (int ww = 0; ww < NW; ++ww) {
-                const uint32_t t = wcnt[ww][d];
-                wcnt[ww][d] = c;
-                c += t;
-            }
-            dcount[d] = c;
-            uint32_t tot;
-            dstart[d] = block_excl_sum<NT>(c, scan_sm, tot);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < KPT; ++i) {
-            const int d = dg[i];
-            if (d < RADIX) {
-                const uint32_t pos = dstart[d] + wcnt[w][d] + rk[i];
-                skey[pos] = k[i];
-                sval[pos] = v[i];
-            }
-        }
-        __syncthreads();
-        const int cnt = (int)(end - tb < (int64_t)TILE ? end - tb : (int64_t)TILE);
-        for (int q = threadIdx.x; q < cnt; q += NT) {
-            const K kk = skey[q];
-            const int d = (int)((unsigned)(kk >> shift) & (RADIX - 1));
-            const int64_t gpos = (int64_t)run[d] + (q - (int)dstart[d]);
-            kdst[gpos] = last ? key_to_bits(kk) : kk;
-            vdst[gpos] = sval[q];
-        }
-        __syncthreads();
-        run[threadIdx.x] += dcount[threadIdx.x];
-        __syncthreads();
+    }
+    __syncthreads();
+    const int cnt = (int)(end - tb);
+    for (int q = threadIdx.x; q < cnt; q += NT) {
+        const K kk = skey[q];
+        const int d = (int)((unsigned)(kk >> shift) & (RADIX - 1));
+        const int64_t gpos = gbase[d] + (q - (int)dstart[d]);
+        kdst[gpos] = last ? key_to_bits(kk) : kk;
+        vdst[gpos] = sval[q];
     }
 }
 
 // ------------------------------------------------------------------ host side
-struct SortPlan {
-    int kpt;
-    int64_t tile, seg;
-    int G;
-};
-
-static SortPlan sort_plan(int64_t n, int f64) {
-    SortPlan p;
-    p.kpt = f64 ? 8 : 16;
-    p.tile = (int64_t)SORT_NT * p.kpt;
-    const int64_t tiles = std::max<int64_t>(1, (n + p.tile - 1) / p.tile);
-    const int64_t G0 = std::min<int64_t>(tiles, 148 * 4);
-    const int64_t per_tiles = (tiles + G0 - 1) / G0;
-    p.seg = per_tiles * p.tile;
-    p.G = (int)std::max<int64_t>(1, (n + p.seg - 1) / p.seg);
-    return p;
-}
+template <typename T> constexpr int sort_kpt() { return sizeof(T) == 8 ? 8 : 16; }
 
 size_t sort_ws_bytes(int64_t n, int f64) {
-    const SortPlan p = sort_plan(n, f64);
+    const int kpt = f64 ? 8 : 16;
+    const int64_t tile = (int64_t)SORT_NT * kpt;
+    const int64_t ntiles = std::max<int64_t>(1, (n + tile - 1) / tile);
     const size_t ks = f64 ? 8 : 4;
+    const int P = f64 ? 8 : 4;
     return Carve::need((size_t)n, ks) + Carve::need((size_t)n, 4) +
-           Carve::need((size_t)RADIX * p.G, 4);
+           Carve::need((size_t)(16 + P * RADIX), 4) + Carve::need((size_t)(ntiles * RADIX), 8);
 }
 
 template <typename T>
@@ -248,30 +271,37 @@ cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws, 
                      uint32_t* status, cudaStream_t st) {
     using K = typename KeyOf<T>::K;
     if (n == 0) return cudaSuccess;
-    const int f64 = sizeof(T) == 8;
-    const SortPlan p = sort_plan(n, f64);
+    constexpr int KPT = sort_kpt<T>();
+    constexpr int P = sizeof(K);
+    const int64_t tile = (int64_t)SORT_NT * KPT;
+    const int64_t ntiles = (n + tile - 1) / tile;
     Carve cv(ws, ws_bytes);
     K* kws = cv.take<K>(n);
     int32_t* vws = cv.take<int32_t>(n);
-    uint32_t* counts = cv.take<uint32_t>((size_t)RADIX * p.G);
+    uint32_t* ctl = cv.take<uint32_t>(16 + P * RADIX);  // [0..P) tickets, [16..) histograms
+    uint64_t* rec = cv.take<uint64_t>(ntiles * RADIX);
     if (!cv.ok) return cudaErrorInvalidValue;
+    uint32_t* tickets = ctl;
+    uint32_t* hist = ctl + 16;
+    cudaError_t e = cudaMemsetAsync(ctl, 0, sizeof(uint32_t) * (16 + P * RADIX), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(rec, 0, sizeof(uint64_t) * ntiles * RADIX, st);
+    if (e != cudaSuccess) return e;
+    {
+        const int64_t blocks = std::min<int64_t>((n + SORT_NT - 1) / SORT_NT, 148 * 8);
+        k_radix_hist<T><<<(unsigned)blocks, SORT_NT, 0, st>>>(a, n, hist, status);
+        k_radix_offsets<<<P, SORT_NT, 0, st>>>(hist);
+    }
     K* kout = reinterpret_cast<K*>(sorted);
-    const int passes = (int)(sizeof(K) * 8 / 8);
     const K* ksrc = nullptr;
     const int32_t* vsrc = nullptr;
-    for (int pass = 0; pass < passes; ++pass) {
-        const bool to_out = ((passes - 1 - pass) % 2) == 0;
+    for (int pass = 0; pass < P; ++pass) {
+        const bool to_out = ((P - 1 - pass) % 2) == 0;
         K* kdst = to_out ? kout : kws;
         int32_t* vdst = to_out ? perm : vws;
-        const int shift = 8 * pass;
-        const int first = pass == 0, last = pass == passes - 1;
-        k_radix_upsweep<T><<<p.G, SORT_NT, 0, st>>>(a, ksrc, n, shift, p.seg, p.G, counts, status,
-                                                     first);
-        k_radix_scan<<<1, 1024, 0, st>>>(counts, (int64_t)RADIX * p.G);
-        constexpr int KPT = sizeof(T) == 8 ? 8 : 16;
-        k_radix_downsweep<T, KPT><<<p.G, SORT_NT, 0, st>>>(a, ksrc, vsrc, n, shift, p.seg, p.G,
-                                                           counts, kdst, vdst, first, last);
-        cudaError_t e = cudaGetLastError();
+        k_onesweep<T, KPT><<<(unsigned)ntiles, SORT_NT, 0, st>>>(
+            a, ksrc, vsrc, n, pass, hist + pass * RADIX, rec, tickets + pass, kdst, vdst,
+            pass == P - 1, status);
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         ksrc = kdst;
         vsrc = vdst;

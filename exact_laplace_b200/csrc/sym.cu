@@ -14,7 +14,7 @@
 #include <algorithm>
 
 #include "laplex_impl.h"
-#include "scan_core.cuh"
+#include "onepass.cuh"
 
 namespace lx {
 
@@ -245,41 +245,9 @@ __global__ void __launch_bounds__(NT) k_sym_final(SymArgs<T> A, const T* __restr
 
 
 // ------------------------------------------------------------------ single pass
-// One launch streams s and x once and writes y once (12 bytes per element for
-// B = 1).  Tiles are taken in order from an atomic ticket.  Each tile
-//   1. scans itself and publishes its forward and backward totals (flag 1),
-//   2. looks back over the tiles to its left for the prefix carry, using an
-//      inclusive prefix (flag 2) where one is published, and stopping as soon
-//      as the decay exp(e_j - e_T) is exactly 0 (then every term further left
-//      is exactly 0 as well), then publishes its own inclusive prefix,
-//   3. looks ahead over at most J tiles to its right for the suffix carry in
-//      the same way, then publishes its inclusive suffix,
-//   4. finishes its elements and writes them.
-// A tile publishes its totals before it waits for anything, and tiles are
-// started in ticket order, so a wait on a left neighbour always ends; a wait on
-// a right neighbour ends as long as J is below the number of co-resident
-// blocks.  Every wait is bounded: an expired look-back sets ST_TIMEOUT; a look-
-// ahead that is too deep or expires marks the tile, which is then completed by
-// k_tile_carries (exact suffix carries from the published totals) and
-// k_sym_fixup (adds exp(s_r - s_end) * carry to the marked tiles' outputs).
-template <typename T>
-struct OnePassWs {
-    uint32_t* ctrl;   // [0] ticket, [1] number of marked tiles, then the flags
-    uint32_t* fflag;  // [ntiles] forward: 1 totals, 2 inclusive
-    uint32_t* bflag;  // [ntiles] backward: 1 totals, 2 inclusive
-    uint32_t* fix;    // [ntiles] 1: suffix carry left to k_sym_fixup
-    T* fagg;
-    T* finc;
-    T* bagg;
-    T* binc;
-    T* carF;          // scratch of k_tile_carries
-    T* carB;          // exact suffix carries (marked tiles only)
-};
-
-constexpr uint32_t LOOKBACK_POLLS = 1u << 25;
-constexpr uint32_t LOOKAHEAD_POLLS = 1u << 16;
-constexpr int LOOKAHEAD_TILES = 64;
-
+// One launch streams the input once and writes y once; carries between tiles
+// follow onepass.cuh (look-back for the prefix, bounded look-ahead for the
+// suffix, exact completion of deferred tiles by k_suffix_carries + k_sym_fixup).
 template <typename T, int NCOL, bool PHASED, int E, int NT>
 __global__ void __launch_bounds__(NT) k_sym_onepass(SymArgs<T> A, OnePassWs<T> W, int64_t ntiles) {
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
@@ -302,81 +270,17 @@ __global__ void __launch_bounds__(NT) k_sym_onepass(SymArgs<T> A, OnePassWs<T> W
     block_excl_fwd<T, C, NT>(s[E - 1], fV, hf, pe, pV, te, tV, smf);
     block_excl_bwd<T, C, NT>(s[0], bW, hb, nf, nW, tf, tW, smb);
     if (threadIdx.x == 0) {
-        const bool first = t == 0, last = t == ntiles - 1;
-#pragma unroll
-        for (int c = 0; c < C; ++c) {
-            W.fagg[t * C + c] = tV[c];
-            W.bagg[t * C + c] = tW[c];
-            if (first) W.finc[c] = tV[c];
-            if (last) W.binc[t * C + c] = tW[c];
-        }
-        st_release(&W.fflag[t], first ? 2u : 1u);
-        st_release(&W.bflag[t], last ? 2u : 1u);
-        // ---- look-back: L at the element before this tile (anchor eT)
-        const T eT = first ? A.s[0] : A.s[tile0 - 1];
-        T acc[C];
-#pragma unroll
-        for (int c = 0; c < C; ++c) acc[c] = T(0);
-        for (int64_t j = t - 1; j >= 0; --j) {
-            const T f = dexp<T>(A.s[(j + 1) * TILE - 1] - eT);
-            if (f == T(0)) break;
-            const uint32_t fl = wait_flag(&W.fflag[j], 1u, LOOKBACK_POLLS);
-            if (fl == 0u) {
-                set_status(A.status, ST_TIMEOUT);
-                break;
-            }
-            const T* src = (fl == 2u ? W.finc : W.fagg) + j * C;
-#pragma unroll
-            for (int c = 0; c < C; ++c) acc[c] = dfma<T>(f, __ldcg(src + c), acc[c]);
-            if (fl == 2u) break;
-        }
-        if (!first) {
-            const T d = dexp<T>(eT - te);
-#pragma unroll
-            for (int c = 0; c < C; ++c) W.finc[t * C + c] = dfma<T>(d, acc[c], tV[c]);
-            st_release(&W.fflag[t], 2u);
-        }
+        const T eT = t == 0 ? A.s[0] : A.s[tile0 - 1];
+        const T fT = t == ntiles - 1 ? A.s[n - 1] : A.s[tile0 + TILE];
+        T acc[C], accb[C];
+        onepass_carries<T, C>(W, t, ntiles, tf, tW, te, tV, eT, fT, acc, accb, A.status);
         sh_e[0] = eT;
-#pragma unroll
-        for (int c = 0; c < C; ++c) sh_c[0][c] = acc[c];
-        // ---- look-ahead: U at the element after this tile (anchor fT)
-        const T fT = last ? A.s[n - 1] : A.s[tile0 + TILE];
-        T accb[C];
-#pragma unroll
-        for (int c = 0; c < C; ++c) accb[c] = T(0);
-        bool defer = false;
-        int depth = 0;
-        for (int64_t j = t + 1; j < ntiles; ++j) {
-            const T f = dexp<T>(fT - A.s[j * TILE]);
-            if (f == T(0)) break;
-            if (++depth > LOOKAHEAD_TILES) {
-                defer = true;
-                break;
-            }
-            const uint32_t fl = wait_flag(&W.bflag[j], 1u, LOOKAHEAD_POLLS);
-            if (fl == 0u) {
-                defer = true;
-                break;
-            }
-            const T* src = (fl == 2u ? W.binc : W.bagg) + j * C;
-#pragma unroll
-            for (int c = 0; c < C; ++c) accb[c] = dfma<T>(f, __ldcg(src + c), accb[c]);
-            if (fl == 2u) break;
-        }
-        if (defer) {
-#pragma unroll
-            for (int c = 0; c < C; ++c) accb[c] = T(0);
-            W.fix[t] = 1u;
-            atomicAdd(&W.ctrl[1], 1u);
-        } else if (!last) {
-            const T d = dexp<T>(tf - fT);
-#pragma unroll
-            for (int c = 0; c < C; ++c) W.binc[t * C + c] = dfma<T>(d, accb[c], tW[c]);
-            st_release(&W.bflag[t], 2u);
-        }
         sh_e[1] = fT;
 #pragma unroll
-        for (int c = 0; c < C; ++c) sh_c[1][c] = accb[c];
+        for (int c = 0; c < C; ++c) {
+            sh_c[0][c] = acc[c];
+            sh_c[1][c] = accb[c];
+        }
     }
     __syncthreads();
     T VT[C], WT[C];
@@ -397,28 +301,29 @@ __global__ void __launch_bounds__(NT) k_sym_onepass(SymArgs<T> A, OnePassWs<T> W
 template <typename T, int NCOL, bool PHASED, int NT>
 __global__ void __launch_bounds__(NT) k_sym_fixup(SymArgs<T> A, OnePassWs<T> W, int64_t tile) {
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
-    if (W.ctrl[1] == 0u) return;
-    const int64_t t = blockIdx.x;
-    if (W.fix[t] == 0u) return;
-    const int64_t n = A.n;
-    const int64_t b = t * tile, e = min(b + tile, n);
-    if (e >= n) return;
-    const T fT = A.s[e];
-    T cr[C];
+    const uint32_t nfix = W.ctrl[1];
+    for (uint32_t q = blockIdx.x; q < nfix; q += gridDim.x) {
+        const int64_t t = W.fix[q];
+        const int64_t n = A.n;
+        const int64_t b = t * tile, e = min(b + tile, n);
+        if (e >= n) continue;
+        const T fT = A.s[e];
+        T cr[C];
 #pragma unroll
-    for (int c = 0; c < C; ++c) cr[c] = W.carB[t * C + c];
-    for (int64_t r = b + threadIdx.x; r < e; r += NT) {
-        const T f = dexp<T>(A.s[r] - fT);
-        if (f == T(0)) continue;
-        const int64_t row = A.pout ? (int64_t)A.pout[r] : r;
-        T* yr = A.y + row * A.ldy + A.col0;
-        if (PHASED) {
-            const int64_t ar = A.paux ? (int64_t)A.paux[r] : r;
-            T sp, cp;
-            dsincos<T>(A.phi[ar], &sp, &cp);
-            for (int c = 0; c < A.ncol; ++c) yr[c] += f * (cp * cr[2 * c] + sp * cr[2 * c + 1]);
-        } else {
-            for (int c = 0; c < A.ncol; ++c) yr[c] += f * cr[c];
+        for (int c = 0; c < C; ++c) cr[c] = W.carB[t * C + c];
+        for (int64_t r = b + threadIdx.x; r < e; r += NT) {
+            const T f = dexp<T>(A.s[r] - fT);
+            if (f == T(0)) continue;
+            const int64_t row = A.pout ? (int64_t)A.pout[r] : r;
+            T* yr = A.y + row * A.ldy + A.col0;
+            if (PHASED) {
+                const int64_t ar = A.paux ? (int64_t)A.paux[r] : r;
+                T sp, cp;
+                dsincos<T>(A.phi[ar], &sp, &cp);
+                for (int c = 0; c < A.ncol; ++c) yr[c] += f * (cp * cr[2 * c] + sp * cr[2 * c + 1]);
+            } else {
+                for (int c = 0; c < A.ncol; ++c) yr[c] += f * cr[c];
+            }
         }
     }
 }
@@ -451,8 +356,9 @@ static SymPlan sym_plan(int64_t n, int64_t B, bool phased, int f64) {
 
 size_t sym_ws_bytes(int64_t n, int64_t B, bool phased, int f64) {
     const SymPlan p = sym_plan(n, B, phased, f64);
-    const size_t es = f64 ? 8 : 4;
-    return Carve::need((size_t)(2 + 3 * p.ntiles), 4) + 6 * Carve::need((size_t)(p.ntiles * p.C), es);
+    const size_t a = onepass_ws_bytes(p.ntiles, p.C, f64 ? 8 : 4);
+    const size_t b = (!phased && B == 1) ? stream_ws_bytes(n, f64) : 0;
+    return a > b ? a : b;
 }
 
 template <typename T, int NCOL, bool PHASED, int E>
@@ -471,12 +377,11 @@ static cudaError_t onepass_launch(const SymArgs<T>& A, int64_t ntiles, const One
                                   cudaStream_t st) {
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
     constexpr int64_t TILE = (int64_t)SYM_NT * E;
-    cudaError_t e = cudaMemsetAsync(W.ctrl, 0, sizeof(uint32_t) * (2 + 3 * ntiles), st);
+    cudaError_t e = onepass_reset(W, ntiles, st);
     if (e != cudaSuccess) return e;
     k_sym_onepass<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, W, ntiles);
-    k_tile_carries<T, C, 1024><<<1, 1024, 0, st>>>(A.s, A.n, TILE, ntiles, W.fagg, W.bagg, W.carF,
-                                                     W.carB, W.ctrl + 1);
-    k_sym_fixup<T, NCOL, PHASED, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, W, TILE);
+    k_suffix_carries<T, C, 1024><<<1, 1024, 0, st>>>(W, ntiles);
+    k_sym_fixup<T, NCOL, PHASED, SYM_NT><<<FIXUP_BLOCKS, SYM_NT, 0, st>>>(A, W, TILE);
     return cudaGetLastError();
 }
 
@@ -484,19 +389,12 @@ template <typename T>
 cudaError_t sym_run(SymArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_bytes,
                     cudaStream_t st) {
     if (A.n == 0) return cudaSuccess;
+    // contiguous single-column input (pre-sorted product): the streaming kernel
+    if (!phased && B == 1 && A.pin == nullptr && A.D == nullptr && A.ldx == 1 && A.ldy == 1)
+        return stream_run<T>(A.s, A.x, A.y, A.pout, A.n, ws, ws_bytes, A.status, st);
     const SymPlan p = sym_plan(A.n, B, phased, sizeof(T) == 8);
     Carve cv(ws, ws_bytes);
-    OnePassWs<T> W;
-    W.ctrl = cv.take<uint32_t>(2 + 3 * p.ntiles);
-    W.fflag = W.ctrl + 2;
-    W.bflag = W.fflag + p.ntiles;
-    W.fix = W.bflag + p.ntiles;
-    W.fagg = cv.take<T>(p.ntiles * p.C);
-    W.finc = cv.take<T>(p.ntiles * p.C);
-    W.bagg = cv.take<T>(p.ntiles * p.C);
-    W.binc = cv.take<T>(p.ntiles * p.C);
-    W.carF = cv.take<T>(p.ntiles * p.C);
-    W.carB = cv.take<T>(p.ntiles * p.C);
+    OnePassWs<T> W = onepass_carve<T>(cv, p.ntiles, p.C);
     if (!cv.ok) return cudaErrorInvalidValue;
     for (int64_t g = 0; g < p.groups; ++g) {
         A.col0 = g * p.ncol;
