@@ -37,7 +37,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "LAPLEX sym matvec Gelem/s at n=2^30 fp32; achieved HBM GB/s vs B200 peak"
 BYTES_PER_ELEM_SYM = 12  # read s (4) + x (4), write y (4): the minimum the product moves
-KERNELS_PER_SYM_CALL = 3  # launches of this library per laplex_matvec_sym call (B <= 8)
+# launches of this library per pre-sorted single-column laplex_matvec_sym call:
+# k_tile_local, k_carry_blocks, k_carry_tiles, k_headtail
+KERNELS_PER_SYM_CALL = 4
 
 
 def parse():
@@ -47,7 +49,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--n", type=int, default=1 << 30)
-    p.add_argument("--rows", default="sort,perm,backward",
+    p.add_argument("--rows", default="sort,perm,backward,c2,c3,c4",
                    help="extra hot-path rows to time (comma list; empty for none)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -241,22 +243,53 @@ def run_ours(args):
         return max_over_ranks(e0.elapsed_time(e1))
 
     # ---------------- headline: pre-sorted symmetric product
+    # events around the dominant kernel (k_tile_local) of every timed call, recorded
+    # by the library on the call's stream (laplex_set_profile_events)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for b, a in kev:  # create the CUDA events
+        b.record(stream)
+        a.record(stream)
+    torch.cuda.synchronize(dev)
+    it = {"i": -1}
+
+    def sym_step():
+        i = it["i"]
+        if 0 <= i < len(kev):
+            X.set_profile_events(kev[i][0], kev[i][1])
+        else:
+            X.set_profile_events(None, None)
+        X.matvec_sym(s_d, x_d, out=y_d)
+
+    def counted():
+        sym_step()
+        it["i"] += 1
+
+    for _ in range(args.warmup):
+        sym_step()
+    it["i"] = 0
     clk = Clocks(local)
-    ms = timed(lambda: X.matvec_sym(s_d, x_d, out=y_d), args.steps, args.warmup)
+    ms = timed(counted, args.steps, 0)
     clocks = clk.stop()
+    X.set_profile_events(None, None)
     X.device_status(dev)
+    kernel_ms = max_over_ranks(sum(b.elapsed_time(a) for b, a in kev) / len(kev))
     ms_step = ms / args.steps
     value = world * n / (ms_step * 1e-3) / 1e9
     hbm, peak_kind = peaks()
-    achieved = BYTES_PER_ELEM_SYM * n / (ms_step * 1e-3) / 1e9
-    sha = src_sha("sym.cu", "scan_core.cuh", "common.cuh")
-    traffic = traffic_from_profile("matvec_sym_presorted_b1", sha, n)
+    achieved = BYTES_PER_ELEM_SYM * n / (kernel_ms * 1e-3) / 1e9
+    sha = src_sha("sym_stream.cu", "scan_core.cuh", "common.cuh")
+    traffic = traffic_from_profile("k_tile_local_presorted_b1", sha, n)
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "traffic": traffic,
             "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
             else "fallback 6650 GB/s",
-            "kernel": "laplex_matvec_sym (whole call)",
-            "algorithmic_bytes_per_launch": BYTES_PER_ELEM_SYM * n}
+            "kernel": "k_tile_local (dominant kernel of laplex_matvec_sym)",
+            "kernel_ms": kernel_ms,
+            "algorithmic_bytes_per_launch": BYTES_PER_ELEM_SYM * n,
+            "whole_call": {"ms": ms_step, "achieved_GB_s": BYTES_PER_ELEM_SYM * n / (ms_step * 1e-3) / 1e9,
+                           "frac": BYTES_PER_ELEM_SYM * n / (ms_step * 1e-3) / 1e9 / hbm,
+                           "kernels": "k_tile_local + k_carry_blocks + k_carry_tiles + k_headtail"}}
 
     # ---------------- other rows on the same data
     rows = {}
@@ -272,16 +305,18 @@ def run_ours(args):
             if "sort" in wanted:
                 ms_s = timed(lambda: X.sort_anchors(a_d, s2, p2), rsteps, 1) / rsteps
                 X.device_status(dev)
-                rows["sort"] = {"ms": ms_s, "Gelem_s": world * n / ms_s / 1e6,
-                                "algorithmic_GB_s": 12 * n / ms_s / 1e6,
-                                "algorithmic_bytes_per_elem": 12}
+                rows["c5_sort"] = {"ms": ms_s, "Gelem_s": world * n / ms_s / 1e6,
+                                   "algorithmic_GB_s": 12 * n / ms_s / 1e6,
+                                   "frac_of_measured_hbm": 12 * n / ms_s / 1e6 / hbm,
+                                   "algorithmic_bytes_per_elem": 12}
             if "perm" in wanted:
                 X.sort_anchors(a_d, s2, p2)
                 ms_p = timed(lambda: X.matvec_sym(s2, x_d, p2, out=y_d), rsteps, 1) / rsteps
                 X.device_status(dev)
-                rows["matvec_perm"] = {"ms": ms_p, "Gelem_s": world * n / ms_p / 1e6,
-                                       "algorithmic_GB_s": 16 * n / ms_p / 1e6,
-                                       "algorithmic_bytes_per_elem": 16}
+                rows["c5_matvec_perm"] = {"ms": ms_p, "Gelem_s": world * n / ms_p / 1e6,
+                                          "algorithmic_GB_s": 16 * n / ms_p / 1e6,
+                                          "frac_of_measured_hbm": 16 * n / ms_p / 1e6 / hbm,
+                                          "algorithmic_bytes_per_elem": 16}
         except X.LaplexError as e:
             rows["sort_error"] = str(e)
         del a_d, s2, p2
@@ -292,13 +327,98 @@ def run_ours(args):
                 da = torch.empty_like(x_d)
                 ms_b = timed(lambda: X.backward(s_d, x_d, g_d, dx_out=dx, da_out=da), rsteps, 1) / rsteps
                 X.device_status(dev)
-                rows["backward"] = {"ms": ms_b, "Gelem_s": world * n / ms_b / 1e6,
-                                    "algorithmic_GB_s": 20 * n / ms_b / 1e6,
-                                    "algorithmic_bytes_per_elem": 20}
+                rows["c5_backward"] = {"ms": ms_b, "Gelem_s": world * n / ms_b / 1e6,
+                                       "algorithmic_GB_s": 20 * n / ms_b / 1e6,
+                                       "frac_of_measured_hbm": 20 * n / ms_b / 1e6 / hbm,
+                                       "algorithmic_bytes_per_elem": 20}
                 del g_d, dx, da
             except X.LaplexError as e:
                 rows["backward_error"] = str(e)
         torch.cuda.empty_cache()
+
+    # ---------------- the other workloads (inputs near or below L2 size: flushed)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed_flush(fn, steps):
+        """Sum of per-call device times, the 126 MB L2 flushed (256 MB write)
+        before every call and outside the timed events."""
+        fn()
+        torch.cuda.synchronize(dev)
+        evs = []
+        for _ in range(steps):
+            flush_buf.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        return max_over_ranks(sum(a.elapsed_time(b) for a, b in evs)) / steps
+
+    def row(ms, elems, bytes_per, note):
+        gbs = bytes_per / ms / 1e6
+        return {"ms": ms, "Gelem_s": world * elems / ms / 1e6, "algorithmic_GB_s": gbs,
+                "frac_of_measured_hbm": gbs / hbm, "algorithmic_bytes": bytes_per, "note": note}
+
+    fsteps = max(3, min(20, args.steps // 10))
+    try:
+        if "c2" in wanted:
+            n2 = 1 << 24
+            for B in (1, 8):
+                a2, x2 = synth.sym_normal(n2, 2000.0, B=B, seed=rank)
+                a2d = torch.from_numpy(a2).to(dev)
+                x2d = torch.from_numpy(x2).to(dev)
+                y2d = torch.empty_like(x2d)
+                s2d = torch.empty_like(a2d)
+                p2d = torch.empty(n2, dtype=torch.int32, device=dev)
+
+                def c2_full():
+                    X.sort_anchors(a2d, s2d, p2d)
+                    X.matvec_sym(s2d, x2d, p2d, out=y2d)
+                ms2 = timed_flush(c2_full, fsteps)
+                rows[f"c2_sort_and_matvec_B{B}"] = row(ms2, n2, n2 * (12 + 16 + 8 * B), "n=2^24, a~N(0,2000^2) unsorted: sort + permuted product")
+                X.sort_anchors(a2d, s2d, p2d)
+                xs = x2d[p2d.long()].contiguous()
+                ms3 = timed_flush(lambda: X.matvec_sym(s2d, xs, out=y2d), fsteps)
+                rows[f"c2_presorted_B{B}"] = row(ms3, n2, n2 * (4 + 8 * B), "n=2^24 pre-sorted product")
+                del a2d, x2d, y2d, s2d, p2d, xs
+            X.device_status(dev)
+        if "c3" in wanted:
+            a3, b3, x3, w3 = synth.general_ties(1 << 22, 1 << 20, -1000.0, 1000.0, seed=rank)
+            a3d, b3d = torch.from_numpy(a3).to(dev), torch.from_numpy(b3).to(dev)
+            sa, pa = X.sort_anchors(a3d)
+            sb, pb = X.sort_anchors(b3d)
+            x3d, w3d = torch.from_numpy(x3).to(dev), torch.from_numpy(w3).to(dev)
+            xs3 = x3d[pb.long()].contiguous()
+            ws3 = w3d[pa.long()].contiguous()
+            y3 = torch.empty_like(ws3)
+            z3 = torch.empty_like(xs3)
+            nn, kk = 1 << 22, 1 << 20
+            ms = timed_flush(lambda: X.matvec_general(sa, sb, xs3, out=y3), fsteps)
+            rows["c3_general_Kx"] = row(ms, nn, 8 * nn + 8 * kk, "n=2^22, k=2^20, pre-sorted, y=Kx")
+            ms = timed_flush(lambda: X.matvec_general(sa, sb, ws3, transpose=True, out=z3), fsteps)
+            rows["c3_general_KTw"] = row(ms, kk, 8 * nn + 8 * kk, "n=2^22, k=2^20, pre-sorted, z=K^T w")
+            X.device_status(dev)
+            del a3d, b3d, sa, pa, sb, pb, x3d, w3d, xs3, ws3, y3, z3
+        if "c4" in wanted:
+            a4, phi4, v4 = synth.phased_image(seed=rank)
+            n4 = a4.size
+            a4d = torch.from_numpy(a4).to(dev)
+            s4, p4 = X.sort_anchors(a4d)
+            phis = torch.from_numpy(phi4).to(dev)[p4.long()].contiguous()
+            vs = torch.from_numpy(v4).to(dev)[p4.long()].contiguous()
+            y4 = torch.empty_like(vs)
+            ms = timed_flush(lambda: X.matvec_phased(s4, phis, vs, out=y4), fsteps)
+            rows["c4_phased_Kv"] = row(ms, n4, 16 * n4, "n=3*1024^2, pre-sorted, phased y=Kv")
+            ms = timed_flush(lambda: X.gram(s4, vs, phi=phis, out=y4), fsteps)
+            rows["c4_gram_KTKv"] = row(ms, n4, 32 * n4, "n=3*1024^2, pre-sorted, K^T K v")
+            X.device_status(dev)
+            del a4d, s4, p4, phis, vs, y4
+    except X.LaplexError as e:
+        rows["rows_error"] = str(e)
+    del flush_buf
+    torch.cuda.empty_cache()
 
     # ---------------- end to end through host buffers (pinned)
     e2e = None

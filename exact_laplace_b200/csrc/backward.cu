@@ -9,209 +9,160 @@
 // strictly-upper exp-weighted sum:  D(v)_r = (L^v_r - P^v_r) - (U^v_r - Q^v_r),
 // where L, U are the inclusive prefix/suffix scans of the symmetric product and
 // P, Q the inclusive prefix/suffix sums over the run of anchors equal to a_r
-// (scan_core.cuh "tie channels").  One single-pass scan of four channels
-// (x, g with exp decay; x, g with tie decay) reads s, x, g once and writes
-// dx, da once: 20 bytes per anchor in fp32.
+// (scan_core.cuh "tie channels").  One scan of four channels (x, g with exp
+// decay; x, g with tie decay) reads s, x, g once and writes dx, da once
+// (20 bytes per anchor in fp32), in the wait-free scheme of threepass.cuh.
 #include <algorithm>
 
 #include "laplex_impl.h"
-#include "onepass.cuh"
+#include "threepass.cuh"
 
 namespace lx {
 
 constexpr int BWD_NT = 256;
 
-template <typename T, int E, int NT>
-__global__ void __launch_bounds__(NT) k_bwd_onepass(const T* __restrict__ s_, const int32_t* __restrict__ perm,
-                                                    int64_t n, const T* __restrict__ x_,
-                                                    const T* __restrict__ g_, T* __restrict__ dx_,
-                                                    T* __restrict__ da_, OnePassWs<T> W, int64_t ntiles,
-                                                    uint32_t* status) {
-    constexpr int C = 4, CT = 2;
-    constexpr int VN = V16<T>::N;
-    constexpr int64_t TILE = (int64_t)NT * E;
-    __shared__ BlockScanSmem<T, C, NT> smf, smb;
-    __shared__ int64_t sh_tile;
-    __shared__ T sh_e[2];
-    __shared__ T sh_c[2][C];
-    if (threadIdx.x == 0) sh_tile = (int64_t)atomicAdd(&W.ctrl[0], 1u);
-    __syncthreads();
-    const int64_t t = sh_tile;
-    const int64_t tile0 = t * TILE;
-    const int64_t r0 = tile0 + (int64_t)threadIdx.x * E;
-    const bool full = r0 + E <= n;
-    T s[E], xv[E], gv[E];
-    if (full) {
+// Policy of threepass.cuh (wait-free: tile-local scans, exact tile carries,
+// carries added to the heads and tails of the tiles).  Channels: x and g with
+// exp decay (L, U), then x and g with tie decay (P, Q).
+template <typename T_, int E_>
+struct BwdTP {
+    using T = T_;
+    static constexpr int C = 4, CT = 2, E = E_, NT = BWD_NT;
+    int64_t n;
+    const T* s;
+    const int32_t* perm;
+    const T* x;
+    const T* g;
+    T* dx;
+    T* da;
+    struct Aux {};
+    __device__ __forceinline__ void load(int64_t r0, T (&sv)[E], T (&v)[E][C], Aux&) const {
+        constexpr int VN = V16<T>::N;
+        const bool full = r0 + E <= n;
+        T xv[E], gv[E];
+        if (full) {
 #pragma unroll
-        for (int i = 0; i < E; i += VN) ld16_stream<T>(s_ + r0 + i, &s[i]);
-    } else {
+            for (int i = 0; i < E; i += VN) ld16_stream<T>(s + r0 + i, &sv[i]);
+        } else {
 #pragma unroll
-        for (int i = 0; i < E; ++i) s[i] = s_[min(r0 + i, n - 1)];
-    }
-    if (full && perm == nullptr) {
-#pragma unroll
-        for (int i = 0; i < E; i += VN) {
-            ld16_stream<T>(x_ + r0 + i, &xv[i]);
-            ld16_stream<T>(g_ + r0 + i, &gv[i]);
+            for (int i = 0; i < E; ++i) sv[i] = s[min(r0 + i, n - 1)];
         }
-    } else {
+        if (full && perm == nullptr) {
+#pragma unroll
+            for (int i = 0; i < E; i += VN) {
+                ld16_stream<T>(x + r0 + i, &xv[i]);
+                ld16_stream<T>(g + r0 + i, &gv[i]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const int64_t r = r0 + i;
+                const int64_t row = r < n ? (perm ? (int64_t)perm[r] : r) : 0;
+                xv[i] = r < n ? x[row] : T(0);
+                gv[i] = r < n ? g[row] : T(0);
+            }
+        }
 #pragma unroll
         for (int i = 0; i < E; ++i) {
-            const int64_t r = r0 + i;
-            if (r < n) {
-                const int64_t row = perm ? (int64_t)perm[r] : r;
-                xv[i] = x_[row];
-                gv[i] = g_[row];
-            } else {
-                xv[i] = T(0);
-                gv[i] = T(0);
+            v[i][0] = xv[i];
+            v[i][1] = gv[i];
+            v[i][2] = xv[i];
+            v[i][3] = gv[i];
+        }
+    }
+    __device__ __forceinline__ void finish(int64_t r0, const T (&sv)[E], const T (&v)[E][C],
+                                           T (&dl)[E], T eprev, const T (&Lp)[C], T enext,
+                                           const T (&Un)[C], Aux&) const {
+        constexpr int VN = V16<T>::N;
+        T Lo[E][C];
+        {
+            T L[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) L[c] = Lp[c];
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const T pv = i == 0 ? eprev : sv[i - 1];
+                const T de = i == 0 ? dexp<T>(eprev - sv[0]) : dl[i];
+                const T dt = pv == sv[i] ? T(1) : T(0);
+#pragma unroll
+                for (int c = 0; c < C; ++c) {
+                    L[c] = dfma<T>(c < 2 ? de : dt, L[c], v[i][c]);
+                    Lo[i][c] = L[c];
+                }
+            }
+        }
+        T dxo[E], dao[E];
+        {
+            T U[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) U[c] = Un[c];
+#pragma unroll
+            for (int i = E - 1; i >= 0; --i) {
+                const T nx = i == E - 1 ? enext : sv[i + 1];
+                const T de = i == E - 1 ? dexp<T>(sv[E - 1] - enext) : dl[i + 1];
+                const T dt = sv[i] == nx ? T(1) : T(0);
+#pragma unroll
+                for (int c = 0; c < C; ++c) U[c] = dfma<T>(c < 2 ? de : dt, U[c], v[i][c]);
+                dxo[i] = Lo[i][1] + U[1] - v[i][1];
+                const T Dx = (Lo[i][0] - Lo[i][2]) - (U[0] - U[2]);
+                const T Dg = (Lo[i][1] - Lo[i][3]) - (U[1] - U[3]);
+                dao[i] = -(v[i][1] * Dx + v[i][0] * Dg);
+            }
+        }
+        if (r0 + E <= n && perm == nullptr) {
+#pragma unroll
+            for (int i = 0; i < E; i += VN) {
+                st16_stream<T>(dx + r0 + i, &dxo[i]);
+                st16_stream<T>(da + r0 + i, &dao[i]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const int64_t r = r0 + i;
+                if (r < n) {
+                    const int64_t row = perm ? (int64_t)perm[r] : r;
+                    dx[row] = dxo[i];
+                    da[row] = dao[i];
+                }
             }
         }
     }
-    T v[E][C], dl[E], fV[C], bW[C];
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-        v[i][0] = xv[i];
-        v[i][1] = gv[i];
-        v[i][2] = xv[i];
-        v[i][3] = gv[i];
+    // A carry c = (L^x, L^g, P^x, P^g) from the left or (U^x, U^g, Q^x, Q^g)
+    // from the right, with exp factor fe and tie factor ft at element r.
+    __device__ __forceinline__ void carry_in(int64_t r, T fe, T ft, const T* c, bool left) const {
+        const int64_t row = perm ? (int64_t)perm[r] : r;
+        const T xr = x[row], gr = g[row];
+        const T dDx = fe * c[0] - ft * c[2];  // change of the strictly-lower (left) or -upper sum
+        const T dDg = fe * c[1] - ft * c[3];
+        dx[row] += fe * c[1];
+        // D(v) = lower - upper: a left carry adds to it, a right carry subtracts
+        if (left) da[row] -= gr * dDx + xr * dDg;
+        else da[row] += gr * dDx + xr * dDg;
     }
-    chunk_aggregates<T, C, E, CT>(s, v, dl, fV, bW);
-    bool hf, hb;
-    T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
-    block_excl_fwd<T, C, NT, CT>(s[E - 1], fV, hf, pe, pV, te, tV, smf);
-    block_excl_bwd<T, C, NT, CT>(s[0], bW, hb, nf, nW, tf, tW, smb);
-    if (threadIdx.x == 0) {
-        const T eT = t == 0 ? s_[0] : s_[tile0 - 1];
-        const T fT = tile0 + TILE < n ? s_[tile0 + TILE] : s_[n - 1];
-        T acc[C], accb[C];
-        onepass_carries<T, C, CT>(W, t, ntiles, tf, tW, te, tV, eT, fT, acc, accb, status);
-        sh_e[0] = eT;
-        sh_e[1] = fT;
-#pragma unroll
-        for (int c = 0; c < C; ++c) {
-            sh_c[0][c] = acc[c];
-            sh_c[1][c] = accb[c];
-        }
-    }
-    __syncthreads();
-    T VT[C], WT[C];
-#pragma unroll
-    for (int c = 0; c < C; ++c) {
-        VT[c] = sh_c[0][c];
-        WT[c] = sh_c[1][c];
-    }
-    T eprev, Lprev[C], enext, Unext[C];
-    apply_carry_fwd<T, C, CT>(hf, pe, pV, sh_e[0], VT, eprev, Lprev);
-    apply_carry_bwd<T, C, CT>(hb, nf, nW, sh_e[1], WT, enext, Unext);
-    // forward: L (exp) and P (tie) at every element
-    T Lo[E][C];
-    {
-        T L[C];
-#pragma unroll
-        for (int c = 0; c < C; ++c) L[c] = Lprev[c];
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-            const T pv = i == 0 ? eprev : s[i - 1];
-            const T de = i == 0 ? dexp<T>(eprev - s[0]) : dl[i];
-            const T dt = pv == s[i] ? T(1) : T(0);
-#pragma unroll
-            for (int c = 0; c < C; ++c) {
-                L[c] = dfma<T>(c < 2 ? de : dt, L[c], v[i][c]);
-                Lo[i][c] = L[c];
-            }
-        }
-    }
-    // backward: U (exp) and Q (tie), and the outputs
-    T dxo[E], dao[E];
-    {
-        T U[C];
-#pragma unroll
-        for (int c = 0; c < C; ++c) U[c] = Unext[c];
-#pragma unroll
-        for (int i = E - 1; i >= 0; --i) {
-            const T nx = i == E - 1 ? enext : s[i + 1];
-            const T de = i == E - 1 ? dexp<T>(s[E - 1] - enext) : dl[i + 1];
-            const T dt = s[i] == nx ? T(1) : T(0);
-#pragma unroll
-            for (int c = 0; c < C; ++c) U[c] = dfma<T>(c < 2 ? de : dt, U[c], v[i][c]);
-            dxo[i] = Lo[i][1] + U[1] - gv[i];
-            const T Dx = (Lo[i][0] - Lo[i][2]) - (U[0] - U[2]);
-            const T Dg = (Lo[i][1] - Lo[i][3]) - (U[1] - U[3]);
-            dao[i] = -(gv[i] * Dx + xv[i] * Dg);
-        }
-    }
-    if (full && perm == nullptr) {
-#pragma unroll
-        for (int i = 0; i < E; i += VN) {
-            st16_stream<T>(dx_ + r0 + i, &dxo[i]);
-            st16_stream<T>(da_ + r0 + i, &dao[i]);
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-            const int64_t r = r0 + i;
-            if (r < n) {
-                const int64_t row = perm ? (int64_t)perm[r] : r;
-                dx_[row] = dxo[i];
-                da_[row] = dao[i];
-            }
-        }
-    }
-}
-
-// Deferred tiles: add the suffix carry (U^x, U^g by exp(s_r - fT), Q^x, Q^g by
-// [s_r == fT]) to dx and da of the tile's anchors.
-template <typename T, int NT>
-__global__ void __launch_bounds__(NT) k_bwd_fixup(const T* __restrict__ s_, const int32_t* __restrict__ perm,
-                                                  int64_t n, const T* __restrict__ x_,
-                                                  const T* __restrict__ g_, T* __restrict__ dx_,
-                                                  T* __restrict__ da_, OnePassWs<T> W, int64_t tile) {
-    const uint32_t nfix = W.ctrl[1];
-    for (uint32_t q = blockIdx.x; q < nfix; q += gridDim.x) {
-        const int64_t t = W.fix[q];
-        const int64_t b = t * tile, e = min(b + tile, n);
-        if (e >= n) continue;
-        const T fT = s_[e];
-        const T cx = W.carB[t * 4 + 0], cg = W.carB[t * 4 + 1];
-        const T qx = W.carB[t * 4 + 2], qg = W.carB[t * 4 + 3];
-        for (int64_t r = b + threadIdx.x; r < e; r += NT) {
-            const T f = dexp<T>(s_[r] - fT);
-            const T qq = s_[r] == fT ? T(1) : T(0);
-            if (f == T(0) && qq == T(0)) continue;
-            const int64_t row = perm ? (int64_t)perm[r] : r;
-            const T dUx = f * cx, dUg = f * cg, dQx = qq * qx, dQg = qq * qg;
-            dx_[row] += dUg;
-            da_[row] += g_[row] * (dUx - dQx) + x_[row] * (dUg - dQg);
-        }
-    }
-}
+};
 
 static constexpr int bwd_E(int es) { return es == 4 ? 8 : 4; }
 
 size_t bwd_ws_bytes(int64_t n, int f64) {
     const int64_t tile = (int64_t)BWD_NT * bwd_E(f64 ? 8 : 4);
     const int64_t ntiles = std::max<int64_t>(1, (n + tile - 1) / tile);
-    return onepass_ws_bytes(ntiles, 4, f64 ? 8 : 4);
+    return tp_ws_bytes(ntiles, 4, f64 ? 8 : 4);
 }
 
 template <typename T>
 cudaError_t bwd_run(const T* s, const int32_t* perm, int64_t n, const T* x, const T* g, T* dx,
                     T* da, void* ws, size_t ws_bytes, uint32_t* status, cudaStream_t st) {
+    (void)status;  // no inter-block waits
     if (n == 0) return cudaSuccess;
-    constexpr int E = bwd_E((int)sizeof(T));
-    const int64_t tile = (int64_t)BWD_NT * E;
-    const int64_t ntiles = (n + tile - 1) / tile;
-    Carve cv(ws, ws_bytes);
-    OnePassWs<T> W = onepass_carve<T>(cv, ntiles, 4);
-    if (!cv.ok) return cudaErrorInvalidValue;
-    cudaError_t e = onepass_reset(W, ntiles, st);
-    if (e != cudaSuccess) return e;
-    k_bwd_onepass<T, E, BWD_NT><<<(unsigned)ntiles, BWD_NT, 0, st>>>(s, perm, n, x, g, dx, da, W,
-                                                                     ntiles, status);
-    k_suffix_carries<T, 4, 1024, 2><<<1, 1024, 0, st>>>(W, ntiles);
-    k_bwd_fixup<T, BWD_NT><<<FIXUP_BLOCKS, BWD_NT, 0, st>>>(s, perm, n, x, g, dx, da, W, tile);
-    return cudaGetLastError();
+    BwdTP<T, bwd_E((int)sizeof(T))> p;
+    p.n = n;
+    p.s = s;
+    p.perm = perm;
+    p.x = x;
+    p.g = g;
+    p.dx = dx;
+    p.da = da;
+    return tp_run(p, ws, ws_bytes, st);
 }
 
 template cudaError_t bwd_run<float>(const float*, const int32_t*, int64_t, const float*,

@@ -104,6 +104,12 @@ uint32_t* ws_status(void* ws) { return static_cast<uint32_t*>(ws); }
 
 }  // namespace
 
+namespace {
+thread_local lx::ProfileEvents g_prof = {nullptr, nullptr};
+}
+
+const lx::ProfileEvents& lx::profile_events() { return g_prof; }
+
 void lx::set_last_error(const char* fmt, ...) {
     va_list ap;
     va_start(ap, fmt);
@@ -128,6 +134,12 @@ const char* laplex_status_string(laplex_status s) {
 }
 
 const char* laplex_last_error(void) { return g_err; }
+
+laplex_status laplex_set_profile_events(void* before, void* after) {
+    g_prof.before = (cudaEvent_t)before;
+    g_prof.after = (cudaEvent_t)after;
+    return ok();
+}
 
 laplex_status laplex_workspace_size(laplex_op op, int64_t n, int64_t k, int64_t B, laplex_dtype dt,
                                     size_t* bytes) {

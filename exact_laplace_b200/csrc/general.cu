@@ -252,7 +252,9 @@ static cudaError_t gen_launch(const GenArgs<T>& A, const GenPlan& p, const OnePa
     constexpr int E = gen_E(C, (int)sizeof(T));
     cudaError_t e = onepass_reset(W, p.ntiles, st);
     if (e != cudaSuccess) return e;
+    profile_before(st);
     k_gen_onepass<T, NCOL, PHASED, E, GEN_NT><<<(unsigned)p.ntiles, GEN_NT, 0, st>>>(A, W, ia, p.ntiles);
+    profile_after(st);
     k_suffix_carries<T, C, 1024><<<1, 1024, 0, st>>>(W, p.ntiles);
     k_gen_fixup<T, NCOL, PHASED, GEN_NT><<<FIXUP_BLOCKS, GEN_NT, 0, st>>>(A, W, ia, p.tile);
     return cudaGetLastError();

@@ -15,6 +15,19 @@ constexpr size_t HEADER_BYTES = 256;
 // Sets the calling thread's message returned by laplex_last_error() (capi.cu).
 void set_last_error(const char* fmt, ...);
 
+// Optional events recorded around a call's dominant kernel (capi.cu, thread-local).
+struct ProfileEvents {
+    cudaEvent_t before;
+    cudaEvent_t after;
+};
+const ProfileEvents& profile_events();
+inline void profile_before(cudaStream_t st) {
+    if (profile_events().before) cudaEventRecord(profile_events().before, st);
+}
+inline void profile_after(cudaStream_t st) {
+    if (profile_events().after) cudaEventRecord(profile_events().after, st);
+}
+
 // Bump allocator over the caller's workspace (256-byte granules).
 struct Carve {
     char* base;

@@ -244,6 +244,174 @@ __device__ __forceinline__ void block_excl_bwd(const T f, const T (&W)[C], bool&
     for (int c = 0; c < C; ++c) tW[c] = sm.tV[c];
 }
 
+// Both exclusive scans of one channel set at once (forward prefix over lower
+// threads, backward suffix over higher threads), sharing two barriers.
+template <typename T, int C, int NT>
+struct BlockScan2Smem {
+    static constexpr int NW = NT / 32;
+    T fe[NW];
+    T fV[NW][C];
+    T be[NW];
+    T bV[NW][C];
+    T pfe[NW];
+    T pfV[NW][C];
+    T pbe[NW];
+    T pbV[NW][C];
+    T tfe, tbe;
+    T tfV[C], tbV[C];
+};
+
+template <typename T, int C, int NT, int CT = 0>
+__device__ __forceinline__ void block_excl_both(const T e, const T (&V)[C], const T f, const T (&W)[C],
+                                                bool& hasf, T& pe, T (&pV)[C], T& te, T (&tV)[C],
+                                                bool& hasb, T& nf, T (&nW)[C], T& tf, T (&tW)[C],
+                                                BlockScan2Smem<T, C, NT>& sm) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    T iV[C], iW[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        iV[c] = V[c];
+        iW[c] = W[c];
+    }
+    warp_incl_fwd<T, C, CT>(e, iV, lane);
+    warp_incl_bwd<T, C, CT>(f, iW, lane);
+    if (lane == 31) {
+        sm.fe[w] = e;
+#pragma unroll
+        for (int c = 0; c < C; ++c) sm.fV[w][c] = iV[c];
+    }
+    if (lane == 0) {
+        sm.be[w] = f;
+#pragma unroll
+        for (int c = 0; c < C; ++c) sm.bV[w][c] = iW[c];
+    }
+    __syncthreads();
+    if (w == 0) {
+        T ge = lane < NW ? sm.fe[lane] : T(0), gV[C];
+        T gf = lane < NW ? sm.be[lane] : T(0), gW[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            gV[c] = lane < NW ? sm.fV[lane][c] : T(0);
+            gW[c] = lane < NW ? sm.bV[lane][c] : T(0);
+        }
+#pragma unroll
+        for (int off = 1; off < NW; off <<= 1) {
+            const T eo = __shfl_up_sync(FULL, ge, off);
+            const T fo = __shfl_down_sync(FULL, gf, off);
+            T Vo[C], Wo[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                Vo[c] = __shfl_up_sync(FULL, gV[c], off);
+                Wo[c] = __shfl_down_sync(FULL, gW[c], off);
+            }
+            if (lane >= off && lane < NW) {
+                const Decay<T, C, CT> d(eo, ge);
+#pragma unroll
+                for (int c = 0; c < C; ++c) gV[c] = dfma<T>(d[c], Vo[c], gV[c]);
+            }
+            if (lane + off < NW) {
+                const Decay<T, C, CT> d(gf, fo);
+#pragma unroll
+                for (int c = 0; c < C; ++c) gW[c] = dfma<T>(d[c], Wo[c], gW[c]);
+            }
+        }
+        const T xe = __shfl_up_sync(FULL, ge, 1);
+        const T xf = __shfl_down_sync(FULL, gf, 1);
+        T xV[C], xW[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            xV[c] = __shfl_up_sync(FULL, gV[c], 1);
+            xW[c] = __shfl_down_sync(FULL, gW[c], 1);
+        }
+        if (lane > 0 && lane < NW) {
+            sm.pfe[lane] = xe;
+#pragma unroll
+            for (int c = 0; c < C; ++c) sm.pfV[lane][c] = xV[c];
+        }
+        if (lane < NW - 1) {
+            sm.pbe[lane] = xf;
+#pragma unroll
+            for (int c = 0; c < C; ++c) sm.pbV[lane][c] = xW[c];
+        }
+        if (lane == NW - 1) {
+            sm.tfe = ge;
+#pragma unroll
+            for (int c = 0; c < C; ++c) sm.tfV[c] = gV[c];
+        }
+        if (lane == 0) {
+            sm.tbe = gf;
+#pragma unroll
+            for (int c = 0; c < C; ++c) sm.tbV[c] = gW[c];
+        }
+    }
+    __syncthreads();
+    // forward: lanes below, then warps below
+    {
+        const T le = __shfl_up_sync(FULL, e, 1);
+        T lV[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) lV[c] = __shfl_up_sync(FULL, iV[c], 1);
+        if (w > 0 && lane > 0) {
+            hasf = true;
+            pe = le;
+            const Decay<T, C, CT> d(sm.pfe[w], le);
+#pragma unroll
+            for (int c = 0; c < C; ++c) pV[c] = dfma<T>(d[c], sm.pfV[w][c], lV[c]);
+        } else if (w > 0) {
+            hasf = true;
+            pe = sm.pfe[w];
+#pragma unroll
+            for (int c = 0; c < C; ++c) pV[c] = sm.pfV[w][c];
+        } else if (lane > 0) {
+            hasf = true;
+            pe = le;
+#pragma unroll
+            for (int c = 0; c < C; ++c) pV[c] = lV[c];
+        } else {
+            hasf = false;
+            pe = T(0);
+#pragma unroll
+            for (int c = 0; c < C; ++c) pV[c] = T(0);
+        }
+        te = sm.tfe;
+#pragma unroll
+        for (int c = 0; c < C; ++c) tV[c] = sm.tfV[c];
+    }
+    // backward: lanes above, then warps above
+    {
+        const T lf = __shfl_down_sync(FULL, f, 1);
+        T lW[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) lW[c] = __shfl_down_sync(FULL, iW[c], 1);
+        if (w < NW - 1 && lane < 31) {
+            hasb = true;
+            nf = lf;
+            const Decay<T, C, CT> d(lf, sm.pbe[w]);
+#pragma unroll
+            for (int c = 0; c < C; ++c) nW[c] = dfma<T>(d[c], sm.pbV[w][c], lW[c]);
+        } else if (w < NW - 1) {
+            hasb = true;
+            nf = sm.pbe[w];
+#pragma unroll
+            for (int c = 0; c < C; ++c) nW[c] = sm.pbV[w][c];
+        } else if (lane < 31) {
+            hasb = true;
+            nf = lf;
+#pragma unroll
+            for (int c = 0; c < C; ++c) nW[c] = lW[c];
+        } else {
+            hasb = false;
+            nf = T(0);
+#pragma unroll
+            for (int c = 0; c < C; ++c) nW[c] = T(0);
+        }
+        tf = sm.tbe;
+#pragma unroll
+        for (int c = 0; c < C; ++c) tW[c] = sm.tbV[c];
+    }
+}
+
 // ---------------------------------------------------------------- chunk level
 // A thread owns E consecutive elements: anchors s[E], values v[E][C].
 // dl[i] = exp(s[i-1] - s[i]) for i = 1..E-1 (dl[0] is set in chunk_final).

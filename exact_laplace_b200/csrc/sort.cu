@@ -294,6 +294,7 @@ cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws, 
     K* kout = reinterpret_cast<K*>(sorted);
     const K* ksrc = nullptr;
     const int32_t* vsrc = nullptr;
+    profile_before(st);
     for (int pass = 0; pass < P; ++pass) {
         const bool to_out = ((P - 1 - pass) % 2) == 0;
         K* kdst = to_out ? kout : kws;
@@ -306,6 +307,7 @@ cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws, 
         ksrc = kdst;
         vsrc = vdst;
     }
+    profile_after(st);
     return cudaSuccess;
 }
 

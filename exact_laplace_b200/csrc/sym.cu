@@ -7,14 +7,16 @@
 // recombines them with cos(phi_i) and sin(phi_i) (cos(p - q) = cos p cos q +
 // sin p sin q).  Each channel is the recurrence pair of scan_core.cuh.
 //
-// Three-phase reduce-then-scan over tiles of NT*E elements:
-//   1. k_sym_reduce   : per-tile forward/backward totals     (reads s, x)
-//   2. k_tile_carries : carries into every tile              (tiny)
-//   3. k_sym_final    : scans each tile again with its carries, writes y
+// Paths:
+//   * one column, x in sorted order or gathered through perm: sym_stream.cu;
+//   * several columns, phases or a scale: the wait-free three-kernel scheme of
+//     threepass.cuh with the SymTP policy below;
+//   * laplex_matvec_sym_noalloc: the three-phase reduce-then-scan below
+//     (k_sym_reduce, k_tile_carries, k_sym_final) with a fixed scratch array.
 #include <algorithm>
 
 #include "laplex_impl.h"
-#include "onepass.cuh"
+#include "threepass.cuh"
 
 namespace lx {
 
@@ -244,89 +246,42 @@ __global__ void __launch_bounds__(NT) k_sym_final(SymArgs<T> A, const T* __restr
 }
 
 
-// ------------------------------------------------------------------ single pass
-// One launch streams the input once and writes y once; carries between tiles
-// follow onepass.cuh (look-back for the prefix, bounded look-ahead for the
-// suffix, exact completion of deferred tiles by k_suffix_carries + k_sym_fixup).
-template <typename T, int NCOL, bool PHASED, int E, int NT>
-__global__ void __launch_bounds__(NT) k_sym_onepass(SymArgs<T> A, OnePassWs<T> W, int64_t ntiles) {
-    constexpr int C = PHASED ? 2 * NCOL : NCOL;
-    constexpr int64_t TILE = (int64_t)NT * E;
-    __shared__ BlockScanSmem<T, C, NT> smf, smb;
-    __shared__ int64_t sh_tile;
-    __shared__ T sh_e[2];
-    __shared__ T sh_c[2][C];
-    if (threadIdx.x == 0) sh_tile = (int64_t)atomicAdd(&W.ctrl[0], 1u);
-    __syncthreads();
-    const int64_t t = sh_tile;
-    const int64_t n = A.n;
-    const int64_t tile0 = t * TILE;
-    const int64_t r0 = tile0 + (int64_t)threadIdx.x * E;
-    T s[E], v[E][C], cph[E], sph[E], dl[E], fV[C], bW[C];
-    sym_load<T, NCOL, PHASED, E>(A, r0, s, v, cph, sph);
-    chunk_aggregates<T, C, E>(s, v, dl, fV, bW);
-    bool hf, hb;
-    T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
-    block_excl_fwd<T, C, NT>(s[E - 1], fV, hf, pe, pV, te, tV, smf);
-    block_excl_bwd<T, C, NT>(s[0], bW, hb, nf, nW, tf, tW, smb);
-    if (threadIdx.x == 0) {
-        const T eT = t == 0 ? A.s[0] : A.s[tile0 - 1];
-        const T fT = t == ntiles - 1 ? A.s[n - 1] : A.s[tile0 + TILE];
-        T acc[C], accb[C];
-        onepass_carries<T, C>(W, t, ntiles, tf, tW, te, tV, eT, fT, acc, accb, A.status);
-        sh_e[0] = eT;
-        sh_e[1] = fT;
-#pragma unroll
-        for (int c = 0; c < C; ++c) {
-            sh_c[0][c] = acc[c];
-            sh_c[1][c] = accb[c];
+// ------------------------------------------------------------------ wait-free path
+// Policy of threepass.cuh for the symmetric/phased product with B columns,
+// an optional scale D and gather/scatter through perm (sym_load/sym_store).
+template <typename T_, int NCOL_, bool PHASED_, int E_, int NT_>
+struct SymTP {
+    using T = T_;
+    static constexpr int NCOL = NCOL_, C = PHASED_ ? 2 * NCOL_ : NCOL_, CT = 0, E = E_, NT = NT_;
+    SymArgs<T> A;
+    int64_t n;
+    const T* s;
+    struct Aux {
+        T cph[E], sph[E];
+    };
+    __device__ __forceinline__ void load(int64_t r0, T (&sv)[E], T (&v)[E][C], Aux& a) const {
+        sym_load<T, NCOL, PHASED_, E>(A, r0, sv, v, a.cph, a.sph);
+    }
+    __device__ __forceinline__ void finish(int64_t r0, const T (&sv)[E], const T (&v)[E][C],
+                                           T (&dl)[E], T eprev, const T (&Lp)[C], T enext,
+                                           const T (&Un)[C], Aux& a) const {
+        T out[E][C];
+        chunk_final<T, C, E>(sv, v, dl, eprev, Lp, enext, Un, out);
+        sym_store<T, NCOL, PHASED_, E>(A, r0, out, a.cph, a.sph);
+    }
+    __device__ __forceinline__ void carry_in(int64_t r, T fe, T, const T* c, bool) const {
+        const int64_t row = A.pout ? (int64_t)A.pout[r] : r;
+        T* yr = A.y + row * A.ldy + A.col0;
+        if (PHASED_) {
+            const int64_t ar = A.paux ? (int64_t)A.paux[r] : r;
+            T sp, cp;
+            dsincos<T>(A.phi[ar], &sp, &cp);
+            for (int k = 0; k < A.ncol; ++k) yr[k] += fe * (cp * c[2 * k] + sp * c[2 * k + 1]);
+        } else {
+            for (int k = 0; k < A.ncol; ++k) yr[k] += fe * c[k];
         }
     }
-    __syncthreads();
-    T VT[C], WT[C];
-#pragma unroll
-    for (int c = 0; c < C; ++c) {
-        VT[c] = sh_c[0][c];
-        WT[c] = sh_c[1][c];
-    }
-    T eprev, Lprev[C], enext, Unext[C], out[E][C];
-    apply_carry_fwd<T, C>(hf, pe, pV, sh_e[0], VT, eprev, Lprev);
-    apply_carry_bwd<T, C>(hb, nf, nW, sh_e[1], WT, enext, Unext);
-    chunk_final<T, C, E>(s, v, dl, eprev, Lprev, enext, Unext, out);
-    sym_store<T, NCOL, PHASED, E>(A, r0, out, cph, sph);
-}
-
-// Adds the suffix carry to the tiles k_sym_onepass marked (exits at once when
-// none is marked).  y_r += exp(s_r - s_end) * carB[t] (phased: recombined).
-template <typename T, int NCOL, bool PHASED, int NT>
-__global__ void __launch_bounds__(NT) k_sym_fixup(SymArgs<T> A, OnePassWs<T> W, int64_t tile) {
-    constexpr int C = PHASED ? 2 * NCOL : NCOL;
-    const uint32_t nfix = W.ctrl[1];
-    for (uint32_t q = blockIdx.x; q < nfix; q += gridDim.x) {
-        const int64_t t = W.fix[q];
-        const int64_t n = A.n;
-        const int64_t b = t * tile, e = min(b + tile, n);
-        if (e >= n) continue;
-        const T fT = A.s[e];
-        T cr[C];
-#pragma unroll
-        for (int c = 0; c < C; ++c) cr[c] = W.carB[t * C + c];
-        for (int64_t r = b + threadIdx.x; r < e; r += NT) {
-            const T f = dexp<T>(A.s[r] - fT);
-            if (f == T(0)) continue;
-            const int64_t row = A.pout ? (int64_t)A.pout[r] : r;
-            T* yr = A.y + row * A.ldy + A.col0;
-            if (PHASED) {
-                const int64_t ar = A.paux ? (int64_t)A.paux[r] : r;
-                T sp, cp;
-                dsincos<T>(A.phi[ar], &sp, &cp);
-                for (int c = 0; c < A.ncol; ++c) yr[c] += f * (cp * cr[2 * c] + sp * cr[2 * c + 1]);
-            } else {
-                for (int c = 0; c < A.ncol; ++c) yr[c] += f * cr[c];
-            }
-        }
-    }
-}
+};
 
 // ------------------------------------------------------------------ host side
 struct SymPlan {
@@ -356,7 +311,7 @@ static SymPlan sym_plan(int64_t n, int64_t B, bool phased, int f64) {
 
 size_t sym_ws_bytes(int64_t n, int64_t B, bool phased, int f64) {
     const SymPlan p = sym_plan(n, B, phased, f64);
-    const size_t a = onepass_ws_bytes(p.ntiles, p.C, f64 ? 8 : 4);
+    const size_t a = tp_ws_bytes(p.ntiles, p.C, f64 ? 8 : 4);
     const size_t b = (!phased && B == 1) ? stream_ws_bytes(n, f64) : 0;
     return a > b ? a : b;
 }
@@ -372,47 +327,37 @@ static cudaError_t sym_launch(const SymArgs<T>& A, int64_t ntiles, T* aggF, T* a
     return cudaGetLastError();
 }
 
-template <typename T, int NCOL, bool PHASED, int E>
-static cudaError_t onepass_launch(const SymArgs<T>& A, int64_t ntiles, const OnePassWs<T>& W,
-                                  cudaStream_t st) {
-    constexpr int C = PHASED ? 2 * NCOL : NCOL;
-    constexpr int64_t TILE = (int64_t)SYM_NT * E;
-    cudaError_t e = onepass_reset(W, ntiles, st);
-    if (e != cudaSuccess) return e;
-    k_sym_onepass<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, W, ntiles);
-    k_suffix_carries<T, C, 1024><<<1, 1024, 0, st>>>(W, ntiles);
-    k_sym_fixup<T, NCOL, PHASED, SYM_NT><<<FIXUP_BLOCKS, SYM_NT, 0, st>>>(A, W, TILE);
-    return cudaGetLastError();
-}
-
 template <typename T>
 cudaError_t sym_run(SymArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_bytes,
                     cudaStream_t st) {
     if (A.n == 0) return cudaSuccess;
-    // contiguous single-column input (pre-sorted product): the streaming kernel
-    if (!phased && B == 1 && A.pin == nullptr && A.D == nullptr && A.ldx == 1 && A.ldy == 1)
+    // single-column input in sorted order, or gathered through perm: the wait-free kernels
+    if (!phased && B == 1 && A.pin == A.pout && A.D == nullptr && A.ldx == 1 && A.ldy == 1)
         return stream_run<T>(A.s, A.x, A.y, A.pout, A.n, ws, ws_bytes, A.status, st);
     const SymPlan p = sym_plan(A.n, B, phased, sizeof(T) == 8);
-    Carve cv(ws, ws_bytes);
-    OnePassWs<T> W = onepass_carve<T>(cv, p.ntiles, p.C);
-    if (!cv.ok) return cudaErrorInvalidValue;
     for (int64_t g = 0; g < p.groups; ++g) {
         A.col0 = g * p.ncol;
         A.ncol = (int)std::min<int64_t>(p.ncol, B - A.col0);
         cudaError_t e;
         constexpr bool D = sizeof(T) == 8;
+        auto run = [&](auto pol) {
+            pol.A = A;
+            pol.n = A.n;
+            pol.s = A.s;
+            return tp_run(pol, ws, ws_bytes, st);
+        };
         if (!phased) {
             switch (p.ncol) {
-                case 1: e = onepass_launch<T, 1, false, D ? 8 : 16>(A, p.ntiles, W, st); break;
-                case 2: e = onepass_launch<T, 2, false, 8>(A, p.ntiles, W, st); break;
-                case 4: e = onepass_launch<T, 4, false, 4>(A, p.ntiles, W, st); break;
-                default: e = onepass_launch<T, 8, false, 4>(A, p.ntiles, W, st); break;
+                case 1: e = run(SymTP<T, 1, false, D ? 8 : 16, SYM_NT>{}); break;
+                case 2: e = run(SymTP<T, 2, false, 8, SYM_NT>{}); break;
+                case 4: e = run(SymTP<T, 4, false, 4, SYM_NT>{}); break;
+                default: e = run(SymTP<T, 8, false, 4, SYM_NT>{}); break;
             }
         } else {
             switch (p.ncol) {
-                case 1: e = onepass_launch<T, 1, true, 8>(A, p.ntiles, W, st); break;
-                case 2: e = onepass_launch<T, 2, true, 4>(A, p.ntiles, W, st); break;
-                default: e = onepass_launch<T, 4, true, 4>(A, p.ntiles, W, st); break;
+                case 1: e = run(SymTP<T, 1, true, 8, SYM_NT>{}); break;
+                case 2: e = run(SymTP<T, 2, true, 4, SYM_NT>{}); break;
+                default: e = run(SymTP<T, 4, true, 4, SYM_NT>{}); break;
             }
         }
         if (e != cudaSuccess) return e;

@@ -62,6 +62,7 @@ SIGNATURES = {
     "laplex_backward": ([_P, _P, _I64, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P],
                         ctypes.c_int),
     "laplex_matvec_sym_noalloc": ([_P, _P, _I64, _P, _P, _P], ctypes.c_int),
+    "laplex_set_profile_events": ([_P, _P], ctypes.c_int),
 }
 
 
@@ -167,6 +168,14 @@ def _ws(op, n, k, B, dtype, device):
     nb = workspace_size(op, n, k, B, dtype)
     buf = Workspace.get(device, nb)
     return buf, buf.numel()
+
+
+def set_profile_events(before=None, after=None) -> None:
+    """Record two torch.cuda.Event objects around the dominant kernel of the
+    following calls on this thread (both recorded once first, so that their CUDA
+    events exist); None, None switches it off."""
+    h = [None if e is None else ctypes.c_void_p(e.cuda_event) for e in (before, after)]
+    _check(lib().laplex_set_profile_events(h[0], h[1]))
 
 
 def device_status(device=None) -> None:

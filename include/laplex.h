@@ -181,6 +181,17 @@ laplex_status laplex_backward(const void* sorted, const int32_t* perm, int64_t n
                               laplex_dtype dtype, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Profiling hook (no counterpart in the paper): for the following calls on the
+ * calling thread, record the CUDA events `before` and `after` (cudaEvent_t
+ * passed as void*, created by the caller) on the call's stream immediately
+ * before and after the call's dominant kernel: the tile-local scan of the
+ * symmetric product and of the backward pass, the four digit passes of the
+ * sort, the merged scan of the general product.  NULL, NULL switches it off.
+ * Host-only bookkeeping; no synchronisation.  Returns LAPLEX_OK.
+ */
+laplex_status laplex_set_profile_events(void* before, void* after);
+
+/*
  * Allocation-free symmetric product, y = K x (fp32, B = 1).  The paper has no
  * counterpart: this entry point exists for callers that cannot allocate device
  * memory -- code running where cudaMalloc is unavailable or forbidden (inside

@@ -52,6 +52,7 @@ def test_ties(dtype):
     check((64.0 * np.round(rng.uniform(0, 2000, n))).astype(dtype), x, g, dtype, "64-apart groups")
     check(np.full(n, 2.0, dtype=dtype), x, g, dtype, "all equal")
     check(rng.uniform(0, 1, n).astype(dtype), x, g, dtype, "dense")
+    check((np.arange(n) * 200.0).astype(dtype), x, g, dtype, "far apart")
 
 
 @pytest.mark.parametrize("dtype", [np.float32, np.float64])
