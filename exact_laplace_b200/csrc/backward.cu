@@ -28,6 +28,11 @@ template <typename T_, int E_>
 struct BwdTP {
     using T = T_;
     static constexpr int C = 4, CT = 2, E = E_, NT = BWD_NT;
+    // halos of 128 (fp32: they span CUT = 104 at spacings above 0.82; fp64,
+    // CUT = 746, would need several times more: none).  Streamed pass 1
+    // (inputs in sorted order): s, x, g in a 2-stage ring.
+    static constexpr int H = sizeof(T_) == 4 ? 128 : 0;
+    static constexpr int NIN = 2, S = 2, MINB = 2;
     int64_t n;
     const T* s;
     const int32_t* perm;
@@ -69,6 +74,13 @@ struct BwdTP {
             v[i][2] = xv[i];
             v[i][3] = gv[i];
         }
+    }
+    __device__ __forceinline__ const T* ring_in(int a) const { return a == 0 ? x : g; }
+    __device__ __forceinline__ void value(const T (&xe)[NIN], T (&vv)[C]) const {
+        vv[0] = xe[0];
+        vv[1] = xe[1];
+        vv[2] = xe[0];
+        vv[3] = xe[1];
     }
     __device__ __forceinline__ void finish(int64_t r0, const T (&sv)[E], const T (&v)[E][C],
                                            T (&dl)[E], T eprev, const T (&Lp)[C], T enext,
@@ -127,17 +139,11 @@ struct BwdTP {
             }
         }
     }
-    // A carry c = (L^x, L^g, P^x, P^g) from the left or (U^x, U^g, Q^x, Q^g)
-    // from the right, with exp factor fe and tie factor ft at element r.
-    __device__ __forceinline__ void carry_in(int64_t r, T fe, T ft, const T* c, bool left) const {
-        const int64_t row = perm ? (int64_t)perm[r] : r;
-        const T xr = x[row], gr = g[row];
-        const T dDx = fe * c[0] - ft * c[2];  // change of the strictly-lower (left) or -upper sum
-        const T dDg = fe * c[1] - ft * c[3];
-        dx[row] += fe * c[1];
-        // D(v) = lower - upper: a left carry adds to it, a right carry subtracts
-        if (left) da[row] -= gr * dDx + xr * dDg;
-        else da[row] += gr * dDx + xr * dDg;
+    __device__ __forceinline__ void load1(int64_t j, T& sj, T (&vv)[C]) const {
+        sj = s[j];
+        const int64_t row = perm ? (int64_t)perm[j] : j;
+        const T xe[NIN] = {x[row], g[row]};
+        value(xe, vv);
     }
 };
 
@@ -152,7 +158,6 @@ size_t bwd_ws_bytes(int64_t n, int f64) {
 template <typename T>
 cudaError_t bwd_run(const T* s, const int32_t* perm, int64_t n, const T* x, const T* g, T* dx,
                     T* da, void* ws, size_t ws_bytes, uint32_t* status, cudaStream_t st) {
-    (void)status;  // no inter-block waits
     if (n == 0) return cudaSuccess;
     BwdTP<T, bwd_E((int)sizeof(T))> p;
     p.n = n;
@@ -162,6 +167,7 @@ cudaError_t bwd_run(const T* s, const int32_t* perm, int64_t n, const T* x, cons
     p.g = g;
     p.dx = dx;
     p.da = da;
+    if (perm == nullptr) return tp_run_ring(p, ws, ws_bytes, status, st);
     return tp_run(p, ws, ws_bytes, st);
 }
 

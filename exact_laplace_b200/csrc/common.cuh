@@ -21,31 +21,6 @@ __device__ __forceinline__ void set_status(uint32_t* st, uint32_t bits) {
     if (st) atomicOr(st, bits);
 }
 
-// Inter-block flags: a release store publishes this thread's earlier writes; an
-// acquire load makes them visible to the reader's later loads (read the payload
-// with __ldcg, i.e. from L2, never from a possibly stale L1 line).
-__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Bounded spin until *p >= want.  Returns the flag, or 0 after `limit` polls
-// (the caller decides whether that is an error or a fallback).
-__device__ __forceinline__ uint32_t wait_flag(const uint32_t* p, uint32_t want, uint32_t limit) {
-    uint32_t v = ld_acquire(p);
-    uint32_t it = 0;
-    while (v < want) {
-        if (++it > limit) return 0u;
-        __nanosleep(32);
-        v = ld_acquire(p);
-    }
-    return v;
-}
-
 // 16-byte vector type for T
 template <typename T> struct V16;
 template <> struct V16<float> { using type = float4; static constexpr int N = 4; };

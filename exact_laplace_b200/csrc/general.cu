@@ -13,14 +13,16 @@
 // sits either before or after it, so every pair is counted once; equal anchors
 // weigh exp(0) = 1 on either side).  Merge order: a_i before b_j iff a_i < b_j.
 //
-// Kernels: k_merge_partition (merge-path split of the merged sequence into
-// tiles), k_gen_onepass (single pass, onepass.cuh carries), k_suffix_carries +
-// k_gen_fixup (only for tiles whose look-ahead was deferred).  K^T is the same
-// product with the roles of a and b exchanged (done by the caller).
+// Kernels (the wait-free scheme of threepass.cuh on the merged sequence):
+// k_merge_partition (merge-path split into tiles), k_gen_local (tile-local
+// scan, outputs at the a-points), k_tp_carry_blocks + k_tp_carry_tiles (exact
+// tile carries), k_gen_headtail (carries added to the a-points of each tile's
+// head and tail reach).  K^T is the same product with the roles of a and b
+// exchanged (done by the caller).
 #include <algorithm>
 
 #include "laplex_impl.h"
-#include "onepass.cuh"
+#include "threepass.cuh"
 
 namespace lx {
 
@@ -46,20 +48,19 @@ __global__ void k_merge_partition(const T* __restrict__ a, int64_t n, const T* _
     ia[t] = lo;
 }
 
+// Tile-local scan of the merged sequence with zero carries from outside the
+// tile (threepass.cuh pass 1 for the merged case).  Outputs go to the
+// a-points; the tile's totals and its reach in a-points (a-points within CUT
+// of the tile's first / last merged anchor) go to the workspace.
 template <typename T, int NCOL, bool PHASED, int E, int NT>
-__global__ void __launch_bounds__(NT) k_gen_onepass(GenArgs<T> A, OnePassWs<T> W,
-                                                    const int64_t* __restrict__ ia, int64_t ntiles) {
+__global__ void __launch_bounds__(NT) k_gen_local(GenArgs<T> A, TPWs<T, PHASED ? 2 * NCOL : NCOL> W,
+                                                  const int64_t* __restrict__ ia) {
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
     constexpr int TILE = NT * E;
-    __shared__ T sh_anc[TILE];          // a-part [0, na), b-part [na, na + nb)
-    __shared__ T sh_val[TILE * C];      // channel values of the b-part
-    __shared__ BlockScanSmem<T, C, NT> smf, smb;
-    __shared__ int64_t sh_tile;
-    __shared__ T sh_e[2];
-    __shared__ T sh_c[2][C];
-    if (threadIdx.x == 0) sh_tile = (int64_t)atomicAdd(&W.ctrl[0], 1u);
-    __syncthreads();
-    const int64_t t = sh_tile;
+    __shared__ T sh_anc[TILE];      // a-part [0, na), b-part [na, na + nb)
+    __shared__ T sh_val[TILE * C];  // channel values of the b-part
+    __shared__ BlockScan2Smem<T, C, NT> sm2;
+    const int64_t t = blockIdx.x;
     const int64_t n = A.n, k = A.k, N = n + k;
     const int64_t p0 = t * TILE, p1 = min(p0 + TILE, N);
     const int64_t i0 = ia[t], i1 = ia[t + 1];
@@ -88,7 +89,8 @@ __global__ void __launch_bounds__(NT) k_gen_onepass(GenArgs<T> A, OnePassWs<T> W
     __syncthreads();
     const T* Aa = sh_anc;
     const T* Bb = sh_anc + na;
-    // this thread's merged range [d0, d0 + E) within the tile: merge-path search
+    const T first = na > 0 && (nb == 0 || Aa[0] <= Bb[0]) ? Aa[0] : Bb[0];
+    const T padA = na > 0 && (nb == 0 || Aa[na - 1] >= Bb[nb - 1]) ? Aa[na - 1] : Bb[nb - 1];
     const int d0 = min((int)threadIdx.x * E, cnt);
     int lo = max(0, d0 - nb), hi = min(d0, na);
     while (lo < hi) {
@@ -97,10 +99,9 @@ __global__ void __launch_bounds__(NT) k_gen_onepass(GenArgs<T> A, OnePassWs<T> W
         else hi = mid;
     }
     int ai = lo, bi = d0 - lo;
-    const T padA = cnt > 0 ? (na > 0 && (nb == 0 || Aa[na - 1] >= Bb[nb - 1]) ? Aa[na - 1] : Bb[nb - 1])
-                           : T(0);
     T s[E], v[E][C], dl[E], fV[C], bW[C];
-    int aidx[E];  // local a index for a-points, -1 otherwise
+    int aidx[E];
+    int h = 0, q = 0;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const bool valid = d0 + e < cnt;
@@ -113,6 +114,8 @@ __global__ void __launch_bounds__(NT) k_gen_onepass(GenArgs<T> A, OnePassWs<T> W
         } else if (takeA) {
             s[e] = Aa[ai];
             aidx[e] = ai;
+            h += (Aa[ai] - first < TPCut<T>::v) ? 1 : 0;
+            q += (padA - Aa[ai] < TPCut<T>::v) ? 1 : 0;
             ++ai;
 #pragma unroll
             for (int c = 0; c < C; ++c) v[e][c] = T(0);
@@ -127,41 +130,28 @@ __global__ void __launch_bounds__(NT) k_gen_onepass(GenArgs<T> A, OnePassWs<T> W
     chunk_aggregates<T, C, E>(s, v, dl, fV, bW);
     bool hf, hb;
     T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
-    block_excl_fwd<T, C, NT>(s[E - 1], fV, hf, pe, pV, te, tV, smf);
-    block_excl_bwd<T, C, NT>(s[0], bW, hb, nf, nW, tf, tW, smb);
+    const int hq[2] = {h, q};
+    int reach[2];
+    (void)block_excl_both_counted<T, C, NT, 0, true>(s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf,
+                                                     nW, tf, tW, hq, reach, false, sm2);
     if (threadIdx.x == 0) {
-        // anchors of the merged elements just before and just after this tile
-        T eT = padA, fT = padA;
-        if (p0 > 0) {
-            if (i0 > 0 && j0 > 0) eT = max(A.sa[i0 - 1], A.sb[j0 - 1]);
-            else eT = i0 > 0 ? A.sa[i0 - 1] : A.sb[j0 - 1];
-        } else if (cnt > 0) {
-            eT = s[0];
-        }
-        if (p1 < N) {
-            if (i1 < n && j1 < k) fT = min(A.sa[i1], A.sb[j1]);
-            else fT = i1 < n ? A.sa[i1] : A.sb[j1];
-        }
-        T acc[C], accb[C];
-        onepass_carries<T, C>(W, t, ntiles, tf, tW, te, tV, eT, fT, acc, accb, A.status);
-        sh_e[0] = eT;
-        sh_e[1] = fT;
+        W.tfirst[t] = tf;
+        W.tlast[t] = te;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            sh_c[0][c] = acc[c];
-            sh_c[1][c] = accb[c];
+            W.fagg[t * C + c] = tV[c];
+            W.bagg[t * C + c] = tW[c];
         }
+        W.st[t].head = reach[0];
+        W.st[t].tail = reach[1];
     }
-    __syncthreads();
-    T VT[C], WT[C];
+    T eprev = hf ? pe : s[0], enext = hb ? nf : s[E - 1];
+    T Lprev[C], Unext[C], out[E][C];
 #pragma unroll
     for (int c = 0; c < C; ++c) {
-        VT[c] = sh_c[0][c];
-        WT[c] = sh_c[1][c];
+        Lprev[c] = hf ? pV[c] : T(0);
+        Unext[c] = hb ? nW[c] : T(0);
     }
-    T eprev, Lprev[C], enext, Unext[C], out[E][C];
-    apply_carry_fwd<T, C>(hf, pe, pV, sh_e[0], VT, eprev, Lprev);
-    apply_carry_bwd<T, C>(hb, nf, nW, sh_e[1], WT, enext, Unext);
     chunk_final<T, C, E>(s, v, dl, eprev, Lprev, enext, Unext, out);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -183,36 +173,55 @@ __global__ void __launch_bounds__(NT) k_gen_onepass(GenArgs<T> A, OnePassWs<T> W
     }
 }
 
-// y_i += exp(a_i - fT) * carB[t] for the a-points of each deferred tile.
-template <typename T, int NCOL, bool PHASED, int NT>
-__global__ void __launch_bounds__(NT) k_gen_fixup(GenArgs<T> A, OnePassWs<T> W,
-                                                  const int64_t* __restrict__ ia, int64_t tile) {
+// Carries into the a-points of each tile's head and tail reach (a warp per tile).
+template <typename T, int NCOL, bool PHASED>
+__global__ void __launch_bounds__(256) k_gen_headtail(GenArgs<T> A, TPWs<T, PHASED ? 2 * NCOL : NCOL> W,
+                                                      const int64_t* __restrict__ ia, int64_t tile,
+                                                      int64_t ntiles) {
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
-    const uint32_t nfix = W.ctrl[1];
-    for (uint32_t q = blockIdx.x; q < nfix; q += gridDim.x) {
-        const int64_t t = W.fix[q];
-        const int64_t n = A.n, k = A.k, N = n + k;
-        const int64_t p1 = min((t + 1) * tile, N);
-        if (p1 >= N) continue;
-        const int64_t i0 = ia[t], i1 = ia[t + 1], j1 = p1 - i1;
-        T fT;
-        if (i1 < n && j1 < k) fT = min(A.sa[i1], A.sb[j1]);
-        else fT = i1 < n ? A.sa[i1] : A.sb[j1];
-        T cr[C];
+    const int lane = threadIdx.x & 31;
+    const int64_t n = A.n, k = A.k, N = n + k;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < ntiles;
+         t += warps) {
+        const int64_t p0 = t * tile, p1 = min(p0 + tile, N);
+        const int64_t i0 = ia[t], i1 = ia[t + 1], j0 = p0 - i0, j1 = p1 - i1;
+        const TPStats stt = W.st[t];
+        for (int side = 0; side < 2; ++side) {
+            const bool left = side == 0;
+            if (left ? t == 0 : t == ntiles - 1) continue;
+            T c[C];
+            bool nz = false;
 #pragma unroll
-        for (int c = 0; c < C; ++c) cr[c] = W.carB[t * C + c];
-        for (int64_t i = i0 + threadIdx.x; i < i1; i += NT) {
-            const T f = dexp<T>(A.sa[i] - fT);
-            if (f == T(0)) continue;
-            const int64_t row = A.pout ? (int64_t)A.pout[i] : i;
-            T* yr = A.y + row * A.ldy + A.col0;
-            if (PHASED) {
-                T sp, cp;
-                gsincos<T>(A.phi[A.pphi ? (int64_t)A.pphi[i] : i], &sp, &cp);
-                for (int c = 0; c < A.ncol; ++c) yr[c] += f * (cp * cr[2 * c] + sp * cr[2 * c + 1]);
-            } else {
-                for (int c = 0; c < A.ncol; ++c) yr[c] += f * cr[c];
+            for (int q = 0; q < C; ++q) {
+                c[q] = (left ? W.carF : W.carB)[t * C + q];
+                nz |= c[q] != T(0);
             }
+            if (!nz) continue;
+            T edge;  // merged anchor just before (left) or just after (right) the tile
+            if (left) {
+                if (i0 > 0 && j0 > 0) edge = max(A.sa[i0 - 1], A.sb[j0 - 1]);
+                else edge = i0 > 0 ? A.sa[i0 - 1] : A.sb[j0 - 1];
+            } else {
+                if (i1 < n && j1 < k) edge = min(A.sa[i1], A.sb[j1]);
+                else edge = i1 < n ? A.sa[i1] : A.sb[j1];
+            }
+            const int64_t len = left ? stt.head : stt.tail;
+            for (int64_t q = lane; q < len; q += 32) {
+                const int64_t i = left ? i0 + q : i1 - 1 - q;
+                const T f = dexp<T>(left ? edge - A.sa[i] : A.sa[i] - edge);
+                if (f == T(0)) continue;
+                const int64_t row = A.pout ? (int64_t)A.pout[i] : i;
+                T* yr = A.y + row * A.ldy + A.col0;
+                if (PHASED) {
+                    T sp, cp;
+                    gsincos<T>(A.phi[A.pphi ? (int64_t)A.pphi[i] : i], &sp, &cp);
+                    for (int q2 = 0; q2 < A.ncol; ++q2) yr[q2] += f * (cp * c[2 * q2] + sp * c[2 * q2 + 1]);
+                } else {
+                    for (int q2 = 0; q2 < A.ncol; ++q2) yr[q2] += f * c[q2];
+                }
+            }
+            __syncwarp();
         }
     }
 }
@@ -242,21 +251,26 @@ static GenPlan gen_plan(int64_t n, int64_t k, int64_t B, bool phased, int es) {
 
 size_t gen_ws_bytes(int64_t n, int64_t k, int64_t B, bool phased, int f64) {
     const GenPlan p = gen_plan(n, k, B, phased, f64 ? 8 : 4);
-    return Carve::need((size_t)(p.ntiles + 1), 8) + onepass_ws_bytes(p.ntiles, p.C, f64 ? 8 : 4);
+    return Carve::need((size_t)(p.ntiles + 1), 8) + tp_ws_bytes(p.ntiles, p.C, f64 ? 8 : 4);
 }
 
 template <typename T, int NCOL, bool PHASED>
-static cudaError_t gen_launch(const GenArgs<T>& A, const GenPlan& p, const OnePassWs<T>& W,
+static cudaError_t gen_launch(const GenArgs<T>& A, const GenPlan& p, void* wsbody, size_t wsb,
                               const int64_t* ia, cudaStream_t st) {
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
     constexpr int E = gen_E(C, (int)sizeof(T));
-    cudaError_t e = onepass_reset(W, p.ntiles, st);
-    if (e != cudaSuccess) return e;
+    Carve cv(wsbody, wsb);
+    TPWs<T, C> W = tp_carve<T, C>(cv, p.ntiles);
+    if (!cv.ok) return cudaErrorInvalidValue;
+    W.redo_count = nullptr;  // every tile takes the carries (reach read-modify-write)
+    const int64_t nb = (p.ntiles + TP_CARRY_BT - 1) / TP_CARRY_BT;
     profile_before(st);
-    k_gen_onepass<T, NCOL, PHASED, E, GEN_NT><<<(unsigned)p.ntiles, GEN_NT, 0, st>>>(A, W, ia, p.ntiles);
+    k_gen_local<T, NCOL, PHASED, E, GEN_NT><<<(unsigned)p.ntiles, GEN_NT, 0, st>>>(A, W, ia);
     profile_after(st);
-    k_suffix_carries<T, C, 1024><<<1, 1024, 0, st>>>(W, p.ntiles);
-    k_gen_fixup<T, NCOL, PHASED, GEN_NT><<<FIXUP_BLOCKS, GEN_NT, 0, st>>>(A, W, ia, p.tile);
+    k_tp_carry_blocks<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, p.ntiles);
+    k_tp_carry_tiles<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, p.ntiles, nb);
+    const int64_t htb = std::max<int64_t>(1, std::min<int64_t>((p.ntiles + 7) / 8, 148 * 8));
+    k_gen_headtail<T, NCOL, PHASED><<<(unsigned)htb, 256, 0, st>>>(A, W, ia, p.tile, p.ntiles);
     return cudaGetLastError();
 }
 
@@ -269,8 +283,9 @@ cudaError_t gen_run(GenArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_by
     const GenPlan p = gen_plan(A.n, A.k, B, phased, (int)sizeof(T));
     Carve cv(ws, ws_bytes);
     int64_t* ia = cv.take<int64_t>(p.ntiles + 1);
-    OnePassWs<T> W = onepass_carve<T>(cv, p.ntiles, p.C);
     if (!cv.ok) return cudaErrorInvalidValue;
+    void* wsbody = cv.base + cv.off;
+    const size_t wsb = cv.cap - cv.off;
     {
         const unsigned blocks = (unsigned)((p.ntiles + 1 + 255) / 256);
         k_merge_partition<T><<<blocks, 256, 0, st>>>(A.sa, A.n, A.sb, A.k, p.tile, p.ntiles, ia);
@@ -281,16 +296,16 @@ cudaError_t gen_run(GenArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_by
         cudaError_t e;
         if (!phased) {
             switch (p.ncol) {
-                case 1: e = gen_launch<T, 1, false>(A, p, W, ia, st); break;
-                case 2: e = gen_launch<T, 2, false>(A, p, W, ia, st); break;
-                case 4: e = gen_launch<T, 4, false>(A, p, W, ia, st); break;
-                default: e = gen_launch<T, 8, false>(A, p, W, ia, st); break;
+                case 1: e = gen_launch<T, 1, false>(A, p, wsbody, wsb, ia, st); break;
+                case 2: e = gen_launch<T, 2, false>(A, p, wsbody, wsb, ia, st); break;
+                case 4: e = gen_launch<T, 4, false>(A, p, wsbody, wsb, ia, st); break;
+                default: e = gen_launch<T, 8, false>(A, p, wsbody, wsb, ia, st); break;
             }
         } else {
             switch (p.ncol) {
-                case 1: e = gen_launch<T, 1, true>(A, p, W, ia, st); break;
-                case 2: e = gen_launch<T, 2, true>(A, p, W, ia, st); break;
-                default: e = gen_launch<T, 4, true>(A, p, W, ia, st); break;
+                case 1: e = gen_launch<T, 1, true>(A, p, wsbody, wsb, ia, st); break;
+                case 2: e = gen_launch<T, 2, true>(A, p, wsbody, wsb, ia, st); break;
+                default: e = gen_launch<T, 4, true>(A, p, wsbody, wsb, ia, st); break;
             }
         }
         if (e != cudaSuccess) return e;

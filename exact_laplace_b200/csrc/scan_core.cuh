@@ -259,14 +259,28 @@ struct BlockScan2Smem {
     T pbV[NW][C];
     T tfe, tbe;
     T tfV[C], tbV[C];
+    int wcnt[NW][4];  // per-warp sums of integer counts (block_excl_both_counted)
+    int tcnt[4];
+    T whs[NW][C];     // per-warp halo sums (one per channel), and their two totals
+    T thL[C], thU[C];
 };
 
-template <typename T, int C, int NT, int CT = 0>
-__device__ __forceinline__ void block_excl_both(const T e, const T (&V)[C], const T f, const T (&W)[C],
-                                                bool& hasf, T& pe, T (&pV)[C], T& te, T (&tV)[C],
-                                                bool& hasb, T& nf, T (&nW)[C], T& tf, T (&tW)[C],
-                                                BlockScan2Smem<T, C, NT>& sm) {
+// block_excl_both_counted: the two scans; it also sums NI <= 4 integer counts
+// over the block (cnt in, tot out, read by every thread) and ORs a flag: if any
+// thread passes bad, the function returns true right after its first barrier,
+// in every thread, with the outputs unset.  COUNTED = false drops the counts
+// and the flag.  HW > 0 also sums HC <= C values hv per thread into two
+// totals: warps [0, HW) into hL, warps [HW, 2 HW) into hU (other warps pass 0).
+template <typename T, int C, int NT, int CT, bool COUNTED, int NI = 2, int HW = 0, int HC = 1>
+__device__ __forceinline__ bool block_excl_both_counted(
+    const T e, const T (&V)[C], const T f, const T (&W)[C], bool& hasf, T& pe, T (&pV)[C], T& te,
+    T (&tV)[C], bool& hasb, T& nf, T (&nW)[C], T& tf, T (&tW)[C], const int (&cnt)[NI], int (&tot)[NI],
+    const bool bad, BlockScan2Smem<T, C, NT>& sm, const T* hv = nullptr, T* hL = nullptr, T* hU = nullptr) {
     constexpr int NW = NT / 32;
+    static_assert(NW <= 32, "one warp scans the warp totals");
+    static_assert(NI >= 1 && NI <= 4, "at most four counts");
+    static_assert(2 * HW <= NW && (HW & (HW - 1)) == 0, "halo warps: a power of two per side");
+    static_assert(HC >= 1 && HC <= C, "halo channels");
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     T iV[C], iW[C];
 #pragma unroll
@@ -281,13 +295,52 @@ __device__ __forceinline__ void block_excl_both(const T e, const T (&V)[C], cons
 #pragma unroll
         for (int c = 0; c < C; ++c) sm.fV[w][c] = iV[c];
     }
+    if (COUNTED) {
+#pragma unroll
+        for (int q = 0; q < NI; ++q) {
+            const int cq = (int)__reduce_add_sync(FULL, (unsigned)cnt[q]);
+            if (lane == 0) sm.wcnt[w][q] = cq;
+        }
+    }
+    if (HW > 0 && w < 2 * HW) {
+#pragma unroll
+        for (int c = 0; c < HC; ++c) {
+            T h = hv[c];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) h += __shfl_xor_sync(FULL, h, off);
+            if (lane == 0) sm.whs[w][c] = h;
+        }
+    }
     if (lane == 0) {
         sm.be[w] = f;
 #pragma unroll
         for (int c = 0; c < C; ++c) sm.bV[w][c] = iW[c];
     }
-    __syncthreads();
+    if (COUNTED) {
+        if (__syncthreads_or(bad)) return true;
+    } else {
+        __syncthreads();
+    }
     if (w == 0) {
+        if (COUNTED) {
+#pragma unroll
+            for (int q = 0; q < NI; ++q) {
+                const int cq = (int)__reduce_add_sync(FULL, lane < NW ? (unsigned)sm.wcnt[lane][q] : 0u);
+                if (lane == 0) sm.tcnt[q] = cq;
+            }
+        }
+        if (HW > 0) {
+            // fixed order: warp sums added in a butterfly over the first HW
+            // lanes (left) and the next HW lanes (right)
+#pragma unroll
+            for (int c = 0; c < HC; ++c) {
+                T hs = lane < 2 * HW ? sm.whs[lane][c] : T(0);
+#pragma unroll
+                for (int off = 1; off < HW; off <<= 1) hs += __shfl_xor_sync(FULL, hs, off);
+                if (lane == 0) sm.thL[c] = hs;
+                if (lane == HW) sm.thU[c] = hs;
+            }
+        }
         T ge = lane < NW ? sm.fe[lane] : T(0), gV[C];
         T gf = lane < NW ? sm.be[lane] : T(0), gW[C];
 #pragma unroll
@@ -410,6 +463,29 @@ __device__ __forceinline__ void block_excl_both(const T e, const T (&V)[C], cons
 #pragma unroll
         for (int c = 0; c < C; ++c) tW[c] = sm.tbV[c];
     }
+    if (COUNTED) {
+#pragma unroll
+        for (int q = 0; q < NI; ++q) tot[q] = sm.tcnt[q];
+    }
+    if (HW > 0) {
+#pragma unroll
+        for (int c = 0; c < HC; ++c) {
+            hL[c] = sm.thL[c];
+            hU[c] = sm.thU[c];
+        }
+    }
+    return false;
+}
+
+template <typename T, int C, int NT, int CT = 0>
+__device__ __forceinline__ void block_excl_both(const T e, const T (&V)[C], const T f, const T (&W)[C],
+                                                bool& hasf, T& pe, T (&pV)[C], T& te, T (&tV)[C],
+                                                bool& hasb, T& nf, T (&nW)[C], T& tf, T (&tW)[C],
+                                                BlockScan2Smem<T, C, NT>& sm) {
+    const int cnt[2] = {0, 0};
+    int tot[2];
+    (void)block_excl_both_counted<T, C, NT, CT, false>(e, V, f, W, hasf, pe, pV, te, tV, hasb, nf, nW,
+                                                       tf, tW, cnt, tot, false, sm);
 }
 
 // ---------------------------------------------------------------- chunk level
@@ -441,7 +517,8 @@ __device__ __forceinline__ void chunk_aggregates(const T (&s)[E], const T (&v)[E
 }
 
 // Given the state just before the chunk (anchor eprev, value Lprev) and just
-// after it (anchor enext, value Unext), out[i][c] = L_i + U_i - v_i.
+// after it (anchor enext, value Unext), out[i][c] = L_i + U_i - v_i, formed as
+// L_i + exp(s_i - s_{i+1}) U_{i+1} (U_i without its own term).
 template <typename T, int C, int E>
 __device__ __forceinline__ void chunk_final(const T (&s)[E], const T (&v)[E][C], T (&dl)[E],
                                             const T eprev, const T (&Lprev)[C], const T enext,
@@ -456,12 +533,12 @@ __device__ __forceinline__ void chunk_final(const T (&s)[E], const T (&v)[E][C],
             L = dfma<T>(dl[i], L, v[i][c]);
             out[i][c] = L;
         }
-        T U = dfma<T>(dn, Unext[c], v[E - 1][c]);
-        out[E - 1][c] += U - v[E - 1][c];
+        T U = Unext[c];
 #pragma unroll
-        for (int i = E - 2; i >= 0; --i) {
-            U = dfma<T>(dl[i + 1], U, v[i][c]);
-            out[i][c] += U - v[i][c];
+        for (int i = E - 1; i >= 0; --i) {
+            const T d = i == E - 1 ? dn : dl[i + 1];
+            out[i][c] = dfma<T>(d, U, out[i][c]);
+            U = dfma<T>(d, U, v[i][c]);
         }
     }
 }

@@ -1,6 +1,7 @@
-// sort.cu -- stable LSD radix sort of the anchors with an index payload
-// ("after sorting the anchors": "LAPLEX - La FFT dei Nuclei di Laplace
-// Apprendibili", technical summary §2.2; the sort is the O(n log n) term).
+// sort.cu -- stable LSD radix sort of the anchors with an index payload (the
+// recurrences run over the anchors in sorted order: "LAPLEX - La FFT dei
+// Nuclei di Laplace Apprendibili", technical summary §2.2; the sort is the
+// O(n log n) term).
 //
 // Key map (monotone, bijective on finite values after -0.0 -> +0.0):
 //     u = bits(a);  u = (u == -0.0) ? +0.0 : u;
@@ -93,12 +94,15 @@ __device__ __forceinline__ uint32_t block_excl_sum(uint32_t v, uint32_t* sm /*NT
     return r;
 }
 
-__device__ __forceinline__ void st_release64(uint64_t* p, uint64_t v) {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+// A look-back record is one 64-bit word (tag in the high half, count in the
+// low half) written and read whole, and nothing else is read on the strength
+// of it, so relaxed accesses suffice and a window of loads can be in flight.
+__device__ __forceinline__ void st_relaxed64(uint64_t* p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-__device__ __forceinline__ uint64_t ld_acquire64(const uint64_t* p) {
+__device__ __forceinline__ uint64_t ld_relaxed64(const uint64_t* p) {
     uint64_t v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 
@@ -139,7 +143,7 @@ __global__ void __launch_bounds__(SORT_NT) k_radix_offsets(uint32_t* __restrict_
 constexpr uint32_t SORT_POLLS = 1u << 25;
 
 template <typename T, int KPT>
-__global__ void __launch_bounds__(SORT_NT) k_onesweep(
+__global__ void __launch_bounds__(SORT_NT, 3) k_onesweep(
     const T* __restrict__ a, const typename KeyOf<T>::K* __restrict__ ksrc,
     const int32_t* __restrict__ vsrc, int64_t n, int pass, const uint32_t* __restrict__ offsets,
     uint64_t* __restrict__ rec, uint32_t* __restrict__ ticket, typename KeyOf<T>::K* __restrict__ kdst,
@@ -165,25 +169,27 @@ __global__ void __launch_bounds__(SORT_NT) k_onesweep(
     const unsigned ltmask = lanemask_lt();
     K k[KPT];
     int32_t v[KPT];
-    int dg[KPT];
     uint32_t rk[KPT];
     bool bad = false;
+    // digit of key i of this thread; RADIX for padding (never placed)
+    const int64_t lane0 = tb + (int64_t)w * 32 * KPT + lane;
+    auto digit = [&](int i) -> int {
+        return lane0 + i * 32 < end ? (int)((unsigned)(k[i] >> shift) & (RADIX - 1)) : RADIX;
+    };
 #pragma unroll
     for (int i = 0; i < KPT; ++i) {
-        const int64_t idx = tb + (int64_t)w * 32 * KPT + i * 32 + lane;
+        const int64_t idx = lane0 + i * 32;
         if (idx < end) {
             k[i] = first ? to_key(a[idx], bad) : ksrc[idx];
             v[i] = first ? (int32_t)idx : vsrc[idx];
-            dg[i] = (int)((unsigned)(k[i] >> shift) & (RADIX - 1));
         } else {
             k[i] = 0;
             v[i] = 0;
-            dg[i] = RADIX;  // padding: never placed
         }
     }
 #pragma unroll
     for (int i = 0; i < KPT; ++i) {
-        const int d = dg[i];
+        const int d = digit(i);
         const unsigned peers = __match_any_sync(FULL, d);
         const uint32_t lower = __popc(peers & ltmask);
         rk[i] = d < RADIX ? wcnt[w][d] + lower : 0u;
@@ -207,26 +213,37 @@ __global__ void __launch_bounds__(SORT_NT) k_onesweep(
         uint64_t* my = rec + t * RADIX + d;
         uint64_t excl = 0;
         if (t == 0) {
-            st_release64(my, tagI | c);
+            st_relaxed64(my, tagI | c);
         } else {
-            st_release64(my, tagA | c);
-            for (int64_t j = t - 1; j >= 0; --j) {
-                const uint64_t* r = rec + j * RADIX + d;
-                uint64_t val = ld_acquire64(r);
-                uint32_t it = 0;
-                while ((val & 0xFFFFFFFF00000000ull) < tagA) {
-                    if (++it > SORT_POLLS) break;
-                    __nanosleep(32);
-                    val = ld_acquire64(r);
+            st_relaxed64(my, tagA | c);
+            // walk back LB records at a time (loads in flight together), adding
+            // counts up to and including the first inclusive record
+            constexpr int LB = 8;
+            bool done = false;
+            for (int64_t j0 = t - 1; !done; j0 -= LB) {
+                uint64_t val[LB];
+#pragma unroll
+                for (int q = 0; q < LB; ++q)
+                    val[q] = j0 - q >= 0 ? ld_relaxed64(rec + (j0 - q) * RADIX + d) : tagI;
+#pragma unroll
+                for (int q = 0; q < LB; ++q) {
+                    if (done) break;
+                    uint32_t it = 0;
+                    while ((val[q] & 0xFFFFFFFF00000000ull) < tagA) {
+                        if (++it > SORT_POLLS) break;
+                        __nanosleep(32);
+                        val[q] = ld_relaxed64(rec + (j0 - q) * RADIX + d);
+                    }
+                    if ((val[q] & 0xFFFFFFFF00000000ull) < tagA) {
+                        set_status(status, ST_TIMEOUT);
+                        done = true;
+                        break;
+                    }
+                    excl += val[q] & 0xFFFFFFFFull;
+                    if ((val[q] & 0xFFFFFFFF00000000ull) == tagI) done = true;
                 }
-                if ((val & 0xFFFFFFFF00000000ull) < tagA) {
-                    set_status(status, ST_TIMEOUT);
-                    break;
-                }
-                excl += val & 0xFFFFFFFFull;
-                if ((val & 0xFFFFFFFF00000000ull) == tagI) break;
             }
-            st_release64(my, tagI | (excl + c));
+            st_relaxed64(my, tagI | (excl + c));
         }
         gbase[d] = (int64_t)offsets[d] + (int64_t)excl;
         uint32_t tot;
@@ -235,7 +252,7 @@ __global__ void __launch_bounds__(SORT_NT) k_onesweep(
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < KPT; ++i) {
-        const int d = dg[i];
+        const int d = digit(i);
         if (d < RADIX) {
             const uint32_t pos = dstart[d] + wcnt[w][d] + rk[i];
             skey[pos] = k[i];

@@ -253,6 +253,9 @@ template <typename T_, int NCOL_, bool PHASED_, int E_, int NT_>
 struct SymTP {
     using T = T_;
     static constexpr int NCOL = NCOL_, C = PHASED_ ? 2 * NCOL_ : NCOL_, CT = 0, E = E_, NT = NT_;
+    // halos of 128 (fp32: they span CUT = 104 at spacings above 0.82); fp64
+    // (CUT = 746) would need several times more: none
+    static constexpr int H = sizeof(T_) == 4 ? 128 : 0;
     SymArgs<T> A;
     int64_t n;
     const T* s;
@@ -269,16 +272,23 @@ struct SymTP {
         chunk_final<T, C, E>(sv, v, dl, eprev, Lp, enext, Un, out);
         sym_store<T, NCOL, PHASED_, E>(A, r0, out, a.cph, a.sph);
     }
-    __device__ __forceinline__ void carry_in(int64_t r, T fe, T, const T* c, bool) const {
-        const int64_t row = A.pout ? (int64_t)A.pout[r] : r;
-        T* yr = A.y + row * A.ldy + A.col0;
-        if (PHASED_) {
-            const int64_t ar = A.paux ? (int64_t)A.paux[r] : r;
-            T sp, cp;
-            dsincos<T>(A.phi[ar], &sp, &cp);
-            for (int k = 0; k < A.ncol; ++k) yr[k] += fe * (cp * c[2 * k] + sp * c[2 * k + 1]);
-        } else {
-            for (int k = 0; k < A.ncol; ++k) yr[k] += fe * c[k];
+    __device__ __forceinline__ void load1(int64_t j, T& sj, T (&vj)[C]) const {
+        sj = A.s[j];
+        const int64_t row = A.pin ? (int64_t)A.pin[j] : j;
+        const int64_t ar = A.paux ? (int64_t)A.paux[j] : j;
+        const T dsc = A.D ? A.D[ar] : T(1);
+        T sp = T(0), cp = T(1);
+        if (PHASED_) dsincos<T>(A.phi[ar], &sp, &cp);
+        const T* xr = A.x + row * A.ldx + A.col0;
+#pragma unroll
+        for (int c = 0; c < NCOL; ++c) {
+            const T val = (c < A.ncol ? xr[c] : T(0)) * dsc;
+            if (PHASED_) {
+                vj[2 * c] = cp * val;
+                vj[2 * c + 1] = sp * val;
+            } else {
+                vj[c] = val;
+            }
         }
     }
 };

@@ -4,50 +4,66 @@
 // x in sorted order, or in the caller's order with perm (gathered on load, y
 // scattered back); several columns, phases or a scale use sym.cu.
 //
-// Three kernels, none of which waits for another block:
-//   1. k_tile_local (streams s and x once, writes y once; persistent blocks,
-//      every tile's s and x brought into a 2-stage shared-memory ring by 1-D
-//      bulk copies (TMA), the next tile loading while one is computed): each tile scans
-//      itself with zero carries and writes y = Lloc + Uloc - x.  It records its
-//      first and last anchors, its forward/backward totals and its reach: how
-//      many elements from each end lie within CUT of that end's anchor.  A carry
-//      from outside the tile reaches element r with a factor exp(-d), d >= the
-//      distance from r to the tile's end anchor, and exp(-d) is exactly 0 for
-//      d >= CUT (fp32: 104, below the smallest subnormal; fp64: 746), so
-//      elements beyond the reach are untouched by the carries, bit for bit.
-//   2. k_carry_blocks, k_carry_tiles: the exact carries into every tile from
-//      the tile totals (block totals, then per-tile carries; the carry into a
-//      block is a walk over the block totals that stops where exp of the gap is
-//      exactly 0).
-//   3. k_headtail: y_r += exp(eT - s_r) L_carry over each tile's head reach and
-//      y_r += exp(s_r - fT) U_carry over its tail reach (read-modify-write of a
-//      few percent of y; one warp per tile at a time).
+// Three passes, none of which waits for another block:
+//   1. k_tile_local<..., 0> (streams s and x once; persistent blocks, every
+//      tile's s and x brought into a 2-stage shared-memory ring by 1-D bulk
+//      copies (TMA), the next tiles loading while one is computed).  The copy
+//      of a tile also brings a halo of H elements on each side.  A carry from
+//      outside the tile reaches element r with a factor exp(-d), d >= the
+//      distance from r to the tile's edge anchor, and exp(-d) is exactly 0 for
+//      d >= CUT (fp32: 104, below the smallest subnormal; fp64: 746).  So when
+//      a halo spans at least CUT, the carry summed over the halo is the exact
+//      carry, and the tile writes its final outputs.  A tile whose halos do
+//      not span CUT (dense anchors) writes nothing and is listed for pass 3.
+//      Every tile records its first and last anchors and its zero-carry
+//      forward/backward totals.
+//   2. k_carry_blocks, k_carry_tiles (only when a tile was listed): the exact
+//      carries into every tile from the tile totals (block totals, then
+//      per-tile carries; the carry into a block is a walk over the block totals
+//      that stops where exp of the gap is exactly 0).
+//   3. k_tile_local<..., 1>: the listed tiles again, with those carries.
+// Sparse anchors (spacing around 1 unit, as in a ~ U(0, n)) finish in pass 1:
+// 12 bytes per element.  Dense anchors take passes 1 and 3: 8 + 12 bytes.
 #include <algorithm>
 
 #include "laplex_impl.h"
+#include "bulk.cuh"
 #include "scan_core.cuh"
 
 namespace lx {
 
-constexpr int LT_NT = 512;     // threads per tile block
+// tile shape of k_tile_local (fp32): threads per block, elements per thread,
+// halo per side, resident blocks per SM
+#ifndef LX_LT_NT
+#define LX_LT_NT 512
+#endif
+#ifndef LX_LT_E
+#define LX_LT_E 12
+#endif
+#ifndef LX_LT_H
+#define LX_LT_H 256
+#endif
+#ifndef LX_LT_MINB
+#define LX_LT_MINB 2
+#endif
+constexpr int LT_NT = LX_LT_NT;  // threads per tile block
 constexpr int CARRY_NT = 256;  // threads per carry block
 constexpr int CARRY_PT = 8;    // tiles per carry thread
 constexpr int CARRY_BT = CARRY_NT * CARRY_PT;
-constexpr int HT_BLOCKS_PER_SM = 8;
 
 template <typename T> struct LocalE;
-template <> struct LocalE<float> { static constexpr int E = 12; };   // 3 x 16 bytes
+template <> struct LocalE<float> { static constexpr int E = LX_LT_E; };  // 3 x 16 bytes
 template <> struct LocalE<double> { static constexpr int E = 6; };   // 3 x 16 bytes
+// halo elements per side: a span of CUT needs about CUT / spacing elements;
+// fp64 (CUT 746) would need several times more, so its tiles have none
+template <typename T> struct LocalH;
+template <> struct LocalH<float> { static constexpr int H = LX_LT_H; };
+template <> struct LocalH<double> { static constexpr int H = 0; };
 constexpr int LT_STAGES = 2;
 
 template <typename T> struct Cut;
 template <> struct Cut<float> { static constexpr float v = 104.0f; };
 template <> struct Cut<double> { static constexpr double v = 746.0; };
-
-struct TileStats {
-    int32_t head;  // elements from the tile start within CUT of the first anchor
-    int32_t tail;  // elements from the tile end within CUT of the last anchor
-};
 
 template <typename T>
 struct LocalWs {
@@ -55,7 +71,8 @@ struct LocalWs {
     T* tlast;
     T* fagg;  // L at the tile's last element, tile only
     T* bagg;  // U at the tile's first element, tile only
-    TileStats* st;
+    int32_t* redo;        // tiles the first pass left for the redo pass (any order)
+    uint32_t* redo_count; // their number (zeroed before the first pass)
     T* bfe;   // per carry-block forward total: last anchor of the block, value
     T* bfv;
     T* bbf;   // per carry-block backward total: first anchor of the block, value
@@ -64,134 +81,136 @@ struct LocalWs {
     T* carB;  // U at the element after tile t
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0u;
-}
-constexpr uint32_t MBAR_POLLS = 1u << 20;
-// bounded wait for phase `parity` of *bar; false if it never completed
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (uint32_t it = 0; it < MBAR_POLLS; ++it)
-        if (mbar_test(bar, parity)) return true;
-    return false;
-}
-// orders this thread's generic-proxy shared-memory accesses before later
-// async-proxy (TMA) accesses to the same memory
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Persistent: block b handles tiles b, b + G, b + 2G, ...; the tile of
-// iteration i sits in ring stage i % S.  Each thread owns E consecutive
-// elements, an odd number of 16-byte units, so 128-bit shared loads of a warp
-// touch distinct banks.  The ragged last tile (if any) is read from global.
+// Persistent: block b handles tiles b, b + G, b + 2G, ... (MODE 1: only the
+// tiles of that sequence marked for the redo pass).  The tile of iteration i
+// sits in ring stage i % S, and the stage is refilled with the block's tile
+// S iterations later as soon as every thread has read it (after the block
+// scan's barriers), so S tiles are in flight while one is computed.  Each
+// thread owns E consecutive elements, an odd number of 16-byte units, so
+// 128-bit shared loads of a warp touch distinct banks.  Two block barriers per
+// tile, both inside the block scan, which also sums the halo terms and checks
+// and carries the copy-timeout flag.
+//
+// MODE 0 (first pass).  The copy of a full tile also brings H elements on each
+// side (halos).  Thread q < 2H takes one halo element: its term of the carry
+// from the left, L_{b-1} = sum_j exp(s_j - s_{b-1}) x_j, or from the right,
+// U_e.  When both halos span at least CUT (or the tile is at an end of the
+// array) these sums are the exact carries and the tile's outputs are final.
+// Otherwise (dense anchors, H = 0, the ragged last tile) nothing is written
+// and the tile is marked for the redo pass.  Every tile publishes its first
+// and last anchors and its zero-carry totals for the carry kernels.
+// MODE 1 (redo pass): the marked tiles again, with the exact carries from the
+// carry kernels.
 // GATHER: x is in the caller's order and y goes back to it through perm (the
 // ring then holds s and perm; x is gathered from global memory).
-template <typename T, int E, int NT, int S, bool GATHER>
-__global__ void __launch_bounds__(NT, 2) k_tile_local(const T* __restrict__ s_, const T* __restrict__ x_,
+template <typename T, int E, int NT, int S, int H, bool GATHER, int MODE>
+__global__ void __launch_bounds__(NT, LX_LT_MINB) k_tile_local(const T* __restrict__ s_, const T* __restrict__ x_,
                                                       T* __restrict__ y_, const int32_t* __restrict__ perm,
                                                       int64_t n, int64_t ntiles, LocalWs<T> W,
                                                       uint32_t* status) {
     constexpr int VN = V16<T>::N;
     constexpr int64_t TILE = (int64_t)NT * E;
+    constexpr int HH = MODE == 0 ? H : 0;     // halo brought by the copies
+    constexpr int64_t STAGE = TILE + 2 * H;   // elements per array per stage
     static_assert(((E / VN) & 1) == 1, "E must be an odd number of 16-byte units");
+    static_assert(H % 32 == 0 && 2 * H <= NT, "halo: whole warps, one element per thread");
     extern __shared__ __align__(128) unsigned char dyn[];
     T* ring_s = reinterpret_cast<T*>(dyn);
-    T* ring_x = ring_s + S * TILE;                              // !GATHER
-    int32_t* ring_p = reinterpret_cast<int32_t*>(ring_s + S * TILE);  // GATHER
-    const int32_t* pout = perm;
+    T* ring_x = ring_s + S * STAGE;                              // !GATHER
+    int32_t* ring_p = reinterpret_cast<int32_t*>(ring_s + S * STAGE);  // GATHER
     __shared__ __align__(8) uint64_t full[S];
+    __shared__ int64_t slot_tile[S];  // tile of each stage, -1: the block is done
+    __shared__ int sh_timeout;
     __shared__ BlockScan2Smem<T, 1, NT> sm2;
-    __shared__ int cnt_head, cnt_tail;
-    __shared__ T sh_first, sh_last;
     const int64_t G = gridDim.x;
+    // thread 0: next candidate tile (MODE 0) or redo-list entry (MODE 1)
+    int64_t cursor = blockIdx.x, listed = 0;
 
     auto issue = [&](int st, int64_t t) {  // one thread
-        if ((t + 1) * TILE <= n) {
+        const int64_t b = t * TILE, e = b + TILE;
+        if (e <= n) {
+            const int64_t hl = (HH > 0 && t > 0) ? HH : 0;
+            const int64_t hr = (HH > 0 && e + HH <= n) ? HH : 0;
+            const int64_t lo = b - hl, cnt = hl + TILE + hr;
+            const int64_t off = st * STAGE + (H - hl);
             if constexpr (GATHER) {
-                mbar_expect_tx(&full[st], (uint32_t)(TILE * (sizeof(T) + sizeof(int32_t))));
-                bulk_g2s(ring_s + st * TILE, s_ + t * TILE, (uint32_t)(TILE * sizeof(T)), &full[st]);
-                bulk_g2s(ring_p + st * TILE, perm + t * TILE, (uint32_t)(TILE * sizeof(int32_t)), &full[st]);
+                mbar_expect_tx(&full[st], (uint32_t)(cnt * (sizeof(T) + sizeof(int32_t))));
+                bulk_g2s(ring_s + off, s_ + lo, (uint32_t)(cnt * sizeof(T)), &full[st]);
+                bulk_g2s(ring_p + off, perm + lo, (uint32_t)(cnt * sizeof(int32_t)), &full[st]);
             } else {
-                mbar_expect_tx(&full[st], (uint32_t)(2 * TILE * sizeof(T)));
-                bulk_g2s(ring_s + st * TILE, s_ + t * TILE, (uint32_t)(TILE * sizeof(T)), &full[st]);
-                bulk_g2s(ring_x + st * TILE, x_ + t * TILE, (uint32_t)(TILE * sizeof(T)), &full[st]);
+                mbar_expect_tx(&full[st], (uint32_t)(2 * cnt * sizeof(T)));
+                bulk_g2s(ring_s + off, s_ + lo, (uint32_t)(cnt * sizeof(T)), &full[st]);
+                bulk_g2s(ring_x + off, x_ + lo, (uint32_t)(cnt * sizeof(T)), &full[st]);
             }
         } else {
             mbar_arrive(&full[st]);  // ragged tile: read from global
         }
     };
+    // thread 0: the block's next tile into stage st (or the end mark)
+    auto next = [&](int st) {
+        int64_t t = -1;
+        if (MODE == 0 ? cursor < ntiles : cursor < listed) t = MODE == 0 ? cursor : (int64_t)W.redo[cursor];
+        cursor += G;
+        slot_tile[st] = t;
+        if (t >= 0) issue(st, t);
+        else mbar_arrive(&full[st]);
+    };
     if (threadIdx.x == 0) {
+        sh_timeout = 0;
+        if (MODE == 1) listed = (int64_t)*(volatile uint32_t*)W.redo_count;
         for (int st = 0; st < S; ++st) mbar_init(&full[st], 1u);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        for (int st = 0; st < S - 1; ++st) {
-            const int64_t t = blockIdx.x + st * G;
-            if (t < ntiles) issue(st, t);
-        }
+        for (int st = 0; st < S; ++st) next(st);
     }
     __syncthreads();
     for (int64_t i = 0;; ++i) {
-        const int64_t t = blockIdx.x + i * G;
-        if (t >= ntiles) break;
         const int st = (int)(i % S);
-        const uint32_t ph = (uint32_t)((i / S) & 1);
-        const bool landed = mbar_wait(&full[st], ph);
-        if (__syncthreads_or(!landed)) {  // a copy never completed: report and stop
-            if (threadIdx.x == 0) {
-                set_status(status, ST_TIMEOUT);
-                for (int k = 1; k < S - 1; ++k) {
-                    const int64_t t2 = blockIdx.x + (i + k) * G;
-                    if (t2 < ntiles) mbar_wait(&full[(i + k) % S], (uint32_t)(((i + k) / S) & 1));
-                }
-            }
-            return;
-        }
+        const bool landed = mbar_wait(&full[st], (uint32_t)((i / S) & 1));
+        // the stage's tile (written before the arrive that completed the
+        // phase); a thread whose wait ran out records it, and the block leaves
+        // the loop together at the block scan's first barrier
+        if (!landed) sh_timeout = 1;
+        const int64_t t = landed ? slot_tile[st] : -1;
+        const bool live = t >= 0;
         const int64_t tile0 = t * TILE;
         const int64_t r0 = tile0 + (int64_t)threadIdx.x * E;
         const bool ragged = tile0 + TILE > n;
+        const T* S0 = ring_s + st * STAGE;  // [left halo | tile | right halo]
+        // MODE 1: the exact carries into the tile (zero at the array's ends)
+        T cL = T(0), cU = T(0), aL = T(0), aU = T(0);
+        if (MODE == 1 && live) {
+            if (t > 0) {
+                cL = W.carF[t];
+                aL = s_[tile0 - 1];
+            }
+            if (t < ntiles - 1) {
+                cU = W.carB[t];
+                aU = s_[tile0 + TILE];
+            }
+        }
         T s[E], v[E][1];
         int32_t pr[GATHER ? E : 1];
         {
             T xv[E];
-            if (!ragged) {
-                const T* ps = ring_s + st * TILE + threadIdx.x * E;
+            if (!live) {
+#pragma unroll
+                for (int k = 0; k < E; ++k) {
+                    s[k] = T(0);
+                    xv[k] = T(0);
+                    if constexpr (GATHER) pr[k] = 0;
+                }
+            } else if (!ragged) {
+                const T* ps = S0 + H + threadIdx.x * E;
 #pragma unroll
                 for (int k = 0; k < E; k += VN) ld16<T>(ps + k, &s[k]);
                 if constexpr (GATHER) {
-                    const int32_t* pp = ring_p + st * TILE + threadIdx.x * E;
+                    const int32_t* pp = ring_p + st * STAGE + H + threadIdx.x * E;
 #pragma unroll
                     for (int k = 0; k < E; ++k) pr[k] = pp[k];
 #pragma unroll
                     for (int k = 0; k < E; ++k) xv[k] = __ldg(x_ + pr[k]);
                 } else {
-                    const T* px = ring_x + st * TILE + threadIdx.x * E;
+                    const T* px = ring_x + st * STAGE + H + threadIdx.x * E;
 #pragma unroll
                     for (int k = 0; k < E; k += VN) ld16<T>(px + k, &xv[k]);
                 }
@@ -199,7 +218,7 @@ __global__ void __launch_bounds__(NT, 2) k_tile_local(const T* __restrict__ s_, 
 #pragma unroll
                 for (int k = 0; k < E; ++k) {
                     const int64_t r = r0 + k;
-                    s[k] = s_[min(r, n - 1)];
+                    s[k] = s_[min(r, n - 1)];  // padded with the last anchor
                     if constexpr (GATHER) {
                         pr[k] = r < n ? perm[r] : 0;
                         xv[k] = r < n ? x_[pr[k]] : T(0);
@@ -211,59 +230,109 @@ __global__ void __launch_bounds__(NT, 2) k_tile_local(const T* __restrict__ s_, 
 #pragma unroll
             for (int k = 0; k < E; ++k) v[k][0] = xv[k];
         }
-        if (threadIdx.x == 0) {
-            cnt_head = 0;
-            cnt_tail = 0;
-            sh_first = ragged ? s_[tile0] : ring_s[st * TILE];
-            sh_last = ragged ? s_[n - 1] : ring_s[st * TILE + TILE - 1];
+        // MODE 0: halo term of this thread (q < H: left, H <= q < 2H: right),
+        // and the checks that each halo spans CUT (thread 0: left, thread H:
+        // right); a tile without usable halos is marked bad on both sides
+        T hv = T(0), ringL = T(0), ringR = T(0);  // s_{b-1}, s_e when in the ring
+        int bad[2] = {0, 0};
+        if constexpr (MODE == 0) {
+            const int q = (int)threadIdx.x;
+            const int64_t e = tile0 + TILE;
+            if constexpr (H > 0) {
+                if (live && !ragged) {
+                    if (t > 0) ringL = S0[H - 1];
+                    if (e + H <= n) ringR = S0[H + TILE];
+                }
+                if (q < 2 * H && live && !ragged) {
+                    const bool left = q < H;
+                    const bool have = left ? t > 0 : e + H <= n;
+                    const int j = left ? q : (int)(H + TILE) + (q - H);  // ring index
+                    if (have) {
+                        const T edge = left ? ringL : ringR;
+                        const T sj = S0[j];
+                        T xj;
+                        if constexpr (GATHER) xj = __ldg(x_ + ring_p[st * STAGE + j]);
+                        else xj = ring_x[st * STAGE + j];
+                        hv = dexp<T>(left ? sj - edge : edge - sj) * xj;
+                        if (q == 0) bad[0] = edge - sj >= Cut<T>::v ? 0 : 1;
+                        if (q == H) bad[1] = S0[2 * H + TILE - 1] - edge >= Cut<T>::v ? 0 : 1;
+                    } else {
+                        // no halo: exact only at the array's own ends
+                        if (q == 0) bad[0] = t == 0 ? 0 : 1;
+                        if (q == H) bad[1] = e == n ? 0 : 1;
+                    }
+                }
+            }
+            if (q == 0 && (H == 0 || ragged)) bad[0] = 1;
         }
-        // Every thread's reads of earlier stages are ordered before the TMA
-        // writes that refill them (generic -> async proxy).  The stage refilled
-        // now is the one of the previous iteration, read before at least one
-        // earlier barrier; the stage just read is refilled one iteration later.
+        // this thread's reads of stage st are ordered before the TMA writes that
+        // refill it (generic -> async proxy); the refill is issued after the
+        // block scan's barriers
         fence_proxy_async();
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            const int64_t t2 = blockIdx.x + (i + S - 1) * G;
-            if (t2 < ntiles) issue((int)((i + S - 1) % S), t2);
-        }
         T dl[E], fV[1], bW[1];
         chunk_aggregates<T, 1, E>(s, v, dl, fV, bW);
         bool hf, hb;
         T pe, pV[1], te, tV[1], nf, nW[1], tf, tW[1];
-        block_excl_both<T, 1, NT>(s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW, sm2);
-        {
-            // reach counts; the chunk is sorted, so only a chunk that straddles
-            // the cut needs a per-element count
-            const T first = sh_first, lastv = sh_last;
-            const int valid = (int)min((int64_t)E, max((int64_t)0, n - r0));
-            int h = 0, q = 0;
-            if (valid > 0) {
-                T sl = s[0];  // last valid anchor of the chunk (static indexing only)
-#pragma unroll
-                for (int k = 1; k < E; ++k)
-                    if (k < valid) sl = s[k];
-                if (sl - first < Cut<T>::v) h = valid;
-                else if (s[0] - first < Cut<T>::v)
-#pragma unroll
-                    for (int k = 0; k < E; ++k) h += (k < valid && s[k] - first < Cut<T>::v) ? 1 : 0;
-                if (lastv - s[0] < Cut<T>::v) q = valid;
-                else if (lastv - sl < Cut<T>::v)
-#pragma unroll
-                    for (int k = 0; k < E; ++k) q += (k < valid && lastv - s[k] < Cut<T>::v) ? 1 : 0;
+        int nbad[2];
+        T hL = T(0), hU = T(0);
+        if (block_excl_both_counted<T, 1, NT, 0, true, 2, (MODE == 0 ? H / 32 : 0)>(
+                s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW, bad, nbad, !live, sm2, &hv,
+                &hL, &hU)) {
+            // the block's last tile is done, or a copy never completed: then
+            // report it and let the copies in flight land before leaving
+            if (threadIdx.x == 0 && sh_timeout) {
+                set_status(status, ST_TIMEOUT);
+                for (int k = 0; k < S; ++k)
+                    if (slot_tile[(i + k) % S] >= 0)
+                        mbar_wait(&full[(i + k) % S], (uint32_t)(((i + k) / S) & 1));
             }
-            if (h) atomicAdd(&cnt_head, h);
-            if (q) atomicAdd(&cnt_tail, q);
+            return;
         }
-        // no carries from outside the tile here (k_headtail adds them): a thread
-        // without a neighbour on one side starts that recurrence from 0
-        T eprev = hf ? pe : s[0], Lprev[1] = {hf ? pV[0] : T(0)};
-        T enext = hb ? nf : s[E - 1], Unext[1] = {hb ? nW[0] : T(0)};
-        T out[E][1];
-        chunk_final<T, 1, E>(s, v, dl, eprev, Lprev, enext, Unext, out);
+        // the carries into the tile, and whether this pass writes it
+        bool out = true;
+        T eT = hf ? pe : s[0], Lc = T(0), fT = hb ? nf : s[E - 1], Uc = T(0);
+        if (MODE == 0) {
+            out = nbad[0] == 0 && nbad[1] == 0;
+            if (H > 0 && out && t > 0) {
+                eT = ringL;
+                Lc = hL;
+            }
+            if (H > 0 && out && tile0 + TILE < n) {
+                fT = ringR;
+                Uc = hU;
+            }
+        } else {
+            if (t > 0) {
+                eT = aL;
+                Lc = cL;
+            }
+            if (t < ntiles - 1) {
+                fT = aU;
+                Uc = cU;
+            }
+        }
+        if (threadIdx.x == 0) {
+            if (MODE == 0) {
+                W.tfirst[t] = tf;
+                W.tlast[t] = te;
+                W.fagg[t] = tV[0];
+                W.bagg[t] = tW[0];
+                if (!out) W.redo[atomicAdd(W.redo_count, 1u)] = (int32_t)t;
+            }
+            next(st);
+        }
+        if (!out) continue;
+        T eprev, Lprev[1], enext, Unext[1];
+        {
+            const T VT[1] = {Lc}, WT[1] = {Uc};
+            apply_carry_fwd<T, 1>(hf, pe, pV, eT, VT, eprev, Lprev);
+            apply_carry_bwd<T, 1>(hb, nf, nW, fT, WT, enext, Unext);
+        }
+        T o4[E][1];
+        chunk_final<T, 1, E>(s, v, dl, eprev, Lprev, enext, Unext, o4);
         T o[E];
 #pragma unroll
-        for (int k = 0; k < E; ++k) o[k] = out[k][0];
+        for (int k = 0; k < E; ++k) o[k] = o4[k][0];
         if constexpr (GATHER) {
 #pragma unroll
             for (int k = 0; k < E; ++k)
@@ -275,15 +344,6 @@ __global__ void __launch_bounds__(NT, 2) k_tile_local(const T* __restrict__ s_, 
 #pragma unroll
             for (int k = 0; k < E; ++k)
                 if (r0 + k < n) y_[r0 + k] = o[k];
-        }
-        __syncthreads();  // the reach counters are complete
-        if (threadIdx.x == 0) {
-            W.tfirst[t] = tf;
-            W.tlast[t] = te;
-            W.fagg[t] = tV[0];
-            W.bagg[t] = tW[0];
-            W.st[t].head = cnt_head;
-            W.st[t].tail = cnt_tail;
         }
     }
 }
@@ -319,6 +379,7 @@ __device__ __forceinline__ void carry_segment(const LocalWs<T>& W, int64_t t0, i
 
 template <typename T>
 __global__ void __launch_bounds__(CARRY_NT) k_carry_blocks(LocalWs<T> W, int64_t ntiles) {
+    if (*(volatile uint32_t*)W.redo_count == 0) return;  // every tile final
     __shared__ BlockScanSmem<T, 1, CARRY_NT> smf, smb;
     const int64_t t0 = (int64_t)blockIdx.x * CARRY_BT + (int64_t)threadIdx.x * CARRY_PT;
     T fe, fv[1], bf, bv[1];
@@ -337,6 +398,7 @@ __global__ void __launch_bounds__(CARRY_NT) k_carry_blocks(LocalWs<T> W, int64_t
 
 template <typename T>
 __global__ void __launch_bounds__(CARRY_NT) k_carry_tiles(LocalWs<T> W, int64_t ntiles, int64_t nblocks) {
+    if (*(volatile uint32_t*)W.redo_count == 0) return;  // every tile final
     __shared__ BlockScanSmem<T, 1, CARRY_NT> smf, smb;
     __shared__ T sh_c[2];
     const int64_t bidx = blockIdx.x;
@@ -405,41 +467,6 @@ __global__ void __launch_bounds__(CARRY_NT) k_carry_tiles(LocalWs<T> W, int64_t 
     }
 }
 
-template <typename T, int TILE>
-__global__ void __launch_bounds__(256) k_headtail(const T* __restrict__ s_, T* __restrict__ y_,
-                                                  const int32_t* __restrict__ pout, int64_t n,
-                                                  LocalWs<T> W, int64_t ntiles) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < ntiles;
-         t += warps) {
-        const int64_t b = t * TILE, e = min(b + (int64_t)TILE, n);
-        const TileStats stt = W.st[t];
-        if (t > 0) {
-            const T c = W.carF[t];
-            if (c != T(0)) {
-                const T eT = s_[b - 1];
-                for (int64_t r = b + lane; r < b + stt.head; r += 32) {
-                    const T f = dexp<T>(eT - s_[r]);
-                    if (f != T(0)) y_[pout ? (int64_t)pout[r] : r] += f * c;
-                }
-            }
-        }
-        __syncwarp();
-        if (t < ntiles - 1) {
-            const T c = W.carB[t];
-            if (c != T(0)) {
-                const T fT = s_[e];
-                for (int64_t r = e - 1 - lane; r >= e - stt.tail; r -= 32) {
-                    const T f = dexp<T>(s_[r] - fT);
-                    if (f != T(0)) y_[pout ? (int64_t)pout[r] : r] += f * c;
-                }
-            }
-        }
-        __syncwarp();
-    }
-}
-
 // ------------------------------------------------------------------ host side
 template <typename T>
 static int64_t local_ntiles(int64_t n) {
@@ -455,7 +482,8 @@ static LocalWs<T> local_carve(Carve& cv, int64_t ntiles) {
     W.tlast = cv.take<T>(ntiles);
     W.fagg = cv.take<T>(ntiles);
     W.bagg = cv.take<T>(ntiles);
-    W.st = cv.take<TileStats>(ntiles);
+    W.redo = cv.take<int32_t>(ntiles);
+    W.redo_count = cv.take<uint32_t>(1);
     W.bfe = cv.take<T>(nb);
     W.bfv = cv.take<T>(nb);
     W.bbf = cv.take<T>(nb);
@@ -469,7 +497,7 @@ size_t stream_ws_bytes(int64_t n, int f64) {
     const int64_t ntiles = f64 ? local_ntiles<double>(n) : local_ntiles<float>(n);
     const int64_t nb = (ntiles + CARRY_BT - 1) / CARRY_BT;
     const size_t es = f64 ? 8 : 4;
-    return 6 * Carve::need((size_t)ntiles, es) + Carve::need((size_t)ntiles, sizeof(TileStats)) +
+    return 6 * Carve::need((size_t)ntiles, es) + Carve::need((size_t)ntiles, 4) + Carve::need(1, 4) +
            4 * Carve::need((size_t)nb, es);
 }
 
@@ -478,7 +506,9 @@ cudaError_t stream_run(const T* s, const T* x, T* y, const int32_t* pout, int64_
                        size_t ws_bytes, uint32_t* status, cudaStream_t st) {
     if (n == 0) return cudaSuccess;
     constexpr int E = LocalE<T>::E;
+    constexpr int H = LocalH<T>::H;
     constexpr int TILE = LT_NT * E;
+    constexpr size_t STAGE = (size_t)TILE + 2 * H;
     const int64_t ntiles = local_ntiles<T>(n);
     const int64_t nb = (ntiles + CARRY_BT - 1) / CARRY_BT;
     Carve cv(ws, ws_bytes);
@@ -493,38 +523,42 @@ cudaError_t stream_run(const T* s, const T* x, T* y, const int32_t* pout, int64_
         e = cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
     }
-    {
-        auto launch = [&](auto kern, size_t smem, const int32_t* pp) -> cudaError_t {
-            static int per_sm[64][2] = {{0}};
-            const int which = pp ? 1 : 0;
-            if (per_sm[dev][which] == 0) {
-                cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-                if (r != cudaSuccess) return r;
-                int per = 0;
-                r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kern, LT_NT, smem);
-                if (r != cudaSuccess) return r;
-                per_sm[dev][which] = std::max(1, per);
-            }
-            const int64_t grid = std::min<int64_t>(ntiles, (int64_t)per_sm[dev][which] * sms_cache[dev]);
-            profile_before(st);
-            kern<<<(unsigned)grid, LT_NT, smem, st>>>(s, x, y, pp, n, ntiles, W, status);
-            profile_after(st);
-            return cudaGetLastError();
-        };
-        if (pout == nullptr)
-            e = launch(k_tile_local<T, E, LT_NT, LT_STAGES, false>,
-                       (size_t)LT_STAGES * TILE * (2 * sizeof(T)), nullptr);
-        else
-            e = launch(k_tile_local<T, E, LT_NT, LT_STAGES, true>,
-                       (size_t)LT_STAGES * TILE * (sizeof(T) + sizeof(int32_t)), pout);
-        if (e != cudaSuccess) return e;
-    }
+    // one persistent launch of k_tile_local<..., GATHER, MODE>; occupancy cached
+    // per device and variant
+    auto launch = [&](auto kern, int variant, size_t smem, const int32_t* pp, bool timed) -> cudaError_t {
+        static int per_sm[64][4] = {{0}};
+        if (per_sm[dev][variant] == 0) {
+            cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (r != cudaSuccess) return r;
+            int per = 0;
+            r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kern, LT_NT, smem);
+            if (r != cudaSuccess) return r;
+            per_sm[dev][variant] = std::max(1, per);
+        }
+        const int64_t grid = std::min<int64_t>(ntiles, (int64_t)per_sm[dev][variant] * sms_cache[dev]);
+        if (timed) profile_before(st);
+        kern<<<(unsigned)grid, LT_NT, smem, st>>>(s, x, y, pp, n, ntiles, W, status);
+        if (timed) profile_after(st);
+        return cudaGetLastError();
+    };
+    e = cudaMemsetAsync(W.redo_count, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess) return e;
+    const size_t smem_x = (size_t)LT_STAGES * STAGE * (2 * sizeof(T));
+    const size_t smem_p = (size_t)LT_STAGES * STAGE * (sizeof(T) + sizeof(int32_t));
+    if (pout == nullptr)
+        e = launch(k_tile_local<T, E, LT_NT, LT_STAGES, H, false, 0>, 0, smem_x, nullptr, true);
+    else
+        e = launch(k_tile_local<T, E, LT_NT, LT_STAGES, H, true, 0>, 1, smem_p, pout, true);
+    if (e != cudaSuccess) return e;
     k_carry_blocks<T><<<(unsigned)nb, CARRY_NT, 0, st>>>(W, ntiles);
     k_carry_tiles<T><<<(unsigned)nb, CARRY_NT, 0, st>>>(W, ntiles, nb);
-    const int64_t htb =
-        std::max<int64_t>(1, std::min<int64_t>((ntiles + 7) / 8, (int64_t)sms_cache[dev] * HT_BLOCKS_PER_SM));
-    k_headtail<T, TILE><<<(unsigned)htb, 256, 0, st>>>(s, y, pout, n, W, ntiles);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (pout == nullptr)
+        e = launch(k_tile_local<T, E, LT_NT, LT_STAGES, H, false, 1>, 2, smem_x, nullptr, false);
+    else
+        e = launch(k_tile_local<T, E, LT_NT, LT_STAGES, H, true, 1>, 3, smem_p, pout, false);
+    return e;
 }
 
 template cudaError_t stream_run<float>(const float*, const float*, float*, const int32_t*, int64_t,

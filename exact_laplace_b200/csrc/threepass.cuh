@@ -1,31 +1,37 @@
-// threepass.cuh -- wait-free three-kernel scheme for the LAPLEX scans, generic
-// over the operation (a policy) and its channels.
+// threepass.cuh -- wait-free scheme for the LAPLEX scans, generic over the
+// operation (a policy) and its channels.
 //
-//   1. k_tp_local: one block per tile; the policy loads the tile (with any
-//      gather through perm), the tile is scanned with zero carries from outside
-//      and the policy writes its outputs.  The tile's first/last anchors, its
-//      forward/backward totals (C channels) and its reach (elements within CUT
-//      of either end anchor) go to the workspace.
-//   2. k_tp_carry_blocks, k_tp_carry_tiles: exact carries into every tile.
-//   3. k_tp_headtail: the policy adds the carries to the elements in each
-//      tile's head and tail reach.  Beyond the reach every carry factor is
-//      exactly 0 (exp of a gap >= CUT underflows; tie factors are 0 for any
-//      gap > 0), so the result equals adding them everywhere.
+//   1. first pass, k_tp_local<P, 0> (one block per tile, register loads) or
+//      k_tp_ring<P> (persistent, TMA ring; inputs in sorted order): each tile
+//      is scanned with the carries from its halos, H elements on each side.
+//      A carry from outside the tile reaches element r with a factor exp(-d),
+//      d >= the distance from r to the tile's edge anchor, and exp(-d) is
+//      exactly 0 for d >= CUT; tie factors are 0 for any d > 0.  So when both
+//      halos span at least CUT (or the tile is at an end of the array) the
+//      halo sums are the exact carries and the tile writes its final outputs.
+//      Otherwise it writes nothing and is appended to the redo list.  Every
+//      tile stores its first/last anchors and its zero-carry totals.
+//   2. k_tp_carry_blocks, k_tp_carry_tiles (skipped when the list is empty):
+//      the exact carries into every tile from the tile totals.
+//   3. k_tp_local<P, 1>: the listed tiles again, with those carries.
 // No kernel waits on another block.
 //
 // A policy P provides
-//   using T;  static constexpr int C, CT, E, NT;   (CT trailing tie channels)
+//   using T;  static constexpr int C, CT, E, NT, H;   (CT trailing tie channels;
+//                                                      halo H: 0, or a multiple
+//                                                      of 32 with 2H <= NT)
 //   int64_t n;  const T* s;
 //   struct Aux { ... }                                  per-thread extra state
 //   __device__ void load(int64_t r0, T (&s)[E], T (&v)[E][C], Aux& a) const
+//        the chunk [r0, r0 + E), padded with the last anchor and value 0
+//   __device__ void load1(int64_t j, T& s, T (&v)[C]) const      one element
 //   __device__ void finish(int64_t r0, const T (&s)[E], const T (&v)[E][C], T (&dl)[E],
 //                          T eprev, const T (&Lp)[C], T enext, const T (&Un)[C], Aux& a) const
-//   __device__ void carry_in(int64_t r, T fe, T ft, const T* c, bool from_left) const
-//        adds, at element r (sorted index), a carry c[C] arriving with the exp
-//        factor fe and the tie factor ft, from the left (prefix) or the right.
+//        writes the outputs of the chunk from the state around it
 #pragma once
 #include <algorithm>
 
+#include "bulk.cuh"
 #include "laplex_impl.h"
 #include "scan_core.cuh"
 
@@ -35,7 +41,7 @@ template <typename T> struct TPCut;
 template <> struct TPCut<float> { static constexpr float v = 104.0f; };   // exp(-104) == 0 in fp32
 template <> struct TPCut<double> { static constexpr double v = 746.0; };  // exp(-746) == 0 in fp64
 
-struct TPStats {
+struct TPStats {  // reach of a tile (general case: elements within CUT of each edge)
     int32_t head;
     int32_t tail;
 };
@@ -50,7 +56,9 @@ struct TPWs {
     T* tlast;    // [ntiles]
     T* fagg;     // [ntiles*C] L at the tile's last element, tile only
     T* bagg;     // [ntiles*C] U at the tile's first element, tile only
-    TPStats* st; // [ntiles]
+    TPStats* st; // [ntiles] (general case)
+    int32_t* redo;         // [ntiles] tiles left for the redo pass, any order
+    uint32_t* redo_count;  // their number; NULL: carries always computed
     T* bfe;      // [nb] last anchor of each carry block
     T* bfv;      // [nb*C]
     T* bbf;      // [nb] first anchor of each carry block
@@ -62,8 +70,8 @@ struct TPWs {
 inline size_t tp_ws_bytes(int64_t ntiles, int C, size_t es) {
     const int64_t nb = (ntiles + TP_CARRY_BT - 1) / TP_CARRY_BT;
     return 2 * Carve::need((size_t)ntiles, es) + 4 * Carve::need((size_t)(ntiles * C), es) +
-           Carve::need((size_t)ntiles, sizeof(TPStats)) + 2 * Carve::need((size_t)nb, es) +
-           2 * Carve::need((size_t)(nb * C), es);
+           Carve::need((size_t)ntiles, sizeof(TPStats)) + Carve::need((size_t)ntiles, 4) + Carve::need(1, 4) +
+           2 * Carve::need((size_t)nb, es) + 2 * Carve::need((size_t)(nb * C), es);
 }
 
 template <typename T, int C>
@@ -75,6 +83,8 @@ inline TPWs<T, C> tp_carve(Carve& cv, int64_t ntiles) {
     W.fagg = cv.take<T>(ntiles * C);
     W.bagg = cv.take<T>(ntiles * C);
     W.st = cv.take<TPStats>(ntiles);
+    W.redo = cv.take<int32_t>(ntiles);
+    W.redo_count = cv.take<uint32_t>(1);
     W.bfe = cv.take<T>(nb);
     W.bfv = cv.take<T>(nb * C);
     W.bbf = cv.take<T>(nb);
@@ -84,75 +94,311 @@ inline TPWs<T, C> tp_carve(Carve& cv, int64_t ntiles) {
     return W;
 }
 
-// ------------------------------------------------------------------ pass 1
+// ------------------------------------------------------------------ pass 1 and 3
+// Halo term of thread q of a tile (q < H: left halo, H <= q < 2H: right halo)
+// and the checks that each halo spans CUT (thread 0: left, thread H: right).
+// A side needs no carry at an end of the array; a side without a halo in the
+// array (the right side of the last-but-one tiles) is marked bad.
 template <class P>
-__global__ void __launch_bounds__(P::NT) k_tp_local(P p, TPWs<typename P::T, P::C> W) {
+__device__ __forceinline__ void tp_halo_term(const P& p, int64_t t, int64_t tile0, int64_t tile1,
+                                             typename P::T (&hv)[P::C], int (&bad)[2]) {
     using T = typename P::T;
-    constexpr int C = P::C, CT = P::CT, E = P::E, NT = P::NT;
-    constexpr int64_t TILE = (int64_t)NT * E;
-    __shared__ BlockScan2Smem<T, C, NT> sm2;
-    __shared__ int cnt_head, cnt_tail;
-    __shared__ T sh_first, sh_last;
+    constexpr int C = P::C, CT = P::CT, H = P::H;
     const int64_t n = p.n;
-    const int64_t t = blockIdx.x;
-    const int64_t tile0 = t * TILE;
+    const int q = (int)threadIdx.x;
+#pragma unroll
+    for (int c = 0; c < C; ++c) hv[c] = T(0);
+    bad[0] = bad[1] = 0;
+    if (H == 0) {
+        if (q == 0) bad[0] = (t > 0 || tile1 < n) ? 1 : 0;  // no halos: final only if alone
+        return;
+    }
+    if (q >= 2 * H) return;
+    const bool left = q < H;
+    const bool need = left ? t > 0 : tile1 < n;
+    if (!need) return;
+    const bool have = left ? true : tile1 + H <= n;  // tile0 >= TILE >= H on the left
+    if (!have) {
+        if (q == H) bad[1] = 1;
+        return;
+    }
+    const int64_t j = left ? tile0 - H + q : tile1 + (q - H);
+    const T edge = left ? p.s[tile0 - 1] : p.s[tile1];
+    T sj, vj[C];
+    p.load1(j, sj, vj);
+    const Decay<T, C, CT> d = left ? Decay<T, C, CT>(sj, edge) : Decay<T, C, CT>(edge, sj);
+#pragma unroll
+    for (int c = 0; c < C; ++c) hv[c] = d[c] * vj[c];
+    if (q == 0) bad[0] = edge - sj >= TPCut<T>::v ? 0 : 1;
+    if (q == H) bad[1] = p.s[tile1 + H - 1] - edge >= TPCut<T>::v ? 0 : 1;
+}
+
+// One tile.  MODE 0: carries from the halos; a tile whose halos fall short is
+// listed for MODE 1 and writes nothing.  MODE 1: carries from the carry kernels.
+template <class P, int MODE>
+__device__ __forceinline__ void tp_tile(const P& p, const TPWs<typename P::T, P::C>& W, int64_t t,
+                                        int64_t ntiles, BlockScan2Smem<typename P::T, P::C, P::NT>& sm2) {
+    using T = typename P::T;
+    constexpr int C = P::C, CT = P::CT, E = P::E, NT = P::NT, H = MODE == 0 ? P::H : 0;
+    constexpr int64_t TILE = (int64_t)NT * E;
+    const int64_t n = p.n;
+    const int64_t tile0 = t * TILE, tile1 = min(tile0 + TILE, n);
     const int64_t r0 = tile0 + (int64_t)threadIdx.x * E;
+    const bool needL = t > 0, needR = tile1 < n;
     T s[E], v[E][C];
     typename P::Aux aux;
     p.load(r0, s, v, aux);
-    if (threadIdx.x == 0) {
-        cnt_head = 0;
-        cnt_tail = 0;
-        sh_first = s[0];
-        sh_last = p.s[min(tile0 + TILE, n) - 1];
-    }
+    T hv[C];
+    int bad[2] = {0, 0};
+    if (MODE == 0) tp_halo_term<P>(p, t, tile0, tile1, hv, bad);
     T dl[E], fV[C], bW[C];
     chunk_aggregates<T, C, E, CT>(s, v, dl, fV, bW);
     bool hf, hb;
     T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
-    block_excl_both<T, C, NT, CT>(s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW,
-                                  sm2);  // its barriers publish sh_first / sh_last
-    {
-        const T first = sh_first, lastv = sh_last;
-        const int valid = (int)min((int64_t)E, max((int64_t)0, n - r0));
-        int h = 0, q = 0;
-        if (valid > 0) {
-            T sl = s[0];
-#pragma unroll
-            for (int k = 1; k < E; ++k)
-                if (k < valid) sl = s[k];
-            if (sl - first < TPCut<T>::v) h = valid;
-            else if (s[0] - first < TPCut<T>::v)
-#pragma unroll
-                for (int k = 0; k < E; ++k) h += (k < valid && s[k] - first < TPCut<T>::v) ? 1 : 0;
-            if (lastv - s[0] < TPCut<T>::v) q = valid;
-            else if (lastv - sl < TPCut<T>::v)
-#pragma unroll
-                for (int k = 0; k < E; ++k) q += (k < valid && lastv - s[k] < TPCut<T>::v) ? 1 : 0;
-        }
-        if (h) atomicAdd(&cnt_head, h);
-        if (q) atomicAdd(&cnt_tail, q);
-    }
-    // zero carries from outside the tile (k_tp_headtail adds them)
-    T eprev = hf ? pe : s[0], enext = hb ? nf : s[E - 1];
-    T Lprev[C], Unext[C];
+    int nbad[2];
+    T hL[C], hU[C];
+    (void)block_excl_both_counted<T, C, NT, CT, true, 2, (H > 0 ? H / 32 : 0), C>(
+        s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW, bad, nbad, false, sm2, hv, hL, hU);
+    bool out = true;
+    T eT = hf ? pe : s[0], fT = hb ? nf : s[E - 1], Lc[C], Uc[C];
 #pragma unroll
     for (int c = 0; c < C; ++c) {
-        Lprev[c] = hf ? pV[c] : T(0);
-        Unext[c] = hb ? nW[c] : T(0);
+        Lc[c] = T(0);
+        Uc[c] = T(0);
     }
+    if (MODE == 0) {
+        out = nbad[0] == 0 && nbad[1] == 0;
+        if (threadIdx.x == 0) {
+            W.tfirst[t] = tf;
+            W.tlast[t] = te;
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                W.fagg[t * C + c] = tV[c];
+                W.bagg[t * C + c] = tW[c];
+            }
+            if (!out) W.redo[atomicAdd(W.redo_count, 1u)] = (int32_t)t;
+        }
+        if (!out) return;
+        if (H > 0 && needL) {
+            eT = p.s[tile0 - 1];
+#pragma unroll
+            for (int c = 0; c < C; ++c) Lc[c] = hL[c];
+        }
+        if (H > 0 && needR) {
+            fT = p.s[tile1];
+#pragma unroll
+            for (int c = 0; c < C; ++c) Uc[c] = hU[c];
+        }
+    } else {
+        if (needL) {
+            eT = p.s[tile0 - 1];
+#pragma unroll
+            for (int c = 0; c < C; ++c) Lc[c] = W.carF[t * C + c];
+        }
+        if (needR) {
+            fT = p.s[tile1];
+#pragma unroll
+            for (int c = 0; c < C; ++c) Uc[c] = W.carB[t * C + c];
+        }
+    }
+    T eprev, Lprev[C], enext, Unext[C];
+    apply_carry_fwd<T, C, CT>(hf, pe, pV, eT, Lc, eprev, Lprev);
+    apply_carry_bwd<T, C, CT>(hb, nf, nW, fT, Uc, enext, Unext);
     p.finish(r0, s, v, dl, eprev, Lprev, enext, Unext, aux);
-    __syncthreads();
+}
+
+// pass 1: one block per tile
+template <class P>
+__global__ void __launch_bounds__(P::NT) k_tp_local(P p, TPWs<typename P::T, P::C> W, int64_t ntiles) {
+    __shared__ BlockScan2Smem<typename P::T, P::C, P::NT> sm2;
+    tp_tile<P, 0>(p, W, (int64_t)blockIdx.x, ntiles, sm2);
+}
+
+// pass 3: the listed tiles, a grid-stride loop over the list
+template <class P>
+__global__ void __launch_bounds__(P::NT) k_tp_redo(P p, TPWs<typename P::T, P::C> W, int64_t ntiles) {
+    __shared__ BlockScan2Smem<typename P::T, P::C, P::NT> sm2;
+    const int64_t listed = (int64_t)*(volatile uint32_t*)W.redo_count;
+    for (int64_t k = blockIdx.x; k < listed; k += gridDim.x) {
+        tp_tile<P, 1>(p, W, (int64_t)W.redo[k], ntiles, sm2);
+        __syncthreads();  // sm2 is reused by the next tile
+    }
+}
+
+// ------------------------------------------------------------------ pass 1, streamed
+// Persistent variant of pass 1 for inputs already in sorted order: s and the
+// policy's NIN value arrays come into a shared-memory ring of S stages by 1-D
+// bulk copies (TMA), each full tile with a halo of H elements on both sides
+// (thread q < 2H takes one halo element, as in k_tp_local).  The ragged last
+// tile goes through the policy's register load and is always listed for the
+// redo pass.
+//
+// Extra policy members:
+//   static constexpr int NIN, S, MINB;         (value arrays, stages, blocks/SM)
+//   __device__ const T* ring_in(int a) const  value array a, sorted order
+//   __device__ void value(const T (&xin)[NIN], T (&v)[C]) const   channels of one element
+template <class P>
+__global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P::T, P::C> W,
+                                                            int64_t ntiles, uint32_t* status) {
+    using T = typename P::T;
+    constexpr int C = P::C, CT = P::CT, E = P::E, NT = P::NT, S = P::S, H = P::H, NIN = P::NIN;
+    constexpr int VN = V16<T>::N, NA = NIN + 1;
+    constexpr int64_t TILE = (int64_t)NT * E, STAGE = TILE + 2 * H;
+    static_assert(E % VN == 0, "E: whole 16-byte units");
+    static_assert(H % 32 == 0 && 2 * H <= NT, "halo: whole warps, one element per thread");
+    extern __shared__ __align__(128) unsigned char dyn[];
+    T* ring = reinterpret_cast<T*>(dyn);  // stage st, array a (0 = s) at ring + (st * NA + a) * STAGE
+    __shared__ __align__(8) uint64_t full[S];
+    __shared__ BlockScan2Smem<T, C, NT> sm2;
+    const int64_t n = p.n;
+    const int64_t G = gridDim.x;
+
+    auto issue = [&](int st, int64_t t) {  // one thread
+        const int64_t b = t * TILE, e = b + TILE;
+        if (e <= n) {
+            const int64_t hl = (H > 0 && t > 0) ? H : 0;
+            const int64_t hr = (H > 0 && e + H <= n) ? H : 0;
+            const int64_t lo = b - hl, cnt = hl + TILE + hr;
+            const uint32_t bytes = (uint32_t)(cnt * sizeof(T));
+            mbar_expect_tx(&full[st], (uint32_t)NA * bytes);
+            bulk_g2s(ring + (int64_t)(st * NA) * STAGE + (H - hl), p.s + lo, bytes, &full[st]);
+#pragma unroll
+            for (int a = 0; a < NIN; ++a)
+                bulk_g2s(ring + (int64_t)(st * NA + 1 + a) * STAGE + (H - hl), p.ring_in(a) + lo, bytes,
+                         &full[st]);
+        } else {
+            mbar_arrive(&full[st]);  // ragged tile: register loads
+        }
+    };
     if (threadIdx.x == 0) {
-        W.tfirst[t] = tf;
-        W.tlast[t] = te;
+        for (int st = 0; st < S; ++st) mbar_init(&full[st], 1u);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int st = 0; st < S; ++st) {
+            const int64_t t = blockIdx.x + st * G;
+            if (t < ntiles) issue(st, t);
+        }
+    }
+    __syncthreads();
+    for (int64_t i = 0;; ++i) {
+        const int64_t t = blockIdx.x + i * G;
+        if (t >= ntiles) break;
+        const int st = (int)(i % S);
+        const bool landed = mbar_wait(&full[st], (uint32_t)((i / S) & 1));
+        const int64_t tile0 = t * TILE, tile1 = min(tile0 + TILE, n);
+        const int64_t r0 = tile0 + (int64_t)threadIdx.x * E;
+        const bool ragged = tile0 + TILE > n;
+        const bool needL = t > 0, needR = tile1 < n;
+        const T* S0 = ring + (int64_t)(st * NA) * STAGE;  // [left halo | tile | right halo]
+        T s[E], v[E][C];
+        typename P::Aux aux;
+        if (!landed) {  // reported at the block scan's first barrier
+#pragma unroll
+            for (int k = 0; k < E; ++k) {
+                s[k] = T(0);
+#pragma unroll
+                for (int c = 0; c < C; ++c) v[k][c] = T(0);
+            }
+        } else if (!ragged) {
+#pragma unroll
+            for (int k = 0; k < E; k += VN) ld16<T>(S0 + H + threadIdx.x * E + k, &s[k]);
+            T xin[NIN][E];
+#pragma unroll
+            for (int a = 0; a < NIN; ++a)
+#pragma unroll
+                for (int k = 0; k < E; k += VN) ld16<T>(S0 + (a + 1) * STAGE + H + threadIdx.x * E + k, &xin[a][k]);
+#pragma unroll
+            for (int k = 0; k < E; ++k) {
+                T xe[NIN];
+#pragma unroll
+                for (int a = 0; a < NIN; ++a) xe[a] = xin[a][k];
+                p.value(xe, v[k]);
+            }
+        } else {
+            p.load(r0, s, v, aux);
+        }
+        // halo term of this thread and the span checks; the edge anchors
+        T hv[C], ringL = T(0), ringR = T(0);
+        int bad[2] = {0, 0};
+#pragma unroll
+        for (int c = 0; c < C; ++c) hv[c] = T(0);
+        {
+            const int q = (int)threadIdx.x;
+            const bool haveR = tile0 + TILE + H <= n;
+            if (H > 0 && landed && !ragged) {
+                if (needL) ringL = S0[H - 1];
+                if (haveR) ringR = S0[H + TILE];
+            }
+            if (H == 0 || ragged) {
+                if (q == 0) bad[0] = (needL || needR) ? 1 : 0;
+            } else if (q < 2 * H && landed) {
+                const bool left = q < H;
+                const bool need = left ? needL : needR;
+                if (need && !left && !haveR) {
+                    if (q == H) bad[1] = 1;
+                } else if (need) {
+                    const int j = left ? q : (int)(H + TILE) + (q - H);  // ring index
+                    const T edge = left ? ringL : ringR;
+                    const T sj = S0[j];
+                    T xe[NIN], vj[C];
+#pragma unroll
+                    for (int a = 0; a < NIN; ++a) xe[a] = S0[(a + 1) * STAGE + j];
+                    p.value(xe, vj);
+                    const Decay<T, C, CT> d = left ? Decay<T, C, CT>(sj, edge) : Decay<T, C, CT>(edge, sj);
+#pragma unroll
+                    for (int c = 0; c < C; ++c) hv[c] = d[c] * vj[c];
+                    if (q == 0) bad[0] = edge - sj >= TPCut<T>::v ? 0 : 1;
+                    if (q == H) bad[1] = S0[2 * H + TILE - 1] - edge >= TPCut<T>::v ? 0 : 1;
+                }
+            }
+        }
+        // this thread's reads of stage st are ordered before the TMA writes
+        // that refill it, issued after the block scan's barriers
+        fence_proxy_async();
+        T dl[E], fV[C], bW[C];
+        chunk_aggregates<T, C, E, CT>(s, v, dl, fV, bW);
+        bool hf, hb;
+        T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
+        int nbad[2];
+        T hL[C], hU[C];
+        if (block_excl_both_counted<T, C, NT, CT, true, 2, (H > 0 ? H / 32 : 0), C>(
+                s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW, bad, nbad, !landed, sm2, hv,
+                hL, hU)) {
+            // a copy never completed: report, let the copies in flight land, stop
+            if (threadIdx.x == 0) {
+                set_status(status, ST_TIMEOUT);
+                for (int k = 0; k < S; ++k) {
+                    const int64_t t2 = blockIdx.x + (i + k) * G;
+                    if (t2 < ntiles) mbar_wait(&full[(i + k) % S], (uint32_t)(((i + k) / S) & 1));
+                }
+            }
+            return;
+        }
+        const bool out = nbad[0] == 0 && nbad[1] == 0;
+        if (threadIdx.x == 0) {
+            const int64_t t2 = t + S * G;
+            if (t2 < ntiles) issue(st, t2);
+            W.tfirst[t] = tf;
+            W.tlast[t] = te;
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                W.fagg[t * C + c] = tV[c];
+                W.bagg[t * C + c] = tW[c];
+            }
+            if (!out) W.redo[atomicAdd(W.redo_count, 1u)] = (int32_t)t;
+        }
+        if (!out) continue;
+        T eT = hf ? pe : s[0], fT = hb ? nf : s[E - 1], Lc[C], Uc[C];
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            W.fagg[t * C + c] = tV[c];
-            W.bagg[t * C + c] = tW[c];
+            Lc[c] = needL ? hL[c] : T(0);
+            Uc[c] = needR ? hU[c] : T(0);
         }
-        W.st[t].head = cnt_head;
-        W.st[t].tail = cnt_tail;
+        if (needL) eT = ringL;
+        if (needR) fT = ringR;
+        T eprev, Lprev[C], enext, Unext[C];
+        apply_carry_fwd<T, C, CT>(hf, pe, pV, eT, Lc, eprev, Lprev);
+        apply_carry_bwd<T, C, CT>(hb, nf, nW, fT, Uc, enext, Unext);
+        p.finish(r0, s, v, dl, eprev, Lprev, enext, Unext, aux);
     }
 }
 
@@ -194,6 +440,7 @@ __device__ __forceinline__ void tp_segment(const TPWs<T, C>& W, int64_t t0, int6
 
 template <typename T, int C, int CT>
 __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_blocks(TPWs<T, C> W, int64_t ntiles) {
+    if (W.redo_count != nullptr && *(volatile uint32_t*)W.redo_count == 0) return;  // every tile final
     __shared__ BlockScan2Smem<T, C, TP_CARRY_NT> sm2;
     const int64_t t0 = (int64_t)blockIdx.x * TP_CARRY_BT + (int64_t)threadIdx.x * TP_CARRY_PT;
     T fe, fv[C], bf, bv[C];
@@ -215,6 +462,7 @@ __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_blocks(TPWs<T, C> W, i
 template <typename T, int C, int CT>
 __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_tiles(TPWs<T, C> W, int64_t ntiles,
                                                                  int64_t nblocks) {
+    if (W.redo_count != nullptr && *(volatile uint32_t*)W.redo_count == 0) return;  // every tile final
     __shared__ BlockScan2Smem<T, C, TP_CARRY_NT> sm2;
     __shared__ T sh_c[2][C];
     const int64_t bidx = blockIdx.x;
@@ -307,73 +555,26 @@ __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_tiles(TPWs<T, C> W, in
     }
 }
 
-// ------------------------------------------------------------------ pass 3
-// One warp per tile at a time (persistent grid).
-template <class P>
-__global__ void __launch_bounds__(256) k_tp_headtail(P p, TPWs<typename P::T, P::C> W, int64_t ntiles) {
-    using T = typename P::T;
-    constexpr int C = P::C, CT = P::CT;
-    constexpr int64_t TILE = (int64_t)P::NT * P::E;
-    const int lane = threadIdx.x & 31;
-    const int64_t n = p.n;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < ntiles;
-         t += warps) {
-        const int64_t b = t * TILE, e = min(b + TILE, n);
-        const TPStats stt = W.st[t];
-        if (t > 0) {
-            T c[C];
-            bool nz = false;
-#pragma unroll
-            for (int k = 0; k < C; ++k) {
-                c[k] = W.carF[t * C + k];
-                nz |= c[k] != T(0);
-            }
-            if (nz) {
-                const T eT = p.s[b - 1];
-                for (int64_t r = b + lane; r < b + stt.head; r += 32) {
-                    const Decay<T, C, CT> d(eT, p.s[r]);
-                    if (d.e != T(0) || (CT > 0 && d.t != T(0))) p.carry_in(r, d.e, CT > 0 ? d.t : T(0), c, true);
-                }
-            }
-        }
-        __syncwarp();
-        if (t < ntiles - 1) {
-            T c[C];
-            bool nz = false;
-#pragma unroll
-            for (int k = 0; k < C; ++k) {
-                c[k] = W.carB[t * C + k];
-                nz |= c[k] != T(0);
-            }
-            if (nz) {
-                const T fT = p.s[e];
-                for (int64_t r = e - 1 - lane; r >= e - stt.tail; r -= 32) {
-                    const Decay<T, C, CT> d(p.s[r], fT);
-                    if (d.e != T(0) || (CT > 0 && d.t != T(0))) p.carry_in(r, d.e, CT > 0 ? d.t : T(0), c, false);
-                }
-            }
-        }
-        __syncwarp();
-    }
-}
-
 template <class P>
 inline int64_t tp_ntiles(int64_t n) {
     const int64_t tile = (int64_t)P::NT * P::E;
     return std::max<int64_t>(1, (n + tile - 1) / tile);
 }
 
+// Passes 2 and 3 after pass 1 (shared by tp_run and tp_run_ring).
 template <class P>
-cudaError_t tp_run(const P& p, void* ws, size_t ws_bytes, cudaStream_t st) {
+cudaError_t tp_finish(const P& p, TPWs<typename P::T, P::C> W, int64_t ntiles, int sms, cudaStream_t st) {
     using T = typename P::T;
     constexpr int C = P::C, CT = P::CT;
-    if (p.n == 0) return cudaSuccess;
-    const int64_t ntiles = tp_ntiles<P>(p.n);
     const int64_t nb = (ntiles + TP_CARRY_BT - 1) / TP_CARRY_BT;
-    Carve cv(ws, ws_bytes);
-    TPWs<T, C> W = tp_carve<T, C>(cv, ntiles);
-    if (!cv.ok) return cudaErrorInvalidValue;
+    k_tp_carry_blocks<T, C, CT><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles);
+    k_tp_carry_tiles<T, C, CT><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles, nb);
+    const int64_t rb = std::max<int64_t>(1, std::min<int64_t>(ntiles, (int64_t)sms * 4));
+    k_tp_redo<P><<<(unsigned)rb, P::NT, 0, st>>>(p, W, ntiles);
+    return cudaGetLastError();
+}
+
+inline cudaError_t tp_sm_count(int& sms) {
     static int sms_cache[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -383,14 +584,64 @@ cudaError_t tp_run(const P& p, void* ws, size_t ws_bytes, cudaStream_t st) {
         e = cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
     }
+    sms = sms_cache[dev];
+    return cudaSuccess;
+}
+
+// The streamed pass 1 (k_tp_ring) for inputs in sorted order, then passes 2-3.
+template <class P>
+cudaError_t tp_run_ring(const P& p, void* ws, size_t ws_bytes, uint32_t* status, cudaStream_t st) {
+    using T = typename P::T;
+    constexpr int C = P::C;
+    if (p.n == 0) return cudaSuccess;
+    const int64_t ntiles = tp_ntiles<P>(p.n);
+    Carve cv(ws, ws_bytes);
+    TPWs<T, C> W = tp_carve<T, C>(cv, ntiles);
+    if (!cv.ok) return cudaErrorInvalidValue;
+    int sms = 0;
+    cudaError_t e = tp_sm_count(sms);
+    if (e != cudaSuccess) return e;
+    constexpr size_t smem = (size_t)P::S * (P::NIN + 1) * ((size_t)P::NT * P::E + 2 * P::H) * sizeof(T);
+    static int per_sm = 0;  // resident blocks per SM (same on every device of one kind)
+    if (per_sm == 0) {
+        e = cudaFuncSetAttribute(k_tp_ring<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        int per = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_tp_ring<P>, P::NT, smem);
+        if (e != cudaSuccess) return e;
+        per_sm = std::max(1, per);
+    }
+    const int64_t grid = std::min<int64_t>(ntiles, (int64_t)per_sm * sms);
+    e = cudaMemsetAsync(W.redo_count, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess) return e;
     profile_before(st);
-    k_tp_local<P><<<(unsigned)ntiles, P::NT, 0, st>>>(p, W);
+    k_tp_ring<P><<<(unsigned)grid, P::NT, smem, st>>>(p, W, ntiles, status);
     profile_after(st);
-    k_tp_carry_blocks<T, C, CT><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles);
-    k_tp_carry_tiles<T, C, CT><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles, nb);
-    const int64_t htb = std::max<int64_t>(1, std::min<int64_t>((ntiles + 7) / 8, (int64_t)sms_cache[dev] * 8));
-    k_tp_headtail<P><<<(unsigned)htb, 256, 0, st>>>(p, W, ntiles);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return tp_finish(p, W, ntiles, sms, st);
+}
+
+template <class P>
+cudaError_t tp_run(const P& p, void* ws, size_t ws_bytes, cudaStream_t st) {
+    using T = typename P::T;
+    constexpr int C = P::C;
+    if (p.n == 0) return cudaSuccess;
+    const int64_t ntiles = tp_ntiles<P>(p.n);
+    Carve cv(ws, ws_bytes);
+    TPWs<T, C> W = tp_carve<T, C>(cv, ntiles);
+    if (!cv.ok) return cudaErrorInvalidValue;
+    int sms = 0;
+    cudaError_t e = tp_sm_count(sms);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(W.redo_count, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess) return e;
+    profile_before(st);
+    k_tp_local<P><<<(unsigned)ntiles, P::NT, 0, st>>>(p, W, ntiles);
+    profile_after(st);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return tp_finish(p, W, ntiles, sms, st);
 }
 
 }  // namespace lx

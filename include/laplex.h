@@ -104,8 +104,8 @@ laplex_status laplex_workspace_init(void* ws, size_t ws_bytes, void* stream);
 laplex_status laplex_get_device_status(void* ws, void* stream);
 
 /*
- * Sort the anchors ("after sorting the anchors", summary §2.2; the O(n log n)
- * term of the method, §2.2 and §3).
+ * Sort the anchors (the recurrences run over them in sorted order, summary
+ * §2.2; the O(n log n) term of the method, §2.2 and §3).
  *   a      [n]   caller's anchors (read only).
  *   sorted [n]   out: the anchors ascending.  -0.0 is stored as +0.0.
  *   perm   [n]   out: int32, sorted[r] == a[perm[r]] (numerically); ties in
@@ -158,8 +158,9 @@ laplex_status laplex_matvec_phased(const void* sa, const int32_t* pa, const void
                                    laplex_dtype dtype, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Gram operator z = K^T diag(D) K v (summary §2.2 "Operatori di Gram"; abstract:
- * "an efficient Gram operator"), as two chained products through the workspace.
+ * Gram operator z = K^T diag(D) K v (summary §2.2 "Operatori di Gram"; the
+ * abstract lists a fast Gram operator), as two chained products through the
+ * workspace.
  *   phi == NULL: unphased K; otherwise the phased K (psi used when sb != NULL).
  *   sb == NULL: symmetric (b = a): v, z [n, B], D [n] or NULL (D = 1).
  *   sb != NULL: v, z [k, B] on the b side, D [n] on the a side or NULL.

@@ -65,7 +65,7 @@ def _cols(x):
 
 
 # ---------------------------------------------------------------------------
-# sort (the O(n log n) step: "after sorting the anchors", summary §2.2)
+# sort (the O(n log n) step; the recurrences run in sorted order, summary §2.2)
 # ---------------------------------------------------------------------------
 
 def stable_sort(a):

@@ -81,3 +81,32 @@ def test_c5_full_size_sampled():
     assert_close(dx[idx], kg, ng, np.float32, "C5 dx")
     da_ref = -(g[idx] * sx + x[idx] * sg)
     assert_close(da[idx], da_ref, np.abs(g[idx]) * nx + np.abs(x[idx]) * ng, np.float32, "C5 da")
+
+
+@pytest.mark.parametrize("case", ["span_below_cut", "span_above_cut", "mixed_ties", "short_right"])
+def test_halo_carries(case):
+    """Streamed tiles (inputs in sorted order) whose carries come from the halos
+    of 256 elements, next to tiles that fall back to the carry kernels: spacing
+    0.40 spans 102 < 104 (fall back), 0.41 spans 104.55 (halo carries), runs of
+    equal anchors inside the halos, and a last-but-one tile without room for
+    a right halo."""
+    rng = np.random.default_rng(21)
+    tile = 256 * 8
+    n = 11 * tile + 77
+    if case == "span_below_cut":
+        a = np.arange(n) * 0.40
+    elif case == "span_above_cut":
+        a = np.arange(n) * 0.41
+    elif case == "mixed_ties":
+        # groups of equal anchors 3 apart, a dense stretch, then unit spacing
+        k = n // 3
+        a = np.concatenate([3.0 * np.repeat(np.arange(k // 8 + 1), 8)[:k],
+                            3.0 * (k // 8 + 2) + np.sort(rng.uniform(0, 5, k)),
+                            3.0 * (k // 8 + 2) + 10 + np.arange(n - 2 * k)])
+    else:
+        n = 9 * tile + 100
+        a = rng.uniform(0, n, n)
+    a = a.astype(np.float32)
+    x = rng.normal(size=n).astype(np.float32)
+    g = rng.normal(size=n).astype(np.float32)
+    check(a, x, g, np.float32, case)

@@ -123,3 +123,52 @@ def test_deep_lookahead_fixup(dtype):
     assert_close(run_sym(a, x, True), O.sym(a, x), O.norm_sym(a, x), dtype, "dense")
     xb = rng.normal(size=(n, 3)).astype(dtype)
     assert_close(run_sym(a, xb, True), O.sym(a, xb), O.norm_sym(a, xb), dtype, "dense B=3")
+
+
+TILE_F32 = 512 * 12  # elements per tile of the single-column fp32 product
+
+
+def _spaced(n, spacing, seed, jitter=0.0):
+    rng = np.random.default_rng(seed)
+    a = np.arange(n) * spacing + rng.uniform(0, jitter, n) if jitter else np.arange(n) * spacing
+    return np.sort(a).astype(np.float32), rng.normal(size=n).astype(np.float32)
+
+
+@pytest.mark.parametrize("use_perm", [False, True])
+@pytest.mark.parametrize("case", ["unit", "span_below_cut", "span_above_cut", "mixed", "far",
+                                  "aligned", "short_right"])
+def test_halo_carries(case, use_perm):
+    """Tiles whose carries come from the halos (sparse anchors: a halo of 256
+    spans at least 104 units) and tiles that fall back to the carry kernels
+    (denser), side by side.  Constant spacing 0.40 gives a halo span of 102
+    (< 104: fall back), 0.41 gives 104.55 (exact halo carries)."""
+    n = 7 * TILE_F32 + 1234
+    if case == "unit":
+        a, x = synth.sym_uniform(n, 0.0, float(n), seed=3)
+    elif case == "span_below_cut":
+        a, x = _spaced(n, 0.40, seed=4)
+    elif case == "span_above_cut":
+        a, x = _spaced(n, 0.41, seed=5)
+    elif case == "mixed":
+        # alternating sparse and dense stretches, with jumps between them
+        rng = np.random.default_rng(6)
+        parts, lo = [], 0.0
+        for k in range(9):
+            m = 3000 + 1500 * k
+            dens = (0.05, 1.0, 2.5, 0.3)[k % 4]
+            parts.append(lo + np.sort(rng.uniform(0, m * dens, m)))
+            lo += m * dens + (0.0 if k % 3 else 50.0)
+        a = np.concatenate(parts).astype(np.float32)
+        n = a.size
+        x = rng.normal(size=n).astype(np.float32)
+    elif case == "far":
+        a, x = _spaced(n, 150.0, seed=7)
+    elif case == "aligned":
+        n = 5 * TILE_F32
+        a, x = synth.sym_uniform(n, 0.0, float(n), seed=8)
+    else:  # the tile before the ragged last one has no room for a right halo
+        n = 6 * TILE_F32 + 100
+        a, x = synth.sym_uniform(n, 0.0, float(n), seed=9)
+    y_ref = O.sym(a, x)
+    norm = O.norm_sym(a, x)
+    assert_close(run_sym(a, x, use_perm), y_ref, norm, np.float32, f"{case} perm={use_perm}")
