@@ -278,7 +278,7 @@ def run_ours(args):
     value = world * n / (ms_step * 1e-3) / 1e9
     hbm, peak_kind = peaks()
     achieved = BYTES_PER_ELEM_SYM * n / (kernel_ms * 1e-3) / 1e9
-    sha = src_sha("sym_stream.cu", "scan_core.cuh", "common.cuh")
+    sha = src_sha("sym_stream.cu", "scan_core.cuh", "common.cuh", "bulk.cuh")
     traffic = traffic_from_profile("k_tile_local_presorted_b1", sha, n)
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "traffic": traffic,
@@ -337,10 +337,10 @@ def run_ours(args):
         torch.cuda.empty_cache()
 
     # ---------------- the other workloads (inputs near or below L2 size: flushed)
-    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_buf = torch.ones(64 << 20, dtype=torch.float32, device=dev)  # 256 MB
 
     def timed_flush(fn, steps):
-        """Sum of per-call device times, the 126 MB L2 flushed (256 MB write)
+        """Sum of per-call device times, the 126 MB L2 flushed (a 256 MB read)
         before every call and outside the timed events.  A spin kernel queued
         first keeps the device behind the host, so the events time the call's
         kernels and not the host's launch latency."""
@@ -349,7 +349,7 @@ def run_ours(args):
         evs = []
         for _ in range(steps):
             torch.cuda._sleep(1_000_000)
-            flush_buf.zero_()
+            flush_buf.sum()  # read: leaves L2 holding clean lines of another buffer
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)

@@ -28,11 +28,11 @@ template <typename T_, int E_>
 struct BwdTP {
     using T = T_;
     static constexpr int C = 4, CT = 2, E = E_, NT = BWD_NT;
-    // halos of 128 (fp32: they span CUT = 104 at spacings above 0.82; fp64,
+    // halos of 128 (fp32: they span CUT = 88 at spacings above 0.7; fp64,
     // CUT = 746, would need several times more: none).  Streamed pass 1
     // (inputs in sorted order): s, x, g in a 2-stage ring.
     static constexpr int H = sizeof(T_) == 4 ? 128 : 0;
-    static constexpr int NIN = 2, S = 2, MINB = 2;
+    static constexpr int NIN = 2, S = 2, MINB = 3;
     int64_t n;
     const T* s;
     const int32_t* perm;

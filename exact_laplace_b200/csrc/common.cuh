@@ -10,10 +10,26 @@ namespace lx {
 constexpr unsigned FULL = 0xffffffffu;
 
 template <typename T> __device__ __forceinline__ T dexp(T v);
-// fp32: the hardware exp2 path (__expf).  A decay exp(d) with d <= 0 only ever
-// multiplies an already-summed value, and terms below FLT_MIN are flushed.
-template <> __device__ __forceinline__ float dexp<float>(float v) { return __expf(v); }
+// fp32: exp(v) = 2^(v log2 e) on the hardware base-2 exponential in
+// flush-to-zero mode (ex2.approx.ftz: relative error about 2^-22; a result
+// below FLT_MIN is 0).  Every factor of the scans is at most 1 and at least
+// the kernel value exp(-|a_i - b_j|) of each term it carries, so a term whose
+// kernel value is >= FLT_MIN is never flushed; only terms below FLT_MIN can
+// be lost (at most their |x|-weighted mass).
+template <> __device__ __forceinline__ float dexp<float>(float v) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v * 1.44269504088896341f));
+    return r;
+}
 template <> __device__ __forceinline__ double dexp<double>(double v) { return exp(v); }
+
+// A distance beyond which dexp(-d) is exactly 0: fp32, 2^(-88 log2 e) =
+// 2^-126.96 < FLT_MIN is flushed (the approximation error of about 2^-22 cannot
+// lift it to FLT_MIN); fp64, exp(-746) rounds to 0 (below the smallest
+// subnormal).  Carries between tiles are cut off there, bit for bit.
+template <typename T> struct ExpCut;
+template <> struct ExpCut<float> { static constexpr float v = 88.0f; };
+template <> struct ExpCut<double> { static constexpr double v = 746.0; };
 
 template <typename T> __device__ __forceinline__ T dfma(T a, T b, T c) { return fma(a, b, c); }
 

@@ -114,8 +114,8 @@ __global__ void __launch_bounds__(NT) k_gen_local(GenArgs<T> A, TPWs<T, PHASED ?
         } else if (takeA) {
             s[e] = Aa[ai];
             aidx[e] = ai;
-            h += (Aa[ai] - first < TPCut<T>::v) ? 1 : 0;
-            q += (padA - Aa[ai] < TPCut<T>::v) ? 1 : 0;
+            h += (Aa[ai] - first < ExpCut<T>::v) ? 1 : 0;
+            q += (padA - Aa[ai] < ExpCut<T>::v) ? 1 : 0;
             ++ai;
 #pragma unroll
             for (int c = 0; c < C; ++c) v[e][c] = T(0);

@@ -321,6 +321,9 @@ __device__ __forceinline__ bool block_excl_both_counted(
     } else {
         __syncthreads();
     }
+    // the serial middle step, split: warp 0 scans the warp totals forward and
+    // sums the counts, warp 1 scans them backward and sums the halo terms
+    constexpr int WB = NW > 1 ? 1 : 0;
     if (w == 0) {
         if (COUNTED) {
 #pragma unroll
@@ -329,6 +332,37 @@ __device__ __forceinline__ bool block_excl_both_counted(
                 if (lane == 0) sm.tcnt[q] = cq;
             }
         }
+        T ge = lane < NW ? sm.fe[lane] : T(0), gV[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) gV[c] = lane < NW ? sm.fV[lane][c] : T(0);
+#pragma unroll
+        for (int off = 1; off < NW; off <<= 1) {
+            const T eo = __shfl_up_sync(FULL, ge, off);
+            T Vo[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) Vo[c] = __shfl_up_sync(FULL, gV[c], off);
+            if (lane >= off && lane < NW) {
+                const Decay<T, C, CT> d(eo, ge);
+#pragma unroll
+                for (int c = 0; c < C; ++c) gV[c] = dfma<T>(d[c], Vo[c], gV[c]);
+            }
+        }
+        const T xe = __shfl_up_sync(FULL, ge, 1);
+        T xV[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) xV[c] = __shfl_up_sync(FULL, gV[c], 1);
+        if (lane > 0 && lane < NW) {
+            sm.pfe[lane] = xe;
+#pragma unroll
+            for (int c = 0; c < C; ++c) sm.pfV[lane][c] = xV[c];
+        }
+        if (lane == NW - 1) {
+            sm.tfe = ge;
+#pragma unroll
+            for (int c = 0; c < C; ++c) sm.tfV[c] = gV[c];
+        }
+    }
+    if (w == WB) {
         if (HW > 0) {
             // fixed order: warp sums added in a butterfly over the first HW
             // lanes (left) and the next HW lanes (right)
@@ -341,56 +375,29 @@ __device__ __forceinline__ bool block_excl_both_counted(
                 if (lane == HW) sm.thU[c] = hs;
             }
         }
-        T ge = lane < NW ? sm.fe[lane] : T(0), gV[C];
         T gf = lane < NW ? sm.be[lane] : T(0), gW[C];
 #pragma unroll
-        for (int c = 0; c < C; ++c) {
-            gV[c] = lane < NW ? sm.fV[lane][c] : T(0);
-            gW[c] = lane < NW ? sm.bV[lane][c] : T(0);
-        }
+        for (int c = 0; c < C; ++c) gW[c] = lane < NW ? sm.bV[lane][c] : T(0);
 #pragma unroll
         for (int off = 1; off < NW; off <<= 1) {
-            const T eo = __shfl_up_sync(FULL, ge, off);
             const T fo = __shfl_down_sync(FULL, gf, off);
-            T Vo[C], Wo[C];
+            T Wo[C];
 #pragma unroll
-            for (int c = 0; c < C; ++c) {
-                Vo[c] = __shfl_up_sync(FULL, gV[c], off);
-                Wo[c] = __shfl_down_sync(FULL, gW[c], off);
-            }
-            if (lane >= off && lane < NW) {
-                const Decay<T, C, CT> d(eo, ge);
-#pragma unroll
-                for (int c = 0; c < C; ++c) gV[c] = dfma<T>(d[c], Vo[c], gV[c]);
-            }
+            for (int c = 0; c < C; ++c) Wo[c] = __shfl_down_sync(FULL, gW[c], off);
             if (lane + off < NW) {
                 const Decay<T, C, CT> d(gf, fo);
 #pragma unroll
                 for (int c = 0; c < C; ++c) gW[c] = dfma<T>(d[c], Wo[c], gW[c]);
             }
         }
-        const T xe = __shfl_up_sync(FULL, ge, 1);
         const T xf = __shfl_down_sync(FULL, gf, 1);
-        T xV[C], xW[C];
+        T xW[C];
 #pragma unroll
-        for (int c = 0; c < C; ++c) {
-            xV[c] = __shfl_up_sync(FULL, gV[c], 1);
-            xW[c] = __shfl_down_sync(FULL, gW[c], 1);
-        }
-        if (lane > 0 && lane < NW) {
-            sm.pfe[lane] = xe;
-#pragma unroll
-            for (int c = 0; c < C; ++c) sm.pfV[lane][c] = xV[c];
-        }
+        for (int c = 0; c < C; ++c) xW[c] = __shfl_down_sync(FULL, gW[c], 1);
         if (lane < NW - 1) {
             sm.pbe[lane] = xf;
 #pragma unroll
             for (int c = 0; c < C; ++c) sm.pbV[lane][c] = xW[c];
-        }
-        if (lane == NW - 1) {
-            sm.tfe = ge;
-#pragma unroll
-            for (int c = 0; c < C; ++c) sm.tfV[c] = gV[c];
         }
         if (lane == 0) {
             sm.tbe = gf;

@@ -11,7 +11,7 @@
 //      of a tile also brings a halo of H elements on each side.  A carry from
 //      outside the tile reaches element r with a factor exp(-d), d >= the
 //      distance from r to the tile's edge anchor, and exp(-d) is exactly 0 for
-//      d >= CUT (fp32: 104, below the smallest subnormal; fp64: 746).  So when
+//      d >= CUT (ExpCut in common.cuh: fp32 88, fp64 746).  So when
 //      a halo spans at least CUT, the carry summed over the halo is the exact
 //      carry, and the tile writes its final outputs.  A tile whose halos do
 //      not span CUT (dense anchors) writes nothing and is listed for pass 3.
@@ -35,16 +35,16 @@ namespace lx {
 // tile shape of k_tile_local (fp32): threads per block, elements per thread,
 // halo per side, resident blocks per SM
 #ifndef LX_LT_NT
-#define LX_LT_NT 512
+#define LX_LT_NT 256
 #endif
 #ifndef LX_LT_E
 #define LX_LT_E 12
 #endif
 #ifndef LX_LT_H
-#define LX_LT_H 256
+#define LX_LT_H 128
 #endif
 #ifndef LX_LT_MINB
-#define LX_LT_MINB 2
+#define LX_LT_MINB 4
 #endif
 constexpr int LT_NT = LX_LT_NT;  // threads per tile block
 constexpr int CARRY_NT = 256;  // threads per carry block
@@ -60,10 +60,6 @@ template <typename T> struct LocalH;
 template <> struct LocalH<float> { static constexpr int H = LX_LT_H; };
 template <> struct LocalH<double> { static constexpr int H = 0; };
 constexpr int LT_STAGES = 2;
-
-template <typename T> struct Cut;
-template <> struct Cut<float> { static constexpr float v = 104.0f; };
-template <> struct Cut<double> { static constexpr double v = 746.0; };
 
 template <typename T>
 struct LocalWs {
@@ -254,8 +250,8 @@ __global__ void __launch_bounds__(NT, LX_LT_MINB) k_tile_local(const T* __restri
                         if constexpr (GATHER) xj = __ldg(x_ + ring_p[st * STAGE + j]);
                         else xj = ring_x[st * STAGE + j];
                         hv = dexp<T>(left ? sj - edge : edge - sj) * xj;
-                        if (q == 0) bad[0] = edge - sj >= Cut<T>::v ? 0 : 1;
-                        if (q == H) bad[1] = S0[2 * H + TILE - 1] - edge >= Cut<T>::v ? 0 : 1;
+                        if (q == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
+                        if (q == H) bad[1] = S0[2 * H + TILE - 1] - edge >= ExpCut<T>::v ? 0 : 1;
                     } else {
                         // no halo: exact only at the array's own ends
                         if (q == 0) bad[0] = t == 0 ? 0 : 1;

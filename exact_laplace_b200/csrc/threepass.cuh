@@ -37,10 +37,6 @@
 
 namespace lx {
 
-template <typename T> struct TPCut;
-template <> struct TPCut<float> { static constexpr float v = 104.0f; };   // exp(-104) == 0 in fp32
-template <> struct TPCut<double> { static constexpr double v = 746.0; };  // exp(-746) == 0 in fp64
-
 struct TPStats {  // reach of a tile (general case: elements within CUT of each edge)
     int32_t head;
     int32_t tail;
@@ -129,8 +125,8 @@ __device__ __forceinline__ void tp_halo_term(const P& p, int64_t t, int64_t tile
     const Decay<T, C, CT> d = left ? Decay<T, C, CT>(sj, edge) : Decay<T, C, CT>(edge, sj);
 #pragma unroll
     for (int c = 0; c < C; ++c) hv[c] = d[c] * vj[c];
-    if (q == 0) bad[0] = edge - sj >= TPCut<T>::v ? 0 : 1;
-    if (q == H) bad[1] = p.s[tile1 + H - 1] - edge >= TPCut<T>::v ? 0 : 1;
+    if (q == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
+    if (q == H) bad[1] = p.s[tile1 + H - 1] - edge >= ExpCut<T>::v ? 0 : 1;
 }
 
 // One tile.  MODE 0: carries from the halos; a tile whose halos fall short is
@@ -346,8 +342,8 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
                     const Decay<T, C, CT> d = left ? Decay<T, C, CT>(sj, edge) : Decay<T, C, CT>(edge, sj);
 #pragma unroll
                     for (int c = 0; c < C; ++c) hv[c] = d[c] * vj[c];
-                    if (q == 0) bad[0] = edge - sj >= TPCut<T>::v ? 0 : 1;
-                    if (q == H) bad[1] = S0[2 * H + TILE - 1] - edge >= TPCut<T>::v ? 0 : 1;
+                    if (q == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
+                    if (q == H) bad[1] = S0[2 * H + TILE - 1] - edge >= ExpCut<T>::v ? 0 : 1;
                 }
             }
         }

@@ -182,3 +182,51 @@ void orc_rows_window(int64_t m, const double* ra, const double* rphi,
         }
     }
 }
+
+/*
+ * One-sided decayed sums at query points (not a step of the method: the mass
+ * of the terms below a threshold, used by the parity criterion of fp32
+ * results).  For anchors sb (ascending, k of them) with values v [k, B] and
+ * query points q (ascending, m of them):
+ *     dir > 0:  out_i = sum_{j: sb_j < q_i} exp(sb_j - q_i) v_j
+ *     dir < 0:  out_i = sum_{j: sb_j > q_i} exp(q_i - sb_j) v_j
+ * by one sweep over the merged order: the running sum at the last anchor
+ * passed, decayed to the query.
+ */
+void orc_onesided_sorted(int64_t k, int64_t m, int64_t B, const double* sb, const double* v,
+                         const double* q, int dir, double* out)
+{
+    double* acc = (double*)calloc((size_t)B, sizeof(double));
+    if (dir > 0) {
+        int64_t j = 0;
+        double last = 0.0;
+        int any = 0;
+        for (int64_t i = 0; i < m; ++i) {
+            while (j < k && sb[j] < q[i]) {
+                const double f = any ? exp(last - sb[j]) : 0.0;
+                for (int64_t c = 0; c < B; ++c) acc[c] = v[j * B + c] + f * acc[c];
+                last = sb[j];
+                any = 1;
+                ++j;
+            }
+            const double f = any ? exp(last - q[i]) : 0.0;
+            for (int64_t c = 0; c < B; ++c) out[i * B + c] = f * acc[c];
+        }
+    } else {
+        int64_t j = k - 1;
+        double last = 0.0;
+        int any = 0;
+        for (int64_t i = m - 1; i >= 0; --i) {
+            while (j >= 0 && sb[j] > q[i]) {
+                const double f = any ? exp(sb[j] - last) : 0.0;
+                for (int64_t c = 0; c < B; ++c) acc[c] = v[j * B + c] + f * acc[c];
+                last = sb[j];
+                any = 1;
+                --j;
+            }
+            const double f = any ? exp(q[i] - last) : 0.0;
+            for (int64_t c = 0; c < B; ++c) out[i * B + c] = f * acc[c];
+        }
+    }
+    free(acc);
+}

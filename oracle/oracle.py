@@ -34,6 +34,10 @@ _I64 = ctypes.c_int64
 #: >= 746 are exactly zero in an fp64 evaluation of the definition.
 CUTOFF_F64 = 746.0
 
+#: -ln(FLT_MIN) = 126 ln 2: a kernel value exp(-d) is below the smallest normal
+#: fp32 number exactly when d > FAR_F32.
+FAR_F32 = 126.0 * float(np.log(2.0))
+
 
 def _L():
     global _lib
@@ -44,8 +48,9 @@ def _L():
         lib.orc_signed_sorted.argtypes = [_I64, _I64, _D, _D, _D]
         lib.orc_rows_window.argtypes = [_I64, _D, _D, _I64, _I64, _D, _D, _D, ctypes.c_double,
                                         _D, _D, _D]
+        lib.orc_onesided_sorted.argtypes = [_I64, _I64, _I64, _D, _D, _D, ctypes.c_int, _D]
         for f in (lib.orc_sym_sorted, lib.orc_general_sorted, lib.orc_signed_sorted,
-                  lib.orc_rows_window):
+                  lib.orc_rows_window, lib.orc_onesided_sorted):
             f.restype = None
         _lib = lib
     return _lib
@@ -266,6 +271,32 @@ def norm_backward(a, x, g):
     x, g = np.abs(_f64(x)), np.abs(_f64(g))
     kx, kg = sym(a, x), sym(a, g)
     return kg, g * kx + x * kg
+
+
+def far_mass(a, v, b=None, dist=FAR_F32):
+    """m_i = sum over j with |a_i - b_j| > dist of exp(-|a_i - b_j|) |v_j|
+    (b = a when None): the |v|-weighted mass of the terms whose kernel value is
+    below exp(-dist) (FLT_MIN for the default).  Not a step of the method: the
+    parity criterion of fp32 results allows terms below FLT_MIN to be lost.
+    Computed as exp(-dist) times one-sided decayed sums at the shifted points
+    a_i - dist and a_i + dist (strict inequalities)."""
+    a = _f64(a)
+    b = a if b is None else _f64(b)
+    v, one = _cols(np.abs(_f64(v)))
+    B = v.shape[1]
+    ob = np.argsort(b, kind="stable")
+    sb = np.ascontiguousarray(b[ob])
+    vs = np.ascontiguousarray(v[ob])
+    out = np.zeros((a.size, B))
+    for dirn, shift in ((1, -dist), (-1, dist)):
+        q = a + shift
+        oq = np.argsort(q, kind="stable")
+        qs = np.ascontiguousarray(q[oq])
+        r = np.zeros((a.size, B))
+        _L().orc_onesided_sorted(sb.size, qs.size, B, _p(sb), _p(vs), _p(qs), dirn, _p(r))
+        out[oq] += r
+    out *= np.exp(-dist)
+    return out[:, 0] if one else out
 
 
 def max_norm_err(y, y_ref, norm):

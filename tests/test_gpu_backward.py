@@ -29,10 +29,12 @@ def run_bwd(a, x, g, use_perm=True):
 def check(a, x, g, dtype, what):
     rdx, rda = O.backward(a, x, g)
     ndx, nda = O.norm_backward(a, x, g)
+    mx, mg = O.far_mass(a, x), O.far_mass(a, g)
+    sda = np.abs(g) * mx + np.abs(x) * mg
     for use_perm in (True, False):
         dx, da = run_bwd(a, x, g, use_perm)
-        assert_close(dx, rdx, ndx, dtype, f"{what} dx perm={use_perm}")
-        assert_close(da, rda, nda, dtype, f"{what} da perm={use_perm}")
+        assert_close(dx, rdx, ndx, dtype, f"{what} dx perm={use_perm}", mg)
+        assert_close(da, rda, nda, dtype, f"{what} da perm={use_perm}", sda)
 
 
 @pytest.mark.parametrize("dtype", [np.float32, np.float64])
@@ -83,20 +85,18 @@ def test_c5_full_size_sampled():
     assert_close(da[idx], da_ref, np.abs(g[idx]) * nx + np.abs(x[idx]) * ng, np.float32, "C5 da")
 
 
-@pytest.mark.parametrize("case", ["span_below_cut", "span_above_cut", "mixed_ties", "short_right"])
+@pytest.mark.parametrize("case", ["spacing_0.69", "spacing_0.70", "spacing_1.0", "mixed_ties", "short_right"])
 def test_halo_carries(case):
-    """Streamed tiles (inputs in sorted order) whose carries come from the halos
-    of 256 elements, next to tiles that fall back to the carry kernels: spacing
-    0.40 spans 102 < 104 (fall back), 0.41 spans 104.55 (halo carries), runs of
-    equal anchors inside the halos, and a last-but-one tile without room for
-    a right halo."""
+    """Tiles whose carries come from the halos of 128 elements, next to tiles
+    that fall back to the carry kernels and the redo pass: spacing 0.69 spans
+    87.6 < 88 (fall back), 0.70 spans 88.9 (halo carries); runs of equal
+    anchors inside the halos; a last-but-one tile without room for a right
+    halo."""
     rng = np.random.default_rng(21)
     tile = 256 * 8
     n = 11 * tile + 77
-    if case == "span_below_cut":
-        a = np.arange(n) * 0.40
-    elif case == "span_above_cut":
-        a = np.arange(n) * 0.41
+    if case.startswith("spacing_"):
+        a = np.arange(n) * float(case.split("_")[1])
     elif case == "mixed_ties":
         # groups of equal anchors 3 apart, a dense stretch, then unit spacing
         k = n // 3

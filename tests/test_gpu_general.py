@@ -29,12 +29,13 @@ def run_general(a, b, x, transpose=False, use_perm=True):
 
 def check(a, b, x, w, dtype, what):
     y_ref = O.general(a, b, x)
-    assert_close(run_general(a, b, x), y_ref, O.norm_general(a, b, x), dtype, what + " Kx")
+    my = O.far_mass(a, x, b)
+    assert_close(run_general(a, b, x), y_ref, O.norm_general(a, b, x), dtype, what + " Kx", my)
     assert_close(run_general(a, b, x, use_perm=False), y_ref, O.norm_general(a, b, x), dtype,
-                 what + " Kx sorted")
+                 what + " Kx sorted", my)
     z_ref = O.general_T(a, b, w)
     assert_close(run_general(a, b, w, transpose=True), z_ref, O.norm_general(b, a, w), dtype,
-                 what + " K^T w")
+                 what + " K^T w", O.far_mass(b, w, a))
 
 
 @pytest.mark.parametrize("dtype", [np.float32, np.float64])

@@ -54,10 +54,12 @@ def test_phased_general_and_transpose(dtype):
     sb, pb = O.stable_sort(b)
     y = host(X.matvec_phased(dev(sa.astype(dtype)), dev(phi), dev(x), pa=_i32(pa),
                              sb=dev(sb.astype(dtype)), psi=dev(psi), pb=_i32(pb)))
-    assert_close(y, O.phased(a, phi, x, b, psi), O.norm_general(a, b, x), dtype, "K x")
+    assert_close(y, O.phased(a, phi, x, b, psi), O.norm_general(a, b, x), dtype, "K x",
+                 O.far_mass(a, x, b))
     z = host(X.matvec_phased(dev(sa.astype(dtype)), dev(phi), dev(w), pa=_i32(pa),
                              sb=dev(sb.astype(dtype)), psi=dev(psi), pb=_i32(pb), transpose=True))
-    assert_close(z, O.phased_T(a, phi, w, b, psi), O.norm_general(b, a, w), dtype, "K^T w")
+    assert_close(z, O.phased_T(a, phi, w, b, psi), O.norm_general(b, a, w), dtype, "K^T w",
+                 O.far_mass(b, w, a))
 
 
 @pytest.mark.parametrize("dtype", [np.float32, np.float64])

@@ -125,7 +125,8 @@ def test_deep_lookahead_fixup(dtype):
     assert_close(run_sym(a, xb, True), O.sym(a, xb), O.norm_sym(a, xb), dtype, "dense B=3")
 
 
-TILE_F32 = 512 * 12  # elements per tile of the single-column fp32 product
+TILE_F32 = 256 * 12  # elements per tile of the single-column fp32 product
+HALO_SPACINGS = [0.30, 0.345, 0.35, 0.40, 0.69, 0.70, 1.0]
 
 
 def _spaced(n, spacing, seed, jitter=0.0):
@@ -135,20 +136,26 @@ def _spaced(n, spacing, seed, jitter=0.0):
 
 
 @pytest.mark.parametrize("use_perm", [False, True])
-@pytest.mark.parametrize("case", ["unit", "span_below_cut", "span_above_cut", "mixed", "far",
-                                  "aligned", "short_right"])
+@pytest.mark.parametrize("spacing", HALO_SPACINGS)
+def test_halo_span_boundary(spacing, use_perm):
+    """Constant anchor spacing around the point where a halo of 128 (or 256)
+    elements spans the cut of 88: 127 x 0.69 = 87.6 falls back to the carry
+    kernels, 127 x 0.70 = 88.9 takes the halo carries (255 x 0.345 = 88.0 and
+    255 x 0.35 = 89.3 for halos of 256)."""
+    n = 9 * TILE_F32 + 1234
+    a, x = _spaced(n, spacing, seed=int(spacing * 1000))
+    assert_close(run_sym(a, x, use_perm), O.sym(a, x), O.norm_sym(a, x), np.float32,
+                 f"spacing {spacing} perm={use_perm}")
+
+
+@pytest.mark.parametrize("use_perm", [False, True])
+@pytest.mark.parametrize("case", ["unit", "mixed", "far", "aligned", "short_right"])
 def test_halo_carries(case, use_perm):
-    """Tiles whose carries come from the halos (sparse anchors: a halo of 256
-    spans at least 104 units) and tiles that fall back to the carry kernels
-    (denser), side by side.  Constant spacing 0.40 gives a halo span of 102
-    (< 104: fall back), 0.41 gives 104.55 (exact halo carries)."""
+    """Tiles whose carries come from the halos (sparse anchors) and tiles that
+    fall back to the carry kernels and the redo pass (denser), side by side."""
     n = 7 * TILE_F32 + 1234
     if case == "unit":
         a, x = synth.sym_uniform(n, 0.0, float(n), seed=3)
-    elif case == "span_below_cut":
-        a, x = _spaced(n, 0.40, seed=4)
-    elif case == "span_above_cut":
-        a, x = _spaced(n, 0.41, seed=5)
     elif case == "mixed":
         # alternating sparse and dense stretches, with jumps between them
         rng = np.random.default_rng(6)

@@ -333,6 +333,56 @@ def test_signed_sums_brute_force():
 
 
 # ---------------------------------------------------------------------------
+# the mass of the terms below a threshold (parity slack of fp32 results)
+# ---------------------------------------------------------------------------
+
+def _far_brute(a, b, v, dist):
+    out = np.zeros((len(a),) + v.shape[1:])
+    for i in range(len(a)):
+        for j in range(len(b)):
+            d = abs(a[i] - b[j])
+            if d > dist:
+                out[i] += math.exp(-d) * np.abs(v[j])
+    return out
+
+
+@pytest.mark.parametrize("dist", [0.0, 0.75, 2.5, 1e9])
+def test_far_mass_brute_force(dist):
+    """far_mass against the double loop, strict inequality included: b_4 sits
+    exactly dist to the right of a_5 and b_9 exactly dist to the left of a_2."""
+    rng = np.random.default_rng(16)
+    a = np.round(rng.uniform(0, 8, 25), 2)
+    b = np.round(rng.uniform(-1, 9, 17), 2)
+    if dist < 1e6:
+        b[4] = a[5] + dist
+        b[9] = a[2] - dist
+    for v in (rng.normal(size=17), rng.normal(size=(17, 3))):
+        np.testing.assert_allclose(O.far_mass(a, v, b, dist), _far_brute(a, b, v, dist), rtol=1e-12,
+                                   atol=1e-300)
+    # symmetric form (b = a), with ties
+    a2 = np.round(rng.uniform(0, 5, 30), 0)
+    v2 = rng.normal(size=30)
+    np.testing.assert_allclose(O.far_mass(a2, v2, dist=dist), _far_brute(a2, a2, v2, dist), rtol=1e-12,
+                               atol=1e-300)
+
+
+def test_far_mass_limits():
+    """dist = 0 on distinct anchors keeps every term: K|v| by the general-case
+    route; dist beyond the spread keeps none; the default threshold is the
+    point where exp(-d) crosses the smallest normal fp32 number."""
+    rng = np.random.default_rng(17)
+    a = rng.uniform(0, 10, 40)
+    b = rng.uniform(0, 10, 33) + 0.001
+    v = rng.normal(size=33)
+    np.testing.assert_allclose(O.far_mass(a, v, b, 0.0), O.general(a, b, np.abs(v)), rtol=1e-12)
+    assert np.all(O.far_mass(a, v, b, 50.0) == 0.0)
+    assert math.exp(-O.FAR_F32) == pytest.approx(float(np.finfo(np.float32).tiny), rel=1e-13)
+    # two anchors 90 apart: each sees the other's term, below FLT_MIN
+    m = O.far_mass(np.array([0.0, 90.0]), np.array([2.0, -3.0]))
+    np.testing.assert_allclose(m, [3.0 * math.exp(-90.0), 2.0 * math.exp(-90.0)], rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------
 # the pins catch planted mistakes (mutants built on the CPU from the oracle)
 # ---------------------------------------------------------------------------
 
