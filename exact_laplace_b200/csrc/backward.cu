@@ -28,10 +28,11 @@ template <typename T_, int E_>
 struct BwdTP {
     using T = T_;
     static constexpr int C = 4, CT = 2, E = E_, NT = BWD_NT;
-    // halos of 128 (fp32: they span CUT = 88 at spacings above 0.7; fp64,
-    // CUT = 746, would need several times more: none).  Streamed pass 1
-    // (inputs in sorted order): s, x, g in a 2-stage ring.
-    static constexpr int H = sizeof(T_) == 4 ? 128 : 0;
+    // halos of 192 (fp32: they span CUT = 88 at spacings above 0.47, and
+    // across runs of up to 64 equal anchors; fp64, CUT = 746, would need
+    // several times more: none).  Streamed pass 1 (inputs in sorted order):
+    // s, x, g in a 2-stage ring.
+    static constexpr int H = sizeof(T_) == 4 ? 192 : 0;
     static constexpr int NIN = 2, S = 2, MINB = 3;
     int64_t n;
     const T* s;

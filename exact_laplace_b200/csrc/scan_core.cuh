@@ -261,25 +261,30 @@ struct BlockScan2Smem {
     T tfV[C], tbV[C];
     int wcnt[NW][4];  // per-warp sums of integer counts (block_excl_both_counted)
     int tcnt[4];
-    T whs[NW][C];     // per-warp halo sums (one per channel), and their two totals
-    T thL[C], thU[C];
+    T whL[NW][C];     // per-warp halo sums (left, right; one per channel)
+    T whU[NW][C];
+    T thL[C], thU[C]; // and their totals
 };
 
 // block_excl_both_counted: the two scans; it also sums NI <= 4 integer counts
 // over the block (cnt in, tot out, read by every thread) and ORs a flag: if any
 // thread passes bad, the function returns true right after its first barrier,
 // in every thread, with the outputs unset.  COUNTED = false drops the counts
-// and the flag.  HW > 0 also sums HC <= C values hv per thread into two
-// totals: warps [0, HW) into hL, warps [HW, 2 HW) into hU (other warps pass 0).
-template <typename T, int C, int NT, int CT, bool COUNTED, int NI = 2, int HW = 0, int HC = 1>
+// and the flag.  HH > 0 (halo elements per side) also sums two sets of HC <= C
+// values per thread, hvL and hvU, into the block totals hL and hU.  The halo
+// element k of the tile (k < HH: left, HH <= k < 2 HH: right) belongs to
+// thread k mod NT, so a warp holds left terms only if one of its k < HH, and
+// right terms only if one of its k lies in [HH, 2 HH).
+template <typename T, int C, int NT, int CT, bool COUNTED, int NI = 2, int HH = 0, int HC = 1>
 __device__ __forceinline__ bool block_excl_both_counted(
     const T e, const T (&V)[C], const T f, const T (&W)[C], bool& hasf, T& pe, T (&pV)[C], T& te,
     T (&tV)[C], bool& hasb, T& nf, T (&nW)[C], T& tf, T (&tW)[C], const int (&cnt)[NI], int (&tot)[NI],
-    const bool bad, BlockScan2Smem<T, C, NT>& sm, const T* hv = nullptr, T* hL = nullptr, T* hU = nullptr) {
+    const bool bad, BlockScan2Smem<T, C, NT>& sm, const T* hvL = nullptr, const T* hvU = nullptr,
+    T* hL = nullptr, T* hU = nullptr) {
     constexpr int NW = NT / 32;
     static_assert(NW <= 32, "one warp scans the warp totals");
     static_assert(NI >= 1 && NI <= 4, "at most four counts");
-    static_assert(2 * HW <= NW && (HW & (HW - 1)) == 0, "halo warps: a power of two per side");
+    static_assert(HH % 32 == 0, "halo: whole warps");
     static_assert(HC >= 1 && HC <= C, "halo channels");
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     T iV[C], iW[C];
@@ -302,13 +307,29 @@ __device__ __forceinline__ bool block_excl_both_counted(
             if (lane == 0) sm.wcnt[w][q] = cq;
         }
     }
-    if (HW > 0 && w < 2 * HW) {
+    if (HH > 0) {
+        bool hasL = false, hasR = false;
+#pragma unroll
+        for (int m = 0; m * NT < 2 * HH; ++m) {
+            const int lo = 32 * w + m * NT;
+            if (lo < HH) hasL = true;
+            else if (lo < 2 * HH) hasR = true;
+        }
 #pragma unroll
         for (int c = 0; c < HC; ++c) {
-            T h = hv[c];
+            T hl = hasL ? hvL[c] : T(0), hu = hasR ? hvU[c] : T(0);
+            if (hasL) {
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) h += __shfl_xor_sync(FULL, h, off);
-            if (lane == 0) sm.whs[w][c] = h;
+                for (int off = 16; off > 0; off >>= 1) hl += __shfl_xor_sync(FULL, hl, off);
+            }
+            if (hasR) {
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) hu += __shfl_xor_sync(FULL, hu, off);
+            }
+            if (lane == 0) {
+                sm.whL[w][c] = hl;
+                sm.whU[w][c] = hu;
+            }
         }
     }
     if (lane == 0) {
@@ -363,16 +384,20 @@ __device__ __forceinline__ bool block_excl_both_counted(
         }
     }
     if (w == WB) {
-        if (HW > 0) {
-            // fixed order: warp sums added in a butterfly over the first HW
-            // lanes (left) and the next HW lanes (right)
+        if (HH > 0) {
+            // warp sums added in a fixed butterfly over the lanes
 #pragma unroll
             for (int c = 0; c < HC; ++c) {
-                T hs = lane < 2 * HW ? sm.whs[lane][c] : T(0);
+                T sl = lane < NW ? sm.whL[lane][c] : T(0), su = lane < NW ? sm.whU[lane][c] : T(0);
 #pragma unroll
-                for (int off = 1; off < HW; off <<= 1) hs += __shfl_xor_sync(FULL, hs, off);
-                if (lane == 0) sm.thL[c] = hs;
-                if (lane == HW) sm.thU[c] = hs;
+                for (int off = 16; off > 0; off >>= 1) {
+                    sl += __shfl_xor_sync(FULL, sl, off);
+                    su += __shfl_xor_sync(FULL, su, off);
+                }
+                if (lane == 0) {
+                    sm.thL[c] = sl;
+                    sm.thU[c] = su;
+                }
             }
         }
         T gf = lane < NW ? sm.be[lane] : T(0), gW[C];
@@ -474,7 +499,7 @@ __device__ __forceinline__ bool block_excl_both_counted(
 #pragma unroll
         for (int q = 0; q < NI; ++q) tot[q] = sm.tcnt[q];
     }
-    if (HW > 0) {
+    if (HH > 0) {
 #pragma unroll
         for (int c = 0; c < HC; ++c) {
             hL[c] = sm.thL[c];

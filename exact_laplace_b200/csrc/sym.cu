@@ -253,9 +253,10 @@ template <typename T_, int NCOL_, bool PHASED_, int E_, int NT_>
 struct SymTP {
     using T = T_;
     static constexpr int NCOL = NCOL_, C = PHASED_ ? 2 * NCOL_ : NCOL_, CT = 0, E = E_, NT = NT_;
-    // halos of 128 (fp32: they span CUT = 88 at spacings above 0.7); fp64
-    // (CUT = 746) would need several times more: none
-    static constexpr int H = sizeof(T_) == 4 ? 128 : 0;
+    // halos of 192 (fp32: they span CUT = 88 at spacings above 0.47, and
+    // across runs of up to 64 equal anchors); fp64 (CUT = 746) would need
+    // several times more: none
+    static constexpr int H = sizeof(T_) == 4 ? 192 : 0;
     SymArgs<T> A;
     int64_t n;
     const T* s;

@@ -41,7 +41,7 @@ namespace lx {
 #define LX_LT_E 12
 #endif
 #ifndef LX_LT_H
-#define LX_LT_H 128
+#define LX_LT_H 192
 #endif
 #ifndef LX_LT_MINB
 #define LX_LT_MINB 4
@@ -88,9 +88,9 @@ struct LocalWs {
 // and carries the copy-timeout flag.
 //
 // MODE 0 (first pass).  The copy of a full tile also brings H elements on each
-// side (halos).  Thread q < 2H takes one halo element: its term of the carry
-// from the left, L_{b-1} = sum_j exp(s_j - s_{b-1}) x_j, or from the right,
-// U_e.  When both halos span at least CUT (or the tile is at an end of the
+// side (halos).  Thread q takes the halo elements q, q + NT, ... < 2H: their
+// terms of the carry from the left, L_{b-1} = sum_j exp(s_j - s_{b-1}) x_j, or
+// from the right, U_e.  When both halos span at least CUT (or the tile is at an end of the
 // array) these sums are the exact carries and the tile's outputs are final.
 // Otherwise (dense anchors, H = 0, the ragged last tile) nothing is written
 // and the tile is marked for the redo pass.  Every tile publishes its first
@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(NT, LX_LT_MINB) k_tile_local(const T* __restri
     constexpr int HH = MODE == 0 ? H : 0;     // halo brought by the copies
     constexpr int64_t STAGE = TILE + 2 * H;   // elements per array per stage
     static_assert(((E / VN) & 1) == 1, "E must be an odd number of 16-byte units");
-    static_assert(H % 32 == 0 && 2 * H <= NT, "halo: whole warps, one element per thread");
+    static_assert(H % 32 == 0 && H <= TILE, "halo: whole warps, at most a tile");
     extern __shared__ __align__(128) unsigned char dyn[];
     T* ring_s = reinterpret_cast<T*>(dyn);
     T* ring_x = ring_s + S * STAGE;                              // !GATHER
@@ -226,36 +226,42 @@ __global__ void __launch_bounds__(NT, LX_LT_MINB) k_tile_local(const T* __restri
 #pragma unroll
             for (int k = 0; k < E; ++k) v[k][0] = xv[k];
         }
-        // MODE 0: halo term of this thread (q < H: left, H <= q < 2H: right),
-        // and the checks that each halo spans CUT (thread 0: left, thread H:
-        // right); a tile without usable halos is marked bad on both sides
-        T hv = T(0), ringL = T(0), ringR = T(0);  // s_{b-1}, s_e when in the ring
+        // MODE 0: the halo terms of this thread (halo element k = q + m NT;
+        // k < H: left, H <= k < 2H: right), and the checks that each halo
+        // spans CUT (by the threads holding k = 0 and k = H)
+        T hvL = T(0), hvU = T(0), ringL = T(0), ringR = T(0);  // s_{b-1}, s_e when in the ring
         int bad[2] = {0, 0};
         if constexpr (MODE == 0) {
             const int q = (int)threadIdx.x;
             const int64_t e = tile0 + TILE;
             if constexpr (H > 0) {
+                const bool haveL = t > 0, haveR = e + H <= n;
                 if (live && !ragged) {
-                    if (t > 0) ringL = S0[H - 1];
-                    if (e + H <= n) ringR = S0[H + TILE];
-                }
-                if (q < 2 * H && live && !ragged) {
-                    const bool left = q < H;
-                    const bool have = left ? t > 0 : e + H <= n;
-                    const int j = left ? q : (int)(H + TILE) + (q - H);  // ring index
-                    if (have) {
+                    if (haveL) ringL = S0[H - 1];
+                    if (haveR) ringR = S0[H + TILE];
+#pragma unroll
+                    for (int m = 0; m * NT < 2 * H; ++m) {
+                        const int k = q + m * NT;
+                        if (k >= 2 * H) break;
+                        const bool left = k < H;
+                        const bool have = left ? haveL : haveR;
+                        const bool need = left ? t > 0 : e < n;
+                        if (!have) {
+                            // no halo: exact only at the array's own ends
+                            if (k == 0 || k == H) bad[left ? 0 : 1] = need ? 1 : 0;
+                            continue;
+                        }
+                        const int j = left ? k : (int)(TILE + k);  // ring index of element k
                         const T edge = left ? ringL : ringR;
                         const T sj = S0[j];
                         T xj;
                         if constexpr (GATHER) xj = __ldg(x_ + ring_p[st * STAGE + j]);
                         else xj = ring_x[st * STAGE + j];
-                        hv = dexp<T>(left ? sj - edge : edge - sj) * xj;
-                        if (q == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
-                        if (q == H) bad[1] = S0[2 * H + TILE - 1] - edge >= ExpCut<T>::v ? 0 : 1;
-                    } else {
-                        // no halo: exact only at the array's own ends
-                        if (q == 0) bad[0] = t == 0 ? 0 : 1;
-                        if (q == H) bad[1] = e == n ? 0 : 1;
+                        const T term = dexp<T>(left ? sj - edge : edge - sj) * xj;
+                        if (left) hvL += term;
+                        else hvU += term;
+                        if (k == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
+                        if (k == H) bad[1] = S0[2 * H + TILE - 1] - edge >= ExpCut<T>::v ? 0 : 1;
                     }
                 }
             }
@@ -271,9 +277,9 @@ __global__ void __launch_bounds__(NT, LX_LT_MINB) k_tile_local(const T* __restri
         T pe, pV[1], te, tV[1], nf, nW[1], tf, tW[1];
         int nbad[2];
         T hL = T(0), hU = T(0);
-        if (block_excl_both_counted<T, 1, NT, 0, true, 2, (MODE == 0 ? H / 32 : 0)>(
-                s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW, bad, nbad, !live, sm2, &hv,
-                &hL, &hU)) {
+        if (block_excl_both_counted<T, 1, NT, 0, true, 2, (MODE == 0 ? H : 0)>(
+                s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW, bad, nbad, !live, sm2, &hvL,
+                &hvU, &hL, &hU)) {
             // the block's last tile is done, or a copy never completed: then
             // report it and let the copies in flight land before leaving
             if (threadIdx.x == 0 && sh_timeout) {

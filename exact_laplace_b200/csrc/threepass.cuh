@@ -19,7 +19,7 @@
 // A policy P provides
 //   using T;  static constexpr int C, CT, E, NT, H;   (CT trailing tie channels;
 //                                                      halo H: 0, or a multiple
-//                                                      of 32 with 2H <= NT)
+//                                                      of 32 up to a tile)
 //   int64_t n;  const T* s;
 //   struct Aux { ... }                                  per-thread extra state
 //   __device__ void load(int64_t r0, T (&s)[E], T (&v)[E][C], Aux& a) const
@@ -91,42 +91,55 @@ inline TPWs<T, C> tp_carve(Carve& cv, int64_t ntiles) {
 }
 
 // ------------------------------------------------------------------ pass 1 and 3
-// Halo term of thread q of a tile (q < H: left halo, H <= q < 2H: right halo)
-// and the checks that each halo spans CUT (thread 0: left, thread H: right).
-// A side needs no carry at an end of the array; a side without a halo in the
-// array (the right side of the last-but-one tiles) is marked bad.
+// Halo terms of thread q of a tile: the halo elements k = q + m NT < 2H
+// (k < H: left halo, H <= k < 2H: right halo), summed per side, and the checks
+// that each halo spans CUT (by the threads holding k = 0 and k = H).  A side
+// needs no carry at an end of the array; a side without a halo in the array
+// (the right side of the last-but-one tiles) is marked bad.
 template <class P>
-__device__ __forceinline__ void tp_halo_term(const P& p, int64_t t, int64_t tile0, int64_t tile1,
-                                             typename P::T (&hv)[P::C], int (&bad)[2]) {
+__device__ __forceinline__ void tp_halo_terms(const P& p, int64_t t, int64_t tile0, int64_t tile1,
+                                              typename P::T (&hvL)[P::C], typename P::T (&hvU)[P::C],
+                                              int (&bad)[2]) {
     using T = typename P::T;
-    constexpr int C = P::C, CT = P::CT, H = P::H;
+    constexpr int C = P::C, CT = P::CT, H = P::H, NT = P::NT;
     const int64_t n = p.n;
     const int q = (int)threadIdx.x;
 #pragma unroll
-    for (int c = 0; c < C; ++c) hv[c] = T(0);
+    for (int c = 0; c < C; ++c) {
+        hvL[c] = T(0);
+        hvU[c] = T(0);
+    }
     bad[0] = bad[1] = 0;
     if (H == 0) {
         if (q == 0) bad[0] = (t > 0 || tile1 < n) ? 1 : 0;  // no halos: final only if alone
         return;
     }
-    if (q >= 2 * H) return;
-    const bool left = q < H;
-    const bool need = left ? t > 0 : tile1 < n;
-    if (!need) return;
-    const bool have = left ? true : tile1 + H <= n;  // tile0 >= TILE >= H on the left
-    if (!have) {
-        if (q == H) bad[1] = 1;
-        return;
-    }
-    const int64_t j = left ? tile0 - H + q : tile1 + (q - H);
-    const T edge = left ? p.s[tile0 - 1] : p.s[tile1];
-    T sj, vj[C];
-    p.load1(j, sj, vj);
-    const Decay<T, C, CT> d = left ? Decay<T, C, CT>(sj, edge) : Decay<T, C, CT>(edge, sj);
+    const bool needL = t > 0, needR = tile1 < n;
+    const bool haveR = tile1 + H <= n;  // the left halo is always in the array (tile0 >= TILE >= H)
+    const T eL = needL ? p.s[tile0 - 1] : T(0), eR = needR && haveR ? p.s[tile1] : T(0);
 #pragma unroll
-    for (int c = 0; c < C; ++c) hv[c] = d[c] * vj[c];
-    if (q == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
-    if (q == H) bad[1] = p.s[tile1 + H - 1] - edge >= ExpCut<T>::v ? 0 : 1;
+    for (int m = 0; m * NT < 2 * H; ++m) {
+        const int k = q + m * NT;
+        if (k >= 2 * H) break;
+        const bool left = k < H;
+        if (!(left ? needL : needR)) continue;
+        if (!left && !haveR) {
+            if (k == H) bad[1] = 1;
+            continue;
+        }
+        const int64_t j = left ? tile0 - H + k : tile1 + (k - H);
+        const T edge = left ? eL : eR;
+        T sj, vj[C];
+        p.load1(j, sj, vj);
+        const Decay<T, C, CT> d = left ? Decay<T, C, CT>(sj, edge) : Decay<T, C, CT>(edge, sj);
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            if (left) hvL[c] += d[c] * vj[c];
+            else hvU[c] += d[c] * vj[c];
+        }
+        if (k == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
+        if (k == H) bad[1] = p.s[tile1 + H - 1] - edge >= ExpCut<T>::v ? 0 : 1;
+    }
 }
 
 // One tile.  MODE 0: carries from the halos; a tile whose halos fall short is
@@ -144,17 +157,19 @@ __device__ __forceinline__ void tp_tile(const P& p, const TPWs<typename P::T, P:
     T s[E], v[E][C];
     typename P::Aux aux;
     p.load(r0, s, v, aux);
-    T hv[C];
+    T hvL[C], hvU[C];
     int bad[2] = {0, 0};
-    if (MODE == 0) tp_halo_term<P>(p, t, tile0, tile1, hv, bad);
+#pragma unroll
+    for (int c = 0; c < C; ++c) hvL[c] = hvU[c] = T(0);
+    if (MODE == 0) tp_halo_terms<P>(p, t, tile0, tile1, hvL, hvU, bad);
     T dl[E], fV[C], bW[C];
     chunk_aggregates<T, C, E, CT>(s, v, dl, fV, bW);
     bool hf, hb;
     T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
     int nbad[2];
     T hL[C], hU[C];
-    (void)block_excl_both_counted<T, C, NT, CT, true, 2, (H > 0 ? H / 32 : 0), C>(
-        s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW, bad, nbad, false, sm2, hv, hL, hU);
+    (void)block_excl_both_counted<T, C, NT, CT, true, 2, H, C>(
+        s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW, bad, nbad, false, sm2, hvL, hvU, hL, hU);
     bool out = true;
     T eT = hf ? pe : s[0], fT = hb ? nf : s[E - 1], Lc[C], Uc[C];
 #pragma unroll
@@ -225,7 +240,7 @@ __global__ void __launch_bounds__(P::NT) k_tp_redo(P p, TPWs<typename P::T, P::C
 // Persistent variant of pass 1 for inputs already in sorted order: s and the
 // policy's NIN value arrays come into a shared-memory ring of S stages by 1-D
 // bulk copies (TMA), each full tile with a halo of H elements on both sides
-// (thread q < 2H takes one halo element, as in k_tp_local).  The ragged last
+// (thread q takes the halo elements q, q + NT, ... < 2H, as in k_tp_local).  The ragged last
 // tile goes through the policy's register load and is always listed for the
 // redo pass.
 //
@@ -241,7 +256,7 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
     constexpr int VN = V16<T>::N, NA = NIN + 1;
     constexpr int64_t TILE = (int64_t)NT * E, STAGE = TILE + 2 * H;
     static_assert(E % VN == 0, "E: whole 16-byte units");
-    static_assert(H % 32 == 0 && 2 * H <= NT, "halo: whole warps, one element per thread");
+    static_assert(H % 32 == 0 && H <= TILE, "halo: whole warps, at most a tile");
     extern __shared__ __align__(128) unsigned char dyn[];
     T* ring = reinterpret_cast<T*>(dyn);  // stage st, array a (0 = s) at ring + (st * NA + a) * STAGE
     __shared__ __align__(8) uint64_t full[S];
@@ -312,11 +327,12 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
         } else {
             p.load(r0, s, v, aux);
         }
-        // halo term of this thread and the span checks; the edge anchors
-        T hv[C], ringL = T(0), ringR = T(0);
+        // halo terms of this thread (elements k = q + m NT < 2H), the span
+        // checks, the edge anchors
+        T hvL[C], hvU[C], ringL = T(0), ringR = T(0);
         int bad[2] = {0, 0};
 #pragma unroll
-        for (int c = 0; c < C; ++c) hv[c] = T(0);
+        for (int c = 0; c < C; ++c) hvL[c] = hvU[c] = T(0);
         {
             const int q = (int)threadIdx.x;
             const bool haveR = tile0 + TILE + H <= n;
@@ -326,13 +342,18 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
             }
             if (H == 0 || ragged) {
                 if (q == 0) bad[0] = (needL || needR) ? 1 : 0;
-            } else if (q < 2 * H && landed) {
-                const bool left = q < H;
-                const bool need = left ? needL : needR;
-                if (need && !left && !haveR) {
-                    if (q == H) bad[1] = 1;
-                } else if (need) {
-                    const int j = left ? q : (int)(H + TILE) + (q - H);  // ring index
+            } else if (landed) {
+#pragma unroll
+                for (int m = 0; m * NT < 2 * H; ++m) {
+                    const int k = q + m * NT;
+                    if (k >= 2 * H) break;
+                    const bool left = k < H;
+                    if (!(left ? needL : needR)) continue;
+                    if (!left && !haveR) {
+                        if (k == H) bad[1] = 1;
+                        continue;
+                    }
+                    const int j = left ? k : (int)TILE + k;  // ring index
                     const T edge = left ? ringL : ringR;
                     const T sj = S0[j];
                     T xe[NIN], vj[C];
@@ -341,9 +362,12 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
                     p.value(xe, vj);
                     const Decay<T, C, CT> d = left ? Decay<T, C, CT>(sj, edge) : Decay<T, C, CT>(edge, sj);
 #pragma unroll
-                    for (int c = 0; c < C; ++c) hv[c] = d[c] * vj[c];
-                    if (q == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
-                    if (q == H) bad[1] = S0[2 * H + TILE - 1] - edge >= ExpCut<T>::v ? 0 : 1;
+                    for (int c = 0; c < C; ++c) {
+                        if (left) hvL[c] += d[c] * vj[c];
+                        else hvU[c] += d[c] * vj[c];
+                    }
+                    if (k == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
+                    if (k == H) bad[1] = S0[2 * H + TILE - 1] - edge >= ExpCut<T>::v ? 0 : 1;
                 }
             }
         }
@@ -356,9 +380,9 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
         T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
         int nbad[2];
         T hL[C], hU[C];
-        if (block_excl_both_counted<T, C, NT, CT, true, 2, (H > 0 ? H / 32 : 0), C>(
-                s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW, bad, nbad, !landed, sm2, hv,
-                hL, hU)) {
+        if (block_excl_both_counted<T, C, NT, CT, true, 2, H, C>(
+                s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf, nW, tf, tW, bad, nbad, !landed, sm2, hvL,
+                hvU, hL, hU)) {
             // a copy never completed: report, let the copies in flight land, stop
             if (threadIdx.x == 0) {
                 set_status(status, ST_TIMEOUT);

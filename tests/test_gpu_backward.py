@@ -85,18 +85,22 @@ def test_c5_full_size_sampled():
     assert_close(da[idx], da_ref, np.abs(g[idx]) * nx + np.abs(x[idx]) * ng, np.float32, "C5 da")
 
 
-@pytest.mark.parametrize("case", ["spacing_0.69", "spacing_0.70", "spacing_1.0", "mixed_ties", "short_right"])
+@pytest.mark.parametrize("case", ["spacing_0.46", "spacing_0.47", "spacing_1.0", "mixed_ties", "short_right",
+                                  "runs_of_64"])
 def test_halo_carries(case):
-    """Tiles whose carries come from the halos of 128 elements, next to tiles
-    that fall back to the carry kernels and the redo pass: spacing 0.69 spans
-    87.6 < 88 (fall back), 0.70 spans 88.9 (halo carries); runs of equal
-    anchors inside the halos; a last-but-one tile without room for a right
-    halo."""
+    """Tiles whose carries come from the halos of 192 elements, next to tiles
+    that fall back to the carry kernels and the redo pass: spacing 0.46 spans
+    87.9 < 88 (fall back), 0.47 spans 89.8 (halo carries); runs of equal
+    anchors inside the halos (and runs of 64 equal anchors 64 apart, the fp32
+    grid of a ~ U(0, 2^30) above 2^29); a last-but-one tile without room for
+    a right halo."""
     rng = np.random.default_rng(21)
     tile = 256 * 8
     n = 11 * tile + 77
     if case.startswith("spacing_"):
         a = np.arange(n) * float(case.split("_")[1])
+    elif case == "runs_of_64":
+        a = 2.0 ** 29 + 64.0 * (np.arange(n) // 64)
     elif case == "mixed_ties":
         # groups of equal anchors 3 apart, a dense stretch, then unit spacing
         k = n // 3

@@ -126,7 +126,7 @@ def test_deep_lookahead_fixup(dtype):
 
 
 TILE_F32 = 256 * 12  # elements per tile of the single-column fp32 product
-HALO_SPACINGS = [0.30, 0.345, 0.35, 0.40, 0.69, 0.70, 1.0]
+HALO_SPACINGS = [0.30, 0.345, 0.35, 0.46, 0.47, 0.69, 0.70, 1.0]
 
 
 def _spaced(n, spacing, seed, jitter=0.0):
@@ -138,10 +138,10 @@ def _spaced(n, spacing, seed, jitter=0.0):
 @pytest.mark.parametrize("use_perm", [False, True])
 @pytest.mark.parametrize("spacing", HALO_SPACINGS)
 def test_halo_span_boundary(spacing, use_perm):
-    """Constant anchor spacing around the point where a halo of 128 (or 256)
-    elements spans the cut of 88: 127 x 0.69 = 87.6 falls back to the carry
-    kernels, 127 x 0.70 = 88.9 takes the halo carries (255 x 0.345 = 88.0 and
-    255 x 0.35 = 89.3 for halos of 256)."""
+    """Constant anchor spacing around the points where a halo spans the cut of
+    88: with 192 elements 191 x 0.46 = 87.9 falls back to the carry kernels
+    and the redo pass, 191 x 0.47 = 89.8 takes the halo carries (0.69 / 0.70
+    for halos of 128, 0.345 / 0.35 for halos of 256)."""
     n = 9 * TILE_F32 + 1234
     a, x = _spaced(n, spacing, seed=int(spacing * 1000))
     assert_close(run_sym(a, x, use_perm), O.sym(a, x), O.norm_sym(a, x), np.float32,
@@ -149,7 +149,7 @@ def test_halo_span_boundary(spacing, use_perm):
 
 
 @pytest.mark.parametrize("use_perm", [False, True])
-@pytest.mark.parametrize("case", ["unit", "mixed", "far", "aligned", "short_right"])
+@pytest.mark.parametrize("case", ["unit", "mixed", "far", "aligned", "short_right", "runs_of_64"])
 def test_halo_carries(case, use_perm):
     """Tiles whose carries come from the halos (sparse anchors) and tiles that
     fall back to the carry kernels and the redo pass (denser), side by side."""
@@ -170,6 +170,10 @@ def test_halo_carries(case, use_perm):
         x = rng.normal(size=n).astype(np.float32)
     elif case == "far":
         a, x = _spaced(n, 150.0, seed=7)
+    elif case == "runs_of_64":
+        # the fp32 grid of a ~ U(0, 2^30) above 2^29: runs of 64 equal anchors
+        a = (2.0 ** 29 + 64.0 * (np.arange(n) // 64)).astype(np.float32)
+        x = np.random.default_rng(10).normal(size=n).astype(np.float32)
     elif case == "aligned":
         n = 5 * TILE_F32
         a, x = synth.sym_uniform(n, 0.0, float(n), seed=8)
