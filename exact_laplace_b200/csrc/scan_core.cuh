@@ -36,35 +36,47 @@ struct Decay {
 };
 
 // ---------------------------------------------------------------- warp level
+// Inclusive scans over the lanes.  At step off a lane combines the partial of
+// lane l - off, whose edge anchor is e_{l-off}, with the decay
+// d_off(l) = exp(e_{l-off} - e_l) (tie channels: [e_{l-off} == e_l]).  Only
+// d_1 takes an exp; d_2off(l) = d_off(l - off) d_off(l) is the product of the
+// previous level's two decays (at most five rounded products; each factor is
+// at least the product, so nothing at or above FLT_MIN is flushed).
 template <typename T, int C, int CT = 0>
 __device__ __forceinline__ void warp_incl_fwd(const T e, T (&V)[C], const int lane) {
+    Decay<T, C, CT> d(__shfl_up_sync(FULL, e, 1), e);  // lane 0: exp(0), unused
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const T eo = __shfl_up_sync(FULL, e, off);
         T Vo[C];
 #pragma unroll
         for (int c = 0; c < C; ++c) Vo[c] = __shfl_up_sync(FULL, V[c], off);
+        const T de = __shfl_up_sync(FULL, d.e, off);
+        const T dt = CT > 0 ? __shfl_up_sync(FULL, d.t, off) : T(0);
         if (lane >= off) {
-            const Decay<T, C, CT> d(eo, e);
 #pragma unroll
             for (int c = 0; c < C; ++c) V[c] = dfma<T>(d[c], Vo[c], V[c]);
         }
+        d.e *= de;
+        if (CT > 0) d.t *= dt;
     }
 }
 
 template <typename T, int C, int CT = 0>
 __device__ __forceinline__ void warp_incl_bwd(const T f, T (&W)[C], const int lane) {
+    Decay<T, C, CT> d(f, __shfl_down_sync(FULL, f, 1));  // lane 31: exp(0), unused
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const T fo = __shfl_down_sync(FULL, f, off);
         T Wo[C];
 #pragma unroll
         for (int c = 0; c < C; ++c) Wo[c] = __shfl_down_sync(FULL, W[c], off);
+        const T de = __shfl_down_sync(FULL, d.e, off);
+        const T dt = CT > 0 ? __shfl_down_sync(FULL, d.t, off) : T(0);
         if (lane + off < 32) {
-            const Decay<T, C, CT> d(f, fo);
 #pragma unroll
             for (int c = 0; c < C; ++c) W[c] = dfma<T>(d[c], Wo[c], W[c]);
         }
+        d.e *= de;
+        if (CT > 0) d.t *= dt;
     }
 }
 

@@ -150,11 +150,12 @@ __global__ void __launch_bounds__(SORT_NT, 3) k_onesweep(
     int32_t* __restrict__ vdst, int last, uint32_t* status) {
     using K = typename KeyOf<T>::K;
     constexpr int NT = SORT_NT, NW = NT / 32, TILE = NT * KPT;
+    static_assert(KPT % 4 == 0, "digits are packed four to a word");
     __shared__ K skey[TILE];
     __shared__ int32_t sval[TILE];
     __shared__ uint32_t wcnt[NW][RADIX];
     __shared__ uint32_t dstart[RADIX];
-    __shared__ int64_t gbase[RADIX];
+    __shared__ int64_t gofs[RADIX];  // global position of staged key q: gofs[digit] + q
     __shared__ uint32_t scan_sm[NT / 32 + 1];
     __shared__ int64_t sh_tile;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -167,104 +168,112 @@ __global__ void __launch_bounds__(SORT_NT, 3) k_onesweep(
     const int64_t tb = t * TILE;
     const int64_t end = min(tb + TILE, n);
     const unsigned ltmask = lanemask_lt();
+    // key i of this thread is element lane0 + 32 i of the tile (coalesced per i)
+    const int64_t lane0 = tb + (int64_t)w * 32 * KPT + lane;
+    const int nvalid = (int)max((int64_t)0, min((int64_t)KPT, (end - lane0 + 31) / 32));
     K k[KPT];
-    int32_t v[KPT];
+    uint32_t dg[KPT / 4];  // the digits, four per word
     uint32_t rk[KPT];
     bool bad = false;
-    // digit of key i of this thread; RADIX for padding (never placed)
-    const int64_t lane0 = tb + (int64_t)w * 32 * KPT + lane;
-    auto digit = [&](int i) -> int {
-        return lane0 + i * 32 < end ? (int)((unsigned)(k[i] >> shift) & (RADIX - 1)) : RADIX;
-    };
 #pragma unroll
     for (int i = 0; i < KPT; ++i) {
         const int64_t idx = lane0 + i * 32;
-        if (idx < end) {
-            k[i] = first ? to_key(a[idx], bad) : ksrc[idx];
-            v[i] = first ? (int32_t)idx : vsrc[idx];
-        } else {
-            k[i] = 0;
-            v[i] = 0;
-        }
+        k[i] = i < nvalid ? (first ? to_key(a[idx], bad) : ksrc[idx]) : K(0);
     }
 #pragma unroll
+    for (int i = 0; i < KPT; i += 4) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) word |= ((uint32_t)(k[i + b] >> shift) & (RADIX - 1)) << (8 * b);
+        dg[i / 4] = word;
+    }
+    auto digit = [&](int i) -> int { return (int)((dg[i / 4] >> (8 * (i % 4))) & (RADIX - 1)); };
+    // stable rank among the keys of this warp with the same digit: lanes in
+    // order within a round, rounds in order.  The lowest lane of each group of
+    // equal digits adds the group to the warp's counter and hands the old
+    // count to the group with one shuffle.
+#pragma unroll
     for (int i = 0; i < KPT; ++i) {
-        const int d = digit(i);
+        const bool valid = i < nvalid;
+        const int d = valid ? digit(i) : RADIX;  // padding ranks apart
         const unsigned peers = __match_any_sync(FULL, d);
-        const uint32_t lower = __popc(peers & ltmask);
-        rk[i] = d < RADIX ? wcnt[w][d] + lower : 0u;
-        __syncwarp();
-        if (d < RADIX && lower == 0) wcnt[w][d] += __popc(peers);
-        __syncwarp();
+        const int leader = __ffs(peers) - 1;
+        uint32_t base = 0;
+        if (valid && lane == leader) base = atomicAdd(&wcnt[w][d], (uint32_t)__popc(peers));
+        base = __shfl_sync(FULL, base, leader);
+        rk[i] = base + __popc(peers & ltmask);
     }
     __syncthreads();
-    {
-        const int d = threadIdx.x;  // NT == RADIX: one digit per thread
-        uint32_t c = 0;
+    const int d = threadIdx.x;  // NT == RADIX: one digit per thread from here on
+    uint32_t c = 0;  // this tile's count of digit d; wcnt[.][d] becomes the warps' exclusive offsets
 #pragma unroll
-        for (int ww = 0; ww < NW; ++ww) {
-            const uint32_t x = wcnt[ww][d];
-            wcnt[ww][d] = c;
-            c += x;
-        }
-        // publish this tile's count of digit d, then look back for the keys of
-        // digit d in all earlier tiles
-        const uint64_t tagA = (uint64_t)(2 * pass + 2) << 32, tagI = (uint64_t)(2 * pass + 3) << 32;
-        uint64_t* my = rec + t * RADIX + d;
-        uint64_t excl = 0;
-        if (t == 0) {
-            st_relaxed64(my, tagI | c);
-        } else {
-            st_relaxed64(my, tagA | c);
-            // walk back LB records at a time (loads in flight together), adding
-            // counts up to and including the first inclusive record
-            constexpr int LB = 8;
-            bool done = false;
-            for (int64_t j0 = t - 1; !done; j0 -= LB) {
-                uint64_t val[LB];
-#pragma unroll
-                for (int q = 0; q < LB; ++q)
-                    val[q] = j0 - q >= 0 ? ld_relaxed64(rec + (j0 - q) * RADIX + d) : tagI;
-#pragma unroll
-                for (int q = 0; q < LB; ++q) {
-                    if (done) break;
-                    uint32_t it = 0;
-                    while ((val[q] & 0xFFFFFFFF00000000ull) < tagA) {
-                        if (++it > SORT_POLLS) break;
-                        __nanosleep(32);
-                        val[q] = ld_relaxed64(rec + (j0 - q) * RADIX + d);
-                    }
-                    if ((val[q] & 0xFFFFFFFF00000000ull) < tagA) {
-                        set_status(status, ST_TIMEOUT);
-                        done = true;
-                        break;
-                    }
-                    excl += val[q] & 0xFFFFFFFFull;
-                    if ((val[q] & 0xFFFFFFFF00000000ull) == tagI) done = true;
-                }
-            }
-            st_relaxed64(my, tagI | (excl + c));
-        }
-        gbase[d] = (int64_t)offsets[d] + (int64_t)excl;
-        uint32_t tot;
-        dstart[d] = block_excl_sum<NT>(c, scan_sm, tot);
+    for (int ww = 0; ww < NW; ++ww) {
+        const uint32_t x = wcnt[ww][d];
+        wcnt[ww][d] = c;
+        c += x;
     }
-    __syncthreads();
+    // publish this tile's count of digit d early; its prefix over earlier tiles
+    // is looked up after the tile is staged, when they have had time to finish
+    const uint64_t tagA = (uint64_t)(2 * pass + 2) << 32, tagI = (uint64_t)(2 * pass + 3) << 32;
+    uint64_t* my = rec + t * RADIX + d;
+    st_relaxed64(my, (t == 0 ? tagI : tagA) | c);
+    uint32_t tot;
+    dstart[d] = block_excl_sum<NT>(c, scan_sm, tot);  // its barriers publish wcnt
+    __syncthreads();                                   // and this one dstart
+    // stage the keys in digit order (rk becomes the staging position), then
+    // the payloads, loaded only now to keep the ranking's registers free
 #pragma unroll
     for (int i = 0; i < KPT; ++i) {
-        const int d = digit(i);
-        if (d < RADIX) {
-            const uint32_t pos = dstart[d] + wcnt[w][d] + rk[i];
-            skey[pos] = k[i];
-            sval[pos] = v[i];
+        if (i < nvalid) {
+            const int di = digit(i);
+            rk[i] += dstart[di] + wcnt[w][di];
+            skey[rk[i]] = k[i];
         }
     }
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+        const int64_t idx = lane0 + i * 32;
+        if (i < nvalid) sval[rk[i]] = first ? (int32_t)idx : vsrc[idx];
+    }
+    // keys of digit d in all earlier tiles: walk back LB records at a time
+    // (loads in flight together), adding counts up to and including the first
+    // inclusive record
+    uint64_t excl = 0;
+    if (t > 0) {
+        constexpr int LB = 8;
+        bool done = false;
+        for (int64_t j0 = t - 1; !done; j0 -= LB) {
+            uint64_t val[LB];
+#pragma unroll
+            for (int q = 0; q < LB; ++q)
+                val[q] = j0 - q >= 0 ? ld_relaxed64(rec + (j0 - q) * RADIX + d) : tagI;
+#pragma unroll
+            for (int q = 0; q < LB; ++q) {
+                if (done) break;
+                uint32_t it = 0;
+                while ((val[q] & 0xFFFFFFFF00000000ull) < tagA) {
+                    if (++it > SORT_POLLS) break;
+                    __nanosleep(64);
+                    val[q] = ld_relaxed64(rec + (j0 - q) * RADIX + d);
+                }
+                if ((val[q] & 0xFFFFFFFF00000000ull) < tagA) {
+                    set_status(status, ST_TIMEOUT);
+                    done = true;
+                    break;
+                }
+                excl += val[q] & 0xFFFFFFFFull;
+                if ((val[q] & 0xFFFFFFFF00000000ull) == tagI) done = true;
+            }
+        }
+        st_relaxed64(my, tagI | (excl + c));
+    }
+    (void)bad;  // non-finite anchors are reported by k_radix_hist
+    gofs[d] = (int64_t)offsets[d] + (int64_t)excl - (int64_t)dstart[d];
     __syncthreads();
     const int cnt = (int)(end - tb);
     for (int q = threadIdx.x; q < cnt; q += NT) {
         const K kk = skey[q];
-        const int d = (int)((unsigned)(kk >> shift) & (RADIX - 1));
-        const int64_t gpos = gbase[d] + (q - (int)dstart[d]);
+        const int64_t gpos = gofs[(unsigned)(kk >> shift) & (RADIX - 1)] + q;
         kdst[gpos] = last ? key_to_bits(kk) : kk;
         vdst[gpos] = sval[q];
     }

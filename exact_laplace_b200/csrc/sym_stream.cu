@@ -91,9 +91,9 @@ struct LocalWs {
 // side (halos).  Thread q takes the halo elements q, q + NT, ... < 2H: their
 // terms of the carry from the left, L_{b-1} = sum_j exp(s_j - s_{b-1}) x_j, or
 // from the right, U_e.  When both halos span at least CUT (or the tile is at an end of the
-// array) these sums are the exact carries and the tile's outputs are final.
-// Otherwise (dense anchors, H = 0, the ragged last tile) nothing is written
-// and the tile is marked for the redo pass.  Every tile publishes its first
+// array, or the halo reaches the end of the array) these sums are the exact
+// carries and the tile's outputs are final.  Otherwise (dense anchors, H = 0)
+// nothing is written and the tile is marked for the redo pass.  Every tile publishes its first
 // and last anchors and its zero-carry totals for the carry kernels.
 // MODE 1 (redo pass): the marked tiles again, with the exact carries from the
 // carry kernels.
@@ -228,44 +228,54 @@ __global__ void __launch_bounds__(NT, LX_LT_MINB) k_tile_local(const T* __restri
         }
         // MODE 0: the halo terms of this thread (halo element k = q + m NT;
         // k < H: left, H <= k < 2H: right), and the checks that each halo
-        // spans CUT (by the threads holding k = 0 and k = H)
-        T hvL = T(0), hvU = T(0), ringL = T(0), ringR = T(0);  // s_{b-1}, s_e when in the ring
+        // spans CUT (by the threads holding k = 0 and k = H).  A halo comes
+        // from the ring when the copy brought it, else from global memory (the
+        // ragged last tile; a right halo cut short by the end of the array,
+        // which then holds every element to the right and needs no check).
+        T hvL = T(0), hvU = T(0), ringL = T(0), ringR = T(0);  // s_{b-1}, s_e
         int bad[2] = {0, 0};
         if constexpr (MODE == 0) {
             const int q = (int)threadIdx.x;
-            const int64_t e = tile0 + TILE;
+            const int64_t e = min(tile0 + TILE, n);
             if constexpr (H > 0) {
-                const bool haveL = t > 0, haveR = e + H <= n;
-                if (live && !ragged) {
-                    if (haveL) ringL = S0[H - 1];
-                    if (haveR) ringR = S0[H + TILE];
+                const bool needL = t > 0, needR = e < n;
+                const bool ringH = !ragged;                    // halos copied with the tile
+                const bool fullR = e + H <= n;                 // a right halo of H elements
+                if (live) {
+                    if (needL) ringL = ringH ? S0[H - 1] : s_[tile0 - 1];
+                    if (needR) ringR = ringH && fullR ? S0[H + TILE] : s_[e];
 #pragma unroll
                     for (int m = 0; m * NT < 2 * H; ++m) {
                         const int k = q + m * NT;
                         if (k >= 2 * H) break;
                         const bool left = k < H;
-                        const bool have = left ? haveL : haveR;
-                        const bool need = left ? t > 0 : e < n;
-                        if (!have) {
-                            // no halo: exact only at the array's own ends
-                            if (k == 0 || k == H) bad[left ? 0 : 1] = need ? 1 : 0;
-                            continue;
+                        if (!(left ? needL : needR)) continue;
+                        const int64_t jg = left ? tile0 - H + k : e + (k - H);  // global index
+                        if (!left && jg >= n) continue;                      // past the end
+                        const bool inring = ringH && (left || fullR);
+                        const int j = left ? k : (int)(TILE + k);            // ring index
+                        T sj, xj;
+                        if (inring) {
+                            sj = S0[j];
+                            if constexpr (GATHER) xj = __ldg(x_ + ring_p[st * STAGE + j]);
+                            else xj = ring_x[st * STAGE + j];
+                        } else {
+                            sj = s_[jg];
+                            if constexpr (GATHER) xj = __ldg(x_ + perm[jg]);
+                            else xj = x_[jg];
                         }
-                        const int j = left ? k : (int)(TILE + k);  // ring index of element k
                         const T edge = left ? ringL : ringR;
-                        const T sj = S0[j];
-                        T xj;
-                        if constexpr (GATHER) xj = __ldg(x_ + ring_p[st * STAGE + j]);
-                        else xj = ring_x[st * STAGE + j];
                         const T term = dexp<T>(left ? sj - edge : edge - sj) * xj;
                         if (left) hvL += term;
                         else hvU += term;
                         if (k == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
-                        if (k == H) bad[1] = S0[2 * H + TILE - 1] - edge >= ExpCut<T>::v ? 0 : 1;
+                        if (k == H && fullR)
+                            bad[1] = (inring ? S0[2 * H + TILE - 1] : s_[e + H - 1]) - edge >= ExpCut<T>::v ? 0 : 1;
                     }
                 }
+            } else {
+                if (q == 0) bad[0] = (t > 0 || tile0 + TILE < n) ? 1 : 0;  // no halos: final only if alone
             }
-            if (q == 0 && (H == 0 || ragged)) bad[0] = 1;
         }
         // this thread's reads of stage st are ordered before the TMA writes that
         // refill it (generic -> async proxy); the refill is issued after the

@@ -94,8 +94,8 @@ inline TPWs<T, C> tp_carve(Carve& cv, int64_t ntiles) {
 // Halo terms of thread q of a tile: the halo elements k = q + m NT < 2H
 // (k < H: left halo, H <= k < 2H: right halo), summed per side, and the checks
 // that each halo spans CUT (by the threads holding k = 0 and k = H).  A side
-// needs no carry at an end of the array; a side without a halo in the array
-// (the right side of the last-but-one tiles) is marked bad.
+// needs no carry at an end of the array, and a halo that reaches the end of
+// the array needs no check.
 template <class P>
 __device__ __forceinline__ void tp_halo_terms(const P& p, int64_t t, int64_t tile0, int64_t tile1,
                                               typename P::T (&hvL)[P::C], typename P::T (&hvU)[P::C],
@@ -115,19 +115,18 @@ __device__ __forceinline__ void tp_halo_terms(const P& p, int64_t t, int64_t til
         return;
     }
     const bool needL = t > 0, needR = tile1 < n;
-    const bool haveR = tile1 + H <= n;  // the left halo is always in the array (tile0 >= TILE >= H)
-    const T eL = needL ? p.s[tile0 - 1] : T(0), eR = needR && haveR ? p.s[tile1] : T(0);
+    // the left halo is always in the array (tile0 >= TILE >= H); a right halo
+    // cut short by the end of the array holds every element to the right
+    const bool fullR = tile1 + H <= n;
+    const T eL = needL ? p.s[tile0 - 1] : T(0), eR = needR ? p.s[tile1] : T(0);
 #pragma unroll
     for (int m = 0; m * NT < 2 * H; ++m) {
         const int k = q + m * NT;
         if (k >= 2 * H) break;
         const bool left = k < H;
         if (!(left ? needL : needR)) continue;
-        if (!left && !haveR) {
-            if (k == H) bad[1] = 1;
-            continue;
-        }
         const int64_t j = left ? tile0 - H + k : tile1 + (k - H);
+        if (j >= n) continue;
         const T edge = left ? eL : eR;
         T sj, vj[C];
         p.load1(j, sj, vj);
@@ -138,7 +137,7 @@ __device__ __forceinline__ void tp_halo_terms(const P& p, int64_t t, int64_t til
             else hvU[c] += d[c] * vj[c];
         }
         if (k == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
-        if (k == H) bad[1] = p.s[tile1 + H - 1] - edge >= ExpCut<T>::v ? 0 : 1;
+        if (k == H && fullR) bad[1] = p.s[tile1 + H - 1] - edge >= ExpCut<T>::v ? 0 : 1;
     }
 }
 
@@ -241,8 +240,7 @@ __global__ void __launch_bounds__(P::NT) k_tp_redo(P p, TPWs<typename P::T, P::C
 // policy's NIN value arrays come into a shared-memory ring of S stages by 1-D
 // bulk copies (TMA), each full tile with a halo of H elements on both sides
 // (thread q takes the halo elements q, q + NT, ... < 2H, as in k_tp_local).  The ragged last
-// tile goes through the policy's register load and is always listed for the
-// redo pass.
+// tile goes through the policy's register loads.
 //
 // Extra policy members:
 //   static constexpr int NIN, S, MINB;         (value arrays, stages, blocks/SM)
@@ -328,38 +326,44 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
             p.load(r0, s, v, aux);
         }
         // halo terms of this thread (elements k = q + m NT < 2H), the span
-        // checks, the edge anchors
+        // checks, the edge anchors.  A halo comes from the ring when the copy
+        // brought it, else through the policy's single-element load (the
+        // ragged last tile; a right halo cut short by the end of the array,
+        // which then holds every element to the right and needs no check).
         T hvL[C], hvU[C], ringL = T(0), ringR = T(0);
         int bad[2] = {0, 0};
 #pragma unroll
         for (int c = 0; c < C; ++c) hvL[c] = hvU[c] = T(0);
         {
             const int q = (int)threadIdx.x;
-            const bool haveR = tile0 + TILE + H <= n;
-            if (H > 0 && landed && !ragged) {
-                if (needL) ringL = S0[H - 1];
-                if (haveR) ringR = S0[H + TILE];
-            }
-            if (H == 0 || ragged) {
+            const bool fullR = tile1 + H <= n;
+            const bool ringH = !ragged;
+            if (H == 0) {
                 if (q == 0) bad[0] = (needL || needR) ? 1 : 0;
             } else if (landed) {
+                if (needL) ringL = ringH ? S0[H - 1] : p.s[tile0 - 1];
+                if (needR) ringR = ringH && fullR ? S0[H + TILE] : p.s[tile1];
 #pragma unroll
                 for (int m = 0; m * NT < 2 * H; ++m) {
                     const int k = q + m * NT;
                     if (k >= 2 * H) break;
                     const bool left = k < H;
                     if (!(left ? needL : needR)) continue;
-                    if (!left && !haveR) {
-                        if (k == H) bad[1] = 1;
-                        continue;
-                    }
+                    const int64_t jg = left ? tile0 - H + k : tile1 + (k - H);
+                    if (!left && jg >= n) continue;
+                    const bool inring = ringH && (left || fullR);
                     const int j = left ? k : (int)TILE + k;  // ring index
                     const T edge = left ? ringL : ringR;
-                    const T sj = S0[j];
-                    T xe[NIN], vj[C];
+                    T sj, vj[C];
+                    if (inring) {
+                        sj = S0[j];
+                        T xe[NIN];
 #pragma unroll
-                    for (int a = 0; a < NIN; ++a) xe[a] = S0[(a + 1) * STAGE + j];
-                    p.value(xe, vj);
+                        for (int a = 0; a < NIN; ++a) xe[a] = S0[(a + 1) * STAGE + j];
+                        p.value(xe, vj);
+                    } else {
+                        p.load1(jg, sj, vj);
+                    }
                     const Decay<T, C, CT> d = left ? Decay<T, C, CT>(sj, edge) : Decay<T, C, CT>(edge, sj);
 #pragma unroll
                     for (int c = 0; c < C; ++c) {
@@ -367,7 +371,8 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
                         else hvU[c] += d[c] * vj[c];
                     }
                     if (k == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
-                    if (k == H) bad[1] = S0[2 * H + TILE - 1] - edge >= ExpCut<T>::v ? 0 : 1;
+                    if (k == H && fullR)
+                        bad[1] = (inring ? S0[2 * H + TILE - 1] : p.s[tile1 + H - 1]) - edge >= ExpCut<T>::v ? 0 : 1;
                 }
             }
         }
