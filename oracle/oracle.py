@@ -222,6 +222,49 @@ def backward(a, x, g):
     return dx, da
 
 
+def _onesided(sq, sb, vs, dirn):
+    """One-sided decayed sums at ascending query points sq over ascending anchors
+    sb with values vs [k, B] (C routine orc_onesided_sorted, strict inequalities)."""
+    out = np.zeros((sq.size, vs.shape[1]))
+    if sq.size and sb.size:
+        _L().orc_onesided_sorted(sb.size, sq.size, vs.shape[1], _p(sb), _p(vs), _p(sq), dirn, _p(out))
+    return out
+
+
+def signed_general(a, b, v):
+    """S_i = sum_j sign(a_i - b_j) exp(-|a_i - b_j|) v_j with sign(0) = 0: the
+    derivative of the general kernel with respect to a_i ("LAPLEX - La FFT dei
+    Nuclei di Laplace Apprendibili", technical summary §2.3: learnable anchors).
+    The b_j below a_i minus the b_j above it, each side a one-sided decayed sum."""
+    sa, pa = stable_sort(a)
+    sb, pb = stable_sort(b)
+    v2, flat = _cols(v)
+    vs = np.ascontiguousarray(v2[pb])
+    ss = _onesided(sa, sb, vs, 1) - _onesided(sa, sb, vs, -1)
+    out = np.empty_like(ss)
+    out[pa] = ss
+    return out.ravel() if flat else out
+
+
+def backward_general(a, b, x, g):
+    """Backward pass of L = <g, K x>, K_ij = exp(-|a_i - b_j|), a in R^n,
+    b in R^k: dx = K^T g, da_i = -g_i S(a <- b, x)_i, db_j = -x_j S(b <- a, g)_j
+    with S the signed sums above (the derivative of exp(-|a_i - b_j|) is
+    -sign(a_i - b_j) exp(-|a_i - b_j|) in a_i and +sign(a_i - b_j) ... in b_j)."""
+    x, g = _f64(x), _f64(g)
+    dx = general_T(a, b, g)
+    da = -g * signed_general(a, b, x)
+    db = -x * signed_general(b, a, g)
+    return dx, da, db
+
+
+def norm_backward_general(a, b, x, g):
+    """Bounds of |dx|, |da|, |db| term by term: K^T|g|, |g| K|x|, |x| K^T|g|."""
+    x, g = np.abs(_f64(x)), np.abs(_f64(g))
+    ktg = general(b, a, g)
+    return ktg, g * general(a, b, x), x * ktg
+
+
 # ---------------------------------------------------------------------------
 # rows of the dense definition at any size (sampled parity)
 # ---------------------------------------------------------------------------

@@ -383,6 +383,56 @@ def test_far_mass_limits():
 
 
 # ---------------------------------------------------------------------------
+# general-case anchor gradients (learnable a and b)
+# ---------------------------------------------------------------------------
+
+def test_signed_general_brute_force():
+    """S(a <- b, v) against the double loop with sign(0) = 0: ties between a and
+    b, ties inside b, several columns, a and b of different sizes."""
+    rng = np.random.default_rng(18)
+    a = np.round(rng.uniform(0, 6, 40), 1)
+    b = np.concatenate([np.round(rng.uniform(-1, 7, 30), 1), a[:5]])
+    v = rng.normal(size=(35, 2))
+    brute = np.zeros((40, 2))
+    for i in range(40):
+        for j in range(35):
+            brute[i] += np.sign(a[i] - b[j]) * math.exp(-abs(a[i] - b[j])) * v[j]
+    np.testing.assert_allclose(O.signed_general(a, b, v), brute, atol=1e-13)
+    # b = a reduces to the symmetric signed sums (a separate C routine)
+    s2 = np.sort(np.round(rng.uniform(0, 6, 50), 0))
+    v2 = rng.normal(size=50)
+    np.testing.assert_allclose(O.signed_general(s2, s2, v2), O.signed_sorted(s2, v2), atol=1e-13)
+
+
+def _loss_general(a, b, x, g):
+    return float(g @ O.dense_matvec(a, x, b=b))
+
+
+def test_backward_general_central_differences():
+    """dx, da, db of L = <g, K(a, b) x> against central differences of the dense
+    definition (distinct anchors; a and b interleaved)."""
+    rng = np.random.default_rng(19)
+    a = rng.uniform(0, 4, 12)
+    b = rng.uniform(0, 4, 9)
+    x, g = rng.normal(size=9), rng.normal(size=12)
+    dx, da, db = O.backward_general(a, b, x, g)
+    np.testing.assert_allclose(dx, O.dense_matrix(a, b=b).T @ g, atol=1e-13)
+    h = 1e-6
+    for i in range(12):
+        ap, am = a.copy(), a.copy()
+        ap[i] += h
+        am[i] -= h
+        fd = (_loss_general(ap, b, x, g) - _loss_general(am, b, x, g)) / (2 * h)
+        assert abs(da[i] - fd) < 1e-7, i
+    for j in range(9):
+        bp, bm = b.copy(), b.copy()
+        bp[j] += h
+        bm[j] -= h
+        fd = (_loss_general(a, bp, x, g) - _loss_general(a, bm, x, g)) / (2 * h)
+        assert abs(db[j] - fd) < 1e-7, j
+
+
+# ---------------------------------------------------------------------------
 # the pins catch planted mistakes (mutants built on the CPU from the oracle)
 # ---------------------------------------------------------------------------
 
