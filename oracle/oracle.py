@@ -103,6 +103,16 @@ def dense_matrix(a, b=None, phi=None, psi=None):
     return K
 
 
+def gram_matrix(a, b, D=None):
+    """M = A diag(D) A^T with A_ij = exp(-|a_i - b_j|) (a in R^n, b in R^k; D = 1
+    when omitted): the weighted Gram matrix of the anchors ("LAPLEX - La FFT dei
+    Nuclei di Laplace Apprendibili", technical summary §2.2 "Operatori di Gram"),
+    by its definition, densely.  Small sizes only."""
+    A = dense_matrix(a, b)
+    d = np.ones(A.shape[1]) if D is None else _f64(D)
+    return (A * d[None, :]) @ A.T
+
+
 def dense_matvec(a, x, b=None, phi=None, psi=None):
     return dense_matrix(a, b, phi, psi) @ _f64(x)
 

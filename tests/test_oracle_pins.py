@@ -433,6 +433,31 @@ def test_backward_general_central_differences():
 
 
 # ---------------------------------------------------------------------------
+# weighted Gram matrix A diag(D) A^T
+# ---------------------------------------------------------------------------
+
+def test_gram_matrix_brute_force_and_structure():
+    """The triple loop of the definition; symmetric, positive semi-definite for
+    D >= 0; one b point gives the rank-one D e^{-|a_i - b|} e^{-|a_j - b|}."""
+    rng = np.random.default_rng(20)
+    a = np.round(rng.uniform(0, 5, 9), 1)
+    b = np.concatenate([np.round(rng.uniform(-1, 6, 6), 1), a[:2]])
+    D = rng.uniform(0.1, 2.0, 8)
+    brute = np.zeros((9, 9))
+    for i in range(9):
+        for j in range(9):
+            brute[i, j] = sum(D[l] * math.exp(-abs(a[i] - b[l])) * math.exp(-abs(a[j] - b[l]))
+                              for l in range(8))
+    M = O.gram_matrix(a, b, D)
+    np.testing.assert_allclose(M, brute, rtol=1e-13)
+    np.testing.assert_allclose(M, M.T, rtol=1e-15)
+    assert np.linalg.eigvalsh(M).min() > -1e-12
+    one = O.gram_matrix(a, np.array([2.3]), np.array([0.7]))
+    u = np.exp(-np.abs(a - 2.3))
+    np.testing.assert_allclose(one, 0.7 * np.outer(u, u), rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------
 # the pins catch planted mistakes (mutants built on the CPU from the oracle)
 # ---------------------------------------------------------------------------
 
