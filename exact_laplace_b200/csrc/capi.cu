@@ -85,6 +85,13 @@ size_t body_bytes(laplex_op op, int64_t n, int64_t k, int64_t B, int f64) {
             return u + m;
         }
         case LAPLEX_OP_BACKWARD: return lx::bwd_ws_bytes(n, f64);
+        case LAPLEX_OP_BACKWARD_GENERAL: {
+            // K^T g first (the general product's workspace), then the two signed
+            // sums one after the other (each over one side)
+            const size_t g = std::max(lx::gen_ws_bytes(n, k, 1, false, f64), lx::gen_ws_bytes(k, n, 1, false, f64));
+            const size_t sg = std::max(lx::sgen_ws_bytes(n, f64), lx::sgen_ws_bytes(k, f64));
+            return std::max(g, sg);
+        }
     }
     return 0;
 }
@@ -147,7 +154,7 @@ laplex_status laplex_workspace_size(laplex_op op, int64_t n, int64_t k, int64_t 
     laplex_status st = check_sizes(n, k, B);
     if (st != LAPLEX_OK) return st;
     if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
-    REQ(op >= LAPLEX_OP_SORT && op <= LAPLEX_OP_BACKWARD, "unknown op %d", (int)op);
+    REQ(op >= LAPLEX_OP_SORT && op <= LAPLEX_OP_BACKWARD_GENERAL, "unknown op %d", (int)op);
     *bytes = lx::HEADER_BYTES + body_bytes(op, n, k, B, dt == LAPLEX_F64);
     return ok();
 }
@@ -439,6 +446,46 @@ laplex_status laplex_backward(const void* sorted, const int32_t* perm, int64_t n
                                   (const double*)g, (double*)dx, (double*)da, ws_body(ws), body,
                                   ws_status(ws), s);
     if (e != cudaSuccess) return cuda_fail(e, "laplex_backward");
+    return ok();
+}
+
+laplex_status laplex_backward_general(const void* sa, const int32_t* pa, int64_t n, const void* sb,
+                                      const int32_t* pb, int64_t k, const void* x, const void* g,
+                                      void* dx, void* da, void* db, laplex_dtype dt, void* ws,
+                                      size_t ws_bytes, void* stream) {
+    laplex_status st = check_sizes(n, k, 1);
+    if (st != LAPLEX_OK) return st;
+    if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
+    REQ_PTR(sa, n > 0);
+    REQ_PTR(sb, k > 0);
+    REQ_PTR(g, n > 0);
+    REQ_PTR(da, n > 0);
+    REQ_PTR(x, k > 0);
+    REQ_PTR(dx, k > 0);
+    REQ_PTR(db, k > 0);
+    if (pa) REQ_PTR(pa, n > 0);
+    if (pb) REQ_PTR(pb, k > 0);
+    if ((st = check_ws(LAPLEX_OP_BACKWARD_GENERAL, n, k, 1, dt, ws, ws_bytes)) != LAPLEX_OK) return st;
+    if (n == 0 && k == 0) return ok();
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    // dx = K^T g (the transposed general product; zero when n = 0)
+    if (k > 0) {
+        e = dt == LAPLEX_F32
+                ? run_gen<float>(sa, pa, n, sb, pb, k, g, dx, 1, 1, nullptr, nullptr, nullptr, nullptr,
+                                 ws, ws_bytes, s, false)
+                : run_gen<double>(sa, pa, n, sb, pb, k, g, dx, 1, 1, nullptr, nullptr, nullptr, nullptr,
+                                  ws, ws_bytes, s, false);
+        if (e != cudaSuccess) return cuda_fail(e, "laplex_backward_general (K^T g)");
+    }
+    const size_t body = ws_bytes - lx::HEADER_BYTES;
+    e = dt == LAPLEX_F32
+            ? lx::sgen_run<float>((const float*)sa, pa, n, (const float*)sb, pb, k, (const float*)x,
+                                  (const float*)g, (float*)da, (float*)db, ws_body(ws), body, s)
+            : lx::sgen_run<double>((const double*)sa, pa, n, (const double*)sb, pb, k,
+                                   (const double*)x, (const double*)g, (double*)da, (double*)db,
+                                   ws_body(ws), body, s);
+    if (e != cudaSuccess) return cuda_fail(e, "laplex_backward_general (signed sums)");
     return ok();
 }
 

@@ -109,4 +109,11 @@ template <typename T>
 cudaError_t bwd_run(const T* s, const int32_t* perm, int64_t n, const T* x, const T* g, T* dx,
                     T* da, void* ws, size_t ws_bytes, uint32_t* status, cudaStream_t st);
 
+// -------------------------------------------------------------- general backward
+size_t sgen_ws_bytes(int64_t len, int f64);
+template <typename T>
+cudaError_t sgen_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, const int32_t* pb,
+                     int64_t k, const T* x, const T* g, T* da, T* db, void* ws, size_t ws_bytes,
+                     cudaStream_t st);
+
 }  // namespace lx

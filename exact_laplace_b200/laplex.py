@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "liblaplex.so")
 
 OK, EINVAL, ENONFINITE, EWORKSPACE, ECUDA, ETIMEOUT = range(6)
 F32, F64 = 0, 1
-OP_SORT, OP_SYM, OP_GENERAL, OP_PHASED, OP_GRAM, OP_BACKWARD = range(6)
+OP_SORT, OP_SYM, OP_GENERAL, OP_PHASED, OP_GRAM, OP_BACKWARD, OP_BACKWARD_GENERAL = range(7)
 
 _lib = None
 _lock = threading.Lock()
@@ -61,6 +61,8 @@ SIGNATURES = {
                      ctypes.c_size_t, _P], ctypes.c_int),
     "laplex_backward": ([_P, _P, _I64, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P],
                         ctypes.c_int),
+    "laplex_backward_general": ([_P, _P, _I64, _P, _P, _I64, _P, _P, _P, _P, _P, ctypes.c_int, _P,
+                                 ctypes.c_size_t, _P], ctypes.c_int),
     "laplex_matvec_sym_noalloc": ([_P, _P, _I64, _P, _P, _P], ctypes.c_int),
     "laplex_set_profile_events": ([_P, _P], ctypes.c_int),
 }
@@ -266,6 +268,21 @@ def backward(sorted_anchors, x, g, perm=None, dx_out=None, da_out=None):
     _check(lib().laplex_backward(_ptr(sorted_anchors), _ptr(perm), n, _ptr(x), _ptr(g), _ptr(dx),
                                  _ptr(da), _dt(x), _ptr(ws), nb, _stream(dev)))
     return dx, da
+
+
+def backward_general(sa, sb, x, g, pa=None, pb=None):
+    """(dx, da, db) of L = <g, K x>, K_ij = exp(-|a_i - b_j|): dx = K^T g and the
+    anchor gradients (sign(0) = 0 at ties).  g, da follow pa; x, dx, db follow pb."""
+    dev = _dev(sa, sb, x, g, _perm(pa), _perm(pb))
+    n, k = sa.numel(), sb.numel()
+    dx = torch.empty_like(x)
+    da = torch.empty_like(g)
+    db = torch.empty_like(x)
+    ws, nb = _ws(OP_BACKWARD_GENERAL, n, k, 1, x.dtype, dev)
+    _check(lib().laplex_backward_general(_ptr(sa), _ptr(pa), n, _ptr(sb), _ptr(pb), k, _ptr(x), _ptr(g),
+                                         _ptr(dx), _ptr(da), _ptr(db), _dt(x), _ptr(ws), nb,
+                                         _stream(dev)))
+    return dx, da, db
 
 
 def matvec_sym_noalloc(sorted_anchors: torch.Tensor, x: torch.Tensor, perm=None, out=None):

@@ -70,7 +70,8 @@ typedef enum {
     LAPLEX_OP_MATVEC_GENERAL = 2,
     LAPLEX_OP_MATVEC_PHASED = 3,
     LAPLEX_OP_GRAM = 4,
-    LAPLEX_OP_BACKWARD = 5
+    LAPLEX_OP_BACKWARD = 5,
+    LAPLEX_OP_BACKWARD_GENERAL = 6
 } laplex_op;
 
 /* Library ABI version (major*10000 + minor*100 + patch). */
@@ -180,6 +181,24 @@ laplex_status laplex_gram(const void* sa, const int32_t* pa, const void* phi, in
 laplex_status laplex_backward(const void* sorted, const int32_t* perm, int64_t n,
                               const void* x, const void* g, void* dx, void* da,
                               laplex_dtype dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Backward pass of the general product: L = <g, K x>, K_ij = exp(-|a_i - b_j|),
+ * a in R^n, b in R^k, with respect to x and both anchor sets (learnable
+ * anchors: summary §2.3):
+ *   dx = K^T g,
+ *   da_i = -g_i sum_j sign(a_i - b_j) K_ij x_j,
+ *   db_j = -x_j sum_i sign(b_j - a_i) K_ij g_i,      sign(0) = 0.
+ *   sa [n], pa [n]|NULL, sb [k], pb [k]|NULL: sorted anchors and perms as in
+ *              laplex_matvec_general; g, da [n] follow pa, x, dx, db [k] follow pb.
+ *   B = 1.  Workspace: laplex_workspace_size(LAPLEX_OP_BACKWARD_GENERAL, n, k, 1, ...).
+ * n = 0 or k = 0: the outputs on the other side are zero.
+ */
+laplex_status laplex_backward_general(const void* sa, const int32_t* pa, int64_t n,
+                                      const void* sb, const int32_t* pb, int64_t k,
+                                      const void* x, const void* g, void* dx, void* da,
+                                      void* db, laplex_dtype dtype, void* ws, size_t ws_bytes,
+                                      void* stream);
 
 /*
  * Profiling hook (no counterpart in the paper): for the following calls on the
