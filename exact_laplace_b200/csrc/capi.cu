@@ -92,6 +92,7 @@ size_t body_bytes(laplex_op op, int64_t n, int64_t k, int64_t B, int f64) {
             const size_t sg = std::max(lx::sgen_ws_bytes(n, f64), lx::sgen_ws_bytes(k, f64));
             return std::max(g, sg);
         }
+        case LAPLEX_OP_GRAM_MATRIX: return lx::grammat_ws_bytes(n, k, f64);
     }
     return 0;
 }
@@ -154,7 +155,7 @@ laplex_status laplex_workspace_size(laplex_op op, int64_t n, int64_t k, int64_t 
     laplex_status st = check_sizes(n, k, B);
     if (st != LAPLEX_OK) return st;
     if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
-    REQ(op >= LAPLEX_OP_SORT && op <= LAPLEX_OP_BACKWARD_GENERAL, "unknown op %d", (int)op);
+    REQ(op >= LAPLEX_OP_SORT && op <= LAPLEX_OP_GRAM_MATRIX, "unknown op %d", (int)op);
     *bytes = lx::HEADER_BYTES + body_bytes(op, n, k, B, dt == LAPLEX_F64);
     return ok();
 }
@@ -486,6 +487,33 @@ laplex_status laplex_backward_general(const void* sa, const int32_t* pa, int64_t
                                    (const double*)x, (const double*)g, (double*)da, (double*)db,
                                    ws_body(ws), body, s);
     if (e != cudaSuccess) return cuda_fail(e, "laplex_backward_general (signed sums)");
+    return ok();
+}
+
+laplex_status laplex_gram_matrix(const void* sa, const int32_t* pa, int64_t n, const void* sb,
+                                 const int32_t* pb, int64_t k, const void* D, void* M, int64_t ldm,
+                                 laplex_dtype dt, void* ws, size_t ws_bytes, void* stream) {
+    laplex_status st = check_sizes(n, k, 1);
+    if (st != LAPLEX_OK) return st;
+    if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
+    REQ(ldm >= n, "ldm = %lld below n = %lld", (long long)ldm, (long long)n);
+    REQ_PTR(sa, n > 0);
+    REQ_PTR(sb, k > 0);
+    REQ_PTR(M, n > 0);
+    if (pa) REQ_PTR(pa, n > 0);
+    if (pb) REQ_PTR(pb, k > 0);
+    if (D) REQ_PTR(D, k > 0);
+    if ((st = check_ws(LAPLEX_OP_GRAM_MATRIX, n, k, 1, dt, ws, ws_bytes)) != LAPLEX_OK) return st;
+    if (n == 0) return ok();
+    const size_t body = ws_bytes - lx::HEADER_BYTES;
+    cudaStream_t s = (cudaStream_t)stream;
+    const cudaError_t e =
+        dt == LAPLEX_F32
+            ? lx::grammat_run<float>((const float*)sa, pa, n, (const float*)sb, pb, k, (const float*)D,
+                                     (float*)M, ldm, ws_body(ws), body, s)
+            : lx::grammat_run<double>((const double*)sa, pa, n, (const double*)sb, pb, k, (const double*)D,
+                                      (double*)M, ldm, ws_body(ws), body, s);
+    if (e != cudaSuccess) return cuda_fail(e, "laplex_gram_matrix");
     return ok();
 }
 

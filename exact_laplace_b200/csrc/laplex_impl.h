@@ -111,6 +111,10 @@ cudaError_t bwd_run(const T* s, const int32_t* perm, int64_t n, const T* x, cons
 
 // -------------------------------------------------------------- general backward
 size_t sgen_ws_bytes(int64_t len, int f64);
+size_t grammat_ws_bytes(int64_t n, int64_t k, int f64);
+template <typename T>
+cudaError_t grammat_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, const int32_t* pb, int64_t k,
+                        const T* D, T* M, int64_t ldm, void* ws, size_t ws_bytes, cudaStream_t st);
 template <typename T>
 cudaError_t sgen_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, const int32_t* pb,
                      int64_t k, const T* x, const T* g, T* da, T* db, void* ws, size_t ws_bytes,

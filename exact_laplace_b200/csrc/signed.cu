@@ -185,6 +185,197 @@ cudaError_t sgen_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, con
     return signed_pass<T>(sa, pa, n, g, sb, pb, k, x, db, ws, ws_bytes, st);
 }
 
+// ------------------------------------------------------------------ weighted Gram matrix
+// M = A diag(D) A^T, A_ij = exp(-|a_i - b_j|) (summary §2.2 "Operatori di
+// Gram").  For a_i <= a_j the terms split at a_i and a_j:
+//     b <= a_i:        D_b exp(-(a_i - b)) exp(-(a_j - b)) = e^{a_i - a_j} D_b e^{-2(a_i - b)}
+//     a_i < b <= a_j:  D_b exp(-(b - a_i)) exp(-(a_j - b)) = e^{a_i - a_j} D_b
+//     b > a_j:         D_b exp(-(b - a_i)) exp(-(b - a_j)) = e^{a_i - a_j} D_b e^{-2(b - a_j)}
+// so M_ij = e^{a_i - a_j} (Lw_i + (P_j - P_i) + Rw_j) with, per a-point,
+// Lw = sum_{b <= a} D e^{-2(a - b)}, Rw = sum_{b > a} D e^{-2(b - a)} (one-sided
+// scans over 2b) and P = sum_{b <= a} D (fp64 prefix sums: their difference
+// must not cancel).  Work: O(k) scans, O(n log k) searches, O(n^2) fill.
+
+constexpr int PS_NT = 256, PS_PT = 16, PS_BT = PS_NT * PS_PT;  // prefix sums: elements per block
+
+template <typename T>
+__global__ void __launch_bounds__(PS_NT) k_psum_blocks(const T* __restrict__ D, const int32_t* __restrict__ pb,
+                                                       int64_t k, double* __restrict__ bsum) {
+    __shared__ double red[PS_NT / 32];
+    const int64_t b0 = (int64_t)blockIdx.x * PS_BT + (int64_t)threadIdx.x * PS_PT;
+    double acc = 0.0;
+    for (int i = 0; i < PS_PT; ++i) {
+        const int64_t r = b0 + i;
+        if (r < k) acc += D ? (double)D[pb ? (int64_t)pb[r] : r] : 1.0;
+    }
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(FULL, acc, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int w = 0; w < PS_NT / 32; ++w) t += red[w];
+        bsum[blockIdx.x] = t;
+    }
+}
+
+// exclusive prefix of the block sums, one block (each thread a run of them)
+__global__ void __launch_bounds__(1024) k_psum_scan(double* __restrict__ bsum, int64_t nb) {
+    __shared__ double part[1024];
+    const int64_t per = (nb + 1023) / 1024;
+    const int64_t b0 = (int64_t)threadIdx.x * per;
+    double acc = 0.0;
+    for (int64_t i = 0; i < per && b0 + i < nb; ++i) acc += bsum[b0 + i];
+    part[threadIdx.x] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double run = 0.0;
+        for (int t = 0; t < 1024; ++t) {
+            const double v = part[t];
+            part[t] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    double run = part[threadIdx.x];
+    for (int64_t i = 0; i < per && b0 + i < nb; ++i) {
+        const double v = bsum[b0 + i];
+        bsum[b0 + i] = run;
+        run += v;
+    }
+}
+
+// P[r] = sum_{l <= r} D_l (sorted order)
+template <typename T>
+__global__ void __launch_bounds__(PS_NT) k_psum_apply(const T* __restrict__ D, const int32_t* __restrict__ pb,
+                                                      int64_t k, const double* __restrict__ boff,
+                                                      double* __restrict__ P) {
+    __shared__ double part[PS_NT];
+    const int64_t b0 = (int64_t)blockIdx.x * PS_BT + (int64_t)threadIdx.x * PS_PT;
+    double v[PS_PT], acc = 0.0;
+    for (int i = 0; i < PS_PT; ++i) {
+        const int64_t r = b0 + i;
+        v[i] = r < k ? (D ? (double)D[pb ? (int64_t)pb[r] : r] : 1.0) : 0.0;
+        acc += v[i];
+    }
+    part[threadIdx.x] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double run = boff[blockIdx.x];
+        for (int t = 0; t < PS_NT; ++t) {
+            const double x = part[t];
+            part[t] = run;
+            run += x;
+        }
+    }
+    __syncthreads();
+    double run = part[threadIdx.x];
+    for (int i = 0; i < PS_PT; ++i) {
+        run += v[i];
+        if (b0 + i < k) P[b0 + i] = run;
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_double(const T* __restrict__ s, int64_t k, T* __restrict__ s2) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < k; r += stride) s2[r] = T(2) * s[r];
+}
+
+// per sorted a-point: Lw, Rw, P (and the inverse of pa)
+template <typename T>
+__global__ void __launch_bounds__(256) k_gram_points(const T* __restrict__ sa, const int32_t* __restrict__ pa,
+                                                     int64_t n, const T* __restrict__ sb, int64_t k,
+                                                     const T* __restrict__ F, const T* __restrict__ G,
+                                                     const double* __restrict__ P, T* __restrict__ Lw,
+                                                     T* __restrict__ Rw, double* __restrict__ Pa,
+                                                     int32_t* __restrict__ inv) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const T q = sa[i];
+        const int64_t ub = bound<T>(sb, k, q, true);  // #{b <= a_i}
+        Lw[i] = ub > 0 ? F[ub - 1] * dexp<T>(T(2) * (sb[ub - 1] - q)) : T(0);
+        Rw[i] = ub < k ? G[ub] * dexp<T>(T(2) * (q - sb[ub])) : T(0);
+        Pa[i] = ub > 0 ? P[ub - 1] : 0.0;
+        if (pa) inv[pa[i]] = (int32_t)i;
+    }
+}
+
+// M[r][c], a block per row r (rows and columns in the order of pa, or sorted
+// order without it)
+template <typename T>
+__global__ void __launch_bounds__(256) k_gram_fill(const T* __restrict__ sa, const int32_t* __restrict__ inv,
+                                                   int64_t n, const T* __restrict__ Lw, const T* __restrict__ Rw,
+                                                   const double* __restrict__ Pa, T* __restrict__ M, int64_t ldm) {
+    const int64_t r = blockIdx.x;
+    const int64_t i = inv ? (int64_t)inv[r] : r;
+    const T ai = sa[i], Li = Lw[i], Ri = Rw[i];
+    const double Pi = Pa[i];
+    T* row = M + r * ldm;
+    for (int64_t c = threadIdx.x; c < n; c += blockDim.x) {
+        const int64_t j = inv ? (int64_t)inv[c] : c;
+        const T aj = sa[j];
+        T v;
+        if (j >= i) v = dexp<T>(ai - aj) * (Li + (T)(Pa[j] - Pi) + Rw[j]);
+        else v = dexp<T>(aj - ai) * (Lw[j] + (T)(Pi - Pa[j]) + Ri);
+        row[c] = v;
+    }
+}
+
+size_t grammat_ws_bytes(int64_t n, int64_t k, int f64) {
+    const size_t es = f64 ? 8 : 4;
+    const int64_t nb = std::max<int64_t>(1, (k + PS_BT - 1) / PS_BT);
+    return Carve::need((size_t)std::max<int64_t>(k, 1), es) + sgen_ws_bytes(k, f64) +
+           Carve::need((size_t)std::max<int64_t>(k, 1), 8) + Carve::need((size_t)nb, 8) +
+           2 * Carve::need((size_t)std::max<int64_t>(n, 1), es) + Carve::need((size_t)std::max<int64_t>(n, 1), 8) +
+           Carve::need((size_t)std::max<int64_t>(n, 1), 4);
+}
+
+template <typename T>
+cudaError_t grammat_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, const int32_t* pb, int64_t k,
+                        const T* D, T* M, int64_t ldm, void* ws, size_t ws_bytes, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    Carve cv(ws, ws_bytes);
+    T* s2 = cv.take<T>(std::max<int64_t>(k, 1));
+    T* F = cv.take<T>(std::max<int64_t>(k, 1));
+    T* G = cv.take<T>(std::max<int64_t>(k, 1));
+    double* P = cv.take<double>(std::max<int64_t>(k, 1));
+    const int64_t nb = std::max<int64_t>(1, (k + PS_BT - 1) / PS_BT);
+    double* bsum = cv.take<double>(nb);
+    T* Lw = cv.take<T>(n);
+    T* Rw = cv.take<T>(n);
+    double* Pa = cv.take<double>(n);
+    int32_t* inv = cv.take<int32_t>(n);
+    if (!cv.ok) return cudaErrorInvalidValue;
+    int sms = 0;
+    cudaError_t e = tp_sm_count(sms);
+    if (e != cudaSuccess) return e;
+    const int64_t gb = std::max<int64_t>(1, (int64_t)sms * 8);
+    if (k > 0) {
+        k_double<T><<<(unsigned)std::min<int64_t>(gb, (k + 255) / 256), 256, 0, st>>>(sb, k, s2);
+        OneSidedTP<T, os_E((int)sizeof(T))> p;
+        p.n = k;
+        p.s = s2;
+        p.perm = pb;
+        p.v = D;
+        p.F = F;
+        p.G = G;
+        e = tp_run(p, cv.base + cv.off, cv.cap - cv.off, st);
+        if (e != cudaSuccess) return e;
+        k_psum_blocks<T><<<(unsigned)nb, PS_NT, 0, st>>>(D, pb, k, bsum);
+        k_psum_scan<<<1, 1024, 0, st>>>(bsum, nb);
+        k_psum_apply<T><<<(unsigned)nb, PS_NT, 0, st>>>(D, pb, k, bsum, P);
+    }
+    k_gram_points<T><<<(unsigned)std::min<int64_t>(gb, (n + 255) / 256), 256, 0, st>>>(sa, pa, n, sb, k, F, G, P,
+                                                                                      Lw, Rw, Pa, inv);
+    k_gram_fill<T><<<(unsigned)n, 256, 0, st>>>(sa, pa ? inv : nullptr, n, Lw, Rw, Pa, M, ldm);  // a block per row
+    return cudaGetLastError();
+}
+
+template cudaError_t grammat_run<float>(const float*, const int32_t*, int64_t, const float*, const int32_t*,
+                                        int64_t, const float*, float*, int64_t, void*, size_t, cudaStream_t);
+template cudaError_t grammat_run<double>(const double*, const int32_t*, int64_t, const double*, const int32_t*,
+                                         int64_t, const double*, double*, int64_t, void*, size_t, cudaStream_t);
+
 template cudaError_t sgen_run<float>(const float*, const int32_t*, int64_t, const float*, const int32_t*,
                                      int64_t, const float*, const float*, float*, float*, void*, size_t,
                                      cudaStream_t);

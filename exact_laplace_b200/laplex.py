@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "liblaplex.so")
 
 OK, EINVAL, ENONFINITE, EWORKSPACE, ECUDA, ETIMEOUT = range(6)
 F32, F64 = 0, 1
-OP_SORT, OP_SYM, OP_GENERAL, OP_PHASED, OP_GRAM, OP_BACKWARD, OP_BACKWARD_GENERAL = range(7)
+OP_SORT, OP_SYM, OP_GENERAL, OP_PHASED, OP_GRAM, OP_BACKWARD, OP_BACKWARD_GENERAL, OP_GRAM_MATRIX = range(8)
 
 _lib = None
 _lock = threading.Lock()
@@ -63,6 +63,8 @@ SIGNATURES = {
                         ctypes.c_int),
     "laplex_backward_general": ([_P, _P, _I64, _P, _P, _I64, _P, _P, _P, _P, _P, ctypes.c_int, _P,
                                  ctypes.c_size_t, _P], ctypes.c_int),
+    "laplex_gram_matrix": ([_P, _P, _I64, _P, _P, _I64, _P, _P, _I64, ctypes.c_int, _P, ctypes.c_size_t, _P],
+                           ctypes.c_int),
     "laplex_matvec_sym_noalloc": ([_P, _P, _I64, _P, _P, _P], ctypes.c_int),
     "laplex_set_profile_events": ([_P, _P], ctypes.c_int),
 }
@@ -283,6 +285,18 @@ def backward_general(sa, sb, x, g, pa=None, pb=None):
                                          _ptr(dx), _ptr(da), _ptr(db), _dt(x), _ptr(ws), nb,
                                          _stream(dev)))
     return dx, da, db
+
+
+def gram_matrix(sa, sb, D=None, pa=None, pb=None, out=None):
+    """M = A diag(D) A^T, A_ij = exp(-|a_i - b_j|), as an [n, n] tensor (rows and
+    columns follow pa; sorted order without it).  D follows pb; None means 1."""
+    dev = _dev(sa, sb, D, _perm(pa), _perm(pb), out)
+    n, k = sa.numel(), sb.numel()
+    M = torch.empty((n, n), dtype=sa.dtype, device=dev) if out is None else out
+    ws, nb = _ws(OP_GRAM_MATRIX, n, k, 1, sa.dtype, dev)
+    _check(lib().laplex_gram_matrix(_ptr(sa), _ptr(pa), n, _ptr(sb), _ptr(pb), k, _ptr(D), _ptr(M),
+                                    M.stride(0) if n else max(n, 1), _dt(sa), _ptr(ws), nb, _stream(dev)))
+    return M
 
 
 def matvec_sym_noalloc(sorted_anchors: torch.Tensor, x: torch.Tensor, perm=None, out=None):

@@ -71,7 +71,8 @@ typedef enum {
     LAPLEX_OP_MATVEC_PHASED = 3,
     LAPLEX_OP_GRAM = 4,
     LAPLEX_OP_BACKWARD = 5,
-    LAPLEX_OP_BACKWARD_GENERAL = 6
+    LAPLEX_OP_BACKWARD_GENERAL = 6,
+    LAPLEX_OP_GRAM_MATRIX = 7
 } laplex_op;
 
 /* Library ABI version (major*10000 + minor*100 + patch). */
@@ -199,6 +200,21 @@ laplex_status laplex_backward_general(const void* sa, const int32_t* pa, int64_t
                                       const void* x, const void* g, void* dx, void* da,
                                       void* db, laplex_dtype dtype, void* ws, size_t ws_bytes,
                                       void* stream);
+
+/*
+ * Weighted Gram matrix M = A diag(D) A^T, A_ij = exp(-|a_i - b_j|) (summary
+ * §2.2 "Operatori di Gram"), in O(n^2 + k log n): per a-point one-sided sums
+ * over b and fp64 prefix sums of D, then
+ *   M_ij = exp(a_i - a_j) (Lw_i + sum_{a_i < b <= a_j} D_b + Rw_j)   (a_i <= a_j).
+ *   sa [n], pa [n]|NULL, sb [k], pb [k]|NULL: sorted anchors and perms.
+ *   D [k]|NULL: weights on b (follow pb); NULL means 1.
+ *   M [n, ldm] row-major, ldm >= n: rows and columns follow pa (sorted order
+ *   when pa is NULL).  Every entry in the first n columns is written.
+ *   Workspace: laplex_workspace_size(LAPLEX_OP_GRAM_MATRIX, n, k, 1, ...).
+ */
+laplex_status laplex_gram_matrix(const void* sa, const int32_t* pa, int64_t n, const void* sb,
+                                 const int32_t* pb, int64_t k, const void* D, void* M, int64_t ldm,
+                                 laplex_dtype dtype, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Profiling hook (no counterpart in the paper): for the following calls on the

@@ -46,9 +46,9 @@ def test_version_and_status_strings(L):
 
 def test_workspace_size_host_only(L):
     from exact_laplace_b200 import laplex as X
-    for op in range(7):
+    for op in range(8):
         for n in (0, 1, 4096, 1 << 24):
-            assert X.workspace_size(op, n, 1000 if op in (2, 3, 4, 6) else 0, 1) >= 256
+            assert X.workspace_size(op, n, 1000 if op in (2, 3, 4, 6, 7) else 0, 1) >= 256
     with pytest.raises(X.LaplexError) as e:
         X.workspace_size(1, -1)
     assert e.value.status == X.EINVAL
