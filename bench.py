@@ -23,6 +23,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -158,6 +159,16 @@ def cpu_baseline(n_total, seed, budget_s=10.0, m=1 << 24):
                       f"workload), fp64 sequential recurrences, {el:.1f} s"}
 
 
+def workload_config(n, world):
+    """The config of the headline workload, the same for both arms."""
+    e = int(round(math.log2(n))) if n > 0 and (n & (n - 1)) == 0 else None
+    size = f"2^{e}" if e is not None else str(n)
+    return {"workload": f"symmetric LAPLEX matvec y=Kx, K_ij=exp(-|a_i-a_j|), n={size} anchors "
+                        f"U(0,{size}) pre-sorted, x~N(0,1), B=1, fp32",
+            "n": n, "B": 1, "seed": "rank", "parallelism": f"replicas x{world}",
+            "l2": f"inputs {12 * n / 1e9:.1f} GB per step vs 126 MB L2 (no flush needed above it)"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -177,11 +188,10 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": "symmetric LAPLEX matvec, pre-sorted anchors U(0,2^30), "
-                                   "x~N(0,1), B=1; reference arm = fp64 CPU oracle on a "
-                                   f"{m}-anchor sample per step", "n": args.n, "B": 1},
+            "config": workload_config(args.n, args.gpus),
             "cpu_baseline": {"value": val, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{m} contiguous anchors per step, same density"},
+                             "sample": f"{m} contiguous anchors of the workload's density per "
+                                       "step, fp64 sequential recurrences on one host core"},
             "e2e": {"value": val, "unit": "Gelem/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -436,10 +446,7 @@ def run_ours(args):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic",
-                "config": {"workload": "symmetric LAPLEX matvec y=Kx, K_ij=exp(-|a_i-a_j|), "
-                                       "n=2^30 anchors U(0,2^30) pre-sorted, x~N(0,1), B=1, fp32",
-                           "n": n, "B": 1, "seed": "rank", "parallelism": f"replicas x{world}",
-                           "l2": "inputs 12.9 GB per step >> 126 MB L2 (no flush needed)"},
+                "config": workload_config(n, world),
                 "roofline": roof, "rows": rows, "e2e": e2e, "cpu_baseline": cpu,
                 "clocks": clocks, "gpu_launches": KERNELS_PER_SYM_CALL * args.steps}
         print(json.dumps(line), flush=True)
