@@ -14,11 +14,13 @@
 // weigh exp(0) = 1 on either side).  Merge order: a_i before b_j iff a_i < b_j.
 //
 // Kernels (the wait-free scheme of threepass.cuh on the merged sequence):
-// k_merge_partition (merge-path split into tiles), k_gen_local (tile-local
-// scan, outputs at the a-points), k_tp_carry_blocks + k_tp_carry_tiles (exact
-// tile carries), k_gen_headtail (carries added to the a-points of each tile's
-// head and tail reach).  K^T is the same product with the roles of a and b
-// exchanged (done by the caller).
+// k_merge_partition (merge-path split into tiles), k_gen_local (tile scan with
+// the carries from halos of b-points, outputs at the a-points), k_tp_carry_blocks
+// + k_tp_carry_tiles (exact tile carries, only when some tile's halos fell
+// short), k_gen_headtail (those carries added to the a-points of such a tile's
+// head and tail reach: on dense anchors a read-modify-write of the output
+// side only, cheaper than scanning the merged tile again).  K^T is the same product with
+// the roles of a and b exchanged (done by the caller).
 #include <algorithm>
 
 #include "laplex_impl.h"
@@ -48,45 +50,104 @@ __global__ void k_merge_partition(const T* __restrict__ a, int64_t n, const T* _
     ia[t] = lo;
 }
 
-// Tile-local scan of the merged sequence with zero carries from outside the
-// tile (threepass.cuh pass 1 for the merged case).  Outputs go to the
-// a-points; the tile's totals and its reach in a-points (a-points within CUT
-// of the tile's first / last merged anchor) go to the workspace.
-template <typename T, int NCOL, bool PHASED, int E, int NT>
-__global__ void __launch_bounds__(NT) k_gen_local(GenArgs<T> A, TPWs<T, PHASED ? 2 * NCOL : NCOL> W,
-                                                  const int64_t* __restrict__ ia) {
+// Channel values of b-point j (x_j times the scale; phased: cos psi_j and
+// sin psi_j times that).
+template <typename T, int NCOL, bool PHASED>
+__device__ __forceinline__ void gen_bvalue(const GenArgs<T>& A, int64_t j, T (&vj)[PHASED ? 2 * NCOL : NCOL]) {
+    const int64_t row = A.pin ? (int64_t)A.pin[j] : j;
+    const T dsc = A.D ? A.D[A.pD ? (int64_t)A.pD[j] : j] : T(1);
+    T cs = T(1), sn = T(0);
+    if (PHASED) gsincos<T>(A.psi[A.ppsi ? (int64_t)A.ppsi[j] : j], &sn, &cs);
+    const T* xr = A.x + row * A.ldx + A.col0;
+#pragma unroll
+    for (int c = 0; c < NCOL; ++c) {
+        const T val = (c < A.ncol ? xr[c] : T(0)) * dsc;
+        if (PHASED) {
+            vj[2 * c] = cs * val;
+            vj[2 * c + 1] = sn * val;
+        } else {
+            vj[c] = val;
+        }
+    }
+}
+
+// One tile of the merged sequence (merged positions [p0, p1)).  The carries
+// come from halos of H b-points on each side (a-points carry 0, so the b-points
+// alone make the halo): the left one, b[j0 - H, j0), gives L at the merged
+// element before the tile as sum_j exp(b_j - eT) x_j, the right one,
+// b[j1, j1 + H), gives U at the element after it.  They are exact when they
+// span CUT or reach the end of b; then the tile's outputs are final and its
+// reach is stored as 0.  Otherwise the outputs are written with zero carries,
+// the tile is counted (so the carry kernels run) and its reach -- the a-points
+// within CUT of its first / last merged anchor -- is stored for k_gen_headtail.
+// Every tile stores its edge anchors and zero-carry totals.
+template <typename T, int NCOL, bool PHASED, int E, int NT, int H>
+__device__ __forceinline__ void gen_tile(const GenArgs<T>& A, const TPWs<T, PHASED ? 2 * NCOL : NCOL>& W,
+                                         const int64_t* __restrict__ ia, int64_t t, T* sh_anc, T* sh_val,
+                                         BlockScan2Smem<T, PHASED ? 2 * NCOL : NCOL, NT>& sm2) {
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
     constexpr int TILE = NT * E;
-    __shared__ T sh_anc[TILE];      // a-part [0, na), b-part [na, na + nb)
-    __shared__ T sh_val[TILE * C];  // channel values of the b-part
-    __shared__ BlockScan2Smem<T, C, NT> sm2;
-    const int64_t t = blockIdx.x;
+    constexpr int HH = H;
     const int64_t n = A.n, k = A.k, N = n + k;
     const int64_t p0 = t * TILE, p1 = min(p0 + TILE, N);
     const int64_t i0 = ia[t], i1 = ia[t + 1];
     const int64_t j0 = p0 - i0, j1 = p1 - i1;
     const int na = (int)(i1 - i0), nb = (int)(j1 - j0), cnt = na + nb;
+    const bool needL = p0 > 0, needR = p1 < N;
+    // merged anchors just before and just after the tile
+    T eT = T(0), fT = T(0);
+    if (needL) eT = (i0 > 0 && j0 > 0) ? max(A.sa[i0 - 1], A.sb[j0 - 1]) : (i0 > 0 ? A.sa[i0 - 1] : A.sb[j0 - 1]);
+    if (needR) fT = (i1 < n && j1 < k) ? min(A.sa[i1], A.sb[j1]) : (i1 < n ? A.sa[i1] : A.sb[j1]);
+    // thread 0 checks from two anchors whether the halos can be exact (they
+    // span CUT or reach the end of b); the halos are only summed when both can
+    __shared__ int sh_ok;
+    if (threadIdx.x == 0) {
+        bool okL = !needL || HH == 0 ? !needL : (j0 - HH <= 0 || eT - A.sb[j0 - HH] >= ExpCut<T>::v);
+        bool okR = !needR || HH == 0 ? !needR : (j1 + HH >= k || A.sb[j1 + HH - 1] - fT >= ExpCut<T>::v);
+        sh_ok = (okL ? 1 : 0) | (okR ? 2 : 0);
+    }
     for (int q = threadIdx.x; q < na; q += NT) sh_anc[q] = A.sa[i0 + q];
     for (int q = threadIdx.x; q < nb; q += NT) {
         const int64_t j = j0 + q;
         sh_anc[na + q] = A.sb[j];
-        const int64_t row = A.pin ? (int64_t)A.pin[j] : j;
-        const T dsc = A.D ? A.D[A.pD ? (int64_t)A.pD[j] : j] : T(1);
-        T cs = T(1), sn = T(0);
-        if (PHASED) gsincos<T>(A.psi[A.ppsi ? (int64_t)A.ppsi[j] : j], &sn, &cs);
-        const T* xr = A.x + row * A.ldx + A.col0;
+        T vj[C];
+        gen_bvalue<T, NCOL, PHASED>(A, j, vj);
 #pragma unroll
-        for (int c = 0; c < NCOL; ++c) {
-            const T val = (c < A.ncol ? xr[c] : T(0)) * dsc;
-            if (PHASED) {
-                sh_val[q * C + 2 * c] = cs * val;
-                sh_val[q * C + 2 * c + 1] = sn * val;
-            } else {
-                sh_val[q * C + c] = val;
+        for (int c = 0; c < C; ++c) sh_val[q * C + c] = vj[c];
+    }
+    __syncthreads();
+    const int ok = sh_ok;
+    // halo terms of this thread (halo element m = q + r NT < 2H; m < H: left,
+    // H <= m < 2H: right), when both halos are exact
+    T hvL[C], hvU[C];
+    int bad[2] = {0, 0};
+    if (threadIdx.x == 0) {
+        bad[0] = (ok & 1) ? 0 : 1;
+        bad[1] = (ok & 2) ? 0 : 1;
+    }
+#pragma unroll
+    for (int c = 0; c < C; ++c) hvL[c] = hvU[c] = T(0);
+    if (HH > 0 && ok == 3) {
+        const int q = (int)threadIdx.x;
+#pragma unroll
+        for (int r = 0; r * NT < 2 * HH; ++r) {
+            const int m = q + r * NT;
+            if (m >= 2 * HH) break;
+            const bool left = m < HH;
+            if (!(left ? needL : needR)) continue;
+            const int64_t j = left ? j0 - HH + m : j1 + (m - HH);
+            if (j < 0 || j >= k) continue;  // the halo reaches the end of b
+            const T bj = A.sb[j];
+            T vj[C];
+            gen_bvalue<T, NCOL, PHASED>(A, j, vj);
+            const T f = dexp<T>(left ? bj - eT : fT - bj);
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                if (left) hvL[c] += f * vj[c];
+                else hvU[c] += f * vj[c];
             }
         }
     }
-    __syncthreads();
     const T* Aa = sh_anc;
     const T* Bb = sh_anc + na;
     const T first = na > 0 && (nb == 0 || Aa[0] <= Bb[0]) ? Aa[0] : Bb[0];
@@ -101,7 +162,7 @@ __global__ void __launch_bounds__(NT) k_gen_local(GenArgs<T> A, TPWs<T, PHASED ?
     int ai = lo, bi = d0 - lo;
     T s[E], v[E][C], dl[E], fV[C], bW[C];
     int aidx[E];
-    int h = 0, q = 0;
+    int cnt4[4] = {bad[0], bad[1], 0, 0};  // span checks, then the reach in a-points
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const bool valid = d0 + e < cnt;
@@ -114,8 +175,8 @@ __global__ void __launch_bounds__(NT) k_gen_local(GenArgs<T> A, TPWs<T, PHASED ?
         } else if (takeA) {
             s[e] = Aa[ai];
             aidx[e] = ai;
-            h += (Aa[ai] - first < ExpCut<T>::v) ? 1 : 0;
-            q += (padA - Aa[ai] < ExpCut<T>::v) ? 1 : 0;
+            cnt4[2] += (Aa[ai] - first < ExpCut<T>::v) ? 1 : 0;
+            cnt4[3] += (padA - Aa[ai] < ExpCut<T>::v) ? 1 : 0;
             ++ai;
 #pragma unroll
             for (int c = 0; c < C; ++c) v[e][c] = T(0);
@@ -130,10 +191,12 @@ __global__ void __launch_bounds__(NT) k_gen_local(GenArgs<T> A, TPWs<T, PHASED ?
     chunk_aggregates<T, C, E>(s, v, dl, fV, bW);
     bool hf, hb;
     T pe, pV[C], te, tV[C], nf, nW[C], tf, tW[C];
-    const int hq[2] = {h, q};
-    int reach[2];
-    (void)block_excl_both_counted<T, C, NT, 0, true>(s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb, nf,
-                                                     nW, tf, tW, hq, reach, false, sm2);
+    int tot4[4];
+    T hL[C], hU[C];
+    (void)block_excl_both_counted<T, C, NT, 0, true, 4, HH, C>(s[E - 1], fV, s[0], bW, hf, pe, pV, te, tV, hb,
+                                                                nf, nW, tf, tW, cnt4, tot4, false, sm2, hvL,
+                                                                hvU, hL, hU);
+    const bool fin = tot4[0] == 0 && tot4[1] == 0;
     if (threadIdx.x == 0) {
         W.tfirst[t] = tf;
         W.tlast[t] = te;
@@ -142,17 +205,21 @@ __global__ void __launch_bounds__(NT) k_gen_local(GenArgs<T> A, TPWs<T, PHASED ?
             W.fagg[t * C + c] = tV[c];
             W.bagg[t * C + c] = tW[c];
         }
-        W.st[t].head = reach[0];
-        W.st[t].tail = reach[1];
+        W.st[t].head = fin ? 0 : tot4[2];
+        W.st[t].tail = fin ? 0 : tot4[3];
+        if (!fin) atomicAdd(W.redo_count, 1u);  // the carry kernels are needed
     }
-    T eprev = hf ? pe : s[0], enext = hb ? nf : s[E - 1];
-    T Lprev[C], Unext[C], out[E][C];
+    T Lc[C], Uc[C];
 #pragma unroll
     for (int c = 0; c < C; ++c) {
-        Lprev[c] = hf ? pV[c] : T(0);
-        Unext[c] = hb ? nW[c] : T(0);
+        Lc[c] = fin && HH > 0 && needL ? hL[c] : T(0);
+        Uc[c] = fin && HH > 0 && needR ? hU[c] : T(0);
     }
-    chunk_final<T, C, E>(s, v, dl, eprev, Lprev, enext, Unext, out);
+    const T eA = fin && needL ? eT : (hf ? pe : s[0]), fA = fin && needR ? fT : (hb ? nf : s[E - 1]);
+    T eprev, Lprev[C], enext, Unext[C], o[E][C];
+    apply_carry_fwd<T, C>(hf, pe, pV, eA, Lc, eprev, Lprev);
+    apply_carry_bwd<T, C>(hb, nf, nW, fA, Uc, enext, Unext);
+    chunk_final<T, C, E>(s, v, dl, eprev, Lprev, enext, Unext, o);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         if (aidx[e] < 0) continue;
@@ -164,13 +231,24 @@ __global__ void __launch_bounds__(NT) k_gen_local(GenArgs<T> A, TPWs<T, PHASED ?
             gsincos<T>(A.phi[A.pphi ? (int64_t)A.pphi[i] : i], &sp, &cp);
 #pragma unroll
             for (int c = 0; c < NCOL; ++c)
-                if (c < A.ncol) yr[c] = cp * out[e][2 * c] + sp * out[e][2 * c + 1];
+                if (c < A.ncol) yr[c] = cp * o[e][2 * c] + sp * o[e][2 * c + 1];
         } else {
 #pragma unroll
             for (int c = 0; c < NCOL; ++c)
-                if (c < A.ncol) yr[c] = out[e][c];
+                if (c < A.ncol) yr[c] = o[e][c];
         }
     }
+}
+
+// one block per merged tile
+template <typename T, int NCOL, bool PHASED, int E, int NT, int H>
+__global__ void __launch_bounds__(NT) k_gen_local(GenArgs<T> A, TPWs<T, PHASED ? 2 * NCOL : NCOL> W,
+                                                  const int64_t* __restrict__ ia) {
+    constexpr int C = PHASED ? 2 * NCOL : NCOL;
+    __shared__ T sh_anc[NT * E];      // a-part [0, na), b-part [na, na + nb)
+    __shared__ T sh_val[NT * E * C];  // channel values of the b-part
+    __shared__ BlockScan2Smem<T, C, NT> sm2;
+    gen_tile<T, NCOL, PHASED, E, NT, H>(A, W, ia, (int64_t)blockIdx.x, sh_anc, sh_val, sm2);
 }
 
 // Carries into the a-points of each tile's head and tail reach (a warp per tile).
@@ -226,6 +304,7 @@ __global__ void __launch_bounds__(256) k_gen_headtail(GenArgs<T> A, TPWs<T, PHAS
     }
 }
 
+
 // ------------------------------------------------------------------ host side
 struct GenPlan {
     int ncol, C, E;
@@ -262,14 +341,19 @@ static cudaError_t gen_launch(const GenArgs<T>& A, const GenPlan& p, void* wsbod
     Carve cv(wsbody, wsb);
     TPWs<T, C> W = tp_carve<T, C>(cv, p.ntiles);
     if (!cv.ok) return cudaErrorInvalidValue;
-    W.redo_count = nullptr;  // every tile takes the carries (reach read-modify-write)
     const int64_t nb = (p.ntiles + TP_CARRY_BT - 1) / TP_CARRY_BT;
+    int sms = 0;
+    cudaError_t e = tp_sm_count(sms);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(W.redo_count, 0, sizeof(uint32_t), st);
+    if (e != cudaSuccess) return e;
+    constexpr int H = sizeof(T) == 4 ? 192 : 0;  // as the symmetric products
     profile_before(st);
-    k_gen_local<T, NCOL, PHASED, E, GEN_NT><<<(unsigned)p.ntiles, GEN_NT, 0, st>>>(A, W, ia);
+    k_gen_local<T, NCOL, PHASED, E, GEN_NT, H><<<(unsigned)p.ntiles, GEN_NT, 0, st>>>(A, W, ia);
     profile_after(st);
     k_tp_carry_blocks<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, p.ntiles);
     k_tp_carry_tiles<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, p.ntiles, nb);
-    const int64_t htb = std::max<int64_t>(1, std::min<int64_t>((p.ntiles + 7) / 8, 148 * 8));
+    const int64_t htb = std::max<int64_t>(1, std::min<int64_t>((p.ntiles + 7) / 8, (int64_t)sms * 8));
     k_gen_headtail<T, NCOL, PHASED><<<(unsigned)htb, 256, 0, st>>>(A, W, ia, p.tile, p.ntiles);
     return cudaGetLastError();
 }

@@ -37,14 +37,14 @@
 
 namespace lx {
 
-struct TPStats {  // reach of a tile (general case: elements within CUT of each edge)
-    int32_t head;
-    int32_t tail;
-};
-
 constexpr int TP_CARRY_NT = 256;
 constexpr int TP_CARRY_PT = 8;
 constexpr int TP_CARRY_BT = TP_CARRY_NT * TP_CARRY_PT;
+
+struct TPStats {  // reach of a tile (general product): elements within CUT of each edge
+    int32_t head;
+    int32_t tail;
+};
 
 template <typename T, int C>
 struct TPWs {
@@ -52,9 +52,9 @@ struct TPWs {
     T* tlast;    // [ntiles]
     T* fagg;     // [ntiles*C] L at the tile's last element, tile only
     T* bagg;     // [ntiles*C] U at the tile's first element, tile only
-    TPStats* st; // [ntiles] (general case)
+    TPStats* st;           // [ntiles] reach (general product)
     int32_t* redo;         // [ntiles] tiles left for the redo pass, any order
-    uint32_t* redo_count;  // their number; NULL: carries always computed
+    uint32_t* redo_count;  // their number (zeroed before pass 1)
     T* bfe;      // [nb] last anchor of each carry block
     T* bfv;      // [nb*C]
     T* bbf;      // [nb] first anchor of each carry block
@@ -93,9 +93,9 @@ inline TPWs<T, C> tp_carve(Carve& cv, int64_t ntiles) {
 // ------------------------------------------------------------------ pass 1 and 3
 // Halo terms of thread q of a tile: the halo elements k = q + m NT < 2H
 // (k < H: left halo, H <= k < 2H: right halo), summed per side, and the checks
-// that each halo spans CUT (by the threads holding k = 0 and k = H).  A side
-// needs no carry at an end of the array, and a halo that reaches the end of
-// the array needs no check.
+// that each halo spans CUT.  A side needs no carry at an end of the array, and
+// a halo that reaches the end of the array needs no check.  Contains a block
+// barrier: every thread of the block calls it.
 template <class P>
 __device__ __forceinline__ void tp_halo_terms(const P& p, int64_t t, int64_t tile0, int64_t tile1,
                                               typename P::T (&hvL)[P::C], typename P::T (&hvU)[P::C],
@@ -116,8 +116,23 @@ __device__ __forceinline__ void tp_halo_terms(const P& p, int64_t t, int64_t til
     }
     const bool needL = t > 0, needR = tile1 < n;
     // the left halo is always in the array (tile0 >= TILE >= H); a right halo
-    // cut short by the end of the array holds every element to the right
+    // cut short by the end of the array holds every element to the right.
+    // Thread 0 checks from two anchors whether both halos can be exact; only
+    // then are they summed (dense anchors skip the loads).
     const bool fullR = tile1 + H <= n;
+    __shared__ int sh_ok;
+    if (q == 0) {
+        const bool okL = !needL || p.s[tile0 - 1] - p.s[tile0 - H] >= ExpCut<T>::v;
+        const bool okR = !needR || !fullR || p.s[tile1 + H - 1] - p.s[tile1] >= ExpCut<T>::v;
+        sh_ok = (okL ? 1 : 0) | (okR ? 2 : 0);
+    }
+    __syncthreads();
+    const int ok = sh_ok;
+    if (q == 0) {
+        bad[0] = (ok & 1) ? 0 : 1;
+        bad[1] = (ok & 2) ? 0 : 1;
+    }
+    if (ok != 3) return;
     const T eL = needL ? p.s[tile0 - 1] : T(0), eR = needR ? p.s[tile1] : T(0);
 #pragma unroll
     for (int m = 0; m * NT < 2 * H; ++m) {
@@ -136,8 +151,6 @@ __device__ __forceinline__ void tp_halo_terms(const P& p, int64_t t, int64_t til
             if (left) hvL[c] += d[c] * vj[c];
             else hvU[c] += d[c] * vj[c];
         }
-        if (k == 0) bad[0] = edge - sj >= ExpCut<T>::v ? 0 : 1;
-        if (k == H && fullR) bad[1] = p.s[tile1 + H - 1] - edge >= ExpCut<T>::v ? 0 : 1;
     }
 }
 
@@ -465,7 +478,7 @@ __device__ __forceinline__ void tp_segment(const TPWs<T, C>& W, int64_t t0, int6
 
 template <typename T, int C, int CT>
 __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_blocks(TPWs<T, C> W, int64_t ntiles) {
-    if (W.redo_count != nullptr && *(volatile uint32_t*)W.redo_count == 0) return;  // every tile final
+    if (*(volatile uint32_t*)W.redo_count == 0) return;  // every tile final
     __shared__ BlockScan2Smem<T, C, TP_CARRY_NT> sm2;
     const int64_t t0 = (int64_t)blockIdx.x * TP_CARRY_BT + (int64_t)threadIdx.x * TP_CARRY_PT;
     T fe, fv[C], bf, bv[C];
@@ -487,7 +500,7 @@ __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_blocks(TPWs<T, C> W, i
 template <typename T, int C, int CT>
 __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_tiles(TPWs<T, C> W, int64_t ntiles,
                                                                  int64_t nblocks) {
-    if (W.redo_count != nullptr && *(volatile uint32_t*)W.redo_count == 0) return;  // every tile final
+    if (*(volatile uint32_t*)W.redo_count == 0) return;  // every tile final
     __shared__ BlockScan2Smem<T, C, TP_CARRY_NT> sm2;
     __shared__ T sh_c[2][C];
     const int64_t bidx = blockIdx.x;

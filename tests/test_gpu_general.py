@@ -93,3 +93,29 @@ def test_c3_full_size():
     a, b, x, w = synth.general_ties(1 << 22, 1 << 20, -1000.0, 1000.0, seed=0)
     assert np.isin(b, a).mean() > 0.009
     check(a, b, x, w, np.float32, "C3")
+
+
+@pytest.mark.parametrize("case", ["sparse", "b_spacing_0.46", "b_spacing_0.47", "b_sparse_a_dense",
+                                  "runs_of_64"])
+def test_halo_carries(case):
+    """Merged tiles whose carries come from halos of 192 b-points (exact when
+    they span the cut of 88 or reach the end of b), next to tiles that fall
+    back to the carry kernels and the redo pass."""
+    rng = np.random.default_rng(29)
+    if case == "sparse":
+        a = rng.uniform(0, 60000, 40000)
+        b = rng.uniform(0, 60000, 30000)
+    elif case.startswith("b_spacing_"):
+        sp = float(case.split("_")[-1])
+        b = np.arange(30000) * sp
+        a = rng.uniform(0, b[-1], 20000)
+    elif case == "b_sparse_a_dense":
+        b = rng.uniform(0, 30000, 20000)
+        a = rng.uniform(1000, 1010, 50000)
+    else:
+        b = 2.0 ** 29 + 64.0 * (np.arange(30000) // 64)
+        a = 2.0 ** 29 + 64.0 * (np.arange(25000) // 50) + 7.0
+    a, b = a.astype(np.float32), b.astype(np.float32)
+    x = rng.normal(size=b.size).astype(np.float32)
+    w = rng.normal(size=a.size).astype(np.float32)
+    check(a, b, x, w, np.float32, case)
