@@ -404,6 +404,15 @@ def run_ours(args):
             rows["c3_general_Kx"] = row(ms, nn, 8 * nn + 8 * kk, "n=2^22, k=2^20, pre-sorted, y=Kx")
             ms = timed_flush(lambda: X.matvec_general(sa, sb, ws3, transpose=True, out=z3), fsteps)
             rows["c3_general_KTw"] = row(ms, kk, 8 * nn + 8 * kk, "n=2^22, k=2^20, pre-sorted, z=K^T w")
+            # anchor gradients of <w, K x> (sorted order): reads a, b, x, w; writes dx, da, db
+            ms = timed_flush(lambda: X.backward_general(sa, sb, xs3, ws3), fsteps)
+            rows["c3_backward_general"] = row(ms, nn + kk, 16 * nn + 16 * kk,
+                                              "n=2^22, k=2^20, pre-sorted: dx = K^T w, da, db")
+            # weighted Gram matrix of 4096 a-points over the 2^20 b-points (output 64 MB)
+            sa4 = sa[:: (nn // 4096)].contiguous()
+            ms = timed_flush(lambda: X.gram_matrix(sa4, sb, xs3.abs()), fsteps)
+            rows["gram_matrix_4096x2^20"] = row(ms, 4096 * 4096, 4 * 4096 * 4096 + 12 * kk,
+                                                "M = A diag(D) A^T, n=4096 of the C3 a-points, k=2^20")
             X.device_status(dev)
             del a3d, b3d, sa, pa, sb, pb, x3d, w3d, xs3, ws3, y3, z3
         if "c4" in wanted:
