@@ -268,6 +268,51 @@ def backward_general(a, b, x, g):
     return dx, da, db
 
 
+def backward_phased(a, phi, x, g, b=None, psi=None):
+    """Backward pass of L = <g, K x> for the phased kernel
+    K_ij = exp(-|a_i - b_j|) cos(phi_i - psi_j) (summary §2.1; trainable anchors
+    and phases, §2.3), w.r.t. x, the phases and the anchors:
+        dx_j   = sum_i K_ij g_i,
+        dphi_i = -g_i sum_j exp(-|a_i - b_j|) sin(phi_i - psi_j) x_j,
+        dpsi_j =  x_j sum_i exp(-|a_i - b_j|) sin(phi_i - psi_j) g_i,
+        da_i   = -g_i sum_j sign(a_i - b_j) K_ij x_j,
+        db_j   = -x_j sum_i sign(b_j - a_i) K_ij g_i          (sign(0) = 0).
+    Through cos(p - q) = cos p cos q + sin p sin q and
+    sin(p - q) = sin p cos q - cos p sin q every sum is a combination of two
+    unphased channels, (cos psi x, sin psi x) seen from a and (cos phi g, sin phi g)
+    seen from b, each summed plainly (general) and signed (signed_general).
+    b = None: the symmetric case (b = a, psi = phi); the anchors and phases are
+    shared, so (dx, dphi + dpsi, da + db) is returned.  Otherwise
+    (dx, dphi, dpsi, da, db)."""
+    sym_case = b is None
+    phi, x, g = _f64(phi), _f64(x), _f64(g)
+    if sym_case:
+        b, psi = a, phi
+    psi = _f64(psi)
+    cphi, sphi, cpsi, spsi = np.cos(phi), np.sin(phi), np.cos(psi), np.sin(psi)
+    xc = np.stack([cpsi * x, spsi * x], axis=1)  # channels on b
+    gc = np.stack([cphi * g, sphi * g], axis=1)  # channels on a
+    Pa, Sa = general(a, b, xc), signed_general(a, b, xc)
+    Pb, Sb = general(b, a, gc), signed_general(b, a, gc)
+    dx = cpsi * Pb[:, 0] + spsi * Pb[:, 1]
+    dphi = g * (cphi * Pa[:, 1] - sphi * Pa[:, 0])
+    dpsi = x * (cpsi * Pb[:, 1] - spsi * Pb[:, 0])
+    da = -g * (cphi * Sa[:, 0] + sphi * Sa[:, 1])
+    db = -x * (cpsi * Sb[:, 0] + spsi * Sb[:, 1])
+    if sym_case:
+        return dx, dphi + dpsi, da + db
+    return dx, dphi, dpsi, da, db
+
+
+def norm_backward_phased(a, x, g, b=None):
+    """Bounds of the phased gradients term by term (|cos|, |sin| <= 1), with the
+    unphased K0: (K0^T|g|, |g| K0|x|, |x| K0^T|g|) for dx, (dphi, da), (dpsi, db);
+    symmetric (b = None): (K0|g|, |g| K0|x| + |x| K0|g|) for dx and the totals."""
+    if b is None:
+        return norm_backward(a, x, g)
+    return norm_backward_general(a, b, x, g)
+
+
 def norm_backward_general(a, b, x, g):
     """Bounds of |dx|, |da|, |db| term by term: K^T|g|, |g| K|x|, |x| K^T|g|."""
     x, g = np.abs(_f64(x)), np.abs(_f64(g))

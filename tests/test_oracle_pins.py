@@ -433,6 +433,79 @@ def test_backward_general_central_differences():
 
 
 # ---------------------------------------------------------------------------
+# phased backward (trainable anchors and phases)
+# ---------------------------------------------------------------------------
+
+def _loss_phased(a, phi, b, psi, x, g):
+    return float(g @ O.dense_matvec(a, x, b=b, phi=phi, psi=psi))
+
+
+def _cd(f, v, i, h=1e-6):
+    vp, vm = v.copy(), v.copy()
+    vp[i] += h
+    vm[i] -= h
+    return (f(vp) - f(vm)) / (2 * h)
+
+
+def test_backward_phased_central_differences():
+    """dx, dphi, dpsi, da, db of L = <g, K x>, K_ij = exp(-|a_i - b_j|) cos(phi_i - psi_j),
+    against central differences of the dense definition (distinct anchors)."""
+    rng = np.random.default_rng(31)
+    a, b = rng.uniform(0, 4, 11), rng.uniform(0, 4, 8)
+    phi, psi = rng.uniform(0, 2 * math.pi, 11), rng.uniform(0, 2 * math.pi, 8)
+    x, g = rng.normal(size=8), rng.normal(size=11)
+    dx, dphi, dpsi, da, db = O.backward_phased(a, phi, x, g, b=b, psi=psi)
+    np.testing.assert_allclose(dx, O.dense_matrix(a, b, phi, psi).T @ g, atol=1e-13)
+    for i in range(11):
+        assert abs(dphi[i] - _cd(lambda v: _loss_phased(a, v, b, psi, x, g), phi, i)) < 1e-7, i
+        assert abs(da[i] - _cd(lambda v: _loss_phased(v, phi, b, psi, x, g), a, i)) < 1e-7, i
+    for j in range(8):
+        assert abs(dpsi[j] - _cd(lambda v: _loss_phased(a, phi, b, v, x, g), psi, j)) < 1e-7, j
+        assert abs(db[j] - _cd(lambda v: _loss_phased(a, phi, v, psi, x, g), b, j)) < 1e-7, j
+
+
+def test_backward_phased_ties_and_invariants():
+    """Tied anchors: the dense derivative with sign(0) = 0, entry by entry.  A
+    common phase shift and a common translation of both anchor sets leave L
+    unchanged, so sum dphi + sum dpsi = 0 and sum da + sum db = 0.  The symmetric
+    case returns the totals of the general one with b = a, psi = phi, and phi = 0
+    reduces it to the unphased backward pass."""
+    rng = np.random.default_rng(32)
+    a = np.round(rng.uniform(0, 3, 10), 1)
+    b = np.concatenate([np.round(rng.uniform(0, 3, 5), 1), a[:3]])
+    phi, psi = rng.uniform(-3, 3, 10), rng.uniform(-3, 3, 8)
+    x, g = rng.normal(size=8), rng.normal(size=10)
+    dx, dphi, dpsi, da, db = O.backward_phased(a, phi, x, g, b=b, psi=psi)
+    for i in range(10):
+        t_phi = t_a = 0.0
+        for j in range(8):
+            e = math.exp(-abs(a[i] - b[j]))
+            t_phi += -g[i] * e * math.sin(phi[i] - psi[j]) * x[j]
+            t_a += -g[i] * np.sign(a[i] - b[j]) * e * math.cos(phi[i] - psi[j]) * x[j]
+        assert abs(dphi[i] - t_phi) < 1e-13 and abs(da[i] - t_a) < 1e-13, i
+    for j in range(8):
+        t_psi = t_b = 0.0
+        for i in range(10):
+            e = math.exp(-abs(a[i] - b[j]))
+            t_psi += x[j] * e * math.sin(phi[i] - psi[j]) * g[i]
+            t_b += -x[j] * np.sign(b[j] - a[i]) * e * math.cos(phi[i] - psi[j]) * g[i]
+        assert abs(dpsi[j] - t_psi) < 1e-13 and abs(db[j] - t_b) < 1e-13, j
+    assert abs(dphi.sum() + dpsi.sum()) < 1e-12
+    assert abs(da.sum() + db.sum()) < 1e-12
+    xs = rng.normal(size=10)
+    sdx, sdphi, sda = O.backward_phased(a, phi, xs, g)
+    gdx, gdphi, gdpsi, gda, gdb = O.backward_phased(a, phi, xs, g, b=a, psi=phi)
+    np.testing.assert_allclose(sdx, gdx, atol=1e-13)
+    np.testing.assert_allclose(sdphi, gdphi + gdpsi, atol=1e-13)
+    np.testing.assert_allclose(sda, gda + gdb, atol=1e-13)
+    udx, uda = O.backward(a, xs, g)
+    zdx, zdphi, zda = O.backward_phased(a, np.zeros(10), xs, g)
+    np.testing.assert_allclose(zdx, udx, atol=1e-13)
+    np.testing.assert_allclose(zda, uda, atol=1e-13)
+    assert np.abs(zdphi).max() < 1e-13
+
+
+# ---------------------------------------------------------------------------
 # weighted Gram matrix A diag(D) A^T
 # ---------------------------------------------------------------------------
 
