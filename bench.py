@@ -413,8 +413,15 @@ def run_ours(args):
             ms = timed_flush(lambda: X.gram_matrix(sa4, sb, xs3.abs()), fsteps)
             rows["gram_matrix_4096x2^20"] = row(ms, 4096 * 4096, 4 * 4096 * 4096 + 12 * kk,
                                                 "M = A diag(D) A^T, n=4096 of the C3 a-points, k=2^20")
+            # phased anchor and phase gradients (phases ~ U(0, 2 pi), sorted order):
+            # reads a, phi, w, b, psi, x; writes dphi, da, dx, dpsi, db
+            phi3 = torch.from_numpy(synth.uniform(nn, 0.0, 2 * math.pi, seed=rank, stream="phi")).to(dev)
+            psi3 = torch.from_numpy(synth.uniform(kk, 0.0, 2 * math.pi, seed=rank, stream="psi")).to(dev)
+            ms = timed_flush(lambda: X.backward_phased(sa, phi3, xs3, ws3, sb=sb, psi=psi3), fsteps)
+            rows["c3_backward_phased"] = row(ms, nn + kk, 20 * nn + 24 * kk,
+                                             "n=2^22, k=2^20, pre-sorted, phased: dx, dphi, dpsi, da, db")
             X.device_status(dev)
-            del a3d, b3d, sa, pa, sb, pb, x3d, w3d, xs3, ws3, y3, z3
+            del a3d, b3d, sa, pa, sb, pb, x3d, w3d, xs3, ws3, y3, z3, phi3, psi3
         if "c4" in wanted:
             a4, phi4, v4 = synth.phased_image(seed=rank)
             n4 = a4.size
@@ -427,8 +434,12 @@ def run_ours(args):
             rows["c4_phased_Kv"] = row(ms, n4, 16 * n4, "n=3*1024^2, pre-sorted, phased y=Kv")
             ms = timed_flush(lambda: X.gram(s4, vs, phi=phis, out=y4), fsteps)
             rows["c4_gram_KTKv"] = row(ms, n4, 32 * n4, "n=3*1024^2, pre-sorted, K^T K v")
+            gs4 = torch.from_numpy(synth.normal(n4, seed=rank, stream="g")).to(dev)
+            ms = timed_flush(lambda: X.backward_phased(s4, phis, vs, gs4), fsteps)
+            rows["c4_backward_phased"] = row(ms, n4, 28 * n4,
+                                             "n=3*1024^2, pre-sorted, symmetric phased: dx, dphi, da")
             X.device_status(dev)
-            del a4d, s4, p4, phis, vs, y4
+            del a4d, s4, p4, phis, vs, y4, gs4
     except X.LaplexError as e:
         rows["rows_error"] = str(e)
     del flush_buf

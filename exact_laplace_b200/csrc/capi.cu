@@ -93,6 +93,7 @@ size_t body_bytes(laplex_op op, int64_t n, int64_t k, int64_t B, int f64) {
             return std::max(g, sg);
         }
         case LAPLEX_OP_GRAM_MATRIX: return lx::grammat_ws_bytes(n, k, f64);
+        case LAPLEX_OP_BACKWARD_PHASED: return std::max(lx::pbwd_ws_bytes(n, f64), lx::pbwd_ws_bytes(k, f64));
     }
     return 0;
 }
@@ -155,7 +156,7 @@ laplex_status laplex_workspace_size(laplex_op op, int64_t n, int64_t k, int64_t 
     laplex_status st = check_sizes(n, k, B);
     if (st != LAPLEX_OK) return st;
     if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
-    REQ(op >= LAPLEX_OP_SORT && op <= LAPLEX_OP_GRAM_MATRIX, "unknown op %d", (int)op);
+    REQ(op >= LAPLEX_OP_SORT && op <= LAPLEX_OP_BACKWARD_PHASED, "unknown op %d", (int)op);
     *bytes = lx::HEADER_BYTES + body_bytes(op, n, k, B, dt == LAPLEX_F64);
     return ok();
 }
@@ -487,6 +488,54 @@ laplex_status laplex_backward_general(const void* sa, const int32_t* pa, int64_t
                                    (const double*)x, (const double*)g, (double*)da, (double*)db,
                                    ws_body(ws), body, s);
     if (e != cudaSuccess) return cuda_fail(e, "laplex_backward_general (signed sums)");
+    return ok();
+}
+
+laplex_status laplex_backward_phased(const void* sa, const int32_t* pa, const void* phi, int64_t n,
+                                     const void* sb, const int32_t* pb, const void* psi, int64_t k,
+                                     const void* x, const void* g, void* dx, void* dphi, void* dpsi,
+                                     void* da, void* db, laplex_dtype dt, void* ws, size_t ws_bytes,
+                                     void* stream) {
+    const bool sym = sb == nullptr;
+    if (sym) {
+        k = n;
+        pb = nullptr;
+        psi = nullptr;
+        dpsi = nullptr;
+        db = nullptr;
+    }
+    laplex_status st = check_sizes(n, k, 1);
+    if (st != LAPLEX_OK) return st;
+    if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
+    REQ_PTR(sa, n > 0);
+    REQ_PTR(phi, n > 0);
+    REQ_PTR(g, n > 0);
+    REQ_PTR(x, k > 0);
+    if (!sym) {
+        REQ_PTR(sb, k > 0);
+        REQ_PTR(psi, k > 0);
+    }
+    if (pa) REQ_PTR(pa, n > 0);
+    if (pb) REQ_PTR(pb, k > 0);
+    if (dphi) REQ_PTR(dphi, n > 0);
+    if (da) REQ_PTR(da, n > 0);
+    if (dx) REQ_PTR(dx, k > 0);
+    if (dpsi) REQ_PTR(dpsi, k > 0);
+    if (db) REQ_PTR(db, k > 0);
+    if ((st = check_ws(LAPLEX_OP_BACKWARD_PHASED, n, k, 1, dt, ws, ws_bytes)) != LAPLEX_OK) return st;
+    if (n == 0 && k == 0) return ok();
+    const size_t body = ws_bytes - lx::HEADER_BYTES;
+    cudaStream_t s = (cudaStream_t)stream;
+    const cudaError_t e =
+        dt == LAPLEX_F32
+            ? lx::pbwd_run<float>((const float*)sa, pa, (const float*)phi, n, (const float*)sb, pb,
+                                  (const float*)psi, k, (const float*)x, (const float*)g, (float*)dx,
+                                  (float*)dphi, (float*)dpsi, (float*)da, (float*)db, ws_body(ws), body, s)
+            : lx::pbwd_run<double>((const double*)sa, pa, (const double*)phi, n, (const double*)sb, pb,
+                                   (const double*)psi, k, (const double*)x, (const double*)g, (double*)dx,
+                                   (double*)dphi, (double*)dpsi, (double*)da, (double*)db, ws_body(ws), body,
+                                   s);
+    if (e != cudaSuccess) return cuda_fail(e, "laplex_backward_phased");
     return ok();
 }
 

@@ -115,6 +115,11 @@ size_t grammat_ws_bytes(int64_t n, int64_t k, int f64);
 template <typename T>
 cudaError_t grammat_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, const int32_t* pb, int64_t k,
                         const T* D, T* M, int64_t ldm, void* ws, size_t ws_bytes, cudaStream_t st);
+size_t pbwd_ws_bytes(int64_t len, int f64);
+template <typename T>
+cudaError_t pbwd_run(const T* sa, const int32_t* pa, const T* phi, int64_t n, const T* sb,
+                     const int32_t* pb, const T* psi, int64_t k, const T* x, const T* g, T* dx, T* dphi,
+                     T* dpsi, T* da, T* db, void* ws, size_t ws_bytes, cudaStream_t st);
 template <typename T>
 cudaError_t sgen_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, const int32_t* pb,
                      int64_t k, const T* x, const T* g, T* da, T* db, void* ws, size_t ws_bytes,

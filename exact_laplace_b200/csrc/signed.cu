@@ -185,6 +185,230 @@ cudaError_t sgen_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, con
     return signed_pass<T>(sa, pa, n, g, sb, pb, k, x, db, ws, ws_bytes, st);
 }
 
+// ------------------------------------------------------------------ phased backward
+// L = <g, K x> with K_ij = exp(-|a_i - b_j|) cos(phi_i - psi_j) (summary §2.1;
+// trainable anchors and phases, §2.3).  By cos(p - q) = cos p cos q + sin p sin q
+// and sin(p - q) = sin p cos q - cos p sin q, with the two channels
+//     P(a <- b) = sum_j exp(-|a - b_j|) (cos psi_j x_j, sin psi_j x_j)
+//     S(a <- b) = sum_j sign(a - b_j) exp(-|a - b_j|) (cos psi_j x_j, sin psi_j x_j)
+// at an a-point with phase phi and weight g:
+//     dphi = g (cos phi P1 - sin phi P0),   da = -g (cos phi S0 + sin phi S1),
+// and, with the roles of the sides swapped (channels cos phi g, sin phi g seen
+// from a b-point with phase psi and weight x):
+//     dx = cos psi P0 + sin psi P1,  dpsi = x (cos psi P1 - sin psi P0),
+//     db = -x (cos psi S0 + sin psi S1).
+// P and S come from the one-sided scans F, G of the two channels (as the signed
+// sums above): P = F_{ub-1} exp(b_{ub-1} - a) + G_{ub} exp(a - b_{ub}),
+// S = F_{lb-1} exp(b_{lb-1} - a) - G_{ub} exp(a - b_{ub}).
+
+static __device__ __forceinline__ void pb_sincos(float t, float* sn, float* cs) { sincosf(t, sn, cs); }
+static __device__ __forceinline__ void pb_sincos(double t, double* sn, double* cs) { sincos(t, sn, cs); }
+
+// Policy of threepass.cuh: channels cos(ph) v and sin(ph) v (v and ph gathered
+// through perm), prefix F and suffix G written interleaved, [n][2], sorted order.
+template <typename T_, int E_>
+struct OneSidedPhasedTP {
+    using T = T_;
+    static constexpr int C = 2, CT = 0, E = E_, NT = OS_NT;
+    static constexpr int H = sizeof(T_) == 4 ? 192 : 0;
+    int64_t n;
+    const T* s;
+    const int32_t* perm;
+    const T* v;
+    const T* ph;
+    T* F;
+    T* G;
+    struct Aux {};
+    __device__ __forceinline__ void value(int64_t r, T (&vj)[C]) const {
+        const int64_t o = perm ? (int64_t)perm[r] : r;
+        T sn, cs;
+        pb_sincos(ph[o], &sn, &cs);
+        const T x = v[o];
+        vj[0] = cs * x;
+        vj[1] = sn * x;
+    }
+    __device__ __forceinline__ void load(int64_t r0, T (&sv)[E], T (&vv)[E][C], Aux&) const {
+        constexpr int VN = V16<T>::N;
+        if (r0 + E <= n) {
+#pragma unroll
+            for (int i = 0; i < E; i += VN) ld16_stream<T>(s + r0 + i, &sv[i]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < E; ++i) sv[i] = s[min(r0 + i, n - 1)];
+        }
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            if (r0 + i < n) {
+                value(r0 + i, vv[i]);
+            } else {
+                vv[i][0] = T(0);
+                vv[i][1] = T(0);
+            }
+        }
+    }
+    __device__ __forceinline__ void load1(int64_t j, T& sj, T (&vj)[C]) const {
+        sj = s[j];
+        value(j, vj);
+    }
+    __device__ __forceinline__ void finish(int64_t r0, const T (&sv)[E], const T (&vv)[E][C],
+                                           T (&dl)[E], T eprev, const T (&Lp)[C], T enext,
+                                           const T (&Un)[C], Aux&) const {
+        constexpr int VN = V16<T>::N;
+        T fo[2 * E], go[2 * E];
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            T L = Lp[c];
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const T d = i == 0 ? dexp<T>(eprev - sv[0]) : dl[i];
+                L = dfma<T>(d, L, vv[i][c]);
+                fo[2 * i + c] = L;
+            }
+            T U = Un[c];
+#pragma unroll
+            for (int i = E - 1; i >= 0; --i) {
+                const T d = i == E - 1 ? dexp<T>(sv[E - 1] - enext) : dl[i + 1];
+                U = dfma<T>(d, U, vv[i][c]);
+                go[2 * i + c] = U;
+            }
+        }
+        if (r0 + E <= n) {
+#pragma unroll
+            for (int i = 0; i < 2 * E; i += VN) {
+                st16<T>(F + 2 * r0 + i, &fo[i]);
+                st16<T>(G + 2 * r0 + i, &go[i]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 2 * E; ++i)
+                if (r0 + i / 2 < n) {
+                    F[2 * r0 + i] = fo[i];
+                    G[2 * r0 + i] = go[i];
+                }
+        }
+    }
+};
+
+static constexpr int pb_E(int es) { return es == 4 ? 8 : 4; }
+
+// Per sorted query anchor r (row pq[r]; phase th and weight w in row order):
+//     prod = cos th P0 + sin th P1,  dph = w (cos th P1 - sin th P0),
+//     dan = -w (cos th S0 + sin th S1),
+// each where its pointer is not NULL: prod written, dph and dan written (acc = 0)
+// or added (acc = 1).  k = 0 gives P = S = 0.
+template <typename T>
+__global__ void __launch_bounds__(256) k_phased_query(const T* __restrict__ sq, const int32_t* __restrict__ pq,
+                                                      int64_t m, const T* __restrict__ th,
+                                                      const T* __restrict__ w, const T* __restrict__ sp,
+                                                      int64_t k, const T* __restrict__ F,
+                                                      const T* __restrict__ G, T* prod, T* dph, T* dan,
+                                                      int acc) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < m; r += stride) {
+        const T q = sq[r];
+        const int64_t lb = bound<T>(sp, k, q, false), ub = bound<T>(sp, k, q, true);
+        T P0 = T(0), P1 = T(0), S0 = T(0), S1 = T(0);
+        if (ub > 0) {
+            const T f = dexp<T>(sp[ub - 1] - q);
+            P0 = F[2 * (ub - 1)] * f;
+            P1 = F[2 * (ub - 1) + 1] * f;
+        }
+        if (lb == ub) {
+            S0 = P0;
+            S1 = P1;
+        } else if (lb > 0) {
+            const T f = dexp<T>(sp[lb - 1] - q);
+            S0 = F[2 * (lb - 1)] * f;
+            S1 = F[2 * (lb - 1) + 1] * f;
+        }
+        if (ub < k) {
+            const T f = dexp<T>(q - sp[ub]);
+            const T g0 = G[2 * ub] * f, g1 = G[2 * ub + 1] * f;
+            P0 += g0;
+            P1 += g1;
+            S0 -= g0;
+            S1 -= g1;
+        }
+        const int64_t row = pq ? (int64_t)pq[r] : r;
+        T sn, cs;
+        pb_sincos(th[row], &sn, &cs);
+        if (prod) prod[row] = cs * P0 + sn * P1;
+        if (dph || dan) {
+            const T wr = w[row];
+            if (dph) {
+                const T v = wr * (cs * P1 - sn * P0);
+                dph[row] = acc ? dph[row] + v : v;
+            }
+            if (dan) {
+                const T v = -wr * (cs * S0 + sn * S1);
+                dan[row] = acc ? dan[row] + v : v;
+            }
+        }
+    }
+}
+
+size_t pbwd_ws_bytes(int64_t len, int f64) {
+    const size_t es = f64 ? 8 : 4;
+    const int64_t tile = (int64_t)OS_NT * pb_E((int)es);
+    const int64_t ntiles = std::max<int64_t>(1, (len + tile - 1) / tile);
+    return 2 * Carve::need((size_t)std::max<int64_t>(2 * len, 1), es) + tp_ws_bytes(ntiles, 2, es);
+}
+
+// The channels of (p-side anchors sp, perm pp, values v, phases php) seen from
+// the query side (sq, pq, phases thq, weights w): prod, dph, dan as in
+// k_phased_query.
+template <typename T>
+static cudaError_t phased_pass(const T* sp, const int32_t* pp, int64_t k, const T* v, const T* php,
+                               const T* sq, const int32_t* pq, int64_t m, const T* thq, const T* w,
+                               T* prod, T* dph, T* dan, int acc, void* ws, size_t ws_bytes,
+                               cudaStream_t st) {
+    if (m == 0 || (prod == nullptr && dph == nullptr && dan == nullptr)) return cudaSuccess;
+    Carve cv(ws, ws_bytes);
+    T* F = cv.take<T>(2 * std::max<int64_t>(k, 1));
+    T* G = cv.take<T>(2 * std::max<int64_t>(k, 1));
+    if (!cv.ok) return cudaErrorInvalidValue;
+    cudaError_t e;
+    if (k > 0) {
+        OneSidedPhasedTP<T, pb_E((int)sizeof(T))> p;
+        p.n = k;
+        p.s = sp;
+        p.perm = pp;
+        p.v = v;
+        p.ph = php;
+        p.F = F;
+        p.G = G;
+        e = tp_run(p, cv.base + cv.off, cv.cap - cv.off, st);
+        if (e != cudaSuccess) return e;
+    }
+    int sms = 0;
+    e = tp_sm_count(sms);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((m + 255) / 256, (int64_t)sms * 16));
+    k_phased_query<T><<<(unsigned)blocks, 256, 0, st>>>(sq, pq, m, thq, w, sp, k, F, G, prod, dph, dan, acc);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t pbwd_run(const T* sa, const int32_t* pa, const T* phi, int64_t n, const T* sb,
+                     const int32_t* pb, const T* psi, int64_t k, const T* x, const T* g, T* dx, T* dphi,
+                     T* dpsi, T* da, T* db, void* ws, size_t ws_bytes, cudaStream_t st) {
+    // sb == NULL: b = a, psi = phi; the b-side gradients are added to the a-side ones
+    const bool sym = sb == nullptr;
+    if (sym) {
+        sb = sa;
+        pb = pa;
+        psi = phi;
+        k = n;
+        dpsi = dphi;
+        db = da;
+    }
+    // a-side: dphi, da from the channels of (x, psi) on b
+    cudaError_t e = phased_pass<T>(sb, pb, k, x, psi, sa, pa, n, phi, g, nullptr, dphi, da, 0, ws, ws_bytes, st);
+    if (e != cudaSuccess) return e;
+    // b-side: dx, dpsi, db from the channels of (g, phi) on a (the workspace is reused)
+    return phased_pass<T>(sa, pa, n, g, phi, sb, pb, k, psi, x, dx, dpsi, db, sym ? 1 : 0, ws, ws_bytes, st);
+}
+
 // ------------------------------------------------------------------ weighted Gram matrix
 // M = A diag(D) A^T, A_ij = exp(-|a_i - b_j|) (summary §2.2 "Operatori di
 // Gram").  For a_i <= a_j the terms split at a_i and a_j:
@@ -382,5 +606,12 @@ template cudaError_t sgen_run<float>(const float*, const int32_t*, int64_t, cons
 template cudaError_t sgen_run<double>(const double*, const int32_t*, int64_t, const double*,
                                       const int32_t*, int64_t, const double*, const double*, double*,
                                       double*, void*, size_t, cudaStream_t);
+
+template cudaError_t pbwd_run<float>(const float*, const int32_t*, const float*, int64_t, const float*,
+                                     const int32_t*, const float*, int64_t, const float*, const float*, float*,
+                                     float*, float*, float*, float*, void*, size_t, cudaStream_t);
+template cudaError_t pbwd_run<double>(const double*, const int32_t*, const double*, int64_t, const double*,
+                                      const int32_t*, const double*, int64_t, const double*, const double*,
+                                      double*, double*, double*, double*, double*, void*, size_t, cudaStream_t);
 
 }  // namespace lx

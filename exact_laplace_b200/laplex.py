@@ -23,7 +23,8 @@ LIB_PATH = os.path.join(_HERE, "liblaplex.so")
 
 OK, EINVAL, ENONFINITE, EWORKSPACE, ECUDA, ETIMEOUT = range(6)
 F32, F64 = 0, 1
-OP_SORT, OP_SYM, OP_GENERAL, OP_PHASED, OP_GRAM, OP_BACKWARD, OP_BACKWARD_GENERAL, OP_GRAM_MATRIX = range(8)
+(OP_SORT, OP_SYM, OP_GENERAL, OP_PHASED, OP_GRAM, OP_BACKWARD, OP_BACKWARD_GENERAL, OP_GRAM_MATRIX,
+ OP_BACKWARD_PHASED) = range(9)
 
 _lib = None
 _lock = threading.Lock()
@@ -63,6 +64,8 @@ SIGNATURES = {
                         ctypes.c_int),
     "laplex_backward_general": ([_P, _P, _I64, _P, _P, _I64, _P, _P, _P, _P, _P, ctypes.c_int, _P,
                                  ctypes.c_size_t, _P], ctypes.c_int),
+    "laplex_backward_phased": ([_P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int,
+                                _P, ctypes.c_size_t, _P], ctypes.c_int),
     "laplex_gram_matrix": ([_P, _P, _I64, _P, _P, _I64, _P, _P, _I64, ctypes.c_int, _P, ctypes.c_size_t, _P],
                            ctypes.c_int),
     "laplex_matvec_sym_noalloc": ([_P, _P, _I64, _P, _P, _P], ctypes.c_int),
@@ -285,6 +288,29 @@ def backward_general(sa, sb, x, g, pa=None, pb=None):
                                          _ptr(dx), _ptr(da), _ptr(db), _dt(x), _ptr(ws), nb,
                                          _stream(dev)))
     return dx, da, db
+
+
+def backward_phased(sa, phi, x, g, pa=None, sb=None, psi=None, pb=None):
+    """Gradients of L = <g, K x>, K_ij = exp(-|a_i - b_j|) cos(phi_i - psi_j).
+
+    sb given: (dx, dphi, dpsi, da, db); phi, g, dphi, da follow pa, and psi, x,
+    dx, dpsi, db follow pb.  sb None (b = a, psi = phi): (dx, dphi, da) with the
+    shared anchors' and phases' total gradients."""
+    dev = _dev(sa, phi, x, g, _perm(pa), sb, psi, _perm(pb))
+    n = sa.numel()
+    sym = sb is None
+    k = n if sym else sb.numel()
+    dx, dphi, da = torch.empty_like(x), torch.empty_like(g), torch.empty_like(g)
+    dpsi = None if sym else torch.empty_like(x)
+    db = None if sym else torch.empty_like(x)
+    ws, nb = _ws(OP_BACKWARD_PHASED, n, k, 1, x.dtype, dev)
+    # a NULL sb selects the symmetric case: an empty b side gets a non-NULL
+    # pointer (the workspace's; nothing is read from it when k = 0)
+    sbp = _ptr(sb) if sym or k > 0 else _ptr(ws)
+    _check(lib().laplex_backward_phased(_ptr(sa), _ptr(pa), _ptr(phi), n, sbp, _ptr(pb), _ptr(psi), k,
+                                        _ptr(x), _ptr(g), _ptr(dx), _ptr(dphi), _ptr(dpsi), _ptr(da), _ptr(db),
+                                        _dt(x), _ptr(ws), nb, _stream(dev)))
+    return (dx, dphi, da) if sym else (dx, dphi, dpsi, da, db)
 
 
 def gram_matrix(sa, sb, D=None, pa=None, pb=None, out=None):

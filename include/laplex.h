@@ -72,7 +72,8 @@ typedef enum {
     LAPLEX_OP_GRAM = 4,
     LAPLEX_OP_BACKWARD = 5,
     LAPLEX_OP_BACKWARD_GENERAL = 6,
-    LAPLEX_OP_GRAM_MATRIX = 7
+    LAPLEX_OP_GRAM_MATRIX = 7,
+    LAPLEX_OP_BACKWARD_PHASED = 8
 } laplex_op;
 
 /* Library ABI version (major*10000 + minor*100 + patch). */
@@ -200,6 +201,31 @@ laplex_status laplex_backward_general(const void* sa, const int32_t* pa, int64_t
                                       const void* x, const void* g, void* dx, void* da,
                                       void* db, laplex_dtype dtype, void* ws, size_t ws_bytes,
                                       void* stream);
+
+/*
+ * Backward pass of the phased product: L = <g, K x>,
+ * K_ij = exp(-|a_i - b_j|) cos(phi_i - psi_j) (summary §2.1; anchors and phases
+ * trainable, §2.3), with respect to x, the phases and the anchors:
+ *   dx_j   = sum_i K_ij g_i,
+ *   dphi_i = -g_i sum_j exp(-|a_i - b_j|) sin(phi_i - psi_j) x_j,
+ *   dpsi_j =  x_j sum_i exp(-|a_i - b_j|) sin(phi_i - psi_j) g_i,
+ *   da_i   = -g_i sum_j sign(a_i - b_j) K_ij x_j,
+ *   db_j   = -x_j sum_i sign(b_j - a_i) K_ij g_i,        sign(0) = 0.
+ *   sa [n], pa [n]|NULL, sb [k], pb [k]|NULL: sorted anchors and perms as in
+ *              laplex_matvec_general; phi, g, dphi, da [n] follow pa; psi, x, dx,
+ *              dpsi, db [k] follow pb.
+ *   sb == NULL: symmetric case (b = a, psi = phi, k = n; k, pb, psi, dpsi, db
+ *              ignored).  The anchors and phases are shared, so dphi and da
+ *              receive the total gradients (both sides' terms); dx = K g.
+ *   Any of dx, dphi, dpsi, da, db may be NULL: that output is not computed.
+ *   B = 1.  Workspace: laplex_workspace_size(LAPLEX_OP_BACKWARD_PHASED, n, k, 1, ...).
+ * n = 0 or k = 0: the outputs on the other side are zero.
+ */
+laplex_status laplex_backward_phased(const void* sa, const int32_t* pa, const void* phi, int64_t n,
+                                     const void* sb, const int32_t* pb, const void* psi, int64_t k,
+                                     const void* x, const void* g, void* dx, void* dphi, void* dpsi,
+                                     void* da, void* db, laplex_dtype dtype, void* ws,
+                                     size_t ws_bytes, void* stream);
 
 /*
  * Weighted Gram matrix M = A diag(D) A^T, A_ij = exp(-|a_i - b_j|) (summary

@@ -46,9 +46,9 @@ def test_version_and_status_strings(L):
 
 def test_workspace_size_host_only(L):
     from exact_laplace_b200 import laplex as X
-    for op in range(8):
+    for op in range(9):
         for n in (0, 1, 4096, 1 << 24):
-            assert X.workspace_size(op, n, 1000 if op in (2, 3, 4, 6, 7) else 0, 1) >= 256
+            assert X.workspace_size(op, n, 1000 if op in (2, 3, 4, 6, 7, 8) else 0, 1) >= 256
     with pytest.raises(X.LaplexError) as e:
         X.workspace_size(1, -1)
     assert e.value.status == X.EINVAL
@@ -58,6 +58,8 @@ def test_workspace_size_host_only(L):
         X.workspace_size(1, 10, 0, 0)
     with pytest.raises(X.LaplexError):
         X.workspace_size(9, 10)
+    with pytest.raises(X.LaplexError):
+        X.workspace_size(-1, 10)
 
 
 def test_argument_errors_return_before_any_launch(L):
@@ -78,6 +80,18 @@ def test_argument_errors_return_before_any_launch(L):
     # NULL workspace
     st = L.laplex_backward(P(256), None, 10, P(256), P(256), P(256), P(256), 0, None, 0, None)
     assert st == X.EINVAL
+    # phased backward: NULL phases with n > 0, misaligned optional output
+    size = ctypes.c_size_t()
+    assert L.laplex_workspace_size(8, 10, 10, 1, 0, ctypes.byref(size)) == 0
+    st = L.laplex_backward_phased(P(256), None, None, 10, P(256), None, P(256), 10, P(256), P(256),
+                                  None, None, None, P(256), None, 0, P(256), size.value, None)
+    assert st == X.EINVAL and b"phi" in L.laplex_last_error()
+    st = L.laplex_backward_phased(P(256), None, P(256), 10, P(256), None, P(256), 10, P(256), P(256),
+                                  None, P(260), None, None, None, 0, P(256), size.value, None)
+    assert st == X.EINVAL and b"dphi" in L.laplex_last_error()
+    st = L.laplex_backward_phased(P(256), None, P(256), 10, None, None, None, 0, P(256), P(256),
+                                  None, None, None, P(256), None, 0, P(256), 300, None)
+    assert st == X.EWORKSPACE
     # n = 0 is a no-op that needs no pointers
     size = ctypes.c_size_t()
     assert L.laplex_workspace_size(1, 0, 0, 1, 0, ctypes.byref(size)) == 0
