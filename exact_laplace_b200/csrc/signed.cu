@@ -291,22 +291,73 @@ struct OneSidedPhasedTP {
 
 static constexpr int pb_E(int es) { return es == 4 ? 8 : 4; }
 
+// [lb, ub): the run of entries equal to sp[r] around index r (ascending sp of
+// length k), by galloping outward from r and bisecting the last step: O(log of
+// the run length) loads instead of a search over the whole array.
+template <typename T>
+__device__ __forceinline__ void tie_run(const T* __restrict__ sp, int64_t k, int64_t r, int64_t& lb, int64_t& ub) {
+    const T q = sp[r];
+    int64_t in = r, out = r, step = 1;  // sp[in] == q; out: below the run, or -1
+    for (;;) {
+        out = r - step;
+        if (out < 0) {
+            out = -1;
+            break;
+        }
+        if (sp[out] < q) break;
+        in = out;
+        step <<= 1;
+    }
+    while (in - out > 1) {
+        const int64_t mid = out + ((in - out) >> 1);
+        if (sp[mid] < q) out = mid;
+        else in = mid;
+    }
+    lb = in;
+    in = r;
+    step = 1;
+    for (;;) {  // out: above the run, or k
+        out = r + step;
+        if (out >= k) {
+            out = k;
+            break;
+        }
+        if (sp[out] > q) break;
+        in = out;
+        step <<= 1;
+    }
+    while (out - in > 1) {
+        const int64_t mid = in + ((out - in) >> 1);
+        if (sp[mid] > q) out = mid;
+        else in = mid;
+    }
+    ub = in + 1;
+}
+
 // Per sorted query anchor r (row pq[r]; phase th and weight w in row order):
 //     prod = cos th P0 + sin th P1,  dph = w (cos th P1 - sin th P0),
 //     dan = -w (cos th S0 + sin th S1),
 // each where its pointer is not NULL: prod written, dph and dan written (acc = 0)
-// or added (acc = 1).  k = 0 gives P = S = 0.
+// or added (acc = 1).  k = 0 gives P = S = 0.  self_q: the queries are the
+// p-side anchors themselves (sq == sp, m == k), so the bounds are the tie run
+// around r.
 template <typename T>
 __global__ void __launch_bounds__(256) k_phased_query(const T* __restrict__ sq, const int32_t* __restrict__ pq,
                                                       int64_t m, const T* __restrict__ th,
                                                       const T* __restrict__ w, const T* __restrict__ sp,
                                                       int64_t k, const T* __restrict__ F,
                                                       const T* __restrict__ G, T* prod, T* dph, T* dan,
-                                                      int acc) {
+                                                      int acc, int self_q) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < m; r += stride) {
         const T q = sq[r];
-        const int64_t lb = bound<T>(sp, k, q, false), ub = bound<T>(sp, k, q, true);
+        int64_t lb, ub;
+        if (self_q) {
+            tie_run<T>(sp, k, r, lb, ub);
+        } else {
+            lb = bound<T>(sp, k, q, false);
+            ub = bound<T>(sp, k, q, true);
+        }
         T P0 = T(0), P1 = T(0), S0 = T(0), S1 = T(0);
         if (ub > 0) {
             const T f = dexp<T>(sp[ub - 1] - q);
@@ -384,7 +435,9 @@ static cudaError_t phased_pass(const T* sp, const int32_t* pp, int64_t k, const 
     e = tp_sm_count(sms);
     if (e != cudaSuccess) return e;
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((m + 255) / 256, (int64_t)sms * 16));
-    k_phased_query<T><<<(unsigned)blocks, 256, 0, st>>>(sq, pq, m, thq, w, sp, k, F, G, prod, dph, dan, acc);
+    const int self_q = sq == sp && m == k ? 1 : 0;
+    k_phased_query<T><<<(unsigned)blocks, 256, 0, st>>>(sq, pq, m, thq, w, sp, k, F, G, prod, dph, dan, acc,
+                                                        self_q);
     return cudaGetLastError();
 }
 
