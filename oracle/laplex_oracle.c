@@ -100,8 +100,9 @@ void orc_general_sorted(int64_t n, int64_t k, int64_t B, const double* sa, const
 }
 
 /*
- * Signed sums for the anchor gradient (spec backward pass; the pages name
- * differentiability w.r.t. the anchors, [IT] §2.3 and §4.1, without a formula).
+ * Signed sums for the anchor gradient of the backward pass ("LAPLEX - La FFT dei
+ * Nuclei di Laplace Apprendibili", technical summary §2.3 and §4.1, name the
+ * differentiability w.r.t. the anchors without a formula).
  * With |.|' = sign and sign(0) = 0,
  *     D_i = sum_j sign(s_i - s_j) exp(-|s_i - s_j|) v_j
  *         = (sum over s_j < s_i) - (sum over s_j > s_i).

@@ -23,7 +23,7 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(laplex_[a-z_0-9]+)\s*\(", text)))
 
 
-def test_header_declares_the_north_star_calls():
+def test_header_declares_the_product_calls():
     names = declared_functions()
     for req in ("laplex_sort_anchors", "laplex_matvec_sym", "laplex_matvec_general",
                 "laplex_matvec_phased", "laplex_gram", "laplex_backward"):

@@ -464,6 +464,38 @@ def test_backward_phased_central_differences():
         assert abs(db[j] - _cd(lambda v: _loss_phased(a, phi, v, psi, x, g), b, j)) < 1e-7, j
 
 
+def test_backward_phased_pins_reject_planted_mistakes():
+    """Plausible slips in the phase and anchor gradients (channels swapped, the
+    sine's sign flipped, the sides' phases exchanged), built from the oracle's own
+    parts, each fail the central differences of the dense definition."""
+    rng = np.random.default_rng(33)
+    a, b = rng.uniform(0, 4, 9), rng.uniform(0, 4, 7)
+    phi, psi = rng.uniform(0, 2 * math.pi, 9), rng.uniform(0, 2 * math.pi, 7)
+    x, g = rng.normal(size=7), rng.normal(size=9)
+    xc = np.stack([np.cos(psi) * x, np.sin(psi) * x], axis=1)
+    P, S = O.general(a, b, xc), O.signed_general(a, b, xc)
+    fd_phi = np.array([_cd(lambda v: _loss_phased(a, v, b, psi, x, g), phi, i) for i in range(9)])
+    fd_a = np.array([_cd(lambda v: _loss_phased(v, phi, b, psi, x, g), a, i) for i in range(9)])
+    c, s = np.cos(phi), np.sin(phi)
+    good_phi = g * (c * P[:, 1] - s * P[:, 0])
+    good_a = -g * (c * S[:, 0] + s * S[:, 1])
+    assert np.abs(good_phi - fd_phi).max() < 1e-7 and np.abs(good_a - fd_a).max() < 1e-7
+    mutants_phi = {
+        "channels swapped": g * (c * P[:, 0] - s * P[:, 1]),
+        "sine sign flipped": g * (s * P[:, 0] - c * P[:, 1]),
+        "cos/sin of the wrong side": g * (np.cos(psi[:1]) * P[:, 1] - np.sin(psi[:1]) * P[:, 0]),
+    }
+    for name, m in mutants_phi.items():
+        assert np.abs(m - fd_phi).max() > 1e-3, name
+    mutants_a = {
+        "plain sums for signed": -g * (c * P[:, 0] + s * P[:, 1]),
+        "sign of the anchor gradient": g * (c * S[:, 0] + s * S[:, 1]),
+        "sine combination": -g * (c * S[:, 1] - s * S[:, 0]),
+    }
+    for name, m in mutants_a.items():
+        assert np.abs(m - fd_a).max() > 1e-3, name
+
+
 def test_backward_phased_ties_and_invariants():
     """Tied anchors: the dense derivative with sign(0) = 0, entry by entry.  A
     common phase shift and a common translation of both anchor sets leave L
