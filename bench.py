@@ -159,6 +159,24 @@ def cpu_baseline(n_total, seed, budget_s=10.0, m=1 << 24):
                       f"workload), fp64 sequential recurrences, {el:.1f} s"}
 
 
+def reduce_max(v, world, device):
+    """v on one rank; over several (torchrun replicas), the maximum over the
+    ranks: the slowest replica decides the job's time."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms):
+    """Whole-job throughput in units/s: every rank processes units_per_rank in
+    the (max-over-ranks) time ms."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def workload_config(n, world):
     """The config of the headline workload, the same for both arms."""
     e = int(round(math.log2(n))) if n > 0 and (n & (n - 1)) == 0 else None
@@ -218,11 +236,7 @@ def run_ours(args):
             dist.barrier()
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, world, dev)
 
     n = args.n
     hi = float(1 << 30)
@@ -277,7 +291,7 @@ def run_ours(args):
     X.device_status(dev)
     kernel_ms = max_over_ranks(sum(b.elapsed_time(a) for b, a in kev) / len(kev))
     ms_step = ms / args.steps
-    value = world * n / (ms_step * 1e-3) / 1e9
+    value = job_throughput(n, world, ms_step) / 1e9
     hbm, peak_kind = peaks()
     achieved = BYTES_PER_ELEM_SYM * n / (kernel_ms * 1e-3) / 1e9
     sha = src_sha("sym_stream.cu", "scan_core.cuh", "common.cuh", "bulk.cuh")
