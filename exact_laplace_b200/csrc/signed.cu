@@ -138,7 +138,8 @@ __global__ void __launch_bounds__(256) k_signed_query(const T* __restrict__ sq, 
     }
 }
 
-// workspace of one signed sum over a side of `len` anchors: F, G and the scan's
+// workspace of one signed sum over a side of `len` anchors: F and G, then the
+// scan's per-tile records (tp_ws_bytes)
 size_t sgen_ws_bytes(int64_t len, int f64) {
     const size_t es = f64 ? 8 : 4;
     const int64_t tile = (int64_t)OS_NT * os_E((int)es);
@@ -398,6 +399,8 @@ __global__ void __launch_bounds__(256) k_phased_query(const T* __restrict__ sq, 
     }
 }
 
+// workspace of one phased pass over a side of `len` anchors: F and G of the two
+// channels, then the scan's per-tile records (tp_ws_bytes)
 size_t pbwd_ws_bytes(int64_t len, int f64) {
     const size_t es = f64 ? 8 : 4;
     const int64_t tile = (int64_t)OS_NT * pb_E((int)es);
