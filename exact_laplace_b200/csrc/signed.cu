@@ -120,16 +120,40 @@ __device__ __forceinline__ int64_t bound(const T* __restrict__ sp, int64_t k, T 
     return lo;
 }
 
+// The queries are ascending, so a block takes them in chunks of QCH consecutive
+// ones and first finds the window [lo, hi) of sp that holds the bounds of all of
+// them: lo = #{sp < sq[r0]}, hi = #{sp <= sq[r1 - 1]}.  Each query then searches
+// only that window.  Contains block barriers: every thread of the block calls it.
+constexpr int QCH = 256;
+
+template <typename T>
+__device__ __forceinline__ void chunk_window(const T* __restrict__ sq, const T* __restrict__ sp, int64_t k,
+                                             int64_t r0, int64_t r1, int64_t& lo, int64_t& hi) {
+    __shared__ int64_t win[2];
+    __syncthreads();  // the previous chunk's threads have read win
+    if (threadIdx.x == 0) win[0] = bound<T>(sp, k, sq[r0], false);
+    if (threadIdx.x == 32) win[1] = bound<T>(sp, k, sq[r1 - 1], true);
+    __syncthreads();
+    lo = win[0];
+    hi = win[1];
+}
+
 // out[row_r] = -w[row_r] S_r for the sorted query anchors sq (rows through pq)
 template <typename T>
-__global__ void __launch_bounds__(256) k_signed_query(const T* __restrict__ sq, const int32_t* __restrict__ pq,
+__global__ void __launch_bounds__(QCH) k_signed_query(const T* __restrict__ sq, const int32_t* __restrict__ pq,
                                                       int64_t m, const T* __restrict__ sp, int64_t k,
                                                       const T* __restrict__ F, const T* __restrict__ G,
                                                       const T* __restrict__ w, T* __restrict__ out) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < m; r += stride) {
+    const int64_t nch = (m + QCH - 1) / QCH;
+    for (int64_t c = blockIdx.x; c < nch; c += gridDim.x) {
+        const int64_t r0 = c * QCH, r1 = min(r0 + QCH, m);
+        int64_t lo, hi;
+        chunk_window<T>(sq, sp, k, r0, r1, lo, hi);
+        const int64_t r = r0 + threadIdx.x;
+        if (r >= r1) continue;
         const T q = sq[r];
-        const int64_t lb = bound<T>(sp, k, q, false), ub = bound<T>(sp, k, q, true);
+        const int64_t lb = lo + bound<T>(sp + lo, hi - lo, q, false);
+        const int64_t ub = lo + bound<T>(sp + lo, hi - lo, q, true);
         T S = T(0);
         if (lb > 0) S = F[lb - 1] * dexp<T>(sp[lb - 1] - q);
         if (ub < k) S -= G[ub] * dexp<T>(q - sp[ub]);
@@ -172,7 +196,7 @@ static cudaError_t signed_pass(const T* sp, const int32_t* pp, int64_t k, const 
     e = tp_sm_count(sms);
     if (e != cudaSuccess) return e;
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((m + 255) / 256, (int64_t)sms * 16));
-    k_signed_query<T><<<(unsigned)blocks, 256, 0, st>>>(sq, pq, m, sp, k, F, G, w, out);
+    k_signed_query<T><<<(unsigned)blocks, QCH, 0, st>>>(sq, pq, m, sp, k, F, G, w, out);
     return cudaGetLastError();
 }
 
@@ -343,21 +367,26 @@ __device__ __forceinline__ void tie_run(const T* __restrict__ sp, int64_t k, int
 // p-side anchors themselves (sq == sp, m == k), so the bounds are the tie run
 // around r.
 template <typename T>
-__global__ void __launch_bounds__(256) k_phased_query(const T* __restrict__ sq, const int32_t* __restrict__ pq,
+__global__ void __launch_bounds__(QCH) k_phased_query(const T* __restrict__ sq, const int32_t* __restrict__ pq,
                                                       int64_t m, const T* __restrict__ th,
                                                       const T* __restrict__ w, const T* __restrict__ sp,
                                                       int64_t k, const T* __restrict__ F,
                                                       const T* __restrict__ G, T* prod, T* dph, T* dan,
                                                       int acc, int self_q) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < m; r += stride) {
+    const int64_t nch = (m + QCH - 1) / QCH;
+    for (int64_t c = blockIdx.x; c < nch; c += gridDim.x) {
+        const int64_t r0 = c * QCH, r1 = min(r0 + QCH, m);
+        int64_t lo = 0, hi = k;
+        if (!self_q) chunk_window<T>(sq, sp, k, r0, r1, lo, hi);  // self_q: the same for the whole grid
+        const int64_t r = r0 + threadIdx.x;
+        if (r >= r1) continue;
         const T q = sq[r];
         int64_t lb, ub;
         if (self_q) {
             tie_run<T>(sp, k, r, lb, ub);
         } else {
-            lb = bound<T>(sp, k, q, false);
-            ub = bound<T>(sp, k, q, true);
+            lb = lo + bound<T>(sp + lo, hi - lo, q, false);
+            ub = lo + bound<T>(sp + lo, hi - lo, q, true);
         }
         T P0 = T(0), P1 = T(0), S0 = T(0), S1 = T(0);
         if (ub > 0) {
@@ -439,7 +468,7 @@ static cudaError_t phased_pass(const T* sp, const int32_t* pp, int64_t k, const 
     if (e != cudaSuccess) return e;
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((m + 255) / 256, (int64_t)sms * 16));
     const int self_q = sq == sp && m == k ? 1 : 0;
-    k_phased_query<T><<<(unsigned)blocks, 256, 0, st>>>(sq, pq, m, thq, w, sp, k, F, G, prod, dph, dan, acc,
+    k_phased_query<T><<<(unsigned)blocks, QCH, 0, st>>>(sq, pq, m, thq, w, sp, k, F, G, prod, dph, dan, acc,
                                                         self_q);
     return cudaGetLastError();
 }
