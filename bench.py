@@ -154,9 +154,16 @@ def cpu_baseline(n_total, seed, budget_s=10.0, m=1 << 24):
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    return {"value": done / el / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+    return {"value": done / el / 1e9, "unit": "Gelem/s", "cores": 1, "of": os.cpu_count(),
+            "kind": "oracle",
             "sample": f"{done // m} x {m} contiguous anchors (same density as the n=2^30 "
                       f"workload), fp64 sequential recurrences, {el:.1f} s"}
+
+
+def crow(ms, bytes_per_call, hbm):
+    """Compact row: time per call (ms) and roofline fraction (algorithmic bytes
+    per call / time / HBM peak), 4 and 3 significant digits."""
+    return {"ms": float(f"{ms:.4g}"), "frac": float(f"{bytes_per_call / (ms * 1e-3) / 1e9 / hbm:.3g}")}
 
 
 def reduce_max(v, world, device):
@@ -207,7 +214,8 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": workload_config(args.n, args.gpus),
-            "cpu_baseline": {"value": val, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": val, "unit": "Gelem/s", "cores": 1, "of": os.cpu_count(),
+                             "kind": "oracle",
                              "sample": f"{m} contiguous anchors of the workload's density per "
                                        "step, fp64 sequential recurrences on one host core"},
             "e2e": {"value": val, "unit": "Gelem/s", "h2d_bytes_per_step": 0,
@@ -321,18 +329,12 @@ def run_ours(args):
             if "sort" in wanted:
                 ms_s = timed(lambda: X.sort_anchors(a_d, s2, p2), rsteps, 1) / rsteps
                 X.device_status(dev)
-                rows["c5_sort"] = {"ms": ms_s, "Gelem_s": world * n / ms_s / 1e6,
-                                   "algorithmic_GB_s": 12 * n / ms_s / 1e6,
-                                   "frac_of_measured_hbm": 12 * n / ms_s / 1e6 / hbm,
-                                   "algorithmic_bytes_per_elem": 12}
+                rows["c5_sort"] = crow(ms_s, 12 * n, hbm)
             if "perm" in wanted:
                 X.sort_anchors(a_d, s2, p2)
                 ms_p = timed(lambda: X.matvec_sym(s2, x_d, p2, out=y_d), rsteps, 1) / rsteps
                 X.device_status(dev)
-                rows["c5_matvec_perm"] = {"ms": ms_p, "Gelem_s": world * n / ms_p / 1e6,
-                                          "algorithmic_GB_s": 16 * n / ms_p / 1e6,
-                                          "frac_of_measured_hbm": 16 * n / ms_p / 1e6 / hbm,
-                                          "algorithmic_bytes_per_elem": 16}
+                rows["c5_matvec_perm"] = crow(ms_p, 16 * n, hbm)
         except X.LaplexError as e:
             rows["sort_error"] = str(e)
         del a_d, s2, p2
@@ -343,10 +345,7 @@ def run_ours(args):
                 da = torch.empty_like(x_d)
                 ms_b = timed(lambda: X.backward(s_d, x_d, g_d, dx_out=dx, da_out=da), rsteps, 1) / rsteps
                 X.device_status(dev)
-                rows["c5_backward"] = {"ms": ms_b, "Gelem_s": world * n / ms_b / 1e6,
-                                       "algorithmic_GB_s": 20 * n / ms_b / 1e6,
-                                       "frac_of_measured_hbm": 20 * n / ms_b / 1e6 / hbm,
-                                       "algorithmic_bytes_per_elem": 20}
+                rows["c5_backward"] = crow(ms_b, 20 * n, hbm)
                 del g_d, dx, da
             except X.LaplexError as e:
                 rows["backward_error"] = str(e)
@@ -375,10 +374,18 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         return max_over_ranks(sum(a.elapsed_time(b) for a, b in evs)) / steps
 
-    def row(ms, elems, bytes_per, note):
-        gbs = bytes_per / ms / 1e6
-        return {"ms": ms, "Gelem_s": world * elems / ms / 1e6, "algorithmic_GB_s": gbs,
-                "frac_of_measured_hbm": gbs / hbm, "algorithmic_bytes": bytes_per, "note": note}
+    def timed_warm(fn, steps):
+        """Mean device time of back-to-back calls (inputs left in L2 by the
+        previous call where they fit)."""
+        return timed(fn, steps, 2) / steps
+
+    def frow(fn, bytes_per, steps):
+        """A row timed both with L2 flushed before every call (ms, frac) and
+        warm (warm_ms, warm_frac); frac = algorithmic bytes / time / HBM peak."""
+        r = crow(timed_flush(fn, steps), bytes_per, hbm)
+        w = crow(timed_warm(fn, steps), bytes_per, hbm)
+        r["warm_ms"], r["warm_frac"] = w["ms"], w["frac"]
+        return r
 
     fsteps = max(3, min(20, args.steps // 10))
     try:
@@ -395,12 +402,10 @@ def run_ours(args):
                 def c2_full():
                     X.sort_anchors(a2d, s2d, p2d)
                     X.matvec_sym(s2d, x2d, p2d, out=y2d)
-                ms2 = timed_flush(c2_full, fsteps)
-                rows[f"c2_sort_and_matvec_B{B}"] = row(ms2, n2, n2 * (12 + 16 + 8 * B), "n=2^24, a~N(0,2000^2) unsorted: sort + permuted product")
+                rows[f"c2_sort_and_matvec_B{B}"] = frow(c2_full, n2 * (12 + 16 + 8 * B), fsteps)
                 X.sort_anchors(a2d, s2d, p2d)
                 xs = x2d[p2d.long()].contiguous()
-                ms3 = timed_flush(lambda: X.matvec_sym(s2d, xs, out=y2d), fsteps)
-                rows[f"c2_presorted_B{B}"] = row(ms3, n2, n2 * (4 + 8 * B), "n=2^24 pre-sorted product")
+                rows[f"c2_presorted_B{B}"] = frow(lambda: X.matvec_sym(s2d, xs, out=y2d), n2 * (4 + 8 * B), fsteps)
                 del a2d, x2d, y2d, s2d, p2d, xs
             X.device_status(dev)
         if "c3" in wanted:
@@ -414,26 +419,18 @@ def run_ours(args):
             y3 = torch.empty_like(ws3)
             z3 = torch.empty_like(xs3)
             nn, kk = 1 << 22, 1 << 20
-            ms = timed_flush(lambda: X.matvec_general(sa, sb, xs3, out=y3), fsteps)
-            rows["c3_general_Kx"] = row(ms, nn, 8 * nn + 8 * kk, "n=2^22, k=2^20, pre-sorted, y=Kx")
-            ms = timed_flush(lambda: X.matvec_general(sa, sb, ws3, transpose=True, out=z3), fsteps)
-            rows["c3_general_KTw"] = row(ms, kk, 8 * nn + 8 * kk, "n=2^22, k=2^20, pre-sorted, z=K^T w")
+            rows["c3_general_Kx"] = frow(lambda: X.matvec_general(sa, sb, xs3, out=y3), 8 * nn + 8 * kk, fsteps)
+            rows["c3_general_KTw"] = frow(lambda: X.matvec_general(sa, sb, ws3, transpose=True, out=z3), 8 * nn + 8 * kk, fsteps)
             # anchor gradients of <w, K x> (sorted order): reads a, b, x, w; writes dx, da, db
-            ms = timed_flush(lambda: X.backward_general(sa, sb, xs3, ws3), fsteps)
-            rows["c3_backward_general"] = row(ms, nn + kk, 16 * nn + 16 * kk,
-                                              "n=2^22, k=2^20, pre-sorted: dx = K^T w, da, db")
+            rows["c3_backward_general"] = frow(lambda: X.backward_general(sa, sb, xs3, ws3), 16 * nn + 16 * kk, fsteps)
             # weighted Gram matrix of 4096 a-points over the 2^20 b-points (output 64 MB)
             sa4 = sa[:: (nn // 4096)].contiguous()
-            ms = timed_flush(lambda: X.gram_matrix(sa4, sb, xs3.abs()), fsteps)
-            rows["gram_matrix_4096x2^20"] = row(ms, 4096 * 4096, 4 * 4096 * 4096 + 12 * kk,
-                                                "M = A diag(D) A^T, n=4096 of the C3 a-points, k=2^20")
+            rows["gram_matrix_4096x2^20"] = frow(lambda: X.gram_matrix(sa4, sb, xs3.abs()), 4 * 4096 * 4096 + 12 * kk, fsteps)
             # phased anchor and phase gradients (phases ~ U(0, 2 pi), sorted order):
             # reads a, phi, w, b, psi, x; writes dphi, da, dx, dpsi, db
             phi3 = torch.from_numpy(synth.uniform(nn, 0.0, 2 * math.pi, seed=rank, stream="phi")).to(dev)
             psi3 = torch.from_numpy(synth.uniform(kk, 0.0, 2 * math.pi, seed=rank, stream="psi")).to(dev)
-            ms = timed_flush(lambda: X.backward_phased(sa, phi3, xs3, ws3, sb=sb, psi=psi3), fsteps)
-            rows["c3_backward_phased"] = row(ms, nn + kk, 20 * nn + 24 * kk,
-                                             "n=2^22, k=2^20, pre-sorted, phased: dx, dphi, dpsi, da, db")
+            rows["c3_backward_phased"] = frow(lambda: X.backward_phased(sa, phi3, xs3, ws3, sb=sb, psi=psi3), 20 * nn + 24 * kk, fsteps)
             X.device_status(dev)
             del a3d, b3d, sa, pa, sb, pb, x3d, w3d, xs3, ws3, y3, z3, phi3, psi3
         if "c4" in wanted:
@@ -444,14 +441,10 @@ def run_ours(args):
             phis = torch.from_numpy(phi4).to(dev)[p4.long()].contiguous()
             vs = torch.from_numpy(v4).to(dev)[p4.long()].contiguous()
             y4 = torch.empty_like(vs)
-            ms = timed_flush(lambda: X.matvec_phased(s4, phis, vs, out=y4), fsteps)
-            rows["c4_phased_Kv"] = row(ms, n4, 16 * n4, "n=3*1024^2, pre-sorted, phased y=Kv")
-            ms = timed_flush(lambda: X.gram(s4, vs, phi=phis, out=y4), fsteps)
-            rows["c4_gram_KTKv"] = row(ms, n4, 32 * n4, "n=3*1024^2, pre-sorted, K^T K v")
+            rows["c4_phased_Kv"] = frow(lambda: X.matvec_phased(s4, phis, vs, out=y4), 16 * n4, fsteps)
+            rows["c4_gram_KTKv"] = frow(lambda: X.gram(s4, vs, phi=phis, out=y4), 32 * n4, fsteps)
             gs4 = torch.from_numpy(synth.normal(n4, seed=rank, stream="g")).to(dev)
-            ms = timed_flush(lambda: X.backward_phased(s4, phis, vs, gs4), fsteps)
-            rows["c4_backward_phased"] = row(ms, n4, 28 * n4,
-                                             "n=3*1024^2, pre-sorted, symmetric phased: dx, dphi, da")
+            rows["c4_backward_phased"] = frow(lambda: X.backward_phased(s4, phis, vs, gs4), 28 * n4, fsteps)
             X.device_status(dev)
             del a4d, s4, p4, phis, vs, y4, gs4
     except X.LaplexError as e:
@@ -462,14 +455,31 @@ def run_ours(args):
     # ---------------- end to end through host buffers (pinned)
     e2e = None
     if not args.no_e2e:
+        # whole steps through host buffers: every step copies its s and x from
+        # pinned host memory and its y back; the streamer overlaps step k's
+        # copy in with step k-1's product and step k-2's copy out
         y_p = torch.empty(n, dtype=torch.float32).pin_memory()
-        esteps = max(2, min(5, args.steps))
-        ms_e = timed(lambda: X.matvec_sym_host(s_p, x_p, device=dev, out=y_p), esteps, 1)
+        esteps = max(3, min(6, args.steps))
+        hs = X.HostStreamer(n, device=dev)
+        hs.submit(s_p, x_p, y_p)  # warm-up step
+        hs.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(hs.h2d)
+        for _ in range(esteps):
+            hs.submit(s_p, x_p, y_p)
+        e1.record(hs.d2h)
+        hs.synchronize()
+        barrier()
+        ms_e = max_over_ranks(e0.elapsed_time(e1))
+        del hs
+        torch.cuda.empty_cache()
         e2e = {"value": world * n / (ms_e / esteps * 1e-3) / 1e9, "unit": "Gelem/s",
                "h2d_bytes_per_step": s_p.numel() * 4 + x_p.numel() * 4,
                "d2h_bytes_per_step": y_p.numel() * 4, "steps": esteps,
-               "path": "exact_laplace_b200.laplex.matvec_sym_host (pinned host -> device, "
-                       "laplex_matvec_sym, device -> pinned host)"}
+               "path": "exact_laplace_b200.laplex.HostStreamer: pinned host -> device, "
+                       "laplex_matvec_sym, device -> pinned host, overlapped across steps"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -481,8 +491,9 @@ def run_ours(args):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic",
                 "config": workload_config(n, world),
-                "roofline": roof, "rows": rows, "e2e": e2e, "cpu_baseline": cpu,
-                "clocks": clocks, "gpu_launches": KERNELS_PER_SYM_CALL * args.steps}
+                "roofline": roof, "e2e": e2e, "cpu_baseline": cpu,
+                "clocks": clocks, "gpu_launches": KERNELS_PER_SYM_CALL * args.steps,
+                "rows": rows}  # last, so that a tail of the line keeps them
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -150,6 +150,11 @@ laplex_status laplex_set_profile_events(void* before, void* after) {
     return ok();
 }
 
+laplex_status laplex_test_set_sort_wait(uint32_t polls, int force_expiry) {
+    lx::set_sort_wait(polls, force_expiry);
+    return ok();
+}
+
 laplex_status laplex_workspace_size(laplex_op op, int64_t n, int64_t k, int64_t B, laplex_dtype dt,
                                     size_t* bytes) {
     REQ(bytes != nullptr, "bytes is NULL");

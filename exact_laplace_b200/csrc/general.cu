@@ -342,8 +342,8 @@ static cudaError_t gen_launch(const GenArgs<T>& A, const GenPlan& p, void* wsbod
     TPWs<T, C> W = tp_carve<T, C>(cv, p.ntiles);
     if (!cv.ok) return cudaErrorInvalidValue;
     const int64_t nb = (p.ntiles + TP_CARRY_BT - 1) / TP_CARRY_BT;
-    int sms = 0;
-    cudaError_t e = tp_sm_count(sms);
+    int dev_ = 0, sms = 0;
+    cudaError_t e = tp_sm_count(dev_, sms);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(W.redo_count, 0, sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;

@@ -78,6 +78,10 @@ cudaError_t stream_run(const T* s, const T* x, T* y, const int32_t* pout, int64_
 
 // -------------------------------------------------------------- sort
 size_t sort_ws_bytes(int64_t n, int f64);
+// bound of each bulk-copy wait of the calling thread's later sorts (0: the
+// default, 2^20 polls), and a test switch under which the first copy of every
+// block of a digit pass is never issued, so that its wait runs to the bound
+void set_sort_wait(uint32_t polls, int force_expiry);
 template <typename T>
 cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws,
                      size_t ws_bytes, uint32_t* status, cudaStream_t st);

@@ -192,8 +192,8 @@ static cudaError_t signed_pass(const T* sp, const int32_t* pp, int64_t k, const 
     p.G = G;
     cudaError_t e = tp_run(p, cv.base + cv.off, cv.cap - cv.off, st);
     if (e != cudaSuccess) return e;
-    int sms = 0;
-    e = tp_sm_count(sms);
+    int dev_ = 0, sms = 0;
+    e = tp_sm_count(dev_, sms);
     if (e != cudaSuccess) return e;
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((m + 255) / 256, (int64_t)sms * 16));
     k_signed_query<T><<<(unsigned)blocks, QCH, 0, st>>>(sq, pq, m, sp, k, F, G, w, out);
@@ -463,8 +463,8 @@ static cudaError_t phased_pass(const T* sp, const int32_t* pp, int64_t k, const 
         e = tp_run(p, cv.base + cv.off, cv.cap - cv.off, st);
         if (e != cudaSuccess) return e;
     }
-    int sms = 0;
-    e = tp_sm_count(sms);
+    int dev_ = 0, sms = 0;
+    e = tp_sm_count(dev_, sms);
     if (e != cudaSuccess) return e;
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((m + 255) / 256, (int64_t)sms * 16));
     const int self_q = sq == sp && m == k ? 1 : 0;
@@ -655,8 +655,8 @@ cudaError_t grammat_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, 
     double* Pa = cv.take<double>(n);
     int32_t* inv = cv.take<int32_t>(n);
     if (!cv.ok) return cudaErrorInvalidValue;
-    int sms = 0;
-    cudaError_t e = tp_sm_count(sms);
+    int dev_ = 0, sms = 0;
+    cudaError_t e = tp_sm_count(dev_, sms);
     if (e != cudaSuccess) return e;
     const int64_t gb = std::max<int64_t>(1, (int64_t)sms * 8);
     if (k > 0) {

@@ -10,45 +10,91 @@
 // and is stable, so equal anchors keep ascending index order and the output
 // permutation is unique.  A NaN or Inf anchor sets ST_NONFINITE.
 //
-// Onesweep (Adinets & Merrill, "Onesweep: A Faster Least Significant Digit
-// Radix Sort for GPUs", 2022):
-//   k_radix_hist    : one read of the keys counts every digit of every pass
-//   k_radix_offsets : exclusive scan of each pass's 256 counts
-//   k_onesweep      : one kernel per pass.  Tiles are taken in ticket order;
-//                     each ranks its keys stably (warp match + per-warp
-//                     counters), publishes its 256 digit counts, and finds how
-//                     many keys of each digit lie in earlier tiles by a
-//                     decoupled look-back over 64-bit records (pass tag in the
-//                     high word, so one memset per call serves every pass).
-//                     Keys are staged in shared memory in digit order, so the
-//                     writes to each digit's run coalesce.
+// Every pass is a reduce-then-scan over tiles of 4096 keys (fp32; 2048 fp64),
+// three launches without any wait between blocks:
+//   k_count      : per tile, the count of each digit; each block walks a
+//                  contiguous range of tiles and keeps running sums, so it
+//                  writes per tile the counts of the earlier tiles of its
+//                  range, and at the end its range's totals
+//   k_count_scan : one block: per digit, the exclusive sums over the ranges,
+//                  plus the digit's start (the exclusive sum over smaller digits)
+//   k_scatter    : persistent blocks, tile t on block t mod G; the tiles'
+//                  keys (and payloads) arrive in a ring of shared-memory stages
+//                  by 1-D bulk copies (TMA), the next ones in flight while one
+//                  is ranked: a stable rank per warp (equal digits found by
+//                  warp match or ballots, one shared atomic per group), staging
+//                  in digit order, then coalesced runs written per digit at the
+//                  offsets k_count_scan gave.
+// The count pass reads the keys once more (4 bytes per key) but leaves the
+// scatter free of the serial look-back of a single-pass sort, whose chain of
+// dependent L2 round trips bounded the tile rate on this GPU.
 // Pass 0 reads the anchors and generates the index payload; the last pass
 // writes the anchors back as values and the payload as perm.
 #include <algorithm>
+#include <type_traits>
 
+#include "bulk.cuh"
 #include "common.cuh"
+#include "devcache.h"
 #include "laplex_impl.h"
+
+// ranking of equal digits in a warp: 0 = warp match, 1 = eight ballots,
+// 3 = shared-memory match masks; 2 = chosen per pass from the digit histogram
+// between the warp match and LX_SORT_HI (1 or 3)
+#ifndef LX_SORT_RANK
+#define LX_SORT_RANK 2
+#endif
+#ifndef LX_SORT_HI
+#define LX_SORT_HI 3
+#endif
+// keys per thread (fp32) and input stages per block
+#ifndef LX_SORT_KPT
+#define LX_SORT_KPT 16
+#endif
+#ifndef LX_SORT_S
+#define LX_SORT_S 1
+#endif
+#ifndef LX_SORT_MINB
+#define LX_SORT_MINB 3
+#endif
+// k_count: one atomic for all lanes sharing lane 0's digit (1) or one per key (0)
+#ifndef LX_COUNT_AGG
+#define LX_COUNT_AGG 1
+#endif
 
 namespace lx {
 
 constexpr int RADIX = 256;
-constexpr int SORT_NT = 256;
+constexpr int SORT_NT = 256;  // threads per block: one digit per thread in the per-digit steps
+constexpr int SORT_NW = SORT_NT / 32;
+
+// bounded wait for phase `parity` of *bar with a caller-chosen bound
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t polls) {
+    for (uint32_t it = 0; it < polls; ++it)
+        if (mbar_test(bar, parity)) return true;
+    return false;
+}
 
 template <typename T> struct KeyOf;
 template <> struct KeyOf<float> { using K = uint32_t; };
 template <> struct KeyOf<double> { using K = uint64_t; };
 
-__device__ __forceinline__ uint32_t to_key(float f, bool& bad) {
-    uint32_t u = __float_as_uint(f);
-    bad |= (u & 0x7F800000u) == 0x7F800000u;
+// keys per thread and input stages (ring of bulk-copy destinations) per block
+template <typename T> struct SortShape;
+template <> struct SortShape<float> { static constexpr int KPT = LX_SORT_KPT, S = LX_SORT_S; };
+template <> struct SortShape<double> { static constexpr int KPT = 8, S = 1; };
+
+__device__ __forceinline__ uint32_t key_of_bits(uint32_t u) {
     if (u == 0x80000000u) u = 0u;
     return (u >> 31) ? ~u : (u | 0x80000000u);
 }
-__device__ __forceinline__ uint64_t to_key(double f, bool& bad) {
-    uint64_t u = (uint64_t)__double_as_longlong(f);
-    bad |= (u & 0x7FF0000000000000ull) == 0x7FF0000000000000ull;
+__device__ __forceinline__ uint64_t key_of_bits(uint64_t u) {
     if (u == 0x8000000000000000ull) u = 0ull;
     return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+__device__ __forceinline__ bool non_finite_bits(uint32_t u) { return (u & 0x7F800000u) == 0x7F800000u; }
+__device__ __forceinline__ bool non_finite_bits(uint64_t u) {
+    return (u & 0x7FF0000000000000ull) == 0x7FF0000000000000ull;
 }
 __device__ __forceinline__ uint32_t key_to_bits(uint32_t k) {
     return (k >> 31) ? (k ^ 0x80000000u) : ~k;
@@ -61,6 +107,68 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     unsigned m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
+}
+
+// Lanes of the warp holding the same digit (0..255; 256 marks padding, which
+// groups only with padding).  Three ways:
+//  - the warp match instruction, whose cost grows with the number of distinct
+//    digits among the 32 lanes (cheap for the few values of an exponent byte,
+//    slow on uniformly spread digits);
+//  - one ballot per digit bit, a fixed cost;
+//  - match masks in shared memory (wmask: this warp's RADIX + 1 words, zero on
+//    entry): every lane ors its bit into its digit's word and reads the word
+//    back; the group's highest lane clears the word at the next call (*clr,
+//    the previous call's word; RADIX + 1 after a clear).
+// use_match is uniform over the grid.
+template <bool RAGGED>
+__device__ __forceinline__ unsigned digit_peers(uint32_t dig, bool use_match, uint32_t* wmask,
+                                                uint32_t& clr, int lane) {
+    constexpr int HI = LX_SORT_RANK == 2 ? LX_SORT_HI : LX_SORT_RANK;
+    if (LX_SORT_RANK == 0 || (LX_SORT_RANK == 2 && use_match)) return __match_any_sync(FULL, dig);
+    if constexpr (HI == 3) {
+        if (clr <= RADIX) wmask[clr] = 0u;
+        __syncwarp();
+        atomicOr(&wmask[dig], 1u << lane);
+        __syncwarp();
+        const unsigned peers = wmask[dig];
+        clr = (peers >> lane) == 1u ? dig : RADIX + 1;  // the highest lane of the group clears
+        return peers;
+    } else {
+        unsigned m = FULL;
+#pragma unroll
+        for (int b = 0; b < (RAGGED ? 9 : 8); ++b) {
+            const bool on = (dig >> b) & 1u;
+            const unsigned bb = __ballot_sync(FULL, on);
+            m &= on ? bb : ~bb;
+        }
+        return m;
+    }
+}
+
+// The expected number of distinct digits among 32 keys drawn from a pass's
+// digit histogram below which the warp match ranks faster than the ballots
+// (measured on B200: about 3 distinct values, match 1.6x faster; about 30,
+// ballots 1.4x faster).
+constexpr float MATCH_BELOW_DISTINCT = 12.0f;
+
+// Predicated shared-memory atomics as single instructions (no branch, so no
+// divergence handling around them): the old value (0 where pred is false),
+// and the add without a result.
+__device__ __forceinline__ uint32_t atom_add_shared_if(bool pred, uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.b32 q, %3, 0;\n mov.b32 %0, 0;\n"
+        " @q atom.shared.add.u32 %0, [%1], %2;\n}\n"
+        : "=&r"(old)
+        : "r"(smem_u32(p)), "r"(v), "r"((uint32_t)pred)
+        : "memory");
+    return old;
+}
+__device__ __forceinline__ void red_add_shared_if(bool pred, uint32_t* p, uint32_t v) {
+    asm volatile("{\n .reg .pred q;\n setp.ne.b32 q, %2, 0;\n @q red.shared.add.u32 [%0], %1;\n}\n" ::"r"(
+                     smem_u32(p)),
+                 "r"(v), "r"((uint32_t)pred)
+                 : "memory");
 }
 
 // exclusive scan of one uint32 per thread over a block of NT threads
@@ -90,206 +198,396 @@ __device__ __forceinline__ uint32_t block_excl_sum(uint32_t v, uint32_t* sm /*NT
     __syncthreads();
     const uint32_t r = sm[w] + inc - v;
     total = sm[NT / 32];
-    __syncthreads();
-    return r;
+    return r;  // sm is written again only after the caller's next barriers
 }
 
-// A look-back record is one 64-bit word (tag in the high half, count in the
-// low half) written and read whole, and nothing else is read on the strength
-// of it, so relaxed accesses suffice and a window of loads can be in flight.
-__device__ __forceinline__ void st_relaxed64(uint64_t* p, uint64_t v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ uint64_t ld_relaxed64(const uint64_t* p) {
-    uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
+// ------------------------------------------------------------------ count
+// grid bound of k_count (sizes its per-block totals in the workspace)
+constexpr int COUNT_MAX_BLOCKS = 4096;
+constexpr int COUNT_BLOCKS_PER_SM = 4;
 
-// Counts of every digit of every pass in one read of the keys.
 template <typename T>
-__global__ void __launch_bounds__(SORT_NT) k_radix_hist(const T* __restrict__ a, int64_t n,
-                                                        uint32_t* __restrict__ hist,
-                                                        uint32_t* status) {
-    using K = typename KeyOf<T>::K;
-    constexpr int P = sizeof(K);
-    __shared__ uint32_t h[P][RADIX];
-    for (int j = threadIdx.x; j < P * RADIX; j += SORT_NT) (&h[0][0])[j] = 0u;
-    __syncthreads();
-    bool bad = false;
-    const int64_t stride = (int64_t)gridDim.x * SORT_NT;
-    for (int64_t i = (int64_t)blockIdx.x * SORT_NT + threadIdx.x; i < n; i += stride) {
-        const K k = to_key(a[i], bad);
-#pragma unroll
-        for (int p = 0; p < P; ++p) atomicAdd(&h[p][(unsigned)(k >> (8 * p)) & (RADIX - 1)], 1u);
+struct CountArgs {
+    const typename KeyOf<T>::K* keys;  // this pass's keys (pass 0: the anchor bits)
+    int64_t n, ntiles, R;              // R: tiles per block
+    int shift;
+    uint32_t* tile_pre;                // [ntiles][RADIX] counts of the earlier tiles of the range
+    uint32_t* blk_tot;                 // [G][RADIX] totals of each range
+    uint32_t* status;
+};
+
+// one key of this warp into the tile histogram; lane 0's digit is counted by
+// one atomic for all lanes that share it (the high digits of real anchors
+// take few values, and same-address shared atomics serialise)
+template <bool FIRST, typename K>
+__device__ __forceinline__ void count_key(K kb, bool valid, int shift, uint32_t* hb, bool& bad) {
+    K k = kb;
+    if constexpr (FIRST) {
+        bad |= valid && non_finite_bits(kb);
+        k = key_of_bits(kb);
     }
-    if (bad) set_status(status, ST_NONFINITE);
-    __syncthreads();
-    for (int j = threadIdx.x; j < P * RADIX; j += SORT_NT) {
-        const uint32_t c = (&h[0][0])[j];
-        if (c) atomicAdd(&hist[j], c);
-    }
+    const uint32_t dig = valid ? ((uint32_t)(k >> shift) & (RADIX - 1)) : (uint32_t)RADIX;
+#if LX_COUNT_AGG
+    const uint32_t d0 = __shfl_sync(FULL, dig, 0);
+    const unsigned same = __ballot_sync(FULL, dig == d0);
+    red_add_shared_if((threadIdx.x & 31) == 0 && d0 < RADIX, &hb[d0 & (RADIX - 1)], (uint32_t)__popc(same));
+    red_add_shared_if(dig != d0 && valid, &hb[dig & (RADIX - 1)], 1u);
+#else
+    red_add_shared_if(valid, &hb[dig & (RADIX - 1)], 1u);
+#endif
 }
 
-// hist[p][d] <- number of keys with a smaller digit d in pass p (one block per pass)
-__global__ void __launch_bounds__(SORT_NT) k_radix_offsets(uint32_t* __restrict__ hist) {
-    __shared__ uint32_t sm[SORT_NT / 32 + 1];
-    uint32_t* h = hist + (int64_t)blockIdx.x * RADIX;
-    uint32_t tot;
-    const uint32_t ex = block_excl_sum<SORT_NT>(h[threadIdx.x], sm, tot);
-    h[threadIdx.x] = ex;
-}
-
-constexpr uint32_t SORT_POLLS = 1u << 25;
-
-template <typename T, int KPT>
-__global__ void __launch_bounds__(SORT_NT, 3) k_onesweep(
-    const T* __restrict__ a, const typename KeyOf<T>::K* __restrict__ ksrc,
-    const int32_t* __restrict__ vsrc, int64_t n, int pass, const uint32_t* __restrict__ offsets,
-    uint64_t* __restrict__ rec, uint32_t* __restrict__ ticket, typename KeyOf<T>::K* __restrict__ kdst,
-    int32_t* __restrict__ vdst, int last, uint32_t* status) {
+template <typename T, bool FIRST>
+__global__ void __launch_bounds__(SORT_NT) k_count(CountArgs<T> A) {
     using K = typename KeyOf<T>::K;
-    constexpr int NT = SORT_NT, NW = NT / 32, TILE = NT * KPT;
-    static_assert(KPT % 4 == 0, "digits are packed four to a word");
-    __shared__ K skey[TILE];
-    __shared__ int32_t sval[TILE];
-    __shared__ uint32_t wcnt[NW][RADIX];
-    __shared__ uint32_t dstart[RADIX];
-    __shared__ int64_t gofs[RADIX];  // global position of staged key q: gofs[digit] + q
-    __shared__ uint32_t scan_sm[NT / 32 + 1];
-    __shared__ int64_t sh_tile;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int shift = 8 * pass;
-    const bool first = pass == 0;
-    if (threadIdx.x == 0) sh_tile = (int64_t)atomicAdd(ticket, 1u);
-    for (int j = threadIdx.x; j < NW * RADIX; j += NT) (&wcnt[0][0])[j] = 0u;
+    constexpr int NT = SORT_NT, TILE = NT * SortShape<T>::KPT;
+    constexpr int KPV = 16 / sizeof(K);          // keys per 16-byte vector
+    constexpr int VPT = TILE / KPV / NT;         // vectors per thread per tile
+    static_assert(VPT * KPV * NT == TILE, "a tile is whole vectors per thread");
+    __shared__ uint32_t h[2][RADIX];  // two tiles' histograms: one barrier per tile
+    const int d = threadIdx.x;
+    h[0][d] = 0u;
+    h[1][d] = 0u;
     __syncthreads();
-    const int64_t t = sh_tile;
-    const int64_t tb = t * TILE;
-    const int64_t end = min(tb + TILE, n);
-    const unsigned ltmask = lanemask_lt();
-    // key i of this thread is element lane0 + 32 i of the tile (coalesced per i)
-    const int64_t lane0 = tb + (int64_t)w * 32 * KPT + lane;
-    const int nvalid = (int)max((int64_t)0, min((int64_t)KPT, (end - lane0 + 31) / 32));
-    K k[KPT];
-    uint32_t dg[KPT / 4];  // the digits, four per word
-    uint32_t rk[KPT];
+    const int64_t t0 = (int64_t)blockIdx.x * A.R, t1 = std::min(t0 + A.R, A.ntiles);
+    const uint4* src = reinterpret_cast<const uint4*>(A.keys);
+    auto full_tile = [&](int64_t t) { return (t + 1) * TILE <= A.n; };
+    auto load = [&](int64_t t, uint4* v) {
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) v[j] = __ldcs(src + t * (TILE / KPV) + j * NT + threadIdx.x);
+    };
     bool bad = false;
+    uint32_t run = 0;
+    uint4 v[VPT];
+    if (t0 < t1 && full_tile(t0)) load(t0, v);
+    for (int64_t t = t0; t < t1; ++t) {
+        uint4 nx[VPT];
+        const bool nfull = t + 1 < t1 && full_tile(t + 1);
+        if (nfull) load(t + 1, nx);
+        uint32_t* hb = h[t & 1];
+        if (full_tile(t)) {
 #pragma unroll
-    for (int i = 0; i < KPT; ++i) {
-        const int64_t idx = lane0 + i * 32;
-        k[i] = i < nvalid ? (first ? to_key(a[idx], bad) : ksrc[idx]) : K(0);
-    }
+            for (int j = 0; j < VPT; ++j) {
+                const K* kv = reinterpret_cast<const K*>(&v[j]);
 #pragma unroll
-    for (int i = 0; i < KPT; i += 4) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) word |= ((uint32_t)(k[i + b] >> shift) & (RADIX - 1)) << (8 * b);
-        dg[i / 4] = word;
-    }
-    auto digit = [&](int i) -> int { return (int)((dg[i / 4] >> (8 * (i % 4))) & (RADIX - 1)); };
-    // stable rank among the keys of this warp with the same digit: lanes in
-    // order within a round, rounds in order.  The lowest lane of each group of
-    // equal digits adds the group to the warp's counter and hands the old
-    // count to the group with one shuffle.
-#pragma unroll
-    for (int i = 0; i < KPT; ++i) {
-        const bool valid = i < nvalid;
-        const int d = valid ? digit(i) : RADIX;  // padding ranks apart
-        const unsigned peers = __match_any_sync(FULL, d);
-        const int leader = __ffs(peers) - 1;
-        uint32_t base = 0;
-        if (valid && lane == leader) base = atomicAdd(&wcnt[w][d], (uint32_t)__popc(peers));
-        base = __shfl_sync(FULL, base, leader);
-        rk[i] = base + __popc(peers & ltmask);
-    }
-    __syncthreads();
-    const int d = threadIdx.x;  // NT == RADIX: one digit per thread from here on
-    uint32_t c = 0;  // this tile's count of digit d; wcnt[.][d] becomes the warps' exclusive offsets
-#pragma unroll
-    for (int ww = 0; ww < NW; ++ww) {
-        const uint32_t x = wcnt[ww][d];
-        wcnt[ww][d] = c;
-        c += x;
-    }
-    // publish this tile's count of digit d early; its prefix over earlier tiles
-    // is looked up after the tile is staged, when they have had time to finish
-    const uint64_t tagA = (uint64_t)(2 * pass + 2) << 32, tagI = (uint64_t)(2 * pass + 3) << 32;
-    uint64_t* my = rec + t * RADIX + d;
-    st_relaxed64(my, (t == 0 ? tagI : tagA) | c);
-    uint32_t tot;
-    dstart[d] = block_excl_sum<NT>(c, scan_sm, tot);  // its barriers publish wcnt
-    __syncthreads();                                   // and this one dstart
-    // stage the keys in digit order (rk becomes the staging position), then
-    // the payloads, loaded only now to keep the ranking's registers free
-#pragma unroll
-    for (int i = 0; i < KPT; ++i) {
-        if (i < nvalid) {
-            const int di = digit(i);
-            rk[i] += dstart[di] + wcnt[w][di];
-            skey[rk[i]] = k[i];
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < KPT; ++i) {
-        const int64_t idx = lane0 + i * 32;
-        if (i < nvalid) sval[rk[i]] = first ? (int32_t)idx : vsrc[idx];
-    }
-    // keys of digit d in all earlier tiles: walk back LB records at a time
-    // (loads in flight together), adding counts up to and including the first
-    // inclusive record
-    uint64_t excl = 0;
-    if (t > 0) {
-        constexpr int LB = 8;
-        bool done = false;
-        for (int64_t j0 = t - 1; !done; j0 -= LB) {
-            uint64_t val[LB];
-#pragma unroll
-            for (int q = 0; q < LB; ++q)
-                val[q] = j0 - q >= 0 ? ld_relaxed64(rec + (j0 - q) * RADIX + d) : tagI;
-#pragma unroll
-            for (int q = 0; q < LB; ++q) {
-                if (done) break;
-                uint32_t it = 0;
-                while ((val[q] & 0xFFFFFFFF00000000ull) < tagA) {
-                    if (++it > SORT_POLLS) break;
-                    __nanosleep(64);
-                    val[q] = ld_relaxed64(rec + (j0 - q) * RADIX + d);
-                }
-                if ((val[q] & 0xFFFFFFFF00000000ull) < tagA) {
-                    set_status(status, ST_TIMEOUT);
-                    done = true;
-                    break;
-                }
-                excl += val[q] & 0xFFFFFFFFull;
-                if ((val[q] & 0xFFFFFFFF00000000ull) == tagI) done = true;
+                for (int e = 0; e < KPV; ++e) count_key<FIRST>(kv[e], true, A.shift, hb, bad);
+            }
+        } else {  // the ragged last tile
+            for (int j = 0; j < TILE / NT; ++j) {
+                const int64_t idx = t * TILE + j * NT + threadIdx.x;
+                const bool valid = idx < A.n;
+                count_key<FIRST>(valid ? A.keys[idx] : K(0), valid, A.shift, hb, bad);
             }
         }
-        st_relaxed64(my, tagI | (excl + c));
+        __syncthreads();
+        const uint32_t c = hb[d];
+        hb[d] = 0u;  // counted into again two tiles later, after this tile's barrier
+        A.tile_pre[t * RADIX + d] = run;
+        run += c;
+        if (nfull) {
+#pragma unroll
+            for (int j = 0; j < VPT; ++j) v[j] = nx[j];
+        }
     }
-    (void)bad;  // non-finite anchors are reported by k_radix_hist
-    gofs[d] = (int64_t)offsets[d] + (int64_t)excl - (int64_t)dstart[d];
+    A.blk_tot[(int64_t)blockIdx.x * RADIX + d] = run;
+    if (FIRST && bad) set_status(A.status, ST_NONFINITE);
+}
+
+// One block of 1024 threads: blk_pre[b][d] = start of digit d + the count of
+// digit d in the ranges before b.  Thread (d, q) owns digit d and the q-th
+// quarter of the ranges.
+__global__ void __launch_bounds__(1024) k_count_scan(const uint32_t* __restrict__ blk_tot,
+                                                     uint32_t* __restrict__ blk_pre, int G,
+                                                     uint32_t* __restrict__ use_match) {
+    __shared__ uint32_t part[4][RADIX];
+    __shared__ uint32_t base[RADIX];
+    const int d = threadIdx.x & (RADIX - 1), q = threadIdx.x >> 8;
+    const int rq = (G + 3) / 4, r0 = std::min(G, q * rq), r1 = std::min(G, r0 + rq);
+    uint32_t sum = 0;
+    int r = r0;
+    for (; r + 8 <= r1; r += 8) {
+        uint32_t x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = blk_tot[(int64_t)(r + u) * RADIX + d];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) sum += x[u];
+    }
+    for (; r < r1; ++r) sum += blk_tot[(int64_t)r * RADIX + d];
+    part[q][d] = sum;
     __syncthreads();
-    const int cnt = (int)(end - tb);
-    for (int q = threadIdx.x; q < cnt; q += NT) {
-        const K kk = skey[q];
-        const int64_t gpos = gofs[(unsigned)(kk >> shift) & (RADIX - 1)] + q;
-        kdst[gpos] = last ? key_to_bits(kk) : kk;
-        vdst[gpos] = sval[q];
+    if (threadIdx.x < 32) {  // warp 0: exclusive scan of the 256 digit totals, 8 per lane
+        const int lane = threadIdx.x;
+        uint32_t tot[8], acc = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int dd = lane * 8 + u;
+            tot[u] = part[0][dd] + part[1][dd] + part[2][dd] + part[3][dd];
+            acc += tot[u];
+        }
+        uint32_t inc = acc;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t o = __shfl_up_sync(FULL, inc, off);
+            if (lane >= off) inc += o;
+        }
+        uint32_t ex = inc - acc;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            base[lane * 8 + u] = ex;
+            ex += tot[u];
+        }
+        // expected distinct digits among 32 keys: sum over d of 1 - (1 - p_d)^32
+        const float all = (float)__shfl_sync(FULL, inc, 31);
+        float ed = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            float q = 1.f - (float)tot[u] / fmaxf(all, 1.f);
+#pragma unroll
+            for (int k = 0; k < 5; ++k) q *= q;  // q^32
+            ed += 1.f - q;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ed += __shfl_xor_sync(FULL, ed, off);
+        if (lane == 0) *use_match = ed < MATCH_BELOW_DISTINCT ? 1u : 0u;
+    }
+    __syncthreads();
+    uint32_t pre = base[d];
+    for (int qq = 0; qq < q; ++qq) pre += part[qq][d];
+    for (r = r0; r < r1; ++r) {
+        const uint32_t x = blk_tot[(int64_t)r * RADIX + d];
+        blk_pre[(int64_t)r * RADIX + d] = pre;
+        pre += x;
+    }
+}
+
+// ------------------------------------------------------------------ scatter
+template <typename T>
+struct ScatterArgs {
+    const typename KeyOf<T>::K* ksrc;  // this pass's keys (pass 0: the anchor bits)
+    const int32_t* vsrc;               // and payloads (not read in pass 0)
+    typename KeyOf<T>::K* kdst;        // the next pass's keys (the last pass: anchor bits)
+    int32_t* vdst;                     // and payloads (the last pass: perm)
+    int64_t n, ntiles, R;              // R: tiles per k_count block
+    int shift;
+    const uint32_t* tile_pre;
+    const uint32_t* blk_pre;
+    const uint32_t* use_match;         // ranking of this pass (k_count_scan's choice)
+    uint32_t* status;
+    uint32_t polls;                    // bound of each copy wait
+    int force_expiry;                  // test hook: every block's first copy is never issued
+};
+
+// Dynamic shared memory of one k_scatter block.
+template <typename T, int KPT, int S, bool FIRST>
+constexpr size_t scatter_smem() {
+    using K = typename KeyOf<T>::K;
+    constexpr size_t TILE = (size_t)SORT_NT * KPT;
+    return S * TILE * sizeof(K) + (FIRST ? 0 : S * TILE * 4) + TILE * (sizeof(K) + 4) +
+           (size_t)SORT_NW * RADIX * 4;
+}
+
+template <typename T, int KPT, int S, bool FIRST, bool LAST>
+__global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<T> A) {
+    using K = typename KeyOf<T>::K;
+    constexpr int NT = SORT_NT, NW = SORT_NW, TILE = NT * KPT;
+    static_assert(32 * KPT * sizeof(K) >= (RADIX + 1) * 4, "a warp's key segment holds its match masks");
+    extern __shared__ __align__(128) unsigned char dyn[];
+    K* stage_k = reinterpret_cast<K*>(dyn);                               // [S][TILE] (pass 0: anchor bits)
+    int32_t* stage_v = reinterpret_cast<int32_t*>(stage_k + S * TILE);   // [S][TILE] (not in pass 0)
+    K* out_k = reinterpret_cast<K*>(stage_v + (FIRST ? 0 : S * TILE));    // [TILE] in digit order
+    int32_t* out_v = reinterpret_cast<int32_t*>(out_k + TILE);            // [TILE]
+    uint32_t* wcnt = reinterpret_cast<uint32_t*>(out_v + TILE);           // [NW][RADIX]
+    __shared__ __align__(8) uint64_t full[S];
+    __shared__ int32_t gofs[RADIX];   // output position of staged key q of digit d: gofs[d] + q
+    __shared__ uint32_t scan_sm[NW + 1];
+    __shared__ int sh_abort;
+
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int d = threadIdx.x;  // the digit of this thread in the per-digit steps
+    const int shift = A.shift;
+    const unsigned ltmask = lanemask_lt();
+    const int64_t G = gridDim.x;
+    const bool use_match = *A.use_match != 0u;
+
+    // thread 0: tile t into stage st (a bulk copy for a full tile; a plain
+    // arrive for the ragged last tile, which is read from global memory)
+    auto refill = [&](int st, int64_t t) {
+        if (t >= A.ntiles) return;
+        const int64_t tb = t * TILE;
+        if (tb + TILE <= A.n) {
+            constexpr uint32_t kb = TILE * sizeof(K), vb = FIRST ? 0u : TILE * 4u;
+            mbar_expect_tx(&full[st], kb + vb);
+            bulk_g2s(stage_k + st * TILE, A.ksrc + tb, kb, &full[st]);
+            if constexpr (!FIRST) bulk_g2s(stage_v + st * TILE, A.vsrc + tb, vb, &full[st]);
+        } else {
+            mbar_arrive(&full[st]);
+        }
+    };
+
+    if (threadIdx.x == 0) {
+        sh_abort = 0;
+        for (int st = 0; st < S; ++st) mbar_init(&full[st], 1u);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int st = 0; st < S; ++st)
+            if (!(A.force_expiry && st == 0)) refill(st, blockIdx.x + st * G);
+    }
+    for (int j = threadIdx.x; j < NW * RADIX; j += NT) wcnt[j] = 0u;
+    __syncthreads();
+
+    for (int64_t i = 0;; ++i) {
+        const int64_t t = blockIdx.x + i * G;
+        if (t >= A.ntiles) return;  // every copy this block issued has been waited for
+        const int st = (int)(i % S);
+        // this tile's output offset of digit d, loaded while its copy lands
+        const uint32_t off = A.blk_pre[(t / A.R) * RADIX + d] + A.tile_pre[t * RADIX + d];
+        // an expired wait is acted on at the first barrier below, together
+        if (!mbar_wait_bounded(&full[st], (uint32_t)((i / S) & 1), A.polls)) sh_abort = 1;
+        const int64_t tb = t * TILE;
+        const int cnt = (int)std::min<int64_t>((int64_t)TILE, A.n - tb);
+
+        auto body = [&](auto full_c) -> bool {
+            constexpr bool FT = decltype(full_c)::value;  // a full tile, staged by the bulk copy
+            const int seg = w * 32 * KPT + lane;          // key i of this thread: seg + 32 i
+            K k[KPT];
+#pragma unroll
+            for (int e = 0; e < KPT; ++e) {
+                const int q = seg + 32 * e;
+                K raw;
+                if constexpr (FT) raw = stage_k[st * TILE + q];
+                else raw = q < cnt ? A.ksrc[tb + q] : K(0);
+                k[e] = FIRST ? key_of_bits(raw) : raw;
+            }
+            // stable rank among the warp's keys of the same digit: rounds in
+            // order, lanes in order within a round; one lane of each group adds
+            // the group to the warp's counter.  The match masks, if used, live
+            // in this warp's own key segment of the stage, read above.
+            uint32_t* wmask = reinterpret_cast<uint32_t*>(stage_k + st * TILE + w * 32 * KPT);
+            __syncwarp();
+            for (int j = lane; j <= RADIX; j += 32) wmask[j] = 0u;
+            uint32_t clr = RADIX + 1;
+            uint32_t rk[KPT];
+#pragma unroll
+            for (int e = 0; e < KPT; ++e) {
+                const bool valid = FT || seg + 32 * e < cnt;
+                const uint32_t dig = valid ? ((uint32_t)(k[e] >> shift) & (RADIX - 1)) : (uint32_t)RADIX;
+                const unsigned peers = digit_peers<!FT>(dig, use_match, wmask, clr, lane);
+                const uint32_t pc = (uint32_t)__popc(peers);
+                const uint32_t lt = (uint32_t)__popc(peers & ltmask);
+                // the group's highest lane adds the group and hands out the old count
+                const uint32_t base =
+                    atom_add_shared_if(valid && lt + 1u == pc, &wcnt[w * RADIX + (dig & (RADIX - 1))], pc);
+                rk[e] = __shfl_sync(FULL, base, 31 - __clz(peers)) + lt;
+            }
+            // the masks were written through the generic proxy; the stage is
+            // refilled by a bulk copy (async proxy) after the next barriers
+            fence_proxy_async();
+            __syncthreads();
+            if (sh_abort) return false;
+            // per digit: the tile's count; wcnt[.][d] becomes the warps' offsets
+            // inside the tile's digit-ordered staging
+            uint32_t c = 0;
+#pragma unroll
+            for (int ww = 0; ww < NW; ++ww) {
+                const uint32_t x = wcnt[ww * RADIX + d];
+                wcnt[ww * RADIX + d] = c;
+                c += x;
+            }
+            uint32_t tot;
+            const uint32_t ds = block_excl_sum<NT>(c, scan_sm, tot);
+#pragma unroll
+            for (int ww = 0; ww < NW; ++ww) wcnt[ww * RADIX + d] += ds;
+            gofs[d] = (int32_t)(off - ds);
+            __syncthreads();
+            // stage keys, then payloads, in digit order
+#pragma unroll
+            for (int e = 0; e < KPT; ++e) {
+                const int q = seg + 32 * e;
+                if (FT || q < cnt) {
+                    rk[e] += wcnt[w * RADIX + ((uint32_t)(k[e] >> shift) & (RADIX - 1))];
+                    out_k[rk[e]] = k[e];
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < KPT; ++e) {
+                const int q = seg + 32 * e;
+                if (FT || q < cnt) {
+                    int32_t v;
+                    if constexpr (FIRST) v = (int32_t)tb + q;  // n < 2^31
+                    else if constexpr (FT) v = stage_v[st * TILE + q];
+                    else v = A.vsrc[tb + q];
+                    out_v[rk[e]] = v;
+                }
+            }
+            __syncthreads();
+            // the stage is consumed: the copy of this block's tile S rounds
+            // later runs while this one is written out
+            if (threadIdx.x == 0) {
+                fence_proxy_async();
+                refill(st, t + S * G);
+            }
+#pragma unroll
+            for (int ww = 0; ww < NW; ++ww) wcnt[ww * RADIX + d] = 0u;
+#pragma unroll
+            for (int j = 0; j < KPT; ++j) {
+                const int q = (int)threadIdx.x + j * NT;
+                if (FT || q < cnt) {
+                    const K kk = out_k[q];
+                    const int64_t g = (int64_t)gofs[(uint32_t)(kk >> shift) & (RADIX - 1)] + q;
+                    A.kdst[g] = LAST ? key_to_bits(kk) : kk;
+                    A.vdst[g] = out_v[q];
+                }
+            }
+            __syncthreads();  // out_k, out_v, gofs, wcnt are the next tile's
+            return true;
+        };
+        const bool ok = cnt == TILE ? body(std::true_type{}) : body(std::false_type{});
+        if (!ok) {
+            // a copy never landed: report it, give this block's copies in
+            // flight (this one included) a bounded time to land, and leave
+            if (threadIdx.x == 0) {
+                set_status(A.status, ST_TIMEOUT);
+                for (int64_t j = 0; j < S; ++j)
+                    if (t + j * G < A.ntiles)
+                        (void)mbar_wait_bounded(&full[(i + j) % S], (uint32_t)(((i + j) / S) & 1), A.polls);
+            }
+            return;
+        }
     }
 }
 
 // ------------------------------------------------------------------ host side
-template <typename T> constexpr int sort_kpt() { return sizeof(T) == 8 ? 8 : 16; }
+namespace {
+thread_local uint32_t g_sort_polls = MBAR_POLLS;
+thread_local int g_sort_force_expiry = 0;
+}  // namespace
+
+void set_sort_wait(uint32_t polls, int force_expiry) {
+    g_sort_polls = polls ? polls : MBAR_POLLS;
+    g_sort_force_expiry = force_expiry;
+}
+
+template <typename T> constexpr int sort_tile() { return SORT_NT * SortShape<T>::KPT; }
 
 size_t sort_ws_bytes(int64_t n, int f64) {
-    const int kpt = f64 ? 8 : 16;
-    const int64_t tile = (int64_t)SORT_NT * kpt;
+    const int64_t tile = f64 ? sort_tile<double>() : sort_tile<float>();
     const int64_t ntiles = std::max<int64_t>(1, (n + tile - 1) / tile);
     const size_t ks = f64 ? 8 : 4;
-    const int P = f64 ? 8 : 4;
     return Carve::need((size_t)n, ks) + Carve::need((size_t)n, 4) +
-           Carve::need((size_t)(16 + P * RADIX), 4) + Carve::need((size_t)(ntiles * RADIX), 8);
+           Carve::need((size_t)(ntiles * RADIX), 4) + 2 * Carve::need((size_t)COUNT_MAX_BLOCKS * RADIX, 4) +
+           Carve::need(1, 4);
+}
+
+template <typename T, bool FIRST, bool LAST>
+static cudaError_t launch_scatter(const ScatterArgs<T>& A, int dev, int sms, cudaStream_t st) {
+    constexpr int KPT = SortShape<T>::KPT, S = SortShape<T>::S;
+    constexpr auto kern = k_scatter<T, KPT, S, FIRST, LAST>;
+    constexpr size_t smem = scatter_smem<T, KPT, S, FIRST>();
+    int per = 0;
+    cudaError_t e = blocks_per_sm<kern>(dev, SORT_NT, smem, &per);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(A.ntiles, (int64_t)per * sms);
+    kern<<<(unsigned)grid, SORT_NT, smem, st>>>(A);
+    return cudaGetLastError();
 }
 
 template <typename T>
@@ -297,41 +595,63 @@ cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws, 
                      uint32_t* status, cudaStream_t st) {
     using K = typename KeyOf<T>::K;
     if (n == 0) return cudaSuccess;
-    constexpr int KPT = sort_kpt<T>();
     constexpr int P = sizeof(K);
-    const int64_t tile = (int64_t)SORT_NT * KPT;
+    const int64_t tile = sort_tile<T>();
     const int64_t ntiles = (n + tile - 1) / tile;
     Carve cv(ws, ws_bytes);
     K* kws = cv.take<K>(n);
     int32_t* vws = cv.take<int32_t>(n);
-    uint32_t* ctl = cv.take<uint32_t>(16 + P * RADIX);  // [0..P) tickets, [16..) histograms
-    uint64_t* rec = cv.take<uint64_t>(ntiles * RADIX);
+    uint32_t* tile_pre = cv.take<uint32_t>(ntiles * RADIX);
+    uint32_t* blk_tot = cv.take<uint32_t>((size_t)COUNT_MAX_BLOCKS * RADIX);
+    uint32_t* blk_pre = cv.take<uint32_t>((size_t)COUNT_MAX_BLOCKS * RADIX);
+    uint32_t* mode = cv.take<uint32_t>(1);
     if (!cv.ok) return cudaErrorInvalidValue;
-    uint32_t* tickets = ctl;
-    uint32_t* hist = ctl + 16;
-    cudaError_t e = cudaMemsetAsync(ctl, 0, sizeof(uint32_t) * (16 + P * RADIX), st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(rec, 0, sizeof(uint64_t) * ntiles * RADIX, st);
+    int dev = 0, sms = 0;
+    cudaError_t e = current_device_sms(&dev, &sms);
     if (e != cudaSuccess) return e;
-    {
-        const int64_t blocks = std::min<int64_t>((n + SORT_NT - 1) / SORT_NT, 148 * 8);
-        k_radix_hist<T><<<(unsigned)blocks, SORT_NT, 0, st>>>(a, n, hist, status);
-        k_radix_offsets<<<P, SORT_NT, 0, st>>>(hist);
-    }
+    // k_count: contiguous ranges of R tiles, every block non-empty
+    const int64_t gmax = std::min<int64_t>((int64_t)COUNT_BLOCKS_PER_SM * sms, COUNT_MAX_BLOCKS);
+    const int64_t R = (ntiles + gmax - 1) / gmax;
+    const int64_t Gc = (ntiles + R - 1) / R;
     K* kout = reinterpret_cast<K*>(sorted);
-    const K* ksrc = nullptr;
-    const int32_t* vsrc = nullptr;
+    CountArgs<T> C;
+    C.n = n;
+    C.ntiles = ntiles;
+    C.R = R;
+    C.tile_pre = tile_pre;
+    C.blk_tot = blk_tot;
+    C.status = status;
+    ScatterArgs<T> A;
+    A.n = n;
+    A.ntiles = ntiles;
+    A.R = R;
+    A.tile_pre = tile_pre;
+    A.blk_pre = blk_pre;
+    A.use_match = mode;
+    A.status = status;
+    A.polls = g_sort_polls;
+    A.force_expiry = g_sort_force_expiry;
+    A.ksrc = reinterpret_cast<const K*>(a);
+    A.vsrc = nullptr;
     profile_before(st);
     for (int pass = 0; pass < P; ++pass) {
-        const bool to_out = ((P - 1 - pass) % 2) == 0;
-        K* kdst = to_out ? kout : kws;
-        int32_t* vdst = to_out ? perm : vws;
-        k_onesweep<T, KPT><<<(unsigned)ntiles, SORT_NT, 0, st>>>(
-            a, ksrc, vsrc, n, pass, hist + pass * RADIX, rec, tickets + pass, kdst, vdst,
-            pass == P - 1, status);
+        const bool to_out = ((P - 1 - pass) % 2) == 0;  // the last pass lands in the outputs
+        C.keys = A.ksrc;
+        C.shift = 8 * pass;
+        if (pass == 0) k_count<T, true><<<(unsigned)Gc, SORT_NT, 0, st>>>(C);
+        else k_count<T, false><<<(unsigned)Gc, SORT_NT, 0, st>>>(C);
+        k_count_scan<<<1, 1024, 0, st>>>(blk_tot, blk_pre, (int)Gc, mode);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        ksrc = kdst;
-        vsrc = vdst;
+        A.kdst = to_out ? kout : kws;
+        A.vdst = to_out ? perm : vws;
+        A.shift = 8 * pass;
+        if (pass == 0) e = launch_scatter<T, true, false>(A, dev, sms, st);
+        else if (pass == P - 1) e = launch_scatter<T, false, true>(A, dev, sms, st);
+        else e = launch_scatter<T, false, false>(A, dev, sms, st);
+        if (e != cudaSuccess) return e;
+        A.ksrc = A.kdst;
+        A.vsrc = A.vdst;
     }
     profile_after(st);
     return cudaSuccess;

@@ -385,6 +385,8 @@ template cudaError_t sym_run<double>(SymArgs<double>, int64_t, bool, void*, size
 // laplex_matvec_sym_noalloc: the three-phase symmetric product (fp32, B = 1)
 // with its per-tile scratch in a fixed device array instead of a caller
 // workspace, for callers that cannot allocate device memory.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "laplex.h"
@@ -402,20 +404,44 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_BYTES];
 constexpr int NOALLOC_MAX_DEVICES = 64;
 static std::mutex g_noalloc_mu;
 static void* g_noalloc_ptr[NOALLOC_MAX_DEVICES];
+static CUcontext g_noalloc_ctx[NOALLOC_MAX_DEVICES];
 
-// Device address of g_noalloc_scratch on the current device (looked up once per
-// device; in host code the array's name is only a host-side handle).
+// The current context (NULL if none or unknown), through the driver entry
+// point that the runtime hands out, so the library needs no link to the driver.
+static CUcontext current_context() {
+    using GetCtx = CUresult (*)(CUcontext*);
+    static GetCtx fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<GetCtx>(f);
+    }();
+    CUcontext ctx = nullptr;
+    if (fn == nullptr || fn(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+    return ctx;
+}
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name is only a host-side handle, so the address is looked up with
+// cudaGetSymbolAddress, once per device and context: a device reset gives the
+// device a new primary context (and reloads the module), and the first call in
+// the new context looks the address up again.
 static cudaError_t noalloc_scratch(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    CUcontext ctx = current_context();
+    if (g_noalloc_ptr[dev] == nullptr || ctx == nullptr || ctx != g_noalloc_ctx[dev]) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // makes the primary context current
         if (e != cudaSuccess) return e;
+        ctx = current_context();
         g_noalloc_ptr[dev] = p;
+        g_noalloc_ctx[dev] = ctx;
     }
     *out = g_noalloc_ptr[dev];
     return cudaSuccess;

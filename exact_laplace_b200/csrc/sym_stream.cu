@@ -28,6 +28,7 @@
 
 #include "laplex_impl.h"
 #include "bulk.cuh"
+#include "devcache.h"
 #include "scan_core.cuh"
 
 namespace lx {
@@ -513,6 +514,23 @@ size_t stream_ws_bytes(int64_t n, int f64) {
            4 * Carve::need((size_t)nb, es);
 }
 
+// One persistent launch of a k_tile_local variant: as many blocks as fit on
+// the device (resident blocks per SM cached per device and variant), or one per
+// tile; `timed` records the profiling events around it.
+template <auto KERN, typename T>
+static cudaError_t launch_tiles(int dev, int sms, size_t smem, bool timed, cudaStream_t st, const T* s,
+                                const T* x, T* y, const int32_t* pp, int64_t n, int64_t ntiles,
+                                const LocalWs<T>& W, uint32_t* status) {
+    int per = 0;
+    cudaError_t e = blocks_per_sm<KERN>(dev, LT_NT, smem, &per);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(ntiles, (int64_t)per * sms);
+    if (timed) profile_before(st);
+    KERN<<<(unsigned)grid, LT_NT, smem, st>>>(s, x, y, pp, n, ntiles, W, status);
+    if (timed) profile_after(st);
+    return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t stream_run(const T* s, const T* x, T* y, const int32_t* pout, int64_t n, void* ws,
                        size_t ws_bytes, uint32_t* status, cudaStream_t st) {
@@ -526,50 +544,26 @@ cudaError_t stream_run(const T* s, const T* x, T* y, const int32_t* pout, int64_
     Carve cv(ws, ws_bytes);
     LocalWs<T> W = local_carve<T>(cv, ntiles);
     if (!cv.ok) return cudaErrorInvalidValue;
-    static int sms_cache[64] = {0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    int dev = 0, sms = 0;
+    cudaError_t e = current_device_sms(&dev, &sms);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (sms_cache[dev] == 0) {
-        e = cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-    }
-    // one persistent launch of k_tile_local<..., GATHER, MODE>; occupancy cached
-    // per device and variant
-    auto launch = [&](auto kern, int variant, size_t smem, const int32_t* pp, bool timed) -> cudaError_t {
-        static int per_sm[64][4] = {{0}};
-        if (per_sm[dev][variant] == 0) {
-            cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (r != cudaSuccess) return r;
-            int per = 0;
-            r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kern, LT_NT, smem);
-            if (r != cudaSuccess) return r;
-            per_sm[dev][variant] = std::max(1, per);
-        }
-        const int64_t grid = std::min<int64_t>(ntiles, (int64_t)per_sm[dev][variant] * sms_cache[dev]);
-        if (timed) profile_before(st);
-        kern<<<(unsigned)grid, LT_NT, smem, st>>>(s, x, y, pp, n, ntiles, W, status);
-        if (timed) profile_after(st);
-        return cudaGetLastError();
-    };
     e = cudaMemsetAsync(W.redo_count, 0, sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;
     const size_t smem_x = (size_t)LT_STAGES * STAGE * (2 * sizeof(T));
     const size_t smem_p = (size_t)LT_STAGES * STAGE * (sizeof(T) + sizeof(int32_t));
     if (pout == nullptr)
-        e = launch(k_tile_local<T, E, LT_NT, LT_STAGES, H, false, 0>, 0, smem_x, nullptr, true);
+        e = launch_tiles<k_tile_local<T, E, LT_NT, LT_STAGES, H, false, 0>>(dev, sms, smem_x, true, st, s, x, y, nullptr, n, ntiles, W, status);
     else
-        e = launch(k_tile_local<T, E, LT_NT, LT_STAGES, H, true, 0>, 1, smem_p, pout, true);
+        e = launch_tiles<k_tile_local<T, E, LT_NT, LT_STAGES, H, true, 0>>(dev, sms, smem_p, true, st, s, x, y, pout, n, ntiles, W, status);
     if (e != cudaSuccess) return e;
     k_carry_blocks<T><<<(unsigned)nb, CARRY_NT, 0, st>>>(W, ntiles);
     k_carry_tiles<T><<<(unsigned)nb, CARRY_NT, 0, st>>>(W, ntiles, nb);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (pout == nullptr)
-        e = launch(k_tile_local<T, E, LT_NT, LT_STAGES, H, false, 1>, 2, smem_x, nullptr, false);
+        e = launch_tiles<k_tile_local<T, E, LT_NT, LT_STAGES, H, false, 1>>(dev, sms, smem_x, false, st, s, x, y, nullptr, n, ntiles, W, status);
     else
-        e = launch(k_tile_local<T, E, LT_NT, LT_STAGES, H, true, 1>, 3, smem_p, pout, false);
+        e = launch_tiles<k_tile_local<T, E, LT_NT, LT_STAGES, H, true, 1>>(dev, sms, smem_p, false, st, s, x, y, pout, n, ntiles, W, status);
     return e;
 }
 

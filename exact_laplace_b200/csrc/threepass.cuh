@@ -32,6 +32,7 @@
 #include <algorithm>
 
 #include "bulk.cuh"
+#include "devcache.h"
 #include "laplex_impl.h"
 #include "scan_core.cuh"
 
@@ -612,19 +613,7 @@ cudaError_t tp_finish(const P& p, TPWs<typename P::T, P::C> W, int64_t ntiles, i
     return cudaGetLastError();
 }
 
-inline cudaError_t tp_sm_count(int& sms) {
-    static int sms_cache[64] = {0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (sms_cache[dev] == 0) {
-        e = cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-    }
-    sms = sms_cache[dev];
-    return cudaSuccess;
-}
+inline cudaError_t tp_sm_count(int& dev, int& sms) { return current_device_sms(&dev, &sms); }
 
 // The streamed pass 1 (k_tp_ring) for inputs in sorted order, then passes 2-3.
 template <class P>
@@ -636,19 +625,13 @@ cudaError_t tp_run_ring(const P& p, void* ws, size_t ws_bytes, uint32_t* status,
     Carve cv(ws, ws_bytes);
     TPWs<T, C> W = tp_carve<T, C>(cv, ntiles);
     if (!cv.ok) return cudaErrorInvalidValue;
-    int sms = 0;
-    cudaError_t e = tp_sm_count(sms);
+    int dev = 0, sms = 0;
+    cudaError_t e = tp_sm_count(dev, sms);
     if (e != cudaSuccess) return e;
     constexpr size_t smem = (size_t)P::S * (P::NIN + 1) * ((size_t)P::NT * P::E + 2 * P::H) * sizeof(T);
-    static int per_sm = 0;  // resident blocks per SM (same on every device of one kind)
-    if (per_sm == 0) {
-        e = cudaFuncSetAttribute(k_tp_ring<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        int per = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, k_tp_ring<P>, P::NT, smem);
-        if (e != cudaSuccess) return e;
-        per_sm = std::max(1, per);
-    }
+    int per_sm = 0;  // resident blocks per SM, cached per device
+    e = blocks_per_sm<k_tp_ring<P>>(dev, P::NT, smem, &per_sm);
+    if (e != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(ntiles, (int64_t)per_sm * sms);
     e = cudaMemsetAsync(W.redo_count, 0, sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;
@@ -669,8 +652,8 @@ cudaError_t tp_run(const P& p, void* ws, size_t ws_bytes, cudaStream_t st) {
     Carve cv(ws, ws_bytes);
     TPWs<T, C> W = tp_carve<T, C>(cv, ntiles);
     if (!cv.ok) return cudaErrorInvalidValue;
-    int sms = 0;
-    cudaError_t e = tp_sm_count(sms);
+    int dev = 0, sms = 0;
+    cudaError_t e = tp_sm_count(dev, sms);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(W.redo_count, 0, sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;

@@ -70,6 +70,7 @@ SIGNATURES = {
                            ctypes.c_int),
     "laplex_matvec_sym_noalloc": ([_P, _P, _I64, _P, _P, _P], ctypes.c_int),
     "laplex_set_profile_events": ([_P, _P], ctypes.c_int),
+    "laplex_test_set_sort_wait": ([ctypes.c_uint32, ctypes.c_int], ctypes.c_int),
 }
 
 
@@ -183,6 +184,12 @@ def set_profile_events(before=None, after=None) -> None:
     events exist); None, None switches it off."""
     h = [None if e is None else ctypes.c_void_p(e.cuda_event) for e in (before, after)]
     _check(lib().laplex_set_profile_events(h[0], h[1]))
+
+
+def test_set_sort_wait(polls: int = 0, force_expiry: bool = False) -> None:
+    """Test hook: bound of the sort's look-back waits on this thread (0: the
+    default) and whether every wait is made to run to that bound."""
+    _check(lib().laplex_test_set_sort_wait(polls, 1 if force_expiry else 0))
 
 
 def device_status(device=None) -> None:
@@ -355,3 +362,59 @@ def matvec_sym_host(sorted_anchors: torch.Tensor, x: torch.Tensor, perm=None, de
         return y_d.cpu()
     out.copy_(y_d, non_blocking=True)
     return out
+
+
+class HostStreamer:
+    """Symmetric products of a stream of host batches (pinned tensors), with the
+    copies overlapped: batch k's host-to-device copy runs on one CUDA stream
+    while batch k-1 is computed on a second and batch k-2's result returns on a
+    third.  Device buffers are double-buffered; events order each buffer's
+    reuse.  Only copies and laplex_matvec_sym calls are enqueued (no host-side
+    arithmetic).
+
+    submit(sorted_h, x_h, y_h, perm_h=None) enqueues one batch and returns at
+    once; y_h is complete after synchronize()."""
+
+    def __init__(self, n: int, B: int = 1, dtype=torch.float32, device="cuda", with_perm=False):
+        self.dev = torch.device(device)
+        self.n, self.B = n, B
+        shape = (n,) if B == 1 else (n, B)
+        self.h2d = torch.cuda.Stream(self.dev)
+        self.comp = torch.cuda.Stream(self.dev)
+        self.d2h = torch.cuda.Stream(self.dev)
+        self.bufs = []
+        for _ in range(2):
+            self.bufs.append({
+                "s": torch.empty(n, dtype=dtype, device=self.dev),
+                "x": torch.empty(shape, dtype=dtype, device=self.dev),
+                "y": torch.empty(shape, dtype=dtype, device=self.dev),
+                "p": torch.empty(n, dtype=torch.int32, device=self.dev) if with_perm else None,
+                "loaded": torch.cuda.Event(), "computed": torch.cuda.Event(),
+                "drained": torch.cuda.Event()})
+        self.k = 0
+
+    def submit(self, sorted_h, x_h, y_h, perm_h=None):
+        b = self.bufs[self.k % 2]
+        with torch.cuda.stream(self.h2d):
+            self.h2d.wait_event(b["computed"])  # s, x, p free once the product that read them is done
+            b["s"].copy_(sorted_h, non_blocking=True)
+            b["x"].copy_(x_h, non_blocking=True)
+            if perm_h is not None:
+                b["p"].copy_(perm_h, non_blocking=True)
+            b["loaded"].record(self.h2d)
+        with torch.cuda.stream(self.comp):
+            self.comp.wait_event(b["loaded"])
+            self.comp.wait_event(b["drained"])  # y free once its last copy back is done
+            matvec_sym(b["s"], b["x"], b["p"] if perm_h is not None else None, out=b["y"])
+            b["computed"].record(self.comp)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(b["computed"])
+            y_h.copy_(b["y"], non_blocking=True)
+            b["drained"].record(self.d2h)
+        self.k += 1
+
+    def synchronize(self):
+        """Wait for every submitted batch; raise if a product recorded a device error."""
+        torch.cuda.synchronize(self.dev)
+        with torch.cuda.stream(self.comp):
+            Workspace.status(self.dev)

@@ -254,6 +254,20 @@ laplex_status laplex_gram_matrix(const void* sa, const int32_t* pa, int64_t n, c
 laplex_status laplex_set_profile_events(void* before, void* after);
 
 /*
+ * Test hook for the bounded waits (no counterpart in the paper).  For the
+ * following laplex_sort_anchors calls on the calling thread: `polls` bounds
+ * every wait of the sort's digit passes for a bulk copy into shared memory
+ * (0 restores the default, 2^20 polls), and a non-zero `force_expiry` leaves
+ * the first copy of every block of a digit pass unissued, so that its wait
+ * runs to the bound.  An expired wait sets LAPLEX_ETIMEOUT in the device
+ * status, and the block lets its other copies land (bounded) and stops; the
+ * outputs are then unspecified, and nothing is written outside them.  It
+ * exists so that tests can check that an expired wait ends with an error
+ * instead of hanging.  Host-only bookkeeping.  Returns LAPLEX_OK.
+ */
+laplex_status laplex_test_set_sort_wait(uint32_t polls, int force_expiry);
+
+/*
  * Allocation-free symmetric product, y = K x (fp32, B = 1).  The paper has no
  * counterpart: this entry point exists for callers that cannot allocate device
  * memory -- code running where cudaMalloc is unavailable or forbidden (inside
@@ -267,7 +281,10 @@ laplex_status laplex_set_profile_events(void* before, void* after);
  * It bounds n to 2^30 (2^18 tiles of 4096 anchors); larger n returns
  * LAPLEX_EINVAL with a message.  The call allocates and frees nothing.
  * The first call on each device looks up the array's device address (with that
- * device current), so make that first call before any stream capture.
+ * device current), so make that first call before any stream capture.  A
+ * device reset (cudaDeviceReset) gives the device a new context; the first
+ * call after it looks the address up again and, likewise, belongs before any
+ * stream capture.
  * Every call shares the one array per device and leaves its last contents
  * there; each call writes every scratch entry before reading it, so nothing
  * needs clearing, but calls that overlap on the GPU (several streams or host

@@ -80,3 +80,21 @@ def test_c5_full_size_properties():
     assert (d >= 0).all()
     tie = d == 0
     assert (np.diff(p)[tie] > 0).all()
+
+
+def test_expired_wait_reports_timeout():
+    """A look-back wait that runs out ends with LAPLEX_ETIMEOUT in the device
+    status instead of hanging: the test hook makes every look-back record count
+    as unwritten and bounds each wait at 16 polls.  The status is cleared once
+    reported, and the next sort (default bound) is exact again."""
+    a = synth.normal(100_000, 0.0, 100.0, seed=5, stream="a")
+    X.test_set_sort_wait(16, True)
+    try:
+        X.sort_anchors(dev(a))
+    finally:
+        X.test_set_sort_wait(0, False)
+    with pytest.raises(X.LaplexError) as e:
+        X.device_status()
+    assert e.value.status == X.ETIMEOUT
+    X.device_status()
+    check_exact(a)
