@@ -335,6 +335,15 @@ def run_ours(args):
                 ms_p = timed(lambda: X.matvec_sym(s2, x_d, p2, out=y_d), rsteps, 1) / rsteps
                 X.device_status(dev)
                 rows["c5_matvec_perm"] = crow(ms_p, 16 * n, hbm)
+                # the plan: inverse permutation once per sort, then products whose
+                # vectors move into and out of sorted order by bucketed scatters
+                inv = torch.empty_like(p2)
+                ms_i = timed(lambda: X.invert_perm(p2, out=inv), rsteps, 1) / rsteps
+                rows["c5_invert_perm"] = crow(ms_i, 8 * n, hbm)
+                ms_q = timed(lambda: X.matvec_sym_planned(s2, p2, inv, x_d, out=y_d), rsteps, 1) / rsteps
+                X.device_status(dev)
+                rows["c5_matvec_planned"] = crow(ms_q, 16 * n, hbm)
+                del inv
         except X.LaplexError as e:
             rows["sort_error"] = str(e)
         del a_d, s2, p2

@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <type_traits>
 
 #include "laplex.h"
 #include "laplex_impl.h"
@@ -94,6 +95,13 @@ size_t body_bytes(laplex_op op, int64_t n, int64_t k, int64_t B, int f64) {
         }
         case LAPLEX_OP_GRAM_MATRIX: return lx::grammat_ws_bytes(n, k, f64);
         case LAPLEX_OP_BACKWARD_PHASED: return std::max(lx::pbwd_ws_bytes(n, f64), lx::pbwd_ws_bytes(k, f64));
+        case LAPLEX_OP_PERMUTE: return lx::permute_ws_bytes(n, f64 ? 8 : 4);
+        case LAPLEX_OP_MATVEC_SYM_PLANNED: {
+            // x and y in sorted order, then the larger of the permutation and the product
+            const size_t es = f64 ? 8 : 4;
+            return 2 * lx::Carve::need((size_t)n, es) +
+                   std::max(lx::permute_ws_bytes(n, (int)es), lx::stream_ws_bytes(n, f64));
+        }
     }
     return 0;
 }
@@ -150,6 +158,40 @@ laplex_status laplex_set_profile_events(void* before, void* after) {
     return ok();
 }
 
+laplex_status laplex_permute(const void* src, const int32_t* idx, int64_t n, laplex_dtype dt, void* dst,
+                             void* ws, size_t ws_bytes, void* stream) {
+    laplex_status st = check_sizes(n, 0, 1);
+    if (st != LAPLEX_OK) return st;
+    if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
+    REQ_PTR(src, n > 0);
+    REQ_PTR(idx, n > 0);
+    REQ_PTR(dst, n > 0);
+    if ((st = check_ws(LAPLEX_OP_PERMUTE, n, 0, 1, dt, ws, ws_bytes)) != LAPLEX_OK) return st;
+    if (n == 0) return ok();
+    const size_t body = ws_bytes - lx::HEADER_BYTES;
+    cudaError_t e = dt == LAPLEX_F32
+                        ? lx::permute_run<int32_t>((const int32_t*)src, idx, n, (int32_t*)dst, ws_body(ws), body,
+                                                   ws_status(ws), (cudaStream_t)stream)
+                        : lx::permute_run<int64_t>((const int64_t*)src, idx, n, (int64_t*)dst, ws_body(ws), body,
+                                                   ws_status(ws), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "laplex_permute");
+    return ok();
+}
+
+laplex_status laplex_invert_perm(const int32_t* perm, int64_t n, int32_t* inv, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    laplex_status st = check_sizes(n, 0, 1);
+    if (st != LAPLEX_OK) return st;
+    REQ_PTR(perm, n > 0);
+    REQ_PTR(inv, n > 0);
+    if ((st = check_ws(LAPLEX_OP_PERMUTE, n, 0, 1, LAPLEX_F32, ws, ws_bytes)) != LAPLEX_OK) return st;
+    if (n == 0) return ok();
+    cudaError_t e = lx::permute_run<int32_t>(nullptr, perm, n, inv, ws_body(ws), ws_bytes - lx::HEADER_BYTES,
+                                             ws_status(ws), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "laplex_invert_perm");
+    return ok();
+}
+
 laplex_status laplex_test_set_sort_wait(uint32_t polls, int force_expiry) {
     lx::set_sort_wait(polls, force_expiry);
     return ok();
@@ -161,7 +203,7 @@ laplex_status laplex_workspace_size(laplex_op op, int64_t n, int64_t k, int64_t 
     laplex_status st = check_sizes(n, k, B);
     if (st != LAPLEX_OK) return st;
     if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
-    REQ(op >= LAPLEX_OP_SORT && op <= LAPLEX_OP_BACKWARD_PHASED, "unknown op %d", (int)op);
+    REQ(op >= LAPLEX_OP_SORT && op <= LAPLEX_OP_MATVEC_SYM_PLANNED, "unknown op %d", (int)op);
     *bytes = lx::HEADER_BYTES + body_bytes(op, n, k, B, dt == LAPLEX_F64);
     return ok();
 }
@@ -260,6 +302,43 @@ laplex_status laplex_matvec_sym(const void* sorted, const int32_t* perm, int64_t
 }
 
 }  // extern "C"
+
+template <typename T>
+static cudaError_t run_sym_planned(const void* sorted, const int32_t* perm, const int32_t* inv, int64_t n,
+                                   const void* x, void* y, void* ws, size_t ws_bytes, cudaStream_t st) {
+    using V = typename std::conditional<sizeof(T) == 8, int64_t, int32_t>::type;
+    lx::Carve cv(ws_body(ws), ws_bytes - lx::HEADER_BYTES);
+    T* xs = cv.take<T>(n);
+    T* ys = cv.take<T>(n);
+    if (!cv.ok) return cudaErrorInvalidValue;
+    void* rest = cv.base + cv.off;
+    const size_t rest_bytes = cv.cap - cv.off;
+    cudaError_t e = lx::permute_run<V>((const V*)x, inv, n, (V*)xs, rest, rest_bytes, ws_status(ws), st);
+    if (e == cudaSuccess)
+        e = lx::stream_run<T>((const T*)sorted, xs, ys, nullptr, n, rest, rest_bytes, ws_status(ws), st);
+    if (e == cudaSuccess) e = lx::permute_run<V>((const V*)ys, perm, n, (V*)y, rest, rest_bytes, ws_status(ws), st);
+    return e;
+}
+
+extern "C" laplex_status laplex_matvec_sym_planned(const void* sorted, const int32_t* perm, const int32_t* inv,
+                                                   int64_t n, const void* x, void* y, laplex_dtype dt, void* ws,
+                                                   size_t ws_bytes, void* stream) {
+    laplex_status st = check_sizes(n, 0, 1);
+    if (st != LAPLEX_OK) return st;
+    if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
+    REQ_PTR(sorted, n > 0);
+    REQ_PTR(perm, n > 0);
+    REQ_PTR(inv, n > 0);
+    REQ_PTR(x, n > 0);
+    REQ_PTR(y, n > 0);
+    if ((st = check_ws(LAPLEX_OP_MATVEC_SYM_PLANNED, n, 0, 1, dt, ws, ws_bytes)) != LAPLEX_OK) return st;
+    if (n == 0) return ok();
+    cudaError_t e = dt == LAPLEX_F32
+                        ? run_sym_planned<float>(sorted, perm, inv, n, x, y, ws, ws_bytes, (cudaStream_t)stream)
+                        : run_sym_planned<double>(sorted, perm, inv, n, x, y, ws, ws_bytes, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "laplex_matvec_sym_planned");
+    return ok();
+}
 
 template <typename T>
 static cudaError_t run_gen(const void* sa, const int32_t* pa, int64_t n, const void* sb,

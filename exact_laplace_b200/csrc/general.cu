@@ -34,20 +34,30 @@ template <typename T> __device__ __forceinline__ void gsincos(T a, T* s, T* c);
 template <> __device__ __forceinline__ void gsincos<float>(float a, float* s, float* c) { sincosf(a, s, c); }
 template <> __device__ __forceinline__ void gsincos<double>(double a, double* s, double* c) { sincos(a, s, c); }
 
-// ia[t] = number of a-points among the first min(t*tile, n+k) merged elements.
+// ia[t] = number of a-points among the first min(t*tile, n+k) merged elements
+// (the merge path of a before b on ties).  One warp per diagonal: each round
+// probes 32 points of the remaining range at once (the test a[i] < b[p-1-i]
+// is true, then false, along it), so a search over 2^20 points takes 4 rounds
+// of dependent loads instead of 20.
 template <typename T>
 __global__ void k_merge_partition(const T* __restrict__ a, int64_t n, const T* __restrict__ b,
                                   int64_t k, int64_t tile, int64_t ntiles, int64_t* __restrict__ ia) {
-    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // uniform per warp
     if (t > ntiles) return;
     const int64_t p = min(t * tile, n + k);
-    int64_t lo = max((int64_t)0, p - k), hi = min(p, n);
+    int64_t lo = max((int64_t)0, p - k), hi = min(p, n);  // the answer is in [lo, hi]
     while (lo < hi) {
-        const int64_t mid = (lo + hi) >> 1;
-        if (a[mid] < b[p - 1 - mid]) lo = mid + 1;
-        else hi = mid;
+        const int64_t span = hi - lo;
+        const int64_t mid = lo + span * lane / 32;
+        const unsigned m = __ballot_sync(FULL, a[mid] < b[p - 1 - mid]);
+        const int c = __popc(m);  // probes 0..c-1 hold the test, c..31 do not
+        const int64_t nlo = c == 0 ? lo : lo + span * (c - 1) / 32 + 1;
+        const int64_t nhi = c == 32 ? hi : lo + span * c / 32;
+        lo = nlo;
+        hi = nhi;
     }
-    ia[t] = lo;
+    if (lane == 0) ia[t] = lo;
 }
 
 // Channel values of b-point j (x_j times the scale; phased: cos psi_j and
@@ -371,7 +381,7 @@ cudaError_t gen_run(GenArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_by
     void* wsbody = cv.base + cv.off;
     const size_t wsb = cv.cap - cv.off;
     {
-        const unsigned blocks = (unsigned)((p.ntiles + 1 + 255) / 256);
+        const unsigned blocks = (unsigned)(((p.ntiles + 1) * 32 + 255) / 256);  // a warp per diagonal
         k_merge_partition<T><<<blocks, 256, 0, st>>>(A.sa, A.n, A.sb, A.k, p.tile, p.ntiles, ia);
     }
     for (int64_t g = 0; g < p.groups; ++g) {

@@ -86,6 +86,14 @@ template <typename T>
 cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws,
                      size_t ws_bytes, uint32_t* status, cudaStream_t st);
 
+// -------------------------------------------------------------- permutation
+// dst[idx[i]] = src[i] for i < n (src NULL: dst[idx[i]] = i); V is a 4- or
+// 8-byte element moved as bits.  Entries of idx outside [0, n) are dropped.
+size_t permute_ws_bytes(int64_t n, int vbytes);
+template <typename V>
+cudaError_t permute_run(const V* src, const int32_t* idx, int64_t n, V* dst, void* ws, size_t ws_bytes,
+                        uint32_t* status, cudaStream_t st);
+
 // -------------------------------------------------------------- general (merged)
 template <typename T>
 struct GenArgs {

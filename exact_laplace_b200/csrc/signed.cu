@@ -590,7 +590,26 @@ __global__ void __launch_bounds__(256) k_double(const T* __restrict__ s, int64_t
     for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < k; r += stride) s2[r] = T(2) * s[r];
 }
 
-// per sorted a-point: Lw, Rw, P (and the inverse of pa)
+// #{b < q} (upper: #{b <= q}) over ascending b[0..k), by one warp: each round
+// probes 32 points of the remaining range at once (4 rounds of dependent loads
+// for k = 2^20, against 20 for a binary search).  lane: this thread's lane.
+template <typename T>
+__device__ __forceinline__ int64_t warp_bound(const T* __restrict__ b, int64_t k, T q, bool upper, int lane) {
+    int64_t lo = 0, hi = k;  // the first index whose element fails the test
+    while (lo < hi) {
+        const int64_t span = hi - lo, mid = lo + span * lane / 32;
+        const T v = b[mid];
+        const unsigned m = __ballot_sync(FULL, upper ? v <= q : v < q);
+        const int c = __popc(m);  // probes 0..c-1 pass, c..31 fail
+        const int64_t nlo = c == 0 ? lo : lo + span * (c - 1) / 32 + 1;
+        const int64_t nhi = c == 32 ? hi : lo + span * c / 32;
+        lo = nlo;
+        hi = nhi;
+    }
+    return lo;
+}
+
+// per sorted a-point (one warp each): Lw, Rw, P (and the inverse of pa)
 template <typename T>
 __global__ void __launch_bounds__(256) k_gram_points(const T* __restrict__ sa, const int32_t* __restrict__ pa,
                                                      int64_t n, const T* __restrict__ sb, int64_t k,
@@ -598,14 +617,17 @@ __global__ void __launch_bounds__(256) k_gram_points(const T* __restrict__ sa, c
                                                      const double* __restrict__ P, T* __restrict__ Lw,
                                                      T* __restrict__ Rw, double* __restrict__ Pa,
                                                      int32_t* __restrict__ inv) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wstride = (int64_t)gridDim.x * (blockDim.x / 32);
+    for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; i < n; i += wstride) {
         const T q = sa[i];
-        const int64_t ub = bound<T>(sb, k, q, true);  // #{b <= a_i}
-        Lw[i] = ub > 0 ? F[ub - 1] * dexp<T>(T(2) * (sb[ub - 1] - q)) : T(0);
-        Rw[i] = ub < k ? G[ub] * dexp<T>(T(2) * (q - sb[ub])) : T(0);
-        Pa[i] = ub > 0 ? P[ub - 1] : 0.0;
-        if (pa) inv[pa[i]] = (int32_t)i;
+        const int64_t ub = warp_bound<T>(sb, k, q, true, lane);  // #{b <= a_i}
+        if (lane == 0) {
+            Lw[i] = ub > 0 ? F[ub - 1] * dexp<T>(T(2) * (sb[ub - 1] - q)) : T(0);
+            Rw[i] = ub < k ? G[ub] * dexp<T>(T(2) * (q - sb[ub])) : T(0);
+            Pa[i] = ub > 0 ? P[ub - 1] : 0.0;
+            if (pa) inv[pa[i]] = (int32_t)i;
+        }
     }
 }
 
@@ -674,7 +696,7 @@ cudaError_t grammat_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, 
         k_psum_scan<<<1, 1024, 0, st>>>(bsum, nb);
         k_psum_apply<T><<<(unsigned)nb, PS_NT, 0, st>>>(D, pb, k, bsum, P);
     }
-    k_gram_points<T><<<(unsigned)std::min<int64_t>(gb, (n + 255) / 256), 256, 0, st>>>(sa, pa, n, sb, k, F, G, P,
+    k_gram_points<T><<<(unsigned)std::max<int64_t>(1, std::min<int64_t>(gb * 8, (n + 7) / 8)), 256, 0, st>>>(sa, pa, n, sb, k, F, G, P,
                                                                                       Lw, Rw, Pa, inv);
     k_gram_fill<T><<<(unsigned)n, 256, 0, st>>>(sa, pa ? inv : nullptr, n, Lw, Rw, Pa, M, ldm);  // a block per row
     return cudaGetLastError();

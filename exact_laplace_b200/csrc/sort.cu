@@ -10,7 +10,7 @@
 // and is stable, so equal anchors keep ascending index order and the output
 // permutation is unique.  A NaN or Inf anchor sets ST_NONFINITE.
 //
-// Every pass is a reduce-then-scan over tiles of 4096 keys (fp32; 2048 fp64),
+// Every pass is a reduce-then-scan over tiles of 6144 keys (fp32; 2048 fp64),
 // three launches without any wait between blocks:
 //   k_count      : per tile, the count of each digit; each block walks a
 //                  contiguous range of tiles and keeps running sums, so it
@@ -18,7 +18,7 @@
 //                  range, and at the end its range's totals
 //   k_count_scan : one block: per digit, the exclusive sums over the ranges,
 //                  plus the digit's start (the exclusive sum over smaller digits)
-//   k_scatter    : persistent blocks, tile t on block t mod G; the tiles'
+//   k_scatter    : persistent blocks, each over a contiguous range of tiles; the tiles'
 //                  keys (and payloads) arrive in a ring of shared-memory stages
 //                  by 1-D bulk copies (TMA), the next ones in flight while one
 //                  is ranked: a stable rank per warp (equal digits found by
@@ -47,15 +47,20 @@
 #ifndef LX_SORT_HI
 #define LX_SORT_HI 3
 #endif
-// keys per thread (fp32) and input stages per block
+// keys per thread (fp32 keys), input stages and resident blocks per SM of
+// k_scatter (24 keys per thread, 2 blocks: measured fastest at n = 2^24 to 2^30)
 #ifndef LX_SORT_KPT
-#define LX_SORT_KPT 16
+#define LX_SORT_KPT 24
 #endif
 #ifndef LX_SORT_S
 #define LX_SORT_S 1
 #endif
 #ifndef LX_SORT_MINB
-#define LX_SORT_MINB 3
+#define LX_SORT_MINB 2
+#endif
+// k_scatter: contiguous tiles per block (1) or round robin (0)
+#ifndef LX_SORT_BLOCKED
+#define LX_SORT_BLOCKED 1
 #endif
 // k_count: one atomic for all lanes sharing lane 0's digit (1) or one per key (0)
 #ifndef LX_COUNT_AGG
@@ -206,9 +211,9 @@ __device__ __forceinline__ uint32_t block_excl_sum(uint32_t v, uint32_t* sm /*NT
 constexpr int COUNT_MAX_BLOCKS = 4096;
 constexpr int COUNT_BLOCKS_PER_SM = 4;
 
-template <typename T>
+template <typename K>
 struct CountArgs {
-    const typename KeyOf<T>::K* keys;  // this pass's keys (pass 0: the anchor bits)
+    const K* keys;                     // this pass's keys (sort pass 0: the anchor bits)
     int64_t n, ntiles, R;              // R: tiles per block
     int shift;
     uint32_t* tile_pre;                // [ntiles][RADIX] counts of the earlier tiles of the range
@@ -219,13 +224,25 @@ struct CountArgs {
 // one key of this warp into the tile histogram; lane 0's digit is counted by
 // one atomic for all lanes that share it (the high digits of real anchors
 // take few values, and same-address shared atomics serialise)
-template <bool FIRST, typename K>
-__device__ __forceinline__ void count_key(K kb, bool valid, int shift, uint32_t* hb, bool& bad) {
-    K k = kb;
-    if constexpr (FIRST) {
-        bad |= valid && non_finite_bits(kb);
-        k = key_of_bits(kb);
-    }
+// key maps of a digit pass's input keys
+enum : int {
+    KM_NONE = 0,
+    KM_ANCHOR = 1,  // anchor bits -> sort key (and a finiteness check)
+    KM_CLAMP = 2,   // index: one outside [0, n) becomes (n - 1) | 2^31 (sorts with the last
+                    // group while its digits below bit 31 are read, and is dropped at the end)
+};
+
+template <int KM, typename K>
+__device__ __forceinline__ K map_key(K kb, int64_t n) {
+    if constexpr (KM == KM_ANCHOR) return key_of_bits(kb);
+    else if constexpr (KM == KM_CLAMP) return (int64_t)kb < n ? kb : (K)((uint64_t)(n - 1) | 0x80000000ull);
+    else return kb;
+}
+
+template <int KM, typename K>
+__device__ __forceinline__ void count_key(K kb, bool valid, int shift, uint32_t* hb, bool& bad, int64_t n) {
+    if constexpr (KM == KM_ANCHOR) bad |= valid && non_finite_bits(kb);
+    const K k = map_key<KM>(kb, n);
     const uint32_t dig = valid ? ((uint32_t)(k >> shift) & (RADIX - 1)) : (uint32_t)RADIX;
 #if LX_COUNT_AGG
     const uint32_t d0 = __shfl_sync(FULL, dig, 0);
@@ -237,10 +254,10 @@ __device__ __forceinline__ void count_key(K kb, bool valid, int shift, uint32_t*
 #endif
 }
 
-template <typename T, bool FIRST>
-__global__ void __launch_bounds__(SORT_NT) k_count(CountArgs<T> A) {
-    using K = typename KeyOf<T>::K;
-    constexpr int NT = SORT_NT, TILE = NT * SortShape<T>::KPT;
+// KM: the map of the input keys (KM_ANCHOR: anchor bits, also checked finite).
+template <typename K, int KPT, int KM>
+__global__ void __launch_bounds__(SORT_NT) k_count(CountArgs<K> A) {
+    constexpr int NT = SORT_NT, TILE = NT * KPT;
     constexpr int KPV = 16 / sizeof(K);          // keys per 16-byte vector
     constexpr int VPT = TILE / KPV / NT;         // vectors per thread per tile
     static_assert(VPT * KPV * NT == TILE, "a tile is whole vectors per thread");
@@ -270,13 +287,13 @@ __global__ void __launch_bounds__(SORT_NT) k_count(CountArgs<T> A) {
             for (int j = 0; j < VPT; ++j) {
                 const K* kv = reinterpret_cast<const K*>(&v[j]);
 #pragma unroll
-                for (int e = 0; e < KPV; ++e) count_key<FIRST>(kv[e], true, A.shift, hb, bad);
+                for (int e = 0; e < KPV; ++e) count_key<KM>(kv[e], true, A.shift, hb, bad, A.n);
             }
         } else {  // the ragged last tile
             for (int j = 0; j < TILE / NT; ++j) {
                 const int64_t idx = t * TILE + j * NT + threadIdx.x;
                 const bool valid = idx < A.n;
-                count_key<FIRST>(valid ? A.keys[idx] : K(0), valid, A.shift, hb, bad);
+                count_key<KM>(valid ? A.keys[idx] : K(0), valid, A.shift, hb, bad, A.n);
             }
         }
         __syncthreads();
@@ -290,39 +307,51 @@ __global__ void __launch_bounds__(SORT_NT) k_count(CountArgs<T> A) {
         }
     }
     A.blk_tot[(int64_t)blockIdx.x * RADIX + d] = run;
-    if (FIRST && bad) set_status(A.status, ST_NONFINITE);
+    if (KM == KM_ANCHOR && bad) set_status(A.status, ST_NONFINITE);
 }
 
 // One block of 1024 threads: blk_pre[b][d] = start of digit d + the count of
-// digit d in the ranges before b.  Thread (d, q) owns digit d and the q-th
-// quarter of the ranges.
+// digit d in the ranges before b.  Thread (g, c) owns the four digits 4g..4g+3
+// (16-byte loads) and the c-th of 16 chunks of the ranges; the ranges' rows
+// are read with 8 loads in flight per thread.
 __global__ void __launch_bounds__(1024) k_count_scan(const uint32_t* __restrict__ blk_tot,
                                                      uint32_t* __restrict__ blk_pre, int G,
                                                      uint32_t* __restrict__ use_match) {
-    __shared__ uint32_t part[4][RADIX];
+    constexpr int CH = 16, U = 8;
+    __shared__ uint4 part[CH][RADIX / 4];
     __shared__ uint32_t base[RADIX];
-    const int d = threadIdx.x & (RADIX - 1), q = threadIdx.x >> 8;
-    const int rq = (G + 3) / 4, r0 = std::min(G, q * rq), r1 = std::min(G, r0 + rq);
-    uint32_t sum = 0;
-    int r = r0;
-    for (; r + 8 <= r1; r += 8) {
-        uint32_t x[8];
+    const int g = threadIdx.x & (RADIX / 4 - 1), c = threadIdx.x >> 6;
+    const int rc = (G + CH - 1) / CH, r0 = std::min(G, c * rc), r1 = std::min(G, r0 + rc);
+    const uint4* tot4 = reinterpret_cast<const uint4*>(blk_tot);
+    uint4* pre4 = reinterpret_cast<uint4*>(blk_pre);
+    uint4 sum = make_uint4(0u, 0u, 0u, 0u);
+    for (int r = r0; r < r1; r += U) {
+        uint4 x[U];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) x[u] = blk_tot[(int64_t)(r + u) * RADIX + d];
+        for (int u = 0; u < U; ++u)
+            x[u] = r + u < r1 ? tot4[(int64_t)(r + u) * (RADIX / 4) + g] : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) sum += x[u];
+        for (int u = 0; u < U; ++u) {
+            sum.x += x[u].x;
+            sum.y += x[u].y;
+            sum.z += x[u].z;
+            sum.w += x[u].w;
+        }
     }
-    for (; r < r1; ++r) sum += blk_tot[(int64_t)r * RADIX + d];
-    part[q][d] = sum;
+    part[c][g] = sum;
     __syncthreads();
     if (threadIdx.x < 32) {  // warp 0: exclusive scan of the 256 digit totals, 8 per lane
         const int lane = threadIdx.x;
+        const uint32_t* pw = reinterpret_cast<const uint32_t*>(&part[0][0]);
         uint32_t tot[8], acc = 0;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int dd = lane * 8 + u;
-            tot[u] = part[0][dd] + part[1][dd] + part[2][dd] + part[3][dd];
-            acc += tot[u];
+            uint32_t t = 0;
+#pragma unroll
+            for (int cc = 0; cc < CH; ++cc) t += pw[cc * RADIX + dd];
+            tot[u] = t;
+            acc += t;
         }
         uint32_t inc = acc;
 #pragma unroll
@@ -351,22 +380,45 @@ __global__ void __launch_bounds__(1024) k_count_scan(const uint32_t* __restrict_
         if (lane == 0) *use_match = ed < MATCH_BELOW_DISTINCT ? 1u : 0u;
     }
     __syncthreads();
-    uint32_t pre = base[d];
-    for (int qq = 0; qq < q; ++qq) pre += part[qq][d];
-    for (r = r0; r < r1; ++r) {
-        const uint32_t x = blk_tot[(int64_t)r * RADIX + d];
-        blk_pre[(int64_t)r * RADIX + d] = pre;
-        pre += x;
+    uint4 pre = make_uint4(base[4 * g], base[4 * g + 1], base[4 * g + 2], base[4 * g + 3]);
+    for (int cc = 0; cc < c; ++cc) {
+        const uint4 p = part[cc][g];
+        pre.x += p.x;
+        pre.y += p.y;
+        pre.z += p.z;
+        pre.w += p.w;
+    }
+    for (int r = r0; r < r1; r += U) {
+        uint4 x[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            x[u] = r + u < r1 ? tot4[(int64_t)(r + u) * (RADIX / 4) + g] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (r + u < r1) pre4[(int64_t)(r + u) * (RADIX / 4) + g] = pre;
+            pre.x += x[u].x;
+            pre.y += x[u].y;
+            pre.z += x[u].z;
+            pre.w += x[u].w;
+        }
     }
 }
 
 // ------------------------------------------------------------------ scatter
-template <typename T>
+// what a k_scatter launch does besides the digit pass
+enum : int {
+    F_KEYMAP = 1,  // the keys are anchor bits: map them to sort keys
+    F_IOTA = 2,    // the payload of key i is its index i (no payload input)
+    F_UNMAP = 4,   // write the keys back as anchor bits
+    F_CLAMP = 8,   // the keys are indices: map them to min(index, n)
+};
+
+template <typename K, typename V>
 struct ScatterArgs {
-    const typename KeyOf<T>::K* ksrc;  // this pass's keys (pass 0: the anchor bits)
-    const int32_t* vsrc;               // and payloads (not read in pass 0)
-    typename KeyOf<T>::K* kdst;        // the next pass's keys (the last pass: anchor bits)
-    int32_t* vdst;                     // and payloads (the last pass: perm)
+    const K* ksrc;                     // this pass's keys (with F_KEYMAP: the anchor bits)
+    const V* vsrc;                     // and payloads (not read with F_IOTA)
+    K* kdst;                           // the keys in digit order (with F_UNMAP: anchor bits)
+    V* vdst;                           // and their payloads
     int64_t n, ntiles, R;              // R: tiles per k_count block
     int shift;
     const uint32_t* tile_pre;
@@ -378,25 +430,25 @@ struct ScatterArgs {
 };
 
 // Dynamic shared memory of one k_scatter block.
-template <typename T, int KPT, int S, bool FIRST>
+template <typename K, typename V, int KPT, int S, int F>
 constexpr size_t scatter_smem() {
-    using K = typename KeyOf<T>::K;
     constexpr size_t TILE = (size_t)SORT_NT * KPT;
-    return S * TILE * sizeof(K) + (FIRST ? 0 : S * TILE * 4) + TILE * (sizeof(K) + 4) +
+    return S * TILE * sizeof(K) + ((F & F_IOTA) ? 0 : S * TILE * sizeof(V)) + TILE * (sizeof(K) + sizeof(V)) +
            (size_t)SORT_NW * RADIX * 4;
 }
 
-template <typename T, int KPT, int S, bool FIRST, bool LAST>
-__global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<T> A) {
-    using K = typename KeyOf<T>::K;
+template <typename K, typename V, int KPT, int S, int F>
+__global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K, V> A) {
+    constexpr bool IOTA = F & F_IOTA, UNMAP = F & F_UNMAP;
+    constexpr int KM = (F & F_KEYMAP) ? KM_ANCHOR : (F & F_CLAMP) ? KM_CLAMP : KM_NONE;
     constexpr int NT = SORT_NT, NW = SORT_NW, TILE = NT * KPT;
     static_assert(32 * KPT * sizeof(K) >= (RADIX + 1) * 4, "a warp's key segment holds its match masks");
     extern __shared__ __align__(128) unsigned char dyn[];
-    K* stage_k = reinterpret_cast<K*>(dyn);                               // [S][TILE] (pass 0: anchor bits)
-    int32_t* stage_v = reinterpret_cast<int32_t*>(stage_k + S * TILE);   // [S][TILE] (not in pass 0)
-    K* out_k = reinterpret_cast<K*>(stage_v + (FIRST ? 0 : S * TILE));    // [TILE] in digit order
-    int32_t* out_v = reinterpret_cast<int32_t*>(out_k + TILE);            // [TILE]
-    uint32_t* wcnt = reinterpret_cast<uint32_t*>(out_v + TILE);           // [NW][RADIX]
+    K* stage_k = reinterpret_cast<K*>(dyn);                    // [S][TILE] (F_KEYMAP: anchor bits)
+    V* stage_v = reinterpret_cast<V*>(stage_k + S * TILE);     // [S][TILE] (not with F_IOTA)
+    K* out_k = reinterpret_cast<K*>(stage_v + (IOTA ? 0 : S * TILE));  // [TILE] in digit order
+    V* out_v = reinterpret_cast<V*>(out_k + TILE);             // [TILE]
+    uint32_t* wcnt = reinterpret_cast<uint32_t*>(out_v + TILE);  // [NW][RADIX]
     __shared__ __align__(8) uint64_t full[S];
     __shared__ int32_t gofs[RADIX];   // output position of staged key q of digit d: gofs[d] + q
     __shared__ uint32_t scan_sm[NW + 1];
@@ -408,17 +460,34 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<T
     const unsigned ltmask = lanemask_lt();
     const int64_t G = gridDim.x;
     const bool use_match = *A.use_match != 0u;
+    // The block's i-th tile (-1 past its share).  Blocked: block b owns the
+    // contiguous tiles [b per, (b + 1) per), so that the tiles in work at one
+    // time are spread over the whole array and so are the runs they write
+    // into each digit's region (round robin would have them all write at one
+    // offset of every region; for digits of equal counts the regions are a
+    // power of two apart, and the concurrent writes then crowd a few DRAM
+    // channels).  Tiles may go in any order: their offsets come precomputed.
+    const int64_t per = (A.ntiles + G - 1) / G;
+    auto tile_of = [&](int64_t i) -> int64_t {
+#if LX_SORT_BLOCKED
+        const int64_t t = (int64_t)blockIdx.x * per + i;
+        return i < per && t < A.ntiles ? t : -1;
+#else
+        const int64_t t = (int64_t)blockIdx.x + i * G;
+        return t < A.ntiles ? t : -1;
+#endif
+    };
 
     // thread 0: tile t into stage st (a bulk copy for a full tile; a plain
     // arrive for the ragged last tile, which is read from global memory)
     auto refill = [&](int st, int64_t t) {
-        if (t >= A.ntiles) return;
+        if (t < 0) return;
         const int64_t tb = t * TILE;
         if (tb + TILE <= A.n) {
-            constexpr uint32_t kb = TILE * sizeof(K), vb = FIRST ? 0u : TILE * 4u;
+            constexpr uint32_t kb = TILE * sizeof(K), vb = IOTA ? 0u : TILE * (uint32_t)sizeof(V);
             mbar_expect_tx(&full[st], kb + vb);
             bulk_g2s(stage_k + st * TILE, A.ksrc + tb, kb, &full[st]);
-            if constexpr (!FIRST) bulk_g2s(stage_v + st * TILE, A.vsrc + tb, vb, &full[st]);
+            if constexpr (!IOTA) bulk_g2s(stage_v + st * TILE, A.vsrc + tb, vb, &full[st]);
         } else {
             mbar_arrive(&full[st]);
         }
@@ -429,14 +498,14 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<T
         for (int st = 0; st < S; ++st) mbar_init(&full[st], 1u);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         for (int st = 0; st < S; ++st)
-            if (!(A.force_expiry && st == 0)) refill(st, blockIdx.x + st * G);
+            if (!(A.force_expiry && st == 0)) refill(st, tile_of(st));
     }
     for (int j = threadIdx.x; j < NW * RADIX; j += NT) wcnt[j] = 0u;
     __syncthreads();
 
     for (int64_t i = 0;; ++i) {
-        const int64_t t = blockIdx.x + i * G;
-        if (t >= A.ntiles) return;  // every copy this block issued has been waited for
+        const int64_t t = tile_of(i);
+        if (t < 0) return;  // every copy this block issued has been waited for
         const int st = (int)(i % S);
         // this tile's output offset of digit d, loaded while its copy lands
         const uint32_t off = A.blk_pre[(t / A.R) * RADIX + d] + A.tile_pre[t * RADIX + d];
@@ -455,7 +524,7 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<T
                 K raw;
                 if constexpr (FT) raw = stage_k[st * TILE + q];
                 else raw = q < cnt ? A.ksrc[tb + q] : K(0);
-                k[e] = FIRST ? key_of_bits(raw) : raw;
+                k[e] = map_key<KM>(raw, A.n);
             }
             // stable rank among the warp's keys of the same digit: rounds in
             // order, lanes in order within a round; one lane of each group adds
@@ -511,8 +580,8 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<T
             for (int e = 0; e < KPT; ++e) {
                 const int q = seg + 32 * e;
                 if (FT || q < cnt) {
-                    int32_t v;
-                    if constexpr (FIRST) v = (int32_t)tb + q;  // n < 2^31
+                    V v;
+                    if constexpr (IOTA) v = (V)((int32_t)tb + q);  // n < 2^31
                     else if constexpr (FT) v = stage_v[st * TILE + q];
                     else v = A.vsrc[tb + q];
                     out_v[rk[e]] = v;
@@ -523,7 +592,7 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<T
             // later runs while this one is written out
             if (threadIdx.x == 0) {
                 fence_proxy_async();
-                refill(st, t + S * G);
+                refill(st, tile_of(i + S));
             }
 #pragma unroll
             for (int ww = 0; ww < NW; ++ww) wcnt[ww * RADIX + d] = 0u;
@@ -533,7 +602,7 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<T
                 if (FT || q < cnt) {
                     const K kk = out_k[q];
                     const int64_t g = (int64_t)gofs[(uint32_t)(kk >> shift) & (RADIX - 1)] + q;
-                    A.kdst[g] = LAST ? key_to_bits(kk) : kk;
+                    A.kdst[g] = UNMAP ? key_to_bits(kk) : kk;
                     A.vdst[g] = out_v[q];
                 }
             }
@@ -547,7 +616,7 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<T
             if (threadIdx.x == 0) {
                 set_status(A.status, ST_TIMEOUT);
                 for (int64_t j = 0; j < S; ++j)
-                    if (t + j * G < A.ntiles)
+                    if (tile_of(i + j) >= 0)
                         (void)mbar_wait_bounded(&full[(i + j) % S], (uint32_t)(((i + j) / S) & 1), A.polls);
             }
             return;
@@ -568,26 +637,81 @@ void set_sort_wait(uint32_t polls, int force_expiry) {
 
 template <typename T> constexpr int sort_tile() { return SORT_NT * SortShape<T>::KPT; }
 
+// Workspace shared by the digit passes over one array: per-tile counts,
+// per-range totals and prefixes, and the pass's ranking choice.
+struct PassWs {
+    uint32_t* tile_pre;
+    uint32_t* blk_tot;
+    uint32_t* blk_pre;
+    uint32_t* mode;
+};
+static size_t pass_ws_bytes(int64_t ntiles) {
+    return Carve::need((size_t)(ntiles * RADIX), 4) + 2 * Carve::need((size_t)COUNT_MAX_BLOCKS * RADIX, 4) +
+           Carve::need(1, 4);
+}
+static PassWs pass_carve(Carve& cv, int64_t ntiles) {
+    PassWs W;
+    W.tile_pre = cv.take<uint32_t>((size_t)(ntiles * RADIX));
+    W.blk_tot = cv.take<uint32_t>((size_t)COUNT_MAX_BLOCKS * RADIX);
+    W.blk_pre = cv.take<uint32_t>((size_t)COUNT_MAX_BLOCKS * RADIX);
+    W.mode = cv.take<uint32_t>(1);
+    return W;
+}
+
+// One stable digit pass, (key >> shift) & 255, of n keys ksrc with payloads
+// vsrc into kdst, vdst: k_count, k_count_scan, k_scatter.
+template <typename K, typename V, int KPT, int S, int F>
+static cudaError_t digit_pass(const K* ksrc, const V* vsrc, K* kdst, V* vdst, int64_t n, int shift,
+                              const PassWs& W, uint32_t* status, int dev, int sms, cudaStream_t st) {
+    const int64_t tile = (int64_t)SORT_NT * KPT;
+    const int64_t ntiles = (n + tile - 1) / tile;
+    // k_count: contiguous ranges of R tiles, every block non-empty
+    const int64_t gmax = std::min<int64_t>((int64_t)COUNT_BLOCKS_PER_SM * sms, COUNT_MAX_BLOCKS);
+    const int64_t R = (ntiles + gmax - 1) / gmax;
+    const int64_t Gc = (ntiles + R - 1) / R;
+    CountArgs<K> C;
+    C.keys = ksrc;
+    C.n = n;
+    C.ntiles = ntiles;
+    C.R = R;
+    C.shift = shift;
+    C.tile_pre = W.tile_pre;
+    C.blk_tot = W.blk_tot;
+    C.status = status;
+    k_count<K, KPT, (F & F_KEYMAP) ? KM_ANCHOR : (F & F_CLAMP) ? KM_CLAMP : KM_NONE><<<(unsigned)Gc, SORT_NT, 0, st>>>(C);
+    k_count_scan<<<1, 1024, 0, st>>>(W.blk_tot, W.blk_pre, (int)Gc, W.mode);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ScatterArgs<K, V> A;
+    A.ksrc = ksrc;
+    A.vsrc = vsrc;
+    A.kdst = kdst;
+    A.vdst = vdst;
+    A.n = n;
+    A.ntiles = ntiles;
+    A.R = R;
+    A.shift = shift;
+    A.tile_pre = W.tile_pre;
+    A.blk_pre = W.blk_pre;
+    A.use_match = W.mode;
+    A.status = status;
+    A.polls = g_sort_polls;
+    A.force_expiry = g_sort_force_expiry;
+    constexpr auto kern = k_scatter<K, V, KPT, S, F>;
+    constexpr size_t smem = scatter_smem<K, V, KPT, S, F>();
+    int per = 0;
+    e = blocks_per_sm<kern>(dev, SORT_NT, smem, &per);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(ntiles, (int64_t)per * sms);
+    kern<<<(unsigned)grid, SORT_NT, smem, st>>>(A);
+    return cudaGetLastError();
+}
+
 size_t sort_ws_bytes(int64_t n, int f64) {
     const int64_t tile = f64 ? sort_tile<double>() : sort_tile<float>();
     const int64_t ntiles = std::max<int64_t>(1, (n + tile - 1) / tile);
     const size_t ks = f64 ? 8 : 4;
-    return Carve::need((size_t)n, ks) + Carve::need((size_t)n, 4) +
-           Carve::need((size_t)(ntiles * RADIX), 4) + 2 * Carve::need((size_t)COUNT_MAX_BLOCKS * RADIX, 4) +
-           Carve::need(1, 4);
-}
-
-template <typename T, bool FIRST, bool LAST>
-static cudaError_t launch_scatter(const ScatterArgs<T>& A, int dev, int sms, cudaStream_t st) {
-    constexpr int KPT = SortShape<T>::KPT, S = SortShape<T>::S;
-    constexpr auto kern = k_scatter<T, KPT, S, FIRST, LAST>;
-    constexpr size_t smem = scatter_smem<T, KPT, S, FIRST>();
-    int per = 0;
-    cudaError_t e = blocks_per_sm<kern>(dev, SORT_NT, smem, &per);
-    if (e != cudaSuccess) return e;
-    const int64_t grid = std::min<int64_t>(A.ntiles, (int64_t)per * sms);
-    kern<<<(unsigned)grid, SORT_NT, smem, st>>>(A);
-    return cudaGetLastError();
+    return Carve::need((size_t)n, ks) + Carve::need((size_t)n, 4) + pass_ws_bytes(ntiles);
 }
 
 template <typename T>
@@ -595,67 +719,183 @@ cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws, 
                      uint32_t* status, cudaStream_t st) {
     using K = typename KeyOf<T>::K;
     if (n == 0) return cudaSuccess;
-    constexpr int P = sizeof(K);
+    constexpr int P = sizeof(K), KPT = SortShape<T>::KPT, S = SortShape<T>::S;
     const int64_t tile = sort_tile<T>();
     const int64_t ntiles = (n + tile - 1) / tile;
     Carve cv(ws, ws_bytes);
     K* kws = cv.take<K>(n);
     int32_t* vws = cv.take<int32_t>(n);
-    uint32_t* tile_pre = cv.take<uint32_t>(ntiles * RADIX);
-    uint32_t* blk_tot = cv.take<uint32_t>((size_t)COUNT_MAX_BLOCKS * RADIX);
-    uint32_t* blk_pre = cv.take<uint32_t>((size_t)COUNT_MAX_BLOCKS * RADIX);
-    uint32_t* mode = cv.take<uint32_t>(1);
+    const PassWs W = pass_carve(cv, ntiles);
     if (!cv.ok) return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t e = current_device_sms(&dev, &sms);
     if (e != cudaSuccess) return e;
-    // k_count: contiguous ranges of R tiles, every block non-empty
-    const int64_t gmax = std::min<int64_t>((int64_t)COUNT_BLOCKS_PER_SM * sms, COUNT_MAX_BLOCKS);
-    const int64_t R = (ntiles + gmax - 1) / gmax;
-    const int64_t Gc = (ntiles + R - 1) / R;
     K* kout = reinterpret_cast<K*>(sorted);
-    CountArgs<T> C;
-    C.n = n;
-    C.ntiles = ntiles;
-    C.R = R;
-    C.tile_pre = tile_pre;
-    C.blk_tot = blk_tot;
-    C.status = status;
-    ScatterArgs<T> A;
-    A.n = n;
-    A.ntiles = ntiles;
-    A.R = R;
-    A.tile_pre = tile_pre;
-    A.blk_pre = blk_pre;
-    A.use_match = mode;
-    A.status = status;
-    A.polls = g_sort_polls;
-    A.force_expiry = g_sort_force_expiry;
-    A.ksrc = reinterpret_cast<const K*>(a);
-    A.vsrc = nullptr;
+    const K* ksrc = reinterpret_cast<const K*>(a);
+    const int32_t* vsrc = nullptr;
     profile_before(st);
     for (int pass = 0; pass < P; ++pass) {
         const bool to_out = ((P - 1 - pass) % 2) == 0;  // the last pass lands in the outputs
-        C.keys = A.ksrc;
-        C.shift = 8 * pass;
-        if (pass == 0) k_count<T, true><<<(unsigned)Gc, SORT_NT, 0, st>>>(C);
-        else k_count<T, false><<<(unsigned)Gc, SORT_NT, 0, st>>>(C);
-        k_count_scan<<<1, 1024, 0, st>>>(blk_tot, blk_pre, (int)Gc, mode);
-        e = cudaGetLastError();
+        K* kdst = to_out ? kout : kws;
+        int32_t* vdst = to_out ? perm : vws;
+        if (pass == 0)
+            e = digit_pass<K, int32_t, KPT, S, F_KEYMAP | F_IOTA>(ksrc, vsrc, kdst, vdst, n, 8 * pass, W, status,
+                                                                  dev, sms, st);
+        else if (pass == P - 1)
+            e = digit_pass<K, int32_t, KPT, S, F_UNMAP>(ksrc, vsrc, kdst, vdst, n, 8 * pass, W, status, dev, sms, st);
+        else
+            e = digit_pass<K, int32_t, KPT, S, 0>(ksrc, vsrc, kdst, vdst, n, 8 * pass, W, status, dev, sms, st);
         if (e != cudaSuccess) return e;
-        A.kdst = to_out ? kout : kws;
-        A.vdst = to_out ? perm : vws;
-        A.shift = 8 * pass;
-        if (pass == 0) e = launch_scatter<T, true, false>(A, dev, sms, st);
-        else if (pass == P - 1) e = launch_scatter<T, false, true>(A, dev, sms, st);
-        else e = launch_scatter<T, false, false>(A, dev, sms, st);
-        if (e != cudaSuccess) return e;
-        A.ksrc = A.kdst;
-        A.vsrc = A.vdst;
+        ksrc = kdst;
+        vsrc = vdst;
     }
     profile_after(st);
     return cudaSuccess;
 }
+
+// ------------------------------------------------------------------ permutation
+// dst[idx[i]] = src[i] (IOTA: dst[idx[i]] = i) for i < n.  Writing 4 or 8
+// bytes at random positions of a large array costs a partial 32-byte sector
+// write each, which the L2 cache does not merge well (measured: 3.3x the
+// bytes written to DRAM, even with the targets grouped into a window of a few
+// MB).  So the elements are first ordered by the group of 2^PERM_GB targets
+// they land in, with stable radix digit passes over the group number
+// (index >> PERM_GB; one pass up to 256 groups, two up to 65536, which covers
+// n <= 2^30 with 4-byte elements), and each block of k_place_group then fills
+// one group's 2^PERM_GB outputs in shared memory and writes them out with
+// whole-sector stores.  Entries of idx outside [0, n) are clamped to n, sort
+// last and are dropped; a position that no entry names is left untouched
+// (a bitmap of the written positions guards the store).
+constexpr int PERM_KPT = 16;
+template <typename V> struct PermGB { static constexpr int v = sizeof(V) == 8 ? 13 : 14; };  // 64 KB of outputs
+
+// group_lo[q] = first position of the ordered keys whose group (index below
+// bit 31, >> gb) is >= q, for q <= ngroups; with ordered == 0 (no digit pass
+// ran: one group) just {0, m}.
+__global__ void __launch_bounds__(256) k_group_bounds(const uint32_t* __restrict__ tk, int64_t m, int gb,
+                                                      int64_t ngroups, int ordered, int64_t* __restrict__ group_lo) {
+    const int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (q > ngroups) return;
+    if (!ordered) {
+        group_lo[q] = q == 0 ? 0 : m;
+        return;
+    }
+    int64_t lo = 0, hi = m;  // first i with group(tk[i]) >= q
+    while (lo < hi) {
+        const int64_t mid = (lo + hi) >> 1;
+        if ((int64_t)((tk[mid] & 0x7FFFFFFFu) >> gb) < q) lo = mid + 1;
+        else hi = mid;
+    }
+    group_lo[q] = lo;
+}
+
+template <typename V, int GB, bool IOTA>
+__global__ void __launch_bounds__(1024) k_place_group(const uint32_t* __restrict__ tk, const V* __restrict__ tv,
+                                                      const int64_t* __restrict__ group_lo, int64_t n,
+                                                      V* __restrict__ dst) {
+    constexpr int GS = 1 << GB;
+    extern __shared__ __align__(16) unsigned char dyn[];
+    V* buf = reinterpret_cast<V*>(dyn);                       // [GS]
+    uint32_t* wrote = reinterpret_cast<uint32_t*>(buf + GS);  // [GS / 32]
+    const int64_t q = blockIdx.x;
+    const int64_t base = q << GB;
+    const int64_t lo = group_lo[q], hi = group_lo[q + 1];
+    for (int j = threadIdx.x; j < GS / 32; j += blockDim.x) wrote[j] = 0u;
+    __syncthreads();
+    for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x) {
+        const uint32_t j = __ldcs(tk + i);
+        if ((int64_t)j < n) {
+            const int p = (int)(j - base);
+            buf[p] = IOTA ? (V)i : __ldcs(tv + i);
+            atomicOr(&wrote[p >> 5], 1u << (p & 31));
+        }
+    }
+    __syncthreads();
+    const int cnt = (int)std::min<int64_t>(GS, n - base);
+    for (int p = threadIdx.x; p < cnt; p += blockDim.x)
+        if ((wrote[p >> 5] >> (p & 31)) & 1u) __stcs(dst + base + p, buf[p]);
+}
+
+template <typename V>
+static int64_t perm_groups(int64_t n) {
+    return ((n + ((int64_t)1 << PermGB<V>::v) - 1) >> PermGB<V>::v);
+}
+
+// digit passes over the group number (of the valid indices 0..n-1)
+template <typename V>
+static int perm_passes(int64_t n) {
+    const int64_t top = (n - 1) >> PermGB<V>::v;  // the largest group number
+    int bits = 0;
+    while (bits < 32 && (top >> bits) > 0) ++bits;
+    return (bits + 7) / 8;
+}
+
+size_t permute_ws_bytes(int64_t n, int vbytes) {
+    const int P = vbytes == 8 ? perm_passes<int64_t>(n) : perm_passes<int32_t>(n);
+    const int64_t ng = vbytes == 8 ? perm_groups<int64_t>(n) : perm_groups<int32_t>(n);
+    const int64_t ntiles = (n + (int64_t)SORT_NT * PERM_KPT - 1) / ((int64_t)SORT_NT * PERM_KPT);
+    const int bufs = P == 0 ? 0 : (P == 1 ? 1 : 2);
+    return bufs * (Carve::need((size_t)n, 4) + Carve::need((size_t)n, (size_t)vbytes)) + pass_ws_bytes(ntiles) +
+           Carve::need((size_t)(ng + 2), 8);
+}
+
+template <typename V>
+cudaError_t permute_run(const V* src, const int32_t* idx, int64_t n, V* dst, void* ws, size_t ws_bytes,
+                        uint32_t* status, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    constexpr int GB = PermGB<V>::v;
+    int dev = 0, sms = 0;
+    cudaError_t e = current_device_sms(&dev, &sms);
+    if (e != cudaSuccess) return e;
+    const bool iota = src == nullptr;
+    const int P = perm_passes<V>(n);
+    const int64_t ng = perm_groups<V>(n);
+    const int64_t ntiles = (n + (int64_t)SORT_NT * PERM_KPT - 1) / ((int64_t)SORT_NT * PERM_KPT);
+    Carve cv(ws, ws_bytes);
+    uint32_t* tk[2] = {nullptr, nullptr};
+    V* tv[2] = {nullptr, nullptr};
+    for (int b = 0; b < (P == 0 ? 0 : (P == 1 ? 1 : 2)); ++b) {
+        tk[b] = cv.take<uint32_t>(n);
+        tv[b] = cv.take<V>(n);
+    }
+    const PassWs W = pass_carve(cv, ntiles);
+    int64_t* group_lo = cv.take<int64_t>(ng + 2);
+    if (!cv.ok) return cudaErrorInvalidValue;
+    const uint32_t* ksrc = reinterpret_cast<const uint32_t*>(idx);
+    const V* vsrc = src;
+    bool vio = iota;  // the payloads are still the indices i, not read from memory
+    for (int p = 0; p < P; ++p) {
+        uint32_t* kd = tk[p & 1];
+        V* vd = tv[p & 1];
+        const int shift = GB + 8 * p;
+        if (p == 0 && vio)
+            e = digit_pass<uint32_t, V, PERM_KPT, 1, F_CLAMP | F_IOTA>(ksrc, nullptr, kd, vd, n, shift, W, status,
+                                                                       dev, sms, st);
+        else if (p == 0)
+            e = digit_pass<uint32_t, V, PERM_KPT, 1, F_CLAMP>(ksrc, vsrc, kd, vd, n, shift, W, status, dev, sms, st);
+        else
+            e = digit_pass<uint32_t, V, PERM_KPT, 1, 0>(ksrc, vsrc, kd, vd, n, shift, W, status, dev, sms, st);
+        if (e != cudaSuccess) return e;
+        ksrc = kd;
+        vsrc = vd;
+        vio = false;
+    }
+    // group boundaries of the ordered keys (with no pass: one group, all of idx)
+    k_group_bounds<<<(unsigned)((ng + 1 + 255) / 256), 256, 0, st>>>(ksrc, n, GB, ng, P > 0 ? 1 : 0, group_lo);
+    constexpr size_t smem = ((size_t)1 << GB) * sizeof(V) + ((size_t)1 << GB) / 8;
+    auto place = [&](auto kern) -> cudaError_t {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (r != cudaSuccess) return r;
+        kern<<<(unsigned)ng, 1024, smem, st>>>(ksrc, vsrc, group_lo, n, dst);
+        return cudaGetLastError();
+    };
+    return vio ? place(k_place_group<V, GB, true>) : place(k_place_group<V, GB, false>);
+}
+
+template cudaError_t permute_run<int32_t>(const int32_t*, const int32_t*, int64_t, int32_t*, void*, size_t,
+                                          uint32_t*, cudaStream_t);
+template cudaError_t permute_run<int64_t>(const int64_t*, const int32_t*, int64_t, int64_t*, void*, size_t,
+                                          uint32_t*, cudaStream_t);
 
 template cudaError_t sort_run<float>(const float*, int64_t, float*, int32_t*, void*, size_t,
                                      uint32_t*, cudaStream_t);

@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_HERE, "liblaplex.so")
 OK, EINVAL, ENONFINITE, EWORKSPACE, ECUDA, ETIMEOUT = range(6)
 F32, F64 = 0, 1
 (OP_SORT, OP_SYM, OP_GENERAL, OP_PHASED, OP_GRAM, OP_BACKWARD, OP_BACKWARD_GENERAL, OP_GRAM_MATRIX,
- OP_BACKWARD_PHASED) = range(9)
+ OP_BACKWARD_PHASED, OP_PERMUTE, OP_SYM_PLANNED) = range(11)
 
 _lib = None
 _lock = threading.Lock()
@@ -71,6 +71,10 @@ SIGNATURES = {
     "laplex_matvec_sym_noalloc": ([_P, _P, _I64, _P, _P, _P], ctypes.c_int),
     "laplex_set_profile_events": ([_P, _P], ctypes.c_int),
     "laplex_test_set_sort_wait": ([ctypes.c_uint32, ctypes.c_int], ctypes.c_int),
+    "laplex_permute": ([_P, _P, _I64, ctypes.c_int, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "laplex_invert_perm": ([_P, _I64, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "laplex_matvec_sym_planned": ([_P, _P, _P, _I64, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P],
+                                  ctypes.c_int),
 }
 
 
@@ -223,6 +227,44 @@ def matvec_sym(sorted_anchors: torch.Tensor, x: torch.Tensor, perm=None, out=Non
     ws, nb = _ws(OP_SYM, n, 0, B, x.dtype, dev)
     _check(lib().laplex_matvec_sym(_ptr(sorted_anchors), _ptr(perm), n, _ptr(x), _ptr(y), B,
                                    _dt(x), _ptr(ws), nb, _stream(dev)))
+    return y
+
+
+def permute(src: torch.Tensor, idx: torch.Tensor, out=None):
+    """dst[idx[i]] = src[i] (4- or 8-byte elements, moved as bits); idx int32."""
+    dev = _dev(src, _perm(idx), out)
+    n = src.numel()
+    if idx.numel() != n or src.element_size() not in (4, 8):
+        raise LaplexError(EINVAL, "src and idx must have n elements; src of 4 or 8 bytes")
+    dst = torch.empty_like(src) if out is None else out
+    dt = F64 if src.element_size() == 8 else F32
+    ws, nb = _ws(OP_PERMUTE, n, 0, 1, torch.float64 if dt == F64 else torch.float32, dev)
+    _check(lib().laplex_permute(_ptr(src), _ptr(idx), n, dt, _ptr(dst), _ptr(ws), nb, _stream(dev)))
+    return dst
+
+
+def invert_perm(perm: torch.Tensor, out=None):
+    """inv with inv[perm[r]] = r (int32)."""
+    dev = _dev(_perm(perm), out)
+    n = perm.numel()
+    inv = torch.empty_like(perm) if out is None else out
+    ws, nb = _ws(OP_PERMUTE, n, 0, 1, torch.float32, dev)
+    _check(lib().laplex_invert_perm(_ptr(perm), n, _ptr(inv), _ptr(ws), nb, _stream(dev)))
+    return inv
+
+
+def matvec_sym_planned(sorted_anchors: torch.Tensor, perm: torch.Tensor, inv: torch.Tensor, x: torch.Tensor,
+                       out=None):
+    """y = K x for x, y in the caller's order (one column), through the plan
+    (sorted, perm, inv): bucketed moves into and out of sorted order."""
+    dev = _dev(sorted_anchors, _perm(perm), _perm(inv), x, out)
+    n = sorted_anchors.numel()
+    if x.numel() != n or x.dtype != sorted_anchors.dtype:
+        raise LaplexError(EINVAL, "x must have n elements and the anchors' dtype")
+    y = torch.empty_like(x) if out is None else out
+    ws, nb = _ws(OP_SYM_PLANNED, n, 0, 1, x.dtype, dev)
+    _check(lib().laplex_matvec_sym_planned(_ptr(sorted_anchors), _ptr(perm), _ptr(inv), n, _ptr(x), _ptr(y),
+                                           _dt(x), _ptr(ws), nb, _stream(dev)))
     return y
 
 

@@ -73,7 +73,9 @@ typedef enum {
     LAPLEX_OP_BACKWARD = 5,
     LAPLEX_OP_BACKWARD_GENERAL = 6,
     LAPLEX_OP_GRAM_MATRIX = 7,
-    LAPLEX_OP_BACKWARD_PHASED = 8
+    LAPLEX_OP_BACKWARD_PHASED = 8,
+    LAPLEX_OP_PERMUTE = 9,           /* laplex_permute and laplex_invert_perm (n elements) */
+    LAPLEX_OP_MATVEC_SYM_PLANNED = 10
 } laplex_op;
 
 /* Library ABI version (major*10000 + minor*100 + patch). */
@@ -120,6 +122,53 @@ laplex_status laplex_get_device_status(void* ws, void* stream);
 laplex_status laplex_sort_anchors(const void* a, int64_t n, laplex_dtype dtype,
                                   void* sorted, int32_t* perm,
                                   void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Permutation by buckets (no counterpart in the paper beyond the sort itself:
+ * the recurrences of summary §2.2 run over the anchors in sorted order, and a
+ * caller whose vectors are in its own order moves them into and out of that
+ * order).  dst[idx[i]] = src[i] for 0 <= i < n.
+ *   src  [n]  elements of 4 bytes (dtype LAPLEX_F32; any 4-byte type, moved
+ *             as bits) or 8 bytes (LAPLEX_F64).
+ *   idx  [n]  int32 destinations, a permutation of 0..n-1; entries outside
+ *             [0, n) are skipped, positions that no entry names keep their
+ *             contents, and for a repeated entry one of its sources is written
+ *             (which one is unspecified).
+ *   dst  [n]  output; must not overlap src or idx.
+ * Writing single elements at random positions of a large array moves a
+ * partial 32-byte sector each; instead, stable radix digit passes over the
+ * group number idx >> 14 (idx >> 13 for 8-byte elements; none for n up to one
+ * group, two up to n = 2^30) order the elements by the group of 64 KiB of
+ * dst they land in, and one block per group fills the group in shared memory
+ * and stores it whole.
+ * Workspace: laplex_workspace_size(LAPLEX_OP_PERMUTE, n, 0, 1, dtype, ...).
+ */
+laplex_status laplex_permute(const void* src, const int32_t* idx, int64_t n, laplex_dtype dtype,
+                             void* dst, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Inverse of a permutation: inv[perm[r]] = r (laplex_permute of the indices
+ * 0..n-1).  With (sorted, perm, inv) a caller holds a plan: vectors in its
+ * own order enter sorted order by laplex_permute(x, inv) and leave it by
+ * laplex_permute(y, perm), both bucketed scatters, instead of the random
+ * gather and scatter of the perm argument of the products.
+ * Workspace: laplex_workspace_size(LAPLEX_OP_PERMUTE, n, 0, 1, LAPLEX_F32, ...).
+ */
+laplex_status laplex_invert_perm(const int32_t* perm, int64_t n, int32_t* inv, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/*
+ * Symmetric product with a plan, y = K x for x, y in the caller's order
+ * (B = 1): x moves into sorted order by laplex_permute(x, inv), the product
+ * runs on the streaming path, and y moves back by laplex_permute(y', perm).
+ * Same result as laplex_matvec_sym(sorted, perm, ...).
+ *   sorted [n], perm [n], inv [n]: from laplex_sort_anchors and laplex_invert_perm.
+ *   x [n], y [n]: caller order.
+ * Workspace: laplex_workspace_size(LAPLEX_OP_MATVEC_SYM_PLANNED, n, 0, 1, dtype, ...).
+ */
+laplex_status laplex_matvec_sym_planned(const void* sorted, const int32_t* perm, const int32_t* inv, int64_t n,
+                                        const void* x, void* y, laplex_dtype dtype, void* ws, size_t ws_bytes,
+                                        void* stream);
 
 /*
  * Symmetric product y = K x, K_ij = exp(-|a_i - a_j|) (summary §2.2, "Caso
