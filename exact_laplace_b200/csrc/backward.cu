@@ -19,6 +19,13 @@
 
 namespace lx {
 
+// elements per thread (fp32: LX_BWD_E32) and resident blocks per SM of the ring pass
+#ifndef LX_BWD_E32
+#define LX_BWD_E32 12
+#endif
+#ifndef LX_BWD_MINB
+#define LX_BWD_MINB 2
+#endif
 constexpr int BWD_NT = 256;
 
 // Policy of threepass.cuh (wait-free: tile-local scans, exact tile carries,
@@ -33,7 +40,7 @@ struct BwdTP {
     // several times more: none).  Streamed pass 1 (inputs in sorted order):
     // s, x, g in a 2-stage ring.
     static constexpr int H = sizeof(T_) == 4 ? 192 : 0;
-    static constexpr int NIN = 2, S = 2, MINB = 3;
+    static constexpr int NIN = 2, S = 2, MINB = LX_BWD_MINB;
     int64_t n;
     const T* s;
     const int32_t* perm;
@@ -83,6 +90,7 @@ struct BwdTP {
         vv[2] = xe[0];
         vv[3] = xe[1];
     }
+    __device__ __forceinline__ void value_chunk(const T (&xe)[NIN], T (&vv)[C], Aux&, int) const { value(xe, vv); }
     __device__ __forceinline__ void finish(int64_t r0, const T (&sv)[E], const T (&v)[E][C],
                                            T (&dl)[E], T eprev, const T (&Lp)[C], T enext,
                                            const T (&Un)[C], Aux&) const {
@@ -148,7 +156,7 @@ struct BwdTP {
     }
 };
 
-static constexpr int bwd_E(int es) { return es == 4 ? 8 : 4; }
+static constexpr int bwd_E(int es) { return es == 4 ? LX_BWD_E32 : 4; }
 
 size_t bwd_ws_bytes(int64_t n, int f64) {
     const int64_t tile = (int64_t)BWD_NT * bwd_E(f64 ? 8 : 4);

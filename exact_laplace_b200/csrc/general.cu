@@ -266,50 +266,87 @@ template <typename T, int NCOL, bool PHASED>
 __global__ void __launch_bounds__(256) k_gen_headtail(GenArgs<T> A, TPWs<T, PHASED ? 2 * NCOL : NCOL> W,
                                                       const int64_t* __restrict__ ia, int64_t tile,
                                                       int64_t ntiles) {
-    constexpr int C = PHASED ? 2 * NCOL : NCOL;
-    const int lane = threadIdx.x & 31;
+    // One block per tile.  Both carries are added in one read-modify-write of
+    // each a-point of the head or tail reach (on dense anchors both reaches
+    // are the whole tile), U = 4 independent a-points per thread and round so
+    // that their loads are in flight together.
+    constexpr int C = PHASED ? 2 * NCOL : NCOL, U = 4;
     const int64_t n = A.n, k = A.k, N = n + k;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < ntiles;
-         t += warps) {
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
         const int64_t p0 = t * tile, p1 = min(p0 + tile, N);
-        const int64_t i0 = ia[t], i1 = ia[t + 1], j0 = p0 - i0, j1 = p1 - i1;
+        const int64_t i0 = ia[t], i1 = ia[t + 1], j0 = p0 - i0, j1 = p1 - i1, na = i1 - i0;
         const TPStats stt = W.st[t];
-        for (int side = 0; side < 2; ++side) {
-            const bool left = side == 0;
-            if (left ? t == 0 : t == ntiles - 1) continue;
-            T c[C];
-            bool nz = false;
+        T cL[C], cR[C];
+        bool nzL = false, nzR = false;
 #pragma unroll
-            for (int q = 0; q < C; ++q) {
-                c[q] = (left ? W.carF : W.carB)[t * C + q];
-                nz |= c[q] != T(0);
+        for (int q = 0; q < C; ++q) {
+            cL[q] = t > 0 ? W.carF[t * C + q] : T(0);
+            cR[q] = t < ntiles - 1 ? W.carB[t * C + q] : T(0);
+            nzL |= cL[q] != T(0);
+            nzR |= cR[q] != T(0);
+        }
+        const int64_t hl = nzL ? min((int64_t)stt.head, na) : 0;   // a-points [0, hl) take the left carry
+        const int64_t tl = nzR ? min((int64_t)stt.tail, na) : 0;   // a-points [na - tl, na) the right one
+        if (hl == 0 && tl == 0) continue;
+        // merged anchors just before and just after the tile
+        T eL = T(0), eR = T(0);
+        if (hl > 0) eL = (i0 > 0 && j0 > 0) ? max(A.sa[i0 - 1], A.sb[j0 - 1]) : (i0 > 0 ? A.sa[i0 - 1] : A.sb[j0 - 1]);
+        if (tl > 0) eR = (i1 < n && j1 < k) ? min(A.sa[i1], A.sb[j1]) : (i1 < n ? A.sa[i1] : A.sb[j1]);
+        // the a-points of the reaches: [0, hl) and [max(hl, na - tl), na)
+        const int64_t gap0 = hl, gap1 = max(hl, na - tl), tot = hl + (na - gap1);
+        for (int64_t q0 = threadIdx.x; q0 < tot; q0 += (int64_t)U * blockDim.x) {
+            int64_t iu[U];
+            T au[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t q = q0 + (int64_t)u * blockDim.x;
+                const int64_t qq = q < gap0 ? q : q - gap0 + gap1;  // skip the middle
+                iu[u] = q < tot ? i0 + qq : -1;
+                au[u] = iu[u] >= 0 ? A.sa[iu[u]] : T(0);
             }
-            if (!nz) continue;
-            T edge;  // merged anchor just before (left) or just after (right) the tile
-            if (left) {
-                if (i0 > 0 && j0 > 0) edge = max(A.sa[i0 - 1], A.sb[j0 - 1]);
-                else edge = i0 > 0 ? A.sa[i0 - 1] : A.sb[j0 - 1];
-            } else {
-                if (i1 < n && j1 < k) edge = min(A.sa[i1], A.sb[j1]);
-                else edge = i1 < n ? A.sa[i1] : A.sb[j1];
+            if constexpr (NCOL == 1 && !PHASED) {
+                // one column: all loads of the round first, then the stores
+                T* yp[U];
+                T yv[U], dv[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    dv[u] = T(0);
+                    yp[u] = nullptr;
+                    if (iu[u] < 0) continue;
+                    const int64_t q = iu[u] - i0;
+                    const T fL = q < hl ? dexp<T>(eL - au[u]) : T(0);
+                    const T fR = q >= na - tl ? dexp<T>(au[u] - eR) : T(0);
+                    if (fL == T(0) && fR == T(0)) continue;
+                    dv[u] = fL * cL[0] + fR * cR[0];
+                    const int64_t row = A.pout ? (int64_t)A.pout[iu[u]] : iu[u];
+                    yp[u] = A.y + row * A.ldy + A.col0;
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) yv[u] = yp[u] ? *yp[u] : T(0);
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (yp[u]) *yp[u] = yv[u] + dv[u];
+                continue;
             }
-            const int64_t len = left ? stt.head : stt.tail;
-            for (int64_t q = lane; q < len; q += 32) {
-                const int64_t i = left ? i0 + q : i1 - 1 - q;
-                const T f = dexp<T>(left ? edge - A.sa[i] : A.sa[i] - edge);
-                if (f == T(0)) continue;
-                const int64_t row = A.pout ? (int64_t)A.pout[i] : i;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (iu[u] < 0) continue;
+                const int64_t q = iu[u] - i0;
+                const T fL = q < hl ? dexp<T>(eL - au[u]) : T(0);
+                const T fR = q >= na - tl ? dexp<T>(au[u] - eR) : T(0);
+                if (fL == T(0) && fR == T(0)) continue;
+                const int64_t row = A.pout ? (int64_t)A.pout[iu[u]] : iu[u];
                 T* yr = A.y + row * A.ldy + A.col0;
                 if (PHASED) {
                     T sp, cp;
-                    gsincos<T>(A.phi[A.pphi ? (int64_t)A.pphi[i] : i], &sp, &cp);
-                    for (int q2 = 0; q2 < A.ncol; ++q2) yr[q2] += f * (cp * c[2 * q2] + sp * c[2 * q2 + 1]);
+                    gsincos<T>(A.phi[A.pphi ? (int64_t)A.pphi[iu[u]] : iu[u]], &sp, &cp);
+                    for (int q2 = 0; q2 < A.ncol; ++q2)
+                        yr[q2] += fL * (cp * cL[2 * q2] + sp * cL[2 * q2 + 1]) +
+                                  fR * (cp * cR[2 * q2] + sp * cR[2 * q2 + 1]);
                 } else {
-                    for (int q2 = 0; q2 < A.ncol; ++q2) yr[q2] += f * c[q2];
+                    for (int q2 = 0; q2 < A.ncol; ++q2) yr[q2] += fL * cL[q2] + fR * cR[q2];
                 }
             }
-            __syncwarp();
         }
     }
 }
@@ -363,7 +400,7 @@ static cudaError_t gen_launch(const GenArgs<T>& A, const GenPlan& p, void* wsbod
     profile_after(st);
     k_tp_carry_blocks<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, p.ntiles);
     k_tp_carry_tiles<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, p.ntiles, nb);
-    const int64_t htb = std::max<int64_t>(1, std::min<int64_t>((p.ntiles + 7) / 8, (int64_t)sms * 8));
+    const int64_t htb = std::max<int64_t>(1, std::min<int64_t>(p.ntiles, (int64_t)sms * 8));
     k_gen_headtail<T, NCOL, PHASED><<<(unsigned)htb, 256, 0, st>>>(A, W, ia, p.tile, p.ntiles);
     return cudaGetLastError();
 }

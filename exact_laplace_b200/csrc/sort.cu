@@ -553,38 +553,58 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
             __syncthreads();
             if (sh_abort) return false;
             // per digit: the tile's count; wcnt[.][d] becomes the warps' offsets
-            // inside the tile's digit-ordered staging
-            uint32_t c = 0;
+            // inside the tile's digit-ordered staging (one read and one write
+            // of each count: the warps' counts stay in registers across the scan)
+            uint32_t xw[NW], c = 0;
 #pragma unroll
             for (int ww = 0; ww < NW; ++ww) {
-                const uint32_t x = wcnt[ww * RADIX + d];
-                wcnt[ww * RADIX + d] = c;
-                c += x;
+                xw[ww] = wcnt[ww * RADIX + d];
+                c += xw[ww];
             }
             uint32_t tot;
             const uint32_t ds = block_excl_sum<NT>(c, scan_sm, tot);
+            {
+                uint32_t pre = ds;
 #pragma unroll
-            for (int ww = 0; ww < NW; ++ww) wcnt[ww * RADIX + d] += ds;
-            gofs[d] = (int32_t)(off - ds);
-            __syncthreads();
-            // stage keys, then payloads, in digit order
-#pragma unroll
-            for (int e = 0; e < KPT; ++e) {
-                const int q = seg + 32 * e;
-                if (FT || q < cnt) {
-                    rk[e] += wcnt[w * RADIX + ((uint32_t)(k[e] >> shift) & (RADIX - 1))];
-                    out_k[rk[e]] = k[e];
+                for (int ww = 0; ww < NW; ++ww) {
+                    wcnt[ww * RADIX + d] = pre;
+                    pre += xw[ww];
                 }
             }
+            gofs[d] = (int32_t)(off - ds);
+            __syncthreads();
+            auto value_of = [&](int q) -> V {
+                if constexpr (IOTA) return (V)((int32_t)tb + q);  // n < 2^31
+                else if constexpr (FT) return stage_v[st * TILE + q];
+                else return A.vsrc[tb + q];
+            };
+            // 4-byte keys and payloads are staged as one 8-byte pair: one
+            // shared store per key, one shared load per key in the write-out
+            constexpr bool PACK = sizeof(K) == 4 && sizeof(V) == 4;
+            uint2* out_kv = reinterpret_cast<uint2*>(out_k);  // out_k and out_v are contiguous
+            if constexpr (PACK) {
 #pragma unroll
-            for (int e = 0; e < KPT; ++e) {
-                const int q = seg + 32 * e;
-                if (FT || q < cnt) {
-                    V v;
-                    if constexpr (IOTA) v = (V)((int32_t)tb + q);  // n < 2^31
-                    else if constexpr (FT) v = stage_v[st * TILE + q];
-                    else v = A.vsrc[tb + q];
-                    out_v[rk[e]] = v;
+                for (int e = 0; e < KPT; ++e) {
+                    const int q = seg + 32 * e;
+                    if (FT || q < cnt) {
+                        rk[e] += wcnt[w * RADIX + ((uint32_t)(k[e] >> shift) & (RADIX - 1))];
+                        out_kv[rk[e]] = make_uint2((uint32_t)k[e], (uint32_t)value_of(q));
+                    }
+                }
+            } else {
+                // stage keys, then payloads, in digit order
+#pragma unroll
+                for (int e = 0; e < KPT; ++e) {
+                    const int q = seg + 32 * e;
+                    if (FT || q < cnt) {
+                        rk[e] += wcnt[w * RADIX + ((uint32_t)(k[e] >> shift) & (RADIX - 1))];
+                        out_k[rk[e]] = k[e];
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < KPT; ++e) {
+                    const int q = seg + 32 * e;
+                    if (FT || q < cnt) out_v[rk[e]] = value_of(q);
                 }
             }
             __syncthreads();
@@ -600,10 +620,19 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
             for (int j = 0; j < KPT; ++j) {
                 const int q = (int)threadIdx.x + j * NT;
                 if (FT || q < cnt) {
-                    const K kk = out_k[q];
+                    K kk;
+                    V vv;
+                    if constexpr (PACK) {
+                        const uint2 kv = out_kv[q];
+                        kk = (K)kv.x;
+                        vv = (V)kv.y;
+                    } else {
+                        kk = out_k[q];
+                        vv = out_v[q];
+                    }
                     const int64_t g = (int64_t)gofs[(uint32_t)(kk >> shift) & (RADIX - 1)] + q;
                     A.kdst[g] = UNMAP ? key_to_bits(kk) : kk;
-                    A.vdst[g] = out_v[q];
+                    A.vdst[g] = vv;
                 }
             }
             __syncthreads();  // out_k, out_v, gofs, wcnt are the next tile's
@@ -665,8 +694,10 @@ static cudaError_t digit_pass(const K* ksrc, const V* vsrc, K* kdst, V* vdst, in
                               const PassWs& W, uint32_t* status, int dev, int sms, cudaStream_t st) {
     const int64_t tile = (int64_t)SORT_NT * KPT;
     const int64_t ntiles = (n + tile - 1) / tile;
-    // k_count: contiguous ranges of R tiles, every block non-empty
-    const int64_t gmax = std::min<int64_t>((int64_t)COUNT_BLOCKS_PER_SM * sms, COUNT_MAX_BLOCKS);
+    // k_count: contiguous ranges of R >= 4 tiles (fewer ranges keep k_count_scan
+    // short on small arrays), every block non-empty
+    const int64_t gmax = std::max<int64_t>(
+        1, std::min<int64_t>(std::min<int64_t>((int64_t)COUNT_BLOCKS_PER_SM * sms, COUNT_MAX_BLOCKS), ntiles / 4));
     const int64_t R = (ntiles + gmax - 1) / gmax;
     const int64_t Gc = (ntiles + R - 1) / R;
     CountArgs<K> C;

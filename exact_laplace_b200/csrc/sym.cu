@@ -257,12 +257,38 @@ struct SymTP {
     // across runs of up to 64 equal anchors); fp64 (CUT = 746) would need
     // several times more: none
     static constexpr int H = sizeof(T_) == 4 ? 192 : 0;
+    // streamed first pass (k_tp_ring: one column in sorted order, no scale):
+    // the value arrays x (and phi), 2 stages, 3 blocks per SM (fp64: 2)
+    static constexpr int NIN = PHASED_ ? 2 : 1, S = 2, MINB = sizeof(T_) == 8 ? 2 : 3;
     SymArgs<T> A;
     int64_t n;
     const T* s;
     struct Aux {
         T cph[E], sph[E];
     };
+    __device__ __forceinline__ const T* ring_in(int a) const { return a == 0 ? A.x : A.phi; }
+    __device__ __forceinline__ void value(const T (&xe)[NIN], T (&vv)[C]) const {
+        if constexpr (PHASED_) {
+            T sp, cp;
+            dsincos<T>(xe[1], &sp, &cp);
+            vv[0] = cp * xe[0];
+            vv[1] = sp * xe[0];
+        } else {
+            vv[0] = xe[0];
+        }
+    }
+    __device__ __forceinline__ void value_chunk(const T (&xe)[NIN], T (&vv)[C], Aux& a, int k) const {
+        if constexpr (PHASED_) {
+            T sp, cp;
+            dsincos<T>(xe[1], &sp, &cp);
+            a.cph[k] = cp;
+            a.sph[k] = sp;
+            vv[0] = cp * xe[0];
+            vv[1] = sp * xe[0];
+        } else {
+            vv[0] = xe[0];
+        }
+    }
     __device__ __forceinline__ void load(int64_t r0, T (&sv)[E], T (&v)[E][C], Aux& a) const {
         sym_load<T, NCOL, PHASED_, E>(A, r0, sv, v, a.cph, a.sph);
     }
@@ -295,6 +321,10 @@ struct SymTP {
 };
 
 // ------------------------------------------------------------------ host side
+// elements per thread of the products with four or more channels
+#ifndef LX_SYM_E_WIDE
+#define LX_SYM_E_WIDE 4
+#endif
 struct SymPlan {
     int ncol;  // template columns per pass
     int C;     // channels per pass
@@ -313,7 +343,7 @@ static SymPlan sym_plan(int64_t n, int64_t B, bool phased, int f64) {
     p.C = phased ? 2 * nc : nc;
     if (p.C == 1) p.E = f64 ? 8 : 16;
     else if (p.C == 2) p.E = 8;
-    else p.E = 4;
+    else p.E = LX_SYM_E_WIDE;
     p.tile = (int64_t)SYM_NT * p.E;
     p.ntiles = (n + p.tile - 1) / p.tile;
     p.groups = (B + nc - 1) / nc;
@@ -351,24 +381,29 @@ cudaError_t sym_run(SymArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_by
         A.ncol = (int)std::min<int64_t>(p.ncol, B - A.col0);
         cudaError_t e;
         constexpr bool D = sizeof(T) == 8;
+        // one column in sorted order without a scale: the streamed (TMA ring) first pass
+        const bool ring = p.ncol == 1 && B == 1 && A.pin == nullptr && A.pout == nullptr && A.paux == nullptr &&
+                          A.D == nullptr && A.ldx == 1 && A.ldy == 1;
         auto run = [&](auto pol) {
             pol.A = A;
             pol.n = A.n;
             pol.s = A.s;
+            if constexpr (decltype(pol)::NCOL == 1)
+                if (ring) return tp_run_ring(pol, ws, ws_bytes, A.status, st);
             return tp_run(pol, ws, ws_bytes, st);
         };
         if (!phased) {
             switch (p.ncol) {
                 case 1: e = run(SymTP<T, 1, false, D ? 8 : 16, SYM_NT>{}); break;
                 case 2: e = run(SymTP<T, 2, false, 8, SYM_NT>{}); break;
-                case 4: e = run(SymTP<T, 4, false, 4, SYM_NT>{}); break;
-                default: e = run(SymTP<T, 8, false, 4, SYM_NT>{}); break;
+                case 4: e = run(SymTP<T, 4, false, LX_SYM_E_WIDE, SYM_NT>{}); break;
+                default: e = run(SymTP<T, 8, false, LX_SYM_E_WIDE, SYM_NT>{}); break;
             }
         } else {
             switch (p.ncol) {
                 case 1: e = run(SymTP<T, 1, true, 8, SYM_NT>{}); break;
-                case 2: e = run(SymTP<T, 2, true, 4, SYM_NT>{}); break;
-                default: e = run(SymTP<T, 4, true, 4, SYM_NT>{}); break;
+                case 2: e = run(SymTP<T, 2, true, LX_SYM_E_WIDE, SYM_NT>{}); break;
+                default: e = run(SymTP<T, 4, true, LX_SYM_E_WIDE, SYM_NT>{}); break;
             }
         }
         if (e != cudaSuccess) return e;

@@ -260,6 +260,8 @@ __global__ void __launch_bounds__(P::NT) k_tp_redo(P p, TPWs<typename P::T, P::C
 //   static constexpr int NIN, S, MINB;         (value arrays, stages, blocks/SM)
 //   __device__ const T* ring_in(int a) const  value array a, sorted order
 //   __device__ void value(const T (&xin)[NIN], T (&v)[C]) const   channels of one element
+//   __device__ void value_chunk(const T (&xin)[NIN], T (&v)[C], Aux& a, int k) const
+//        the same for element k of this thread's chunk, also filling Aux
 template <class P>
 __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P::T, P::C> W,
                                                             int64_t ntiles, uint32_t* status) {
@@ -334,7 +336,7 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
                 T xe[NIN];
 #pragma unroll
                 for (int a = 0; a < NIN; ++a) xe[a] = xin[a][k];
-                p.value(xe, v[k]);
+                p.value_chunk(xe, v[k], aux, k);
             }
         } else {
             p.load(r0, s, v, aux);
