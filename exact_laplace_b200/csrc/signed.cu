@@ -107,15 +107,36 @@ struct OneSidedTP {
 
 static constexpr int os_E(int es) { return es == 4 ? 12 : 6; }
 
-// first index in [0, k) with sp[index] >= q (strict = false) or > q (strict = true)
+// first index in [0, k) with sp[index] >= q (strict = false) or > q (strict =
+// true); k < 2^31, so 32-bit indices, and selects instead of branches
 template <typename T>
 __device__ __forceinline__ int64_t bound(const T* __restrict__ sp, int64_t k, T q, bool strict) {
-    int64_t lo = 0, hi = k;
+    uint32_t lo = 0, len = (uint32_t)k;
+    while (len > 0) {
+        const uint32_t half = len >> 1;
+        const T v = sp[lo + half];
+        const bool go = strict ? v <= q : v < q;
+        lo = go ? lo + half + 1 : lo;
+        len = go ? len - half - 1 : half;
+    }
+    return (int64_t)lo;
+}
+
+// #{b < q} (upper: #{b <= q}) over ascending b[0..k), by one warp: each round
+// probes 32 points of the remaining range at once (4 rounds of dependent loads
+// for k = 2^20, against 20 for a binary search).  lane: this thread's lane.
+template <typename T>
+__device__ __forceinline__ int64_t warp_bound(const T* __restrict__ b, int64_t k, T q, bool upper, int lane) {
+    int64_t lo = 0, hi = k;  // the first index whose element fails the test
     while (lo < hi) {
-        const int64_t mid = (lo + hi) >> 1;
-        const T v = sp[mid];
-        if (strict ? v <= q : v < q) lo = mid + 1;
-        else hi = mid;
+        const int64_t span = hi - lo, mid = lo + span * lane / 32;
+        const T v = b[mid];
+        const unsigned m = __ballot_sync(FULL, upper ? v <= q : v < q);
+        const int c = __popc(m);  // probes 0..c-1 pass, c..31 fail
+        const int64_t nlo = c == 0 ? lo : lo + span * (c - 1) / 32 + 1;
+        const int64_t nhi = c == 32 ? hi : lo + span * c / 32;
+        lo = nlo;
+        hi = nhi;
     }
     return lo;
 }
@@ -131,11 +152,35 @@ __device__ __forceinline__ void chunk_window(const T* __restrict__ sq, const T* 
                                              int64_t r0, int64_t r1, int64_t& lo, int64_t& hi) {
     __shared__ int64_t win[2];
     __syncthreads();  // the previous chunk's threads have read win
-    if (threadIdx.x == 0) win[0] = bound<T>(sp, k, sq[r0], false);
-    if (threadIdx.x == 32) win[1] = bound<T>(sp, k, sq[r1 - 1], true);
+    // warps 0 and 1 each search the whole of sp, 32 probes per round
+    const int wq = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (wq < 2) {
+        const int64_t v = warp_bound<T>(sp, k, sq[wq == 0 ? r0 : r1 - 1], wq == 1, lane);
+        if (lane == 0) win[wq] = v;
+    }
     __syncthreads();
     lo = win[0];
     hi = win[1];
+}
+
+// A window of at most QWIN points of sp is copied to shared memory, and the
+// queries search it there (a few shared loads instead of dependent global ones).
+constexpr int QWIN = 2048;
+
+template <typename T>
+__device__ __forceinline__ void stage_window(const T* __restrict__ sp, int64_t lo, int64_t hi, T* swin) {
+    if (hi - lo <= QWIN)
+        for (int64_t j = threadIdx.x; j < hi - lo; j += blockDim.x) swin[j] = sp[lo + j];
+    __syncthreads();
+}
+
+// lb = #{sp < q}, ub = #{sp <= q} for a query whose bounds lie in [lo, hi]
+template <typename T>
+__device__ __forceinline__ void window_bounds(const T* __restrict__ sp, int64_t lo, int64_t hi, const T* swin, T q,
+                                              int64_t& lb, int64_t& ub) {
+    const T* base = hi - lo <= QWIN ? swin : sp + lo;
+    lb = lo + bound<T>(base, hi - lo, q, false);
+    ub = lo + bound<T>(base, hi - lo, q, true);
 }
 
 // out[row_r] = -w[row_r] S_r for the sorted query anchors sq (rows through pq)
@@ -144,16 +189,18 @@ __global__ void __launch_bounds__(QCH) k_signed_query(const T* __restrict__ sq, 
                                                       int64_t m, const T* __restrict__ sp, int64_t k,
                                                       const T* __restrict__ F, const T* __restrict__ G,
                                                       const T* __restrict__ w, T* __restrict__ out) {
+    __shared__ T swin[QWIN];
     const int64_t nch = (m + QCH - 1) / QCH;
     for (int64_t c = blockIdx.x; c < nch; c += gridDim.x) {
         const int64_t r0 = c * QCH, r1 = min(r0 + QCH, m);
         int64_t lo, hi;
         chunk_window<T>(sq, sp, k, r0, r1, lo, hi);
+        stage_window<T>(sp, lo, hi, swin);
         const int64_t r = r0 + threadIdx.x;
         if (r >= r1) continue;
         const T q = sq[r];
-        const int64_t lb = lo + bound<T>(sp + lo, hi - lo, q, false);
-        const int64_t ub = lo + bound<T>(sp + lo, hi - lo, q, true);
+        int64_t lb, ub;
+        window_bounds<T>(sp, lo, hi, swin, q, lb, ub);
         T S = T(0);
         if (lb > 0) S = F[lb - 1] * dexp<T>(sp[lb - 1] - q);
         if (ub < k) S -= G[ub] * dexp<T>(q - sp[ub]);
@@ -373,11 +420,15 @@ __global__ void __launch_bounds__(QCH) k_phased_query(const T* __restrict__ sq, 
                                                       int64_t k, const T* __restrict__ F,
                                                       const T* __restrict__ G, T* prod, T* dph, T* dan,
                                                       int acc, int self_q) {
+    __shared__ T swin[QWIN];
     const int64_t nch = (m + QCH - 1) / QCH;
     for (int64_t c = blockIdx.x; c < nch; c += gridDim.x) {
         const int64_t r0 = c * QCH, r1 = min(r0 + QCH, m);
         int64_t lo = 0, hi = k;
-        if (!self_q) chunk_window<T>(sq, sp, k, r0, r1, lo, hi);  // self_q: the same for the whole grid
+        if (!self_q) {  // self_q: the same for the whole grid
+            chunk_window<T>(sq, sp, k, r0, r1, lo, hi);
+            stage_window<T>(sp, lo, hi, swin);
+        }
         const int64_t r = r0 + threadIdx.x;
         if (r >= r1) continue;
         const T q = sq[r];
@@ -385,8 +436,7 @@ __global__ void __launch_bounds__(QCH) k_phased_query(const T* __restrict__ sq, 
         if (self_q) {
             tie_run<T>(sp, k, r, lb, ub);
         } else {
-            lb = lo + bound<T>(sp + lo, hi - lo, q, false);
-            ub = lo + bound<T>(sp + lo, hi - lo, q, true);
+            window_bounds<T>(sp, lo, hi, swin, q, lb, ub);
         }
         T P0 = T(0), P1 = T(0), S0 = T(0), S1 = T(0);
         if (ub > 0) {
@@ -588,25 +638,6 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_double(const T* __restrict__ s, int64_t k, T* __restrict__ s2) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < k; r += stride) s2[r] = T(2) * s[r];
-}
-
-// #{b < q} (upper: #{b <= q}) over ascending b[0..k), by one warp: each round
-// probes 32 points of the remaining range at once (4 rounds of dependent loads
-// for k = 2^20, against 20 for a binary search).  lane: this thread's lane.
-template <typename T>
-__device__ __forceinline__ int64_t warp_bound(const T* __restrict__ b, int64_t k, T q, bool upper, int lane) {
-    int64_t lo = 0, hi = k;  // the first index whose element fails the test
-    while (lo < hi) {
-        const int64_t span = hi - lo, mid = lo + span * lane / 32;
-        const T v = b[mid];
-        const unsigned m = __ballot_sync(FULL, upper ? v <= q : v < q);
-        const int c = __popc(m);  // probes 0..c-1 pass, c..31 fail
-        const int64_t nlo = c == 0 ? lo : lo + span * (c - 1) / 32 + 1;
-        const int64_t nhi = c == 32 ? hi : lo + span * c / 32;
-        lo = nlo;
-        hi = nhi;
-    }
-    return lo;
 }
 
 // per sorted a-point (one warp each): Lw, Rw, P (and the inverse of pa)

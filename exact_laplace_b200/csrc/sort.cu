@@ -116,38 +116,81 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 
 // Lanes of the warp holding the same digit (0..255; 256 marks padding, which
 // groups only with padding).  Three ways:
-//  - the warp match instruction, whose cost grows with the number of distinct
-//    digits among the 32 lanes (cheap for the few values of an exponent byte,
-//    slow on uniformly spread digits);
-//  - one ballot per digit bit, a fixed cost;
-//  - match masks in shared memory (wmask: this warp's RADIX + 1 words, zero on
-//    entry): every lane ors its bit into its digit's word and reads the word
-//    back; the group's highest lane clears the word at the next call (*clr,
-//    the previous call's word; RADIX + 1 after a clear).
-// use_match is uniform over the grid.
+//  - RANK_MATCH: the warp match instruction, whose cost grows with the number
+//    of distinct digits among the 32 lanes (cheap for the few values of an
+//    exponent byte, slow on uniformly spread digits);
+//  - RANK_BALLOT: one ballot per digit bit, a fixed cost;
+//  - RANK_MASK: match masks in shared memory (wmask: this warp's RADIX + 1
+//    words, zero on entry): every lane ors its bit into its digit's word and
+//    reads the word back; the group's highest lane clears the word at the next
+//    call (clr: the previous call's word, RADIX + 1 for none).
+// The shared-memory and rank steps are single PTX blocks, so that no branch
+// (and no reconvergence point) surrounds the warp-wide steps.
+enum : int { RANK_MATCH = 0, RANK_BALLOT = 1, RANK_MASK = 3 };
+
 template <bool RAGGED>
-__device__ __forceinline__ unsigned digit_peers(uint32_t dig, bool use_match, uint32_t* wmask,
-                                                uint32_t& clr, int lane) {
-    constexpr int HI = LX_SORT_RANK == 2 ? LX_SORT_HI : LX_SORT_RANK;
-    if (LX_SORT_RANK == 0 || (LX_SORT_RANK == 2 && use_match)) return __match_any_sync(FULL, dig);
-    if constexpr (HI == 3) {
-        if (clr <= RADIX) wmask[clr] = 0u;
-        __syncwarp();
-        atomicOr(&wmask[dig], 1u << lane);
-        __syncwarp();
-        const unsigned peers = wmask[dig];
-        clr = (peers >> lane) == 1u ? dig : RADIX + 1;  // the highest lane of the group clears
-        return peers;
-    } else {
-        unsigned m = FULL;
+__device__ __forceinline__ unsigned ballot_peers(uint32_t dig) {
+    unsigned m = FULL;
 #pragma unroll
-        for (int b = 0; b < (RAGGED ? 9 : 8); ++b) {
-            const bool on = (dig >> b) & 1u;
-            const unsigned bb = __ballot_sync(FULL, on);
-            m &= on ? bb : ~bb;
-        }
-        return m;
+    for (int b = 0; b < (RAGGED ? 9 : 8); ++b) {
+        const bool on = (dig >> b) & 1u;
+        const unsigned bb = __ballot_sync(FULL, on);
+        m &= on ? bb : ~bb;
     }
+    return m;
+}
+
+__device__ __forceinline__ unsigned mask_peers(uint32_t dig, uint32_t* wmask, uint32_t& clr, uint32_t lanebit,
+                                               uint32_t gtmask) {
+    unsigned peers;
+    asm volatile(
+        "{\n"
+        " .reg .b32 a;\n"
+        " .reg .pred pc;\n"
+        " setp.le.u32 pc, %2, 256;\n"
+        " mad.lo.u32 a, %2, 4, %3;\n"
+        " @pc st.shared.u32 [a], 0;\n"
+        " bar.warp.sync 0xffffffff;\n"
+        " mad.lo.u32 a, %1, 4, %3;\n"
+        " red.shared.or.b32 [a], %4;\n"
+        " bar.warp.sync 0xffffffff;\n"
+        " ld.shared.u32 %0, [a];\n"
+        "}\n"
+        : "=r"(peers)
+        : "r"(dig), "r"(clr), "r"(smem_u32(wmask)), "r"(lanebit)
+        : "memory");
+    clr = (peers & gtmask) == 0u ? dig : (uint32_t)(RADIX + 1);
+    return peers;
+}
+
+// Stable rank of this lane's key among the warp's keys of its digit in this
+// and the earlier rounds: the group's highest lane adds the group's size to
+// the warp's counter of the digit and hands the old count to the group.
+__device__ __forceinline__ uint32_t group_rank(unsigned peers, uint32_t dig, bool valid, uint32_t* wcnt_w,
+                                               unsigned ltmask) {
+    uint32_t r;
+    asm volatile(
+        "{\n"
+        " .reg .b32 pc, ltb, lt, old, hi, a, b;\n"
+        " .reg .pred ld;\n"
+        " popc.b32 pc, %1;\n"
+        " and.b32 ltb, %1, %4;\n"
+        " popc.b32 lt, ltb;\n"
+        " add.u32 a, lt, 1;\n"
+        " setp.eq.u32 ld, a, pc;\n"
+        " setp.ne.and.u32 ld, %3, 0, ld;\n"
+        " and.b32 a, %2, 255;\n"
+        " mad.lo.u32 a, a, 4, %5;\n"
+        " mov.b32 old, 0;\n"
+        " @ld atom.shared.add.u32 old, [a], pc;\n"
+        " bfind.u32 hi, %1;\n"
+        " shfl.sync.idx.b32 b, old, hi, 0x1f, 0xffffffff;\n"
+        " add.u32 %0, b, lt;\n"
+        "}\n"
+        : "=r"(r)
+        : "r"(peers), "r"(dig), "r"((uint32_t)valid), "r"(ltmask), "r"(smem_u32(wcnt_w))
+        : "memory");
+    return r;
 }
 
 // The expected number of distinct digits among 32 keys drawn from a pass's
@@ -156,19 +199,7 @@ __device__ __forceinline__ unsigned digit_peers(uint32_t dig, bool use_match, ui
 // ballots 1.4x faster).
 constexpr float MATCH_BELOW_DISTINCT = 12.0f;
 
-// Predicated shared-memory atomics as single instructions (no branch, so no
-// divergence handling around them): the old value (0 where pred is false),
-// and the add without a result.
-__device__ __forceinline__ uint32_t atom_add_shared_if(bool pred, uint32_t* p, uint32_t v) {
-    uint32_t old;
-    asm volatile(
-        "{\n .reg .pred q;\n setp.ne.b32 q, %3, 0;\n mov.b32 %0, 0;\n"
-        " @q atom.shared.add.u32 %0, [%1], %2;\n}\n"
-        : "=&r"(old)
-        : "r"(smem_u32(p)), "r"(v), "r"((uint32_t)pred)
-        : "memory");
-    return old;
-}
+// A predicated shared-memory add without a result, as one instruction.
 __device__ __forceinline__ void red_add_shared_if(bool pred, uint32_t* p, uint32_t v) {
     asm volatile("{\n .reg .pred q;\n setp.ne.b32 q, %2, 0;\n @q red.shared.add.u32 [%0], %1;\n}\n" ::"r"(
                      smem_u32(p)),
@@ -239,16 +270,41 @@ __device__ __forceinline__ K map_key(K kb, int64_t n) {
     else return kb;
 }
 
+// One key per lane into the tile histogram hb (dig = RADIX: no key).  The
+// lanes holding lane 0's digit are counted by one add of lane 0 (the high
+// digits of real anchors take few values, and same-address shared atomics
+// serialise), the others add 1 each.  Written as one PTX block so that no
+// branch, and no reconvergence point, surrounds the warp-wide steps.
+__device__ __forceinline__ void count_digit(uint32_t dig, uint32_t* hb, uint32_t lane0) {
+    asm volatile(
+        "{\n"
+        " .reg .b32 d0, same, cnt, a0, a1;\n"
+        " .reg .pred p, np, q, r;\n"
+        " shfl.sync.idx.b32 d0, %0, 0, 0x1f, 0xffffffff;\n"
+        " setp.eq.u32 p, %0, d0;\n"
+        " vote.sync.ballot.b32 same, p, 0xffffffff;\n"
+        " popc.b32 cnt, same;\n"
+        " setp.lt.u32 q, d0, 256;\n"
+        " setp.ne.and.u32 q, %2, 0, q;\n"
+        " mad.lo.u32 a0, d0, 4, %1;\n"
+        " @q red.shared.add.u32 [a0], cnt;\n"
+        " not.pred np, p;\n"
+        " setp.lt.and.u32 r, %0, 256, np;\n"
+        " mad.lo.u32 a1, %0, 4, %1;\n"
+        " @r red.shared.add.u32 [a1], 1;\n"
+        "}\n" ::"r"(dig),
+        "r"(smem_u32(hb)), "r"(lane0)
+        : "memory");
+}
+
 template <int KM, typename K>
-__device__ __forceinline__ void count_key(K kb, bool valid, int shift, uint32_t* hb, bool& bad, int64_t n) {
-    if constexpr (KM == KM_ANCHOR) bad |= valid && non_finite_bits(kb);
+__device__ __forceinline__ void count_key(K kb, bool valid, int shift, uint32_t* hb, bool& bad, int64_t n,
+                                          uint32_t lane0) {
+    if constexpr (KM == KM_ANCHOR) bad |= valid & non_finite_bits(kb);
     const K k = map_key<KM>(kb, n);
     const uint32_t dig = valid ? ((uint32_t)(k >> shift) & (RADIX - 1)) : (uint32_t)RADIX;
 #if LX_COUNT_AGG
-    const uint32_t d0 = __shfl_sync(FULL, dig, 0);
-    const unsigned same = __ballot_sync(FULL, dig == d0);
-    red_add_shared_if((threadIdx.x & 31) == 0 && d0 < RADIX, &hb[d0 & (RADIX - 1)], (uint32_t)__popc(same));
-    red_add_shared_if(dig != d0 && valid, &hb[dig & (RADIX - 1)], 1u);
+    count_digit(dig, hb, lane0);
 #else
     red_add_shared_if(valid, &hb[dig & (RADIX - 1)], 1u);
 #endif
@@ -263,6 +319,7 @@ __global__ void __launch_bounds__(SORT_NT) k_count(CountArgs<K> A) {
     static_assert(VPT * KPV * NT == TILE, "a tile is whole vectors per thread");
     __shared__ uint32_t h[2][RADIX];  // two tiles' histograms: one barrier per tile
     const int d = threadIdx.x;
+    const uint32_t lane0 = (threadIdx.x & 31) == 0 ? 1u : 0u;
     h[0][d] = 0u;
     h[1][d] = 0u;
     __syncthreads();
@@ -287,13 +344,13 @@ __global__ void __launch_bounds__(SORT_NT) k_count(CountArgs<K> A) {
             for (int j = 0; j < VPT; ++j) {
                 const K* kv = reinterpret_cast<const K*>(&v[j]);
 #pragma unroll
-                for (int e = 0; e < KPV; ++e) count_key<KM>(kv[e], true, A.shift, hb, bad, A.n);
+                for (int e = 0; e < KPV; ++e) count_key<KM>(kv[e], true, A.shift, hb, bad, A.n, lane0);
             }
         } else {  // the ragged last tile
             for (int j = 0; j < TILE / NT; ++j) {
                 const int64_t idx = t * TILE + j * NT + threadIdx.x;
                 const bool valid = idx < A.n;
-                count_key<KM>(valid ? A.keys[idx] : K(0), valid, A.shift, hb, bad, A.n);
+                count_key<KM>(valid ? A.keys[idx] : K(0), valid, A.shift, hb, bad, A.n, lane0);
             }
         }
         __syncthreads();
@@ -442,7 +499,7 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
     constexpr bool IOTA = F & F_IOTA, UNMAP = F & F_UNMAP;
     constexpr int KM = (F & F_KEYMAP) ? KM_ANCHOR : (F & F_CLAMP) ? KM_CLAMP : KM_NONE;
     constexpr int NT = SORT_NT, NW = SORT_NW, TILE = NT * KPT;
-    static_assert(32 * KPT * sizeof(K) >= (RADIX + 1) * 4, "a warp's key segment holds its match masks");
+    static_assert(TILE * (sizeof(K) + sizeof(V)) >= NW * (RADIX + 1) * 4, "the staging area holds the match masks");
     extern __shared__ __align__(128) unsigned char dyn[];
     K* stage_k = reinterpret_cast<K*>(dyn);                    // [S][TILE] (F_KEYMAP: anchor bits)
     V* stage_v = reinterpret_cast<V*>(stage_k + S * TILE);     // [S][TILE] (not with F_IOTA)
@@ -458,6 +515,7 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
     const int d = threadIdx.x;  // the digit of this thread in the per-digit steps
     const int shift = A.shift;
     const unsigned ltmask = lanemask_lt();
+    const uint32_t lanebit = 1u << lane, gtmask = ~(ltmask | lanebit);
     const int64_t G = gridDim.x;
     const bool use_match = *A.use_match != 0u;
     // The block's i-th tile (-1 past its share).  Blocked: block b owns the
@@ -514,8 +572,9 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
         const int64_t tb = t * TILE;
         const int cnt = (int)std::min<int64_t>((int64_t)TILE, A.n - tb);
 
-        auto body = [&](auto full_c) -> bool {
+        auto body = [&](auto full_c, auto rank_c) -> bool {
             constexpr bool FT = decltype(full_c)::value;  // a full tile, staged by the bulk copy
+            constexpr int RM = decltype(rank_c)::value;   // how equal digits are found
             const int seg = w * 32 * KPT + lane;          // key i of this thread: seg + 32 i
             K k[KPT];
 #pragma unroll
@@ -527,29 +586,26 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
                 k[e] = map_key<KM>(raw, A.n);
             }
             // stable rank among the warp's keys of the same digit: rounds in
-            // order, lanes in order within a round; one lane of each group adds
-            // the group to the warp's counter.  The match masks, if used, live
-            // in this warp's own key segment of the stage, read above.
-            uint32_t* wmask = reinterpret_cast<uint32_t*>(stage_k + st * TILE + w * 32 * KPT);
-            __syncwarp();
-            for (int j = lane; j <= RADIX; j += 32) wmask[j] = 0u;
+            // order, lanes in order within a round.  The match masks, if used,
+            // live in the staging area (free until the staging below; only
+            // generic-proxy accesses touch it, so no proxy fence is needed).
+            uint32_t* wmask = reinterpret_cast<uint32_t*>(out_k) + w * (RADIX + 1);
+            if constexpr (RM == RANK_MASK) {
+                __syncwarp();
+                for (int j = lane; j <= RADIX; j += 32) wmask[j] = 0u;
+            }
             uint32_t clr = RADIX + 1;
             uint32_t rk[KPT];
 #pragma unroll
             for (int e = 0; e < KPT; ++e) {
                 const bool valid = FT || seg + 32 * e < cnt;
                 const uint32_t dig = valid ? ((uint32_t)(k[e] >> shift) & (RADIX - 1)) : (uint32_t)RADIX;
-                const unsigned peers = digit_peers<!FT>(dig, use_match, wmask, clr, lane);
-                const uint32_t pc = (uint32_t)__popc(peers);
-                const uint32_t lt = (uint32_t)__popc(peers & ltmask);
-                // the group's highest lane adds the group and hands out the old count
-                const uint32_t base =
-                    atom_add_shared_if(valid && lt + 1u == pc, &wcnt[w * RADIX + (dig & (RADIX - 1))], pc);
-                rk[e] = __shfl_sync(FULL, base, 31 - __clz(peers)) + lt;
+                unsigned peers;
+                if constexpr (RM == RANK_MATCH) peers = __match_any_sync(FULL, dig);
+                else if constexpr (RM == RANK_MASK) peers = mask_peers(dig, wmask, clr, lanebit, gtmask);
+                else peers = ballot_peers<!FT>(dig);
+                rk[e] = group_rank(peers, dig, valid, wcnt + w * RADIX, ltmask);
             }
-            // the masks were written through the generic proxy; the stage is
-            // refilled by a bulk copy (async proxy) after the next barriers
-            fence_proxy_async();
             __syncthreads();
             if (sh_abort) return false;
             // per digit: the tile's count; wcnt[.][d] becomes the warps' offsets
@@ -638,7 +694,12 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
             __syncthreads();  // out_k, out_v, gofs, wcnt are the next tile's
             return true;
         };
-        const bool ok = cnt == TILE ? body(std::true_type{}) : body(std::false_type{});
+        // the ranking of this pass (uniform over the grid), and full or ragged tile
+        using HiRank = std::integral_constant<int, LX_SORT_RANK == 2 ? LX_SORT_HI : LX_SORT_RANK>;
+        using MatchRank = std::integral_constant<int, LX_SORT_RANK == 2 ? RANK_MATCH : LX_SORT_RANK>;
+        bool ok;
+        if (cnt == TILE) ok = use_match ? body(std::true_type{}, MatchRank{}) : body(std::true_type{}, HiRank{});
+        else ok = use_match ? body(std::false_type{}, MatchRank{}) : body(std::false_type{}, HiRank{});
         if (!ok) {
             // a copy never landed: report it, give this block's copies in
             // flight (this one included) a bounded time to land, and leave
