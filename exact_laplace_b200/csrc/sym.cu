@@ -215,6 +215,12 @@ __global__ void __launch_bounds__(NT) k_tile_carries(const T* __restrict__ s, in
     }
 }
 
+}  // namespace lx
+
+#include "cols.cuh"
+
+namespace lx {
+
 template <typename T, int NCOL, bool PHASED, int E, int NT>
 __global__ void __launch_bounds__(NT) k_sym_final(SymArgs<T> A, const T* __restrict__ carF,
                                                   const T* __restrict__ carB) {
@@ -354,7 +360,8 @@ size_t sym_ws_bytes(int64_t n, int64_t B, bool phased, int f64) {
     const SymPlan p = sym_plan(n, B, phased, f64);
     const size_t a = tp_ws_bytes(p.ntiles, p.C, f64 ? 8 : 4);
     const size_t b = (!phased && B == 1) ? stream_ws_bytes(n, f64) : 0;
-    return a > b ? a : b;
+    const size_t c = phased ? 0 : cols_ws_bytes(n, B, f64);
+    return std::max(a, std::max(b, c));
 }
 
 template <typename T, int NCOL, bool PHASED, int E>
@@ -375,6 +382,10 @@ cudaError_t sym_run(SymArgs<T> A, int64_t B, bool phased, void* ws, size_t ws_by
     // single-column input in sorted order, or gathered through perm: the wait-free kernels
     if (!phased && B == 1 && A.pin == A.pout && A.D == nullptr && A.ldx == 1 && A.ldy == 1)
         return stream_run<T>(A.s, A.x, A.y, A.pout, A.n, ws, ws_bytes, A.status, st);
+    // 2, 4 or 8 columns in sorted order without a scale: the column-parallel kernels
+    if (!phased && cols_supported(B) && A.pin == nullptr && A.pout == nullptr && A.D == nullptr && A.ldx == B &&
+        A.ldy == B)
+        return cols_run<T>(A.s, A.n, A.x, A.y, B, ws, ws_bytes, st);
     const SymPlan p = sym_plan(A.n, B, phased, sizeof(T) == 8);
     for (int64_t g = 0; g < p.groups; ++g) {
         A.col0 = g * p.ncol;
