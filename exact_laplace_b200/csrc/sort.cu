@@ -62,9 +62,10 @@
 #ifndef LX_SORT_BLOCKED
 #define LX_SORT_BLOCKED 1
 #endif
-// k_count: one atomic for all lanes sharing lane 0's digit (1) or one per key (0)
+// k_count: one atomic for all lanes sharing lane 0's digit (1) or one per key (0: measured
+// faster on B200, the high exponent digits included)
 #ifndef LX_COUNT_AGG
-#define LX_COUNT_AGG 1
+#define LX_COUNT_AGG 0
 #endif
 
 namespace lx {
