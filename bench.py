@@ -390,10 +390,9 @@ def run_ours(args):
 
     def frow(fn, bytes_per, steps):
         """A row timed both with L2 flushed before every call (ms, frac) and
-        warm (warm_ms, warm_frac); frac = algorithmic bytes / time / HBM peak."""
+        warm (warm_ms); frac = algorithmic bytes / time / HBM peak."""
         r = crow(timed_flush(fn, steps), bytes_per, hbm)
-        w = crow(timed_warm(fn, steps), bytes_per, hbm)
-        r["warm_ms"], r["warm_frac"] = w["ms"], w["frac"]
+        r["warm_ms"] = crow(timed_warm(fn, steps), bytes_per, hbm)["ms"]
         return r
 
     fsteps = max(3, min(20, args.steps // 10))
@@ -502,7 +501,9 @@ def run_ours(args):
                 "config": workload_config(n, world),
                 "roofline": roof, "e2e": e2e, "cpu_baseline": cpu,
                 "clocks": clocks, "gpu_launches": KERNELS_PER_SYM_CALL * args.steps,
-                "rows": rows}  # last, so that a tail of the line keeps them
+                # last, so that a tail of the line keeps them; the n = 2^30 rows at the very end
+                "rows": {**{k: v for k, v in rows.items() if not k.startswith("c5")},
+                         **{k: v for k, v in rows.items() if k.startswith("c5")}}}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
