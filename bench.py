@@ -50,7 +50,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--n", type=int, default=1 << 30)
-    p.add_argument("--rows", default="sort,perm,backward,c2,c3,c4",
+    p.add_argument("--rows", default="sort,perm,carry,backward,c2,c3,c4",
                    help="extra hot-path rows to time (comma list; empty for none)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -344,6 +344,18 @@ def run_ours(args):
                 X.device_status(dev)
                 rows["c5_matvec_planned"] = crow(ms_q, 16 * n, hbm)
                 del inv
+            if "carry" in wanted:
+                # anchors that change every step: the sort carrying x, then the
+                # one-call product (sort carrying x, product, y back to caller order)
+                xs = torch.empty_like(x_d)
+                ms_c = timed(lambda: X.sort_anchors_carry(a_d, x_d, s2, p2, xs), rsteps, 1) / rsteps
+                X.device_status(dev)
+                rows["c5_sort_carry"] = crow(ms_c, 20 * n, hbm)
+                del xs
+                ms_u = timed(lambda: X.matvec_sym_unsorted(a_d, x_d, out=y_d, sorted_out=s2, perm_out=p2),
+                             rsteps, 1) / rsteps
+                X.device_status(dev)
+                rows["c5_matvec_unsorted"] = crow(ms_u, 20 * n, hbm)
         except X.LaplexError as e:
             rows["sort_error"] = str(e)
         del a_d, s2, p2

@@ -61,6 +61,13 @@ laplex_status check_dtype(laplex_dtype dt) {
     return LAPLEX_OK;
 }
 
+// the sort carrying a value: fp32 in the digit passes; fp64 as the sort, then
+// inv (n int32) and the permutation of x by inv
+size_t sort_carry_body(int64_t n, int f64) {
+    if (!f64) return lx::sort_carry_ws_bytes(n);
+    return lx::Carve::need((size_t)n, 4) + std::max(lx::sort_ws_bytes(n, 1), lx::permute_ws_bytes(n, 8));
+}
+
 size_t body_bytes(laplex_op op, int64_t n, int64_t k, int64_t B, int f64) {
     switch (op) {
         case LAPLEX_OP_SORT: return lx::sort_ws_bytes(n, f64);
@@ -96,6 +103,14 @@ size_t body_bytes(laplex_op op, int64_t n, int64_t k, int64_t B, int f64) {
         case LAPLEX_OP_GRAM_MATRIX: return lx::grammat_ws_bytes(n, k, f64);
         case LAPLEX_OP_BACKWARD_PHASED: return std::max(lx::pbwd_ws_bytes(n, f64), lx::pbwd_ws_bytes(k, f64));
         case LAPLEX_OP_PERMUTE: return lx::permute_ws_bytes(n, f64 ? 8 : 4);
+        case LAPLEX_OP_SORT_CARRY: return sort_carry_body(n, f64);
+        case LAPLEX_OP_MATVEC_SYM_UNSORTED: {
+            // xs and y' in sorted order, then the larger of the sort, the product and the permutation
+            const size_t es = f64 ? 8 : 4;
+            return 2 * lx::Carve::need((size_t)n, es) +
+                   std::max(sort_carry_body(n, f64),
+                            std::max(lx::permute_ws_bytes(n, (int)es), lx::stream_ws_bytes(n, f64)));
+        }
         case LAPLEX_OP_MATVEC_SYM_PLANNED: {
             // x and y in sorted order, then the larger of the permutation and the product
             const size_t es = f64 ? 8 : 4;
@@ -203,7 +218,7 @@ laplex_status laplex_workspace_size(laplex_op op, int64_t n, int64_t k, int64_t 
     laplex_status st = check_sizes(n, k, B);
     if (st != LAPLEX_OK) return st;
     if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
-    REQ(op >= LAPLEX_OP_SORT && op <= LAPLEX_OP_MATVEC_SYM_PLANNED, "unknown op %d", (int)op);
+    REQ(op >= LAPLEX_OP_SORT && op <= LAPLEX_OP_MATVEC_SYM_UNSORTED, "unknown op %d", (int)op);
     *bytes = lx::HEADER_BYTES + body_bytes(op, n, k, B, dt == LAPLEX_F64);
     return ok();
 }
@@ -302,6 +317,80 @@ laplex_status laplex_matvec_sym(const void* sorted, const int32_t* perm, int64_t
 }
 
 }  // extern "C"
+
+// xs[r] = x[perm[r]] with the sort (see sort_carry_body for the layout)
+static cudaError_t run_sort_carry(const void* a, const void* x, int64_t n, bool f64, void* sorted, int32_t* perm,
+                                  void* xs, void* body, size_t body_bytes, uint32_t* status, cudaStream_t st) {
+    if (!f64)
+        return lx::sort_carry_run((const float*)a, (const float*)x, n, (float*)sorted, perm, (float*)xs, body,
+                                  body_bytes, status, st);
+    lx::Carve cv(body, body_bytes);
+    int32_t* inv = cv.take<int32_t>(n);
+    if (!cv.ok) return cudaErrorInvalidValue;
+    void* rest = cv.base + cv.off;
+    const size_t rest_bytes = cv.cap - cv.off;
+    cudaError_t e = lx::sort_run<double>((const double*)a, n, (double*)sorted, perm, rest, rest_bytes, status, st);
+    if (e == cudaSuccess) e = lx::permute_run<int32_t>(nullptr, perm, n, inv, rest, rest_bytes, status, st);
+    if (e == cudaSuccess)
+        e = lx::permute_run<int64_t>((const int64_t*)x, inv, n, (int64_t*)xs, rest, rest_bytes, status, st);
+    return e;
+}
+
+extern "C" laplex_status laplex_sort_anchors_carry(const void* a, const void* x, int64_t n, laplex_dtype dt,
+                                                   void* sorted, int32_t* perm, void* xs, void* ws, size_t ws_bytes,
+                                                   void* stream) {
+    laplex_status st = check_sizes(n, 0, 1);
+    if (st != LAPLEX_OK) return st;
+    if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
+    REQ_PTR(a, n > 0);
+    REQ_PTR(x, n > 0);
+    REQ_PTR(sorted, n > 0);
+    REQ_PTR(perm, n > 0);
+    REQ_PTR(xs, n > 0);
+    if ((st = check_ws(LAPLEX_OP_SORT_CARRY, n, 0, 1, dt, ws, ws_bytes)) != LAPLEX_OK) return st;
+    if (n == 0) return ok();
+    cudaError_t e = run_sort_carry(a, x, n, dt == LAPLEX_F64, sorted, perm, xs, ws_body(ws),
+                                   ws_bytes - lx::HEADER_BYTES, ws_status(ws), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "laplex_sort_anchors_carry");
+    return ok();
+}
+
+template <typename T>
+static cudaError_t run_sym_unsorted(const void* a, const void* x, int64_t n, void* y, void* sorted, int32_t* perm,
+                                    void* ws, size_t ws_bytes, cudaStream_t st) {
+    using V = typename std::conditional<sizeof(T) == 8, int64_t, int32_t>::type;
+    lx::Carve cv(ws_body(ws), ws_bytes - lx::HEADER_BYTES);
+    T* xs = cv.take<T>(n);
+    T* ys = cv.take<T>(n);
+    if (!cv.ok) return cudaErrorInvalidValue;
+    void* rest = cv.base + cv.off;
+    const size_t rest_bytes = cv.cap - cv.off;
+    cudaError_t e = run_sort_carry(a, x, n, sizeof(T) == 8, sorted, perm, xs, rest, rest_bytes, ws_status(ws), st);
+    if (e == cudaSuccess)
+        e = lx::stream_run<T>((const T*)sorted, xs, ys, nullptr, n, rest, rest_bytes, ws_status(ws), st);
+    if (e == cudaSuccess) e = lx::permute_run<V>((const V*)ys, perm, n, (V*)y, rest, rest_bytes, ws_status(ws), st);
+    return e;
+}
+
+extern "C" laplex_status laplex_matvec_sym_unsorted(const void* a, const void* x, int64_t n, laplex_dtype dt,
+                                                    void* y, void* sorted, int32_t* perm, void* ws, size_t ws_bytes,
+                                                    void* stream) {
+    laplex_status st = check_sizes(n, 0, 1);
+    if (st != LAPLEX_OK) return st;
+    if ((st = check_dtype(dt)) != LAPLEX_OK) return st;
+    REQ_PTR(a, n > 0);
+    REQ_PTR(x, n > 0);
+    REQ_PTR(y, n > 0);
+    REQ_PTR(sorted, n > 0);
+    REQ_PTR(perm, n > 0);
+    if ((st = check_ws(LAPLEX_OP_MATVEC_SYM_UNSORTED, n, 0, 1, dt, ws, ws_bytes)) != LAPLEX_OK) return st;
+    if (n == 0) return ok();
+    cudaError_t e = dt == LAPLEX_F32
+                        ? run_sym_unsorted<float>(a, x, n, y, sorted, perm, ws, ws_bytes, (cudaStream_t)stream)
+                        : run_sym_unsorted<double>(a, x, n, y, sorted, perm, ws, ws_bytes, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "laplex_matvec_sym_unsorted");
+    return ok();
+}
 
 template <typename T>
 static cudaError_t run_sym_planned(const void* sorted, const int32_t* perm, const int32_t* inv, int64_t n,

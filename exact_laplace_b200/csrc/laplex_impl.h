@@ -86,6 +86,11 @@ template <typename T>
 cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws,
                      size_t ws_bytes, uint32_t* status, cudaStream_t st);
 
+// fp32 sort whose values x ride along: xs[r] = x[perm[r]]
+size_t sort_carry_ws_bytes(int64_t n);
+cudaError_t sort_carry_run(const float* a, const float* x, int64_t n, float* sorted, int32_t* perm, float* xs,
+                           void* ws, size_t ws_bytes, uint32_t* status, cudaStream_t st);
+
 // -------------------------------------------------------------- permutation
 // dst[idx[i]] = src[i] for i < n (src NULL: dst[idx[i]] = i); V is a 4- or
 // 8-byte element moved as bits.  Entries of idx outside [0, n) are dropped.

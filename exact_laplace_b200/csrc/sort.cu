@@ -469,6 +469,7 @@ enum : int {
     F_IOTA = 2,    // the payload of key i is its index i (no payload input)
     F_UNMAP = 4,   // write the keys back as anchor bits
     F_CLAMP = 8,   // the keys are indices: map them to min(index, n)
+    F_PAIR = 16,   // a second 4-byte payload array rides along (v2src -> v2dst)
 };
 
 template <typename K, typename V>
@@ -477,6 +478,8 @@ struct ScatterArgs {
     const V* vsrc;                     // and payloads (not read with F_IOTA)
     K* kdst;                           // the keys in digit order (with F_UNMAP: anchor bits)
     V* vdst;                           // and their payloads
+    const uint32_t* v2src;             // with F_PAIR: the second payload, in and out
+    uint32_t* v2dst;
     int64_t n, ntiles, R;              // R: tiles per k_count block
     int shift;
     const uint32_t* tile_pre;
@@ -490,23 +493,26 @@ struct ScatterArgs {
 // Dynamic shared memory of one k_scatter block.
 template <typename K, typename V, int KPT, int S, int F>
 constexpr size_t scatter_smem() {
-    constexpr size_t TILE = (size_t)SORT_NT * KPT;
-    return S * TILE * sizeof(K) + ((F & F_IOTA) ? 0 : S * TILE * sizeof(V)) + TILE * (sizeof(K) + sizeof(V)) +
-           (size_t)SORT_NW * RADIX * 4;
+    constexpr size_t TILE = (size_t)SORT_NT * KPT, W2 = (F & F_PAIR) ? 4 : 0;
+    return S * TILE * sizeof(K) + ((F & F_IOTA) ? 0 : S * TILE * sizeof(V)) + S * TILE * W2 +
+           TILE * (sizeof(K) + sizeof(V) + W2) + (size_t)SORT_NW * RADIX * 4;
 }
 
 template <typename K, typename V, int KPT, int S, int F>
 __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K, V> A) {
-    constexpr bool IOTA = F & F_IOTA, UNMAP = F & F_UNMAP;
+    constexpr bool IOTA = F & F_IOTA, UNMAP = F & F_UNMAP, PAIR = F & F_PAIR;
     constexpr int KM = (F & F_KEYMAP) ? KM_ANCHOR : (F & F_CLAMP) ? KM_CLAMP : KM_NONE;
     constexpr int NT = SORT_NT, NW = SORT_NW, TILE = NT * KPT;
     static_assert(TILE * (sizeof(K) + sizeof(V)) >= NW * (RADIX + 1) * 4, "the staging area holds the match masks");
+    static_assert(!PAIR || (sizeof(K) == 4 && sizeof(V) == 4), "a second payload rides with 4-byte keys and payloads");
     extern __shared__ __align__(128) unsigned char dyn[];
     K* stage_k = reinterpret_cast<K*>(dyn);                    // [S][TILE] (F_KEYMAP: anchor bits)
     V* stage_v = reinterpret_cast<V*>(stage_k + S * TILE);     // [S][TILE] (not with F_IOTA)
-    K* out_k = reinterpret_cast<K*>(stage_v + (IOTA ? 0 : S * TILE));  // [TILE] in digit order
+    uint32_t* stage_v2 = reinterpret_cast<uint32_t*>(stage_v + (IOTA ? 0 : S * TILE));  // [S][TILE] (F_PAIR)
+    K* out_k = reinterpret_cast<K*>(stage_v2 + (PAIR ? S * TILE : 0));  // [TILE] in digit order
     V* out_v = reinterpret_cast<V*>(out_k + TILE);             // [TILE]
-    uint32_t* wcnt = reinterpret_cast<uint32_t*>(out_v + TILE);  // [NW][RADIX]
+    uint32_t* out_v2 = reinterpret_cast<uint32_t*>(out_v + TILE);  // [TILE] (F_PAIR)
+    uint32_t* wcnt = out_v2 + (PAIR ? TILE : 0);               // [NW][RADIX]
     __shared__ __align__(8) uint64_t full[S];
     __shared__ int32_t gofs[RADIX];   // output position of staged key q of digit d: gofs[d] + q
     __shared__ uint32_t scan_sm[NW + 1];
@@ -543,10 +549,12 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
         if (t < 0) return;
         const int64_t tb = t * TILE;
         if (tb + TILE <= A.n) {
-            constexpr uint32_t kb = TILE * sizeof(K), vb = IOTA ? 0u : TILE * (uint32_t)sizeof(V);
-            mbar_expect_tx(&full[st], kb + vb);
+            constexpr uint32_t kb = TILE * sizeof(K), vb = IOTA ? 0u : TILE * (uint32_t)sizeof(V),
+                               wb = PAIR ? TILE * 4u : 0u;
+            mbar_expect_tx(&full[st], kb + vb + wb);
             bulk_g2s(stage_k + st * TILE, A.ksrc + tb, kb, &full[st]);
             if constexpr (!IOTA) bulk_g2s(stage_v + st * TILE, A.vsrc + tb, vb, &full[st]);
+            if constexpr (PAIR) bulk_g2s(stage_v2 + st * TILE, A.v2src + tb, wb, &full[st]);
         } else {
             mbar_arrive(&full[st]);
         }
@@ -635,6 +643,10 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
                 else if constexpr (FT) return stage_v[st * TILE + q];
                 else return A.vsrc[tb + q];
             };
+            auto value2_of = [&](int q) -> uint32_t {
+                if constexpr (FT) return stage_v2[st * TILE + q];
+                else return A.v2src[tb + q];
+            };
             // 4-byte keys and payloads are staged as one 8-byte pair: one
             // shared store per key, one shared load per key in the write-out
             constexpr bool PACK = sizeof(K) == 4 && sizeof(V) == 4;
@@ -646,6 +658,13 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
                     if (FT || q < cnt) {
                         rk[e] += wcnt[w * RADIX + ((uint32_t)(k[e] >> shift) & (RADIX - 1))];
                         out_kv[rk[e]] = make_uint2((uint32_t)k[e], (uint32_t)value_of(q));
+                    }
+                }
+                if constexpr (PAIR) {
+#pragma unroll
+                    for (int e = 0; e < KPT; ++e) {
+                        const int q = seg + 32 * e;
+                        if (FT || q < cnt) out_v2[rk[e]] = value2_of(q);
                     }
                 }
             } else {
@@ -690,6 +709,7 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
                     const int64_t g = (int64_t)gofs[(uint32_t)(kk >> shift) & (RADIX - 1)] + q;
                     A.kdst[g] = UNMAP ? key_to_bits(kk) : kk;
                     A.vdst[g] = vv;
+                    if constexpr (PAIR) A.v2dst[g] = out_v2[q];
                 }
             }
             __syncthreads();  // out_k, out_v, gofs, wcnt are the next tile's
@@ -753,7 +773,8 @@ static PassWs pass_carve(Carve& cv, int64_t ntiles) {
 // vsrc into kdst, vdst: k_count, k_count_scan, k_scatter.
 template <typename K, typename V, int KPT, int S, int F>
 static cudaError_t digit_pass(const K* ksrc, const V* vsrc, K* kdst, V* vdst, int64_t n, int shift,
-                              const PassWs& W, uint32_t* status, int dev, int sms, cudaStream_t st) {
+                              const PassWs& W, uint32_t* status, int dev, int sms, cudaStream_t st,
+                              const uint32_t* v2src = nullptr, uint32_t* v2dst = nullptr) {
     const int64_t tile = (int64_t)SORT_NT * KPT;
     const int64_t ntiles = (n + tile - 1) / tile;
     // k_count: contiguous ranges of R >= 4 tiles (fewer ranges keep k_count_scan
@@ -780,6 +801,8 @@ static cudaError_t digit_pass(const K* ksrc, const V* vsrc, K* kdst, V* vdst, in
     A.vsrc = vsrc;
     A.kdst = kdst;
     A.vdst = vdst;
+    A.v2src = v2src;
+    A.v2dst = v2dst;
     A.n = n;
     A.ntiles = ntiles;
     A.R = R;
@@ -841,6 +864,61 @@ cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws, 
         if (e != cudaSuccess) return e;
         ksrc = kdst;
         vsrc = vdst;
+    }
+    profile_after(st);
+    return cudaSuccess;
+}
+
+// ------------------------------------------------------------------ sort carrying a value
+// The fp32 sort with a second payload: the value x[i] of each anchor rides
+// through the digit passes beside its index, so that the values arrive in
+// sorted order (xs[r] = x[perm[r]]) with coalesced writes, instead of a random
+// gather after the sort.  16 keys per thread: three staged arrays per tile.
+constexpr int CARRY_KPT = 16;
+
+size_t sort_carry_ws_bytes(int64_t n) {
+    const int64_t tile = (int64_t)SORT_NT * CARRY_KPT;
+    const int64_t ntiles = std::max<int64_t>(1, (n + tile - 1) / tile);
+    return 3 * Carve::need((size_t)n, 4) + pass_ws_bytes(ntiles);
+}
+
+cudaError_t sort_carry_run(const float* a, const float* x, int64_t n, float* sorted, int32_t* perm, float* xs,
+                           void* ws, size_t ws_bytes, uint32_t* status, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    constexpr int P = 4, KPT = CARRY_KPT;
+    const int64_t tile = (int64_t)SORT_NT * KPT;
+    const int64_t ntiles = (n + tile - 1) / tile;
+    Carve cv(ws, ws_bytes);
+    uint32_t* kws = cv.take<uint32_t>(n);
+    int32_t* vws = cv.take<int32_t>(n);
+    uint32_t* wws = cv.take<uint32_t>(n);
+    const PassWs W = pass_carve(cv, ntiles);
+    if (!cv.ok) return cudaErrorInvalidValue;
+    int dev = 0, sms = 0;
+    cudaError_t e = current_device_sms(&dev, &sms);
+    if (e != cudaSuccess) return e;
+    const uint32_t* ksrc = reinterpret_cast<const uint32_t*>(a);
+    const int32_t* vsrc = nullptr;
+    const uint32_t* wsrc = reinterpret_cast<const uint32_t*>(x);
+    profile_before(st);
+    for (int pass = 0; pass < P; ++pass) {
+        const bool to_out = ((P - 1 - pass) % 2) == 0;  // the last pass lands in the outputs
+        uint32_t* kdst = to_out ? reinterpret_cast<uint32_t*>(sorted) : kws;
+        int32_t* vdst = to_out ? perm : vws;
+        uint32_t* wdst = to_out ? reinterpret_cast<uint32_t*>(xs) : wws;
+        if (pass == 0)
+            e = digit_pass<uint32_t, int32_t, KPT, 1, F_KEYMAP | F_IOTA | F_PAIR>(ksrc, vsrc, kdst, vdst, n, 0, W,
+                                                                                  status, dev, sms, st, wsrc, wdst);
+        else if (pass == P - 1)
+            e = digit_pass<uint32_t, int32_t, KPT, 1, F_UNMAP | F_PAIR>(ksrc, vsrc, kdst, vdst, n, 8 * pass, W,
+                                                                        status, dev, sms, st, wsrc, wdst);
+        else
+            e = digit_pass<uint32_t, int32_t, KPT, 1, F_PAIR>(ksrc, vsrc, kdst, vdst, n, 8 * pass, W, status, dev,
+                                                              sms, st, wsrc, wdst);
+        if (e != cudaSuccess) return e;
+        ksrc = kdst;
+        vsrc = vdst;
+        wsrc = wdst;
     }
     profile_after(st);
     return cudaSuccess;

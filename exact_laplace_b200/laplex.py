@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_HERE, "liblaplex.so")
 OK, EINVAL, ENONFINITE, EWORKSPACE, ECUDA, ETIMEOUT = range(6)
 F32, F64 = 0, 1
 (OP_SORT, OP_SYM, OP_GENERAL, OP_PHASED, OP_GRAM, OP_BACKWARD, OP_BACKWARD_GENERAL, OP_GRAM_MATRIX,
- OP_BACKWARD_PHASED, OP_PERMUTE, OP_SYM_PLANNED) = range(11)
+ OP_BACKWARD_PHASED, OP_PERMUTE, OP_SYM_PLANNED, OP_SORT_CARRY, OP_SYM_UNSORTED) = range(13)
 
 _lib = None
 _lock = threading.Lock()
@@ -75,6 +75,10 @@ SIGNATURES = {
     "laplex_invert_perm": ([_P, _I64, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "laplex_matvec_sym_planned": ([_P, _P, _P, _I64, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P],
                                   ctypes.c_int),
+    "laplex_sort_anchors_carry": ([_P, _P, _I64, ctypes.c_int, _P, _P, _P, _P, ctypes.c_size_t, _P],
+                                  ctypes.c_int),
+    "laplex_matvec_sym_unsorted": ([_P, _P, _I64, ctypes.c_int, _P, _P, _P, _P, ctypes.c_size_t, _P],
+                                   ctypes.c_int),
 }
 
 
@@ -213,6 +217,38 @@ def sort_anchors(a: torch.Tensor, sorted_out=None, perm_out=None):
     _check(lib().laplex_sort_anchors(_ptr(a), n, _dt(a), _ptr(s), _ptr(p), _ptr(ws), nb,
                                      _stream(dev)))
     return s, p
+
+
+def sort_anchors_carry(a: torch.Tensor, x: torch.Tensor, sorted_out=None, perm_out=None, xs_out=None):
+    """(sorted, perm, xs): the sort of laplex_sort_anchors with x carried along,
+    xs[r] = x[perm[r]]."""
+    dev = _dev(a, x, sorted_out, perm_out, xs_out)
+    n = a.numel()
+    if x.numel() != n or x.dtype != a.dtype:
+        raise LaplexError(EINVAL, "x must have n elements and the anchors' dtype")
+    s = torch.empty_like(a) if sorted_out is None else sorted_out
+    p = torch.empty(n, dtype=torch.int32, device=dev) if perm_out is None else perm_out
+    xs = torch.empty_like(x) if xs_out is None else xs_out
+    ws, nb = _ws(OP_SORT_CARRY, n, 0, 1, a.dtype, dev)
+    _check(lib().laplex_sort_anchors_carry(_ptr(a), _ptr(x), n, _dt(a), _ptr(s), _ptr(p), _ptr(xs), _ptr(ws), nb,
+                                           _stream(dev)))
+    return s, p, xs
+
+
+def matvec_sym_unsorted(a: torch.Tensor, x: torch.Tensor, out=None, sorted_out=None, perm_out=None):
+    """(y, sorted, perm): y = K x on anchors and x in the caller's order (one
+    column), in one call: the sort carrying x, the product, y back to caller order."""
+    dev = _dev(a, x, out, sorted_out, perm_out)
+    n = a.numel()
+    if x.numel() != n or x.dtype != a.dtype:
+        raise LaplexError(EINVAL, "x must have n elements and the anchors' dtype")
+    y = torch.empty_like(x) if out is None else out
+    s = torch.empty_like(a) if sorted_out is None else sorted_out
+    p = torch.empty(n, dtype=torch.int32, device=dev) if perm_out is None else perm_out
+    ws, nb = _ws(OP_SYM_UNSORTED, n, 0, 1, a.dtype, dev)
+    _check(lib().laplex_matvec_sym_unsorted(_ptr(a), _ptr(x), n, _dt(a), _ptr(y), _ptr(s), _ptr(p), _ptr(ws), nb,
+                                            _stream(dev)))
+    return y, s, p
 
 
 def matvec_sym(sorted_anchors: torch.Tensor, x: torch.Tensor, perm=None, out=None):

@@ -75,7 +75,9 @@ typedef enum {
     LAPLEX_OP_GRAM_MATRIX = 7,
     LAPLEX_OP_BACKWARD_PHASED = 8,
     LAPLEX_OP_PERMUTE = 9,           /* laplex_permute and laplex_invert_perm (n elements) */
-    LAPLEX_OP_MATVEC_SYM_PLANNED = 10
+    LAPLEX_OP_MATVEC_SYM_PLANNED = 10,
+    LAPLEX_OP_SORT_CARRY = 11,       /* laplex_sort_anchors_carry (n anchors and values) */
+    LAPLEX_OP_MATVEC_SYM_UNSORTED = 12
 } laplex_op;
 
 /* Library ABI version (major*10000 + minor*100 + patch). */
@@ -122,6 +124,36 @@ laplex_status laplex_get_device_status(void* ws, void* stream);
 laplex_status laplex_sort_anchors(const void* a, int64_t n, laplex_dtype dtype,
                                   void* sorted, int32_t* perm,
                                   void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Sort the anchors and carry a value per anchor along (summary §2.2: the
+ * recurrences run over the anchors in sorted order, and so over the entries of
+ * the vector they weigh).  As laplex_sort_anchors, and
+ *   x  [n]  in: one value per anchor, caller order (dtype).
+ *   xs [n]  out: xs[r] == x[perm[r]], bit for bit.
+ * fp32: the value rides through the digit passes beside the index payload, so
+ * it reaches sorted order with coalesced writes (no random gather).  fp64: the
+ * sort, then xs by laplex_invert_perm and laplex_permute inside the call.
+ * sorted, perm, xs must not overlap a, x or each other.
+ * Workspace: laplex_workspace_size(LAPLEX_OP_SORT_CARRY, n, 0, 1, dtype, ...).
+ */
+laplex_status laplex_sort_anchors_carry(const void* a, const void* x, int64_t n, laplex_dtype dtype,
+                                        void* sorted, int32_t* perm, void* xs,
+                                        void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Symmetric product y = K x on anchors in the caller's order, in one call
+ * (B = 1; summary §2.2: sort, then the two recurrences): the sort carrying x
+ * (laplex_sort_anchors_carry), the streaming product in sorted order, and y
+ * back to caller order by laplex_permute(y', perm).
+ *   a [n], x [n]: caller order.    y [n]: out, caller order.
+ *   sorted [n], perm [n]: out, as laplex_sort_anchors writes them (for the
+ *   backward pass or later products).
+ * Same result as laplex_sort_anchors followed by laplex_matvec_sym(sorted, perm, ...).
+ * Workspace: laplex_workspace_size(LAPLEX_OP_MATVEC_SYM_UNSORTED, n, 0, 1, dtype, ...).
+ */
+laplex_status laplex_matvec_sym_unsorted(const void* a, const void* x, int64_t n, laplex_dtype dtype, void* y,
+                                         void* sorted, int32_t* perm, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Permutation by buckets (no counterpart in the paper beyond the sort itself:

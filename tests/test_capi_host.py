@@ -46,7 +46,7 @@ def test_version_and_status_strings(L):
 
 def test_workspace_size_host_only(L):
     from exact_laplace_b200 import laplex as X
-    for op in range(11):
+    for op in range(13):
         for n in (0, 1, 4096, 1 << 24):
             assert X.workspace_size(op, n, 1000 if op in (2, 3, 4, 6, 7, 8) else 0, 1) >= 256
     with pytest.raises(X.LaplexError) as e:
@@ -57,7 +57,7 @@ def test_workspace_size_host_only(L):
     with pytest.raises(X.LaplexError):
         X.workspace_size(1, 10, 0, 0)
     with pytest.raises(X.LaplexError):
-        X.workspace_size(11, 10)
+        X.workspace_size(13, 10)
     with pytest.raises(X.LaplexError):
         X.workspace_size(-1, 10)
 
