@@ -26,6 +26,9 @@ namespace lx {
 #ifndef LX_BWD_MINB
 #define LX_BWD_MINB 2
 #endif
+#ifndef LX_BWD_S
+#define LX_BWD_S 2
+#endif
 constexpr int BWD_NT = 256;
 
 // Policy of threepass.cuh (wait-free: tile-local scans, exact tile carries,
@@ -40,7 +43,7 @@ struct BwdTP {
     // several times more: none).  Streamed pass 1 (inputs in sorted order):
     // s, x, g in a 2-stage ring.
     static constexpr int H = sizeof(T_) == 4 ? 192 : 0;
-    static constexpr int NIN = 2, S = 2, MINB = LX_BWD_MINB;
+    static constexpr int NIN = 2, S = LX_BWD_S, MINB = LX_BWD_MINB;
     int64_t n;
     const T* s;
     const int32_t* perm;

@@ -9,9 +9,10 @@
 // U at the element whose anchor is f".  Runs combine associatively:
 //     forward   P (+) A  = (e_A, V_A + exp(e_P - e_A) V_P)      P left of A
 //     backward  A (+) S  = (f_A, W_A + exp(f_A - f_S) W_S)      A left of S
-// The decay across any number of elements is one exp of an anchor difference,
-// never a product of rounded per-step decays, so fp32 error does not grow with
-// the distance between tiles.  Elements past the end are padded with the last
+// Between two runs the decay is one exp of the difference of their edge
+// anchors, so between tiles and between warps of a block fp32 error does not
+// grow with the distance; inside a warp's shuffle scan a decay is a product of
+// at most five rounded factors (see the warp level below).  Elements past the end are padded with the last
 // anchor and value 0, which is neutral in both directions.
 //
 // The last CT channels ("tie channels") use the decay [e_P == e_A] instead of

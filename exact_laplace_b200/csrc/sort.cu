@@ -874,7 +874,10 @@ cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws, 
 // through the digit passes beside its index, so that the values arrive in
 // sorted order (xs[r] = x[perm[r]]) with coalesced writes, instead of a random
 // gather after the sort.  16 keys per thread: three staged arrays per tile.
-constexpr int CARRY_KPT = 16;
+#ifndef LX_CARRY_KPT
+#define LX_CARRY_KPT 16
+#endif
+constexpr int CARRY_KPT = LX_CARRY_KPT;
 
 size_t sort_carry_ws_bytes(int64_t n) {
     const int64_t tile = (int64_t)SORT_NT * CARRY_KPT;

@@ -114,3 +114,21 @@ def test_halo_carries(case):
     x = rng.normal(size=n).astype(np.float32)
     g = rng.normal(size=n).astype(np.float32)
     check(a, x, g, np.float32, case)
+
+
+@pytest.mark.parametrize("L", [2, 5, 12, 13, 37, 64, 100, 191, 193, 385, 3072, 5000])
+@pytest.mark.parametrize("n", [7 * 3072 + 1234, 7 * 3072 + 100])
+def test_runs_across_chunks_and_tiles(L, n):
+    """Runs of L equal anchors, L apart (about one unit per element, so the
+    halos of the exp channels span the cut for short runs), shifted so that
+    run boundaries fall at several offsets from the chunk (12 elements) and
+    tile (3072) boundaries: the run sums of the sorted-order pass cross
+    neighbouring chunks, the tile edges and the halos; runs longer than 32
+    chunks or than a halo list their tiles for the four-channel redo pass.
+    n = 7 * 3072 + 100 leaves the last full tile without room for a right halo."""
+    rng = np.random.default_rng(L)
+    for off in (0, 7):
+        a = (float(L) * ((np.arange(n) + off) // L)).astype(np.float32)
+        x = rng.normal(size=n).astype(np.float32)
+        g = rng.normal(size=n).astype(np.float32)
+        check(a, x, g, np.float32, f"L={L} off={off}")
