@@ -50,7 +50,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--n", type=int, default=1 << 30)
-    p.add_argument("--rows", default="sort,perm,carry,backward,c2,c3,c4",
+    p.add_argument("--rows", default="sort,perm,carry,noalloc,backward,c2,c3,c4",
                    help="extra hot-path rows to time (comma list; empty for none)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -359,6 +359,11 @@ def run_ours(args):
         except X.LaplexError as e:
             rows["sort_error"] = str(e)
         del a_d, s2, p2
+        if "noalloc" in wanted:
+            # the allocation-free entry point on the headline's data
+            ms_n = timed(lambda: X.matvec_sym_noalloc(s_d, x_d, out=y_d), rsteps, 1) / rsteps
+            X.device_status(dev)
+            rows["c5_matvec_noalloc"] = crow(ms_n, BYTES_PER_ELEM_SYM * n, hbm)
         if "backward" in wanted:
             try:
                 g_d = torch.from_numpy(synth.normal(n, seed=rank, stream="g")).to(dev)

@@ -469,7 +469,8 @@ enum : int {
     F_IOTA = 2,    // the payload of key i is its index i (no payload input)
     F_UNMAP = 4,   // write the keys back as anchor bits
     F_CLAMP = 8,   // the keys are indices: map them to min(index, n)
-    F_PAIR = 16,   // a second 4-byte payload array rides along (v2src -> v2dst)
+    F_PAIR = 16,   // a second 4-byte payload array rides along (v2src -> v2dst), staged in a
+                   // second round through the staging area after the keys and payloads
 };
 
 template <typename K, typename V>
@@ -493,9 +494,9 @@ struct ScatterArgs {
 // Dynamic shared memory of one k_scatter block.
 template <typename K, typename V, int KPT, int S, int F>
 constexpr size_t scatter_smem() {
-    constexpr size_t TILE = (size_t)SORT_NT * KPT, W2 = (F & F_PAIR) ? 4 : 0;
-    return S * TILE * sizeof(K) + ((F & F_IOTA) ? 0 : S * TILE * sizeof(V)) + S * TILE * W2 +
-           TILE * (sizeof(K) + sizeof(V) + W2) + (size_t)SORT_NW * RADIX * 4;
+    constexpr size_t TILE = (size_t)SORT_NT * KPT;
+    return S * TILE * sizeof(K) + ((F & F_IOTA) ? 0 : S * TILE * sizeof(V)) + TILE * (sizeof(K) + sizeof(V)) +
+           (size_t)SORT_NW * RADIX * 4;
 }
 
 template <typename K, typename V, int KPT, int S, int F>
@@ -508,11 +509,9 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
     extern __shared__ __align__(128) unsigned char dyn[];
     K* stage_k = reinterpret_cast<K*>(dyn);                    // [S][TILE] (F_KEYMAP: anchor bits)
     V* stage_v = reinterpret_cast<V*>(stage_k + S * TILE);     // [S][TILE] (not with F_IOTA)
-    uint32_t* stage_v2 = reinterpret_cast<uint32_t*>(stage_v + (IOTA ? 0 : S * TILE));  // [S][TILE] (F_PAIR)
-    K* out_k = reinterpret_cast<K*>(stage_v2 + (PAIR ? S * TILE : 0));  // [TILE] in digit order
+    K* out_k = reinterpret_cast<K*>(stage_v + (IOTA ? 0 : S * TILE));  // [TILE] in digit order
     V* out_v = reinterpret_cast<V*>(out_k + TILE);             // [TILE]
-    uint32_t* out_v2 = reinterpret_cast<uint32_t*>(out_v + TILE);  // [TILE] (F_PAIR)
-    uint32_t* wcnt = out_v2 + (PAIR ? TILE : 0);               // [NW][RADIX]
+    uint32_t* wcnt = reinterpret_cast<uint32_t*>(out_v + TILE);  // [NW][RADIX]
     __shared__ __align__(8) uint64_t full[S];
     __shared__ int32_t gofs[RADIX];   // output position of staged key q of digit d: gofs[d] + q
     __shared__ uint32_t scan_sm[NW + 1];
@@ -549,12 +548,10 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
         if (t < 0) return;
         const int64_t tb = t * TILE;
         if (tb + TILE <= A.n) {
-            constexpr uint32_t kb = TILE * sizeof(K), vb = IOTA ? 0u : TILE * (uint32_t)sizeof(V),
-                               wb = PAIR ? TILE * 4u : 0u;
-            mbar_expect_tx(&full[st], kb + vb + wb);
+            constexpr uint32_t kb = TILE * sizeof(K), vb = IOTA ? 0u : TILE * (uint32_t)sizeof(V);
+            mbar_expect_tx(&full[st], kb + vb);
             bulk_g2s(stage_k + st * TILE, A.ksrc + tb, kb, &full[st]);
             if constexpr (!IOTA) bulk_g2s(stage_v + st * TILE, A.vsrc + tb, vb, &full[st]);
-            if constexpr (PAIR) bulk_g2s(stage_v2 + st * TILE, A.v2src + tb, wb, &full[st]);
         } else {
             mbar_arrive(&full[st]);
         }
@@ -643,10 +640,6 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
                 else if constexpr (FT) return stage_v[st * TILE + q];
                 else return A.vsrc[tb + q];
             };
-            auto value2_of = [&](int q) -> uint32_t {
-                if constexpr (FT) return stage_v2[st * TILE + q];
-                else return A.v2src[tb + q];
-            };
             // 4-byte keys and payloads are staged as one 8-byte pair: one
             // shared store per key, one shared load per key in the write-out
             constexpr bool PACK = sizeof(K) == 4 && sizeof(V) == 4;
@@ -658,13 +651,6 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
                     if (FT || q < cnt) {
                         rk[e] += wcnt[w * RADIX + ((uint32_t)(k[e] >> shift) & (RADIX - 1))];
                         out_kv[rk[e]] = make_uint2((uint32_t)k[e], (uint32_t)value_of(q));
-                    }
-                }
-                if constexpr (PAIR) {
-#pragma unroll
-                    for (int e = 0; e < KPT; ++e) {
-                        const int q = seg + 32 * e;
-                        if (FT || q < cnt) out_v2[rk[e]] = value2_of(q);
                     }
                 }
             } else {
@@ -709,7 +695,28 @@ __global__ void __launch_bounds__(SORT_NT, LX_SORT_MINB) k_scatter(ScatterArgs<K
                     const int64_t g = (int64_t)gofs[(uint32_t)(kk >> shift) & (RADIX - 1)] + q;
                     A.kdst[g] = UNMAP ? key_to_bits(kk) : kk;
                     A.vdst[g] = vv;
-                    if constexpr (PAIR) A.v2dst[g] = out_v2[q];
+                    // F_PAIR: position q's output offset replaces its key (read only by this thread)
+                    if constexpr (PAIR) out_kv[q].x = (uint32_t)g;  // n < 2^31
+                }
+            }
+            if constexpr (PAIR) {
+                // second round: the second payload (read from global memory,
+                // coalesced) into the payload slots of the staging area, at the
+                // same positions; each slot pairs it with its output offset
+                __syncthreads();  // the first round's payloads have been read
+#pragma unroll
+                for (int e = 0; e < KPT; ++e) {
+                    const int q = seg + 32 * e;
+                    if (FT || q < cnt) out_kv[rk[e]].y = __ldcs(A.v2src + tb + q);
+                }
+                __syncthreads();
+#pragma unroll
+                for (int j = 0; j < KPT; ++j) {
+                    const int q = (int)threadIdx.x + j * NT;
+                    if (FT || q < cnt) {
+                        const uint2 gw = out_kv[q];
+                        A.v2dst[gw.x] = gw.y;
+                    }
                 }
             }
             __syncthreads();  // out_k, out_v, gofs, wcnt are the next tile's
@@ -873,9 +880,10 @@ cudaError_t sort_run(const T* a, int64_t n, T* sorted, int32_t* perm, void* ws, 
 // The fp32 sort with a second payload: the value x[i] of each anchor rides
 // through the digit passes beside its index, so that the values arrive in
 // sorted order (xs[r] = x[perm[r]]) with coalesced writes, instead of a random
-// gather after the sort.  16 keys per thread: three staged arrays per tile.
+// gather after the sort.  Each pass stages the keys with the indices, then the
+// values through the same staging area (the same shared memory as the plain sort).
 #ifndef LX_CARRY_KPT
-#define LX_CARRY_KPT 16
+#define LX_CARRY_KPT 24
 #endif
 constexpr int CARRY_KPT = LX_CARRY_KPT;
 

@@ -289,6 +289,18 @@ def invert_perm(perm: torch.Tensor, out=None):
     return inv
 
 
+def matvec_sym_noalloc(sorted_anchors: torch.Tensor, x: torch.Tensor, perm=None, out=None):
+    """laplex_matvec_sym_noalloc: y = K x (fp32, one column) with the library's
+    fixed device scratch instead of a workspace (n <= 2^30)."""
+    dev = _dev(sorted_anchors, x, _perm(perm), out)
+    n = sorted_anchors.numel()
+    if x.numel() != n or x.dtype != torch.float32 or sorted_anchors.dtype != torch.float32:
+        raise LaplexError(EINVAL, "fp32 anchors and x with n elements")
+    y = torch.empty_like(x) if out is None else out
+    _check(lib().laplex_matvec_sym_noalloc(_ptr(sorted_anchors), _ptr(perm), n, _ptr(x), _ptr(y), _stream(dev)))
+    return y
+
+
 def matvec_sym_planned(sorted_anchors: torch.Tensor, perm: torch.Tensor, inv: torch.Tensor, x: torch.Tensor,
                        out=None):
     """y = K x for x, y in the caller's order (one column), through the plan
