@@ -4,6 +4,11 @@ Every .cu under csrc/ is compiled with
     nvcc -gencode arch=compute_100a,code=sm_100a -O3 -lineinfo -std=c++17 -Xcompiler -fPIC
 and linked (static CUDA runtime) into exact_laplace_b200/liblaplex.so.
 Objects go to exact_laplace_b200/_build/ (git-ignored).
+
+LAPLEX_ACCURATE_EXP=1 in the environment builds the fp32 decays on CUDA's
+expf (with --ftz=true, so that exp(-d) for d >= 88 is still exactly 0)
+instead of the hardware base-2 exponential: a smaller scan error (below the
+dense fp32 product's at the pages' C1 size) for a slower headline product.
 """
 from __future__ import annotations
 
@@ -22,6 +27,10 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include"), "-I", CSRC]
+ACCURATE = os.environ.get("LAPLEX_ACCURATE_EXP", "0") == "1"
+if ACCURATE:
+    FLAGS += ["-DLX_ACCURATE_EXP", "--ftz=true"]
+MODE_FILE = os.path.join(BUILD, "mode.txt")
 
 
 def _deps_mtime() -> float:
@@ -44,7 +53,9 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
+    mode = "accurate-exp" if ACCURATE else "default"
+    same_mode = os.path.exists(MODE_FILE) and open(MODE_FILE).read().strip() == mode
+    if not force and same_mode and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
         return LIB
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     with ThreadPoolExecutor(max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
@@ -55,6 +66,8 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    with open(MODE_FILE, "w") as f:
+        f.write(mode + "\n")
     return LIB
 
 

@@ -151,7 +151,15 @@ void lx::set_last_error(const char* fmt, ...) {
 
 extern "C" {
 
-int laplex_version(void) { return 10000; }
+int laplex_version(void) { return 10100; }
+
+int laplex_build_flags(void) {
+#ifdef LX_ACCURATE_EXP
+    return LAPLEX_BUILD_ACCURATE_EXP;
+#else
+    return 0;
+#endif
+}
 
 const char* laplex_status_string(laplex_status s) {
     switch (s) {

@@ -16,11 +16,18 @@ template <typename T> __device__ __forceinline__ T dexp(T v);
 // the kernel value exp(-|a_i - b_j|) of each term it carries, so a term whose
 // kernel value is >= FLT_MIN is never flushed; only terms below FLT_MIN can
 // be lost (at most their |x|-weighted mass).
+// Built with LX_ACCURATE_EXP (and --ftz=true): CUDA's expf, whose smaller
+// error takes the scan's error below the dense fp32 product's, for a slower
+// product; the flush of results below FLT_MIN, and so the cut below, hold.
+#ifdef LX_ACCURATE_EXP
+template <> __device__ __forceinline__ float dexp<float>(float v) { return expf(v); }
+#else
 template <> __device__ __forceinline__ float dexp<float>(float v) {
     float r;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v * 1.44269504088896341f));
     return r;
 }
+#endif
 template <> __device__ __forceinline__ double dexp<double>(double v) { return exp(v); }
 
 // A distance beyond which dexp(-d) is exactly 0: fp32, 2^(-88 log2 e) =

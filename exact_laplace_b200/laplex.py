@@ -22,6 +22,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblaplex.so")
 
 OK, EINVAL, ENONFINITE, EWORKSPACE, ECUDA, ETIMEOUT = range(6)
+BUILD_ACCURATE_EXP = 1  # laplex_build_flags() bit
 F32, F64 = 0, 1
 (OP_SORT, OP_SYM, OP_GENERAL, OP_PHASED, OP_GRAM, OP_BACKWARD, OP_BACKWARD_GENERAL, OP_GRAM_MATRIX,
  OP_BACKWARD_PHASED, OP_PERMUTE, OP_SYM_PLANNED, OP_SORT_CARRY, OP_SYM_UNSORTED) = range(13)
@@ -45,6 +46,7 @@ _STATUS_NAMES = {OK: "LAPLEX_OK", EINVAL: "LAPLEX_EINVAL", ENONFINITE: "LAPLEX_E
 #: every symbol include/laplex.h declares, with its ctypes signature
 SIGNATURES = {
     "laplex_version": ([], ctypes.c_int),
+    "laplex_build_flags": ([], ctypes.c_int),
     "laplex_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "laplex_last_error": ([], ctypes.c_char_p),
     "laplex_workspace_size": ([ctypes.c_int, _I64, _I64, _I64, ctypes.c_int,

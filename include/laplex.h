@@ -83,6 +83,12 @@ typedef enum {
 /* Library ABI version (major*10000 + minor*100 + patch). */
 int laplex_version(void);
 
+/* How the library was built: LAPLEX_BUILD_ACCURATE_EXP set when the fp32
+ * decays use CUDA's expf (more accurate, slower) instead of the hardware
+ * base-2 exponential.  No side effects; callable without a GPU. */
+#define LAPLEX_BUILD_ACCURATE_EXP 1
+int laplex_build_flags(void);
+
 /* Human-readable name of a status code (static string). */
 const char* laplex_status_string(laplex_status s);
 

@@ -40,6 +40,7 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_version_and_status_strings(L):
     assert L.laplex_version() >= 10000
+    assert L.laplex_build_flags() in (0, 1)
     assert L.laplex_status_string(0) == b"LAPLEX_OK"
     assert L.laplex_status_string(5) == b"LAPLEX_ETIMEOUT"
 

@@ -140,3 +140,23 @@ def test_c5_full_size():
     r = np.concatenate([np.arange(64), n - 64 + np.arange(64), synth.randint(4096, n, seed=1, stream="misc")])
     out, _, absn = rows_local(s, xs, r)
     assert_close(y[p[r]], out, absn, np.float32, "C5 unsorted sampled rows")
+
+
+def test_carry_expired_wait_reports_timeout():
+    """The carrying sort's copy waits are bounded like the plain sort's: with
+    every block's first copy left unissued and a bound of 16 polls, the call
+    returns, the status is LAPLEX_ETIMEOUT (cleared once read), and the next
+    call is exact."""
+    n = 100_000
+    a = synth.normal(n, 0.0, 100.0, seed=5, stream="a")
+    x = bits(n, np.float32, 6)
+    X.test_set_sort_wait(16, True)
+    try:
+        X.sort_anchors_carry(dev(a), dev(x))
+    finally:
+        X.test_set_sort_wait(0, False)
+    with pytest.raises(X.LaplexError) as e:
+        X.device_status()
+    assert e.value.status == X.ETIMEOUT
+    X.device_status()
+    check_carry(a, x)
