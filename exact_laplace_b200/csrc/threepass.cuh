@@ -444,10 +444,33 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
 }
 
 // ------------------------------------------------------------------ pass 2
+// The records of a thread's TP_CARRY_PT consecutive tiles, loaded at once (the
+// loads are independent; a tile past the end repeats the last one and is
+// masked out by `valid`).
+template <typename T, int C>
+struct TPSeg {
+    T tl[TP_CARRY_PT], tf[TP_CARRY_PT];
+    T fa[TP_CARRY_PT][C], ba[TP_CARRY_PT][C];
+    __device__ __forceinline__ void load(const TPWs<T, C>& W, int64_t t0, int64_t ntiles) {
+#pragma unroll
+        for (int k = 0; k < TP_CARRY_PT; ++k) {
+            const int64_t t = min(t0 + k, ntiles - 1);
+            tl[k] = W.tlast[t];
+            tf[k] = W.tfirst[t];
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                fa[k][c] = W.fagg[t * C + c];
+                ba[k][c] = W.bagg[t * C + c];
+            }
+        }
+    }
+};
+
+// The thread's segment summaries: forward (fe, fv) and backward (bf, bv);
+// a thread with no tile holds the neutral summary (the last anchor, 0).
 template <typename T, int C, int CT>
-__device__ __forceinline__ void tp_segment(const TPWs<T, C>& W, int64_t t0, int64_t ntiles, T& fe,
+__device__ __forceinline__ void tp_segment(const TPSeg<T, C>& g, int64_t t0, int64_t ntiles, T pad, T& fe,
                                            T (&fv)[C], T& bf, T (&bv)[C]) {
-    const T pad = W.tlast[ntiles - 1];
     fe = pad;
     bf = pad;
 #pragma unroll
@@ -456,24 +479,24 @@ __device__ __forceinline__ void tp_segment(const TPWs<T, C>& W, int64_t t0, int6
         bv[c] = T(0);
     }
     bool any = false;
+#pragma unroll
     for (int k = 0; k < TP_CARRY_PT; ++k) {
-        const int64_t t = t0 + k;
-        if (t >= ntiles) break;
-        const T e = W.tlast[t];
+        if (t0 + k >= ntiles) break;
+        const T e = g.tl[k];
         const Decay<T, C, CT> d(fe, e);
 #pragma unroll
-        for (int c = 0; c < C; ++c) fv[c] = dfma<T>(any ? d[c] : T(0), fv[c], W.fagg[t * C + c]);
+        for (int c = 0; c < C; ++c) fv[c] = dfma<T>(any ? d[c] : T(0), fv[c], g.fa[k][c]);
         fe = e;
         any = true;
     }
     any = false;
+#pragma unroll
     for (int k = TP_CARRY_PT - 1; k >= 0; --k) {
-        const int64_t t = t0 + k;
-        if (t >= ntiles) continue;
-        const T f = W.tfirst[t];
+        if (t0 + k >= ntiles) continue;
+        const T f = g.tf[k];
         const Decay<T, C, CT> d(f, bf);
 #pragma unroll
-        for (int c = 0; c < C; ++c) bv[c] = dfma<T>(any ? d[c] : T(0), bv[c], W.bagg[t * C + c]);
+        for (int c = 0; c < C; ++c) bv[c] = dfma<T>(any ? d[c] : T(0), bv[c], g.ba[k][c]);
         bf = f;
         any = true;
     }
@@ -484,8 +507,10 @@ __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_blocks(TPWs<T, C> W, i
     if (*(volatile uint32_t*)W.redo_count == 0) return;  // every tile final
     __shared__ BlockScan2Smem<T, C, TP_CARRY_NT> sm2;
     const int64_t t0 = (int64_t)blockIdx.x * TP_CARRY_BT + (int64_t)threadIdx.x * TP_CARRY_PT;
+    TPSeg<T, C> g;
+    g.load(W, t0, ntiles);
     T fe, fv[C], bf, bv[C];
-    tp_segment<T, C, CT>(W, t0, ntiles, fe, fv, bf, bv);
+    tp_segment<T, C, CT>(g, t0, ntiles, W.tlast[ntiles - 1], fe, fv, bf, bv);
     bool hf, hb;
     T pe, pv[C], te, tv[C], nf, nv[C], tf, tw[C];
     block_excl_both<T, C, TP_CARRY_NT, CT>(fe, fv, bf, bv, hf, pe, pv, te, tv, hb, nf, nv, tf, tw, sm2);
@@ -541,8 +566,10 @@ __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_tiles(TPWs<T, C> W, in
         }
     }
     const int64_t t0 = bidx * TP_CARRY_BT + (int64_t)threadIdx.x * TP_CARRY_PT;
+    TPSeg<T, C> g;
+    g.load(W, t0, ntiles);
     T fe, fv[C], bf, bv[C];
-    tp_segment<T, C, CT>(W, t0, ntiles, fe, fv, bf, bv);
+    tp_segment<T, C, CT>(g, t0, ntiles, W.tlast[ntiles - 1], fe, fv, bf, bv);
     bool hf, hb;
     T pe, pv[C], te, tv[C], nf, nv[C], tf, tw[C];
     block_excl_both<T, C, TP_CARRY_NT, CT>(fe, fv, bf, bv, hf, pe, pv, te, tv, hb, nf, nv, tf, tw,
@@ -560,15 +587,16 @@ __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_tiles(TPWs<T, C> W, in
 #pragma unroll
         for (int c = 0; c < C; ++c) cv[c] = sh_c[0][c];
     }
+#pragma unroll
     for (int k = 0; k < TP_CARRY_PT; ++k) {
         const int64_t t = t0 + k;
         if (t >= ntiles) break;
 #pragma unroll
         for (int c = 0; c < C; ++c) W.carF[t * C + c] = t == 0 ? T(0) : cv[c];
-        const T e = W.tlast[t];
+        const T e = g.tl[k];
         const Decay<T, C, CT> d(ce, e);
 #pragma unroll
-        for (int c = 0; c < C; ++c) cv[c] = dfma<T>(d[c], cv[c], W.fagg[t * C + c]);
+        for (int c = 0; c < C; ++c) cv[c] = dfma<T>(d[c], cv[c], g.fa[k][c]);
         ce = e;
     }
     const T fBlk = bidx + 1 < nblocks ? W.bbf[bidx + 1] : W.tlast[ntiles - 1];
@@ -583,15 +611,16 @@ __global__ void __launch_bounds__(TP_CARRY_NT) k_tp_carry_tiles(TPWs<T, C> W, in
 #pragma unroll
         for (int c = 0; c < C; ++c) cw[c] = sh_c[1][c];
     }
+#pragma unroll
     for (int k = TP_CARRY_PT - 1; k >= 0; --k) {
         const int64_t t = t0 + k;
         if (t >= ntiles) continue;
 #pragma unroll
         for (int c = 0; c < C; ++c) W.carB[t * C + c] = t == ntiles - 1 ? T(0) : cw[c];
-        const T f = W.tfirst[t];
+        const T f = g.tf[k];
         const Decay<T, C, CT> d(f, cf);
 #pragma unroll
-        for (int c = 0; c < C; ++c) cw[c] = dfma<T>(d[c], cw[c], W.bagg[t * C + c]);
+        for (int c = 0; c < C; ++c) cw[c] = dfma<T>(d[c], cw[c], g.ba[k][c]);
         cf = f;
     }
 }
