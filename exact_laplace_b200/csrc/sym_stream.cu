@@ -361,30 +361,46 @@ __global__ void __launch_bounds__(NT, LX_LT_MINB) k_tile_local(const T* __restri
     }
 }
 
+// The records of this thread's CARRY_PT tiles, loaded in one round of
+// independent loads (a tile past the end repeats the last one; it is skipped).
+template <typename T>
+struct CarrySeg {
+    T tl[CARRY_PT], tf[CARRY_PT], fa[CARRY_PT], ba[CARRY_PT];
+    __device__ __forceinline__ void load(const LocalWs<T>& W, int64_t t0, int64_t ntiles) {
+#pragma unroll
+        for (int k = 0; k < CARRY_PT; ++k) {
+            const int64_t t = min(t0 + k, ntiles - 1);
+            tl[k] = W.tlast[t];
+            tf[k] = W.tfirst[t];
+            fa[k] = W.fagg[t];
+            ba[k] = W.bagg[t];
+        }
+    }
+};
+
 // This thread's forward and backward totals over its CARRY_PT tiles.
 template <typename T>
-__device__ __forceinline__ void carry_segment(const LocalWs<T>& W, int64_t t0, int64_t ntiles,
+__device__ __forceinline__ void carry_segment(const CarrySeg<T>& g, int64_t t0, int64_t ntiles, T pad,
                                               T& fe, T (&fv)[1], T& bf, T (&bv)[1]) {
-    const T pad = W.tlast[ntiles - 1];
     fe = pad;
     bf = pad;
     fv[0] = T(0);
     bv[0] = T(0);
     bool any = false;
+#pragma unroll
     for (int k = 0; k < CARRY_PT; ++k) {
-        const int64_t t = t0 + k;
-        if (t >= ntiles) break;
-        const T e = W.tlast[t];
-        fv[0] = dfma<T>(any ? dexp<T>(fe - e) : T(0), fv[0], W.fagg[t]);
+        if (t0 + k >= ntiles) break;
+        const T e = g.tl[k];
+        fv[0] = dfma<T>(any ? dexp<T>(fe - e) : T(0), fv[0], g.fa[k]);
         fe = e;
         any = true;
     }
     any = false;
+#pragma unroll
     for (int k = CARRY_PT - 1; k >= 0; --k) {
-        const int64_t t = t0 + k;
-        if (t >= ntiles) continue;
-        const T f = W.tfirst[t];
-        bv[0] = dfma<T>(any ? dexp<T>(f - bf) : T(0), bv[0], W.bagg[t]);
+        if (t0 + k >= ntiles) continue;
+        const T f = g.tf[k];
+        bv[0] = dfma<T>(any ? dexp<T>(f - bf) : T(0), bv[0], g.ba[k]);
         bf = f;
         any = true;
     }
@@ -395,8 +411,10 @@ __global__ void __launch_bounds__(CARRY_NT) k_carry_blocks(LocalWs<T> W, int64_t
     if (*(volatile uint32_t*)W.redo_count == 0) return;  // every tile final
     __shared__ BlockScanSmem<T, 1, CARRY_NT> smf, smb;
     const int64_t t0 = (int64_t)blockIdx.x * CARRY_BT + (int64_t)threadIdx.x * CARRY_PT;
+    CarrySeg<T> g;
+    g.load(W, t0, ntiles);
     T fe, fv[1], bf, bv[1];
-    carry_segment<T>(W, t0, ntiles, fe, fv, bf, bv);
+    carry_segment<T>(g, t0, ntiles, W.tlast[ntiles - 1], fe, fv, bf, bv);
     bool h;
     T pe, pv[1], te, tv[1], nf, nv[1], tf, tw[1];
     block_excl_fwd<T, 1, CARRY_NT>(fe, fv, h, pe, pv, te, tv, smf);
@@ -438,8 +456,10 @@ __global__ void __launch_bounds__(CARRY_NT) k_carry_tiles(LocalWs<T> W, int64_t 
         sh_c[1] = accb;
     }
     const int64_t t0 = bidx * CARRY_BT + (int64_t)threadIdx.x * CARRY_PT;
+    CarrySeg<T> g;
+    g.load(W, t0, ntiles);
     T fe, fv[1], bf, bv[1];
-    carry_segment<T>(W, t0, ntiles, fe, fv, bf, bv);
+    carry_segment<T>(g, t0, ntiles, W.tlast[ntiles - 1], fe, fv, bf, bv);
     bool hf, hb;
     T pe, pv[1], te, tv[1], nf, nv[1], tf, tw[1];
     block_excl_fwd<T, 1, CARRY_NT>(fe, fv, hf, pe, pv, te, tv, smf);  // its barriers publish sh_c
@@ -453,12 +473,13 @@ __global__ void __launch_bounds__(CARRY_NT) k_carry_tiles(LocalWs<T> W, int64_t 
         ce = eBlk;
         cv = sh_c[0];
     }
+#pragma unroll
     for (int k = 0; k < CARRY_PT; ++k) {
         const int64_t t = t0 + k;
         if (t >= ntiles) break;
         W.carF[t] = t == 0 ? T(0) : cv;
-        const T e = W.tlast[t];
-        cv = dfma<T>(dexp<T>(ce - e), cv, W.fagg[t]);
+        const T e = g.tl[k];
+        cv = dfma<T>(dexp<T>(ce - e), cv, g.fa[k]);
         ce = e;
     }
     const T fBlk = bidx + 1 < nblocks ? W.bbf[bidx + 1] : W.tlast[ntiles - 1];
@@ -470,12 +491,13 @@ __global__ void __launch_bounds__(CARRY_NT) k_carry_tiles(LocalWs<T> W, int64_t 
         cf = fBlk;
         cw = sh_c[1];
     }
+#pragma unroll
     for (int k = CARRY_PT - 1; k >= 0; --k) {
         const int64_t t = t0 + k;
         if (t >= ntiles) continue;
         W.carB[t] = t == ntiles - 1 ? T(0) : cw;
-        const T f = W.tfirst[t];
-        cw = dfma<T>(dexp<T>(f - cf), cw, W.bagg[t]);
+        const T f = g.tf[k];
+        cw = dfma<T>(dexp<T>(f - cf), cw, g.ba[k]);
         cf = f;
     }
 }
