@@ -40,6 +40,21 @@ template <> struct ExpCut<double> { static constexpr double v = 746.0; };
 
 template <typename T> __device__ __forceinline__ T dfma(T a, T b, T c) { return fma(a, b, c); }
 
+// sin and cos of a phase.  fp32: the phase is first reduced to [-pi, pi] by
+// Cody and Waite's two-constant reduction (t - k 2pi with 2pi split into the
+// nearest float and its remainder, each step one fused multiply-add), then the
+// hardware sine and cosine (absolute error about 2^-21 on [-pi, pi]); fp64:
+// sincos.
+template <typename T> __device__ __forceinline__ void psincos(T t, T* s, T* c);
+template <> __device__ __forceinline__ void psincos<float>(float t, float* s, float* c) {
+    constexpr float TWO_PI_HI = 6.28318548202514648f;   // the float nearest 2 pi
+    constexpr float TWO_PI_LO = -1.7484555314695172e-7f;  // 2 pi - TWO_PI_HI
+    const float k = rintf(t * 0.159154943091895336f);     // t / (2 pi), rounded
+    const float r = fmaf(-k, TWO_PI_LO, fmaf(-k, TWO_PI_HI, t));
+    __sincosf(r, s, c);
+}
+template <> __device__ __forceinline__ void psincos<double>(double t, double* s, double* c) { sincos(t, s, c); }
+
 __device__ __forceinline__ void set_status(uint32_t* st, uint32_t bits) {
     if (st) atomicOr(st, bits);
 }

@@ -30,9 +30,6 @@ namespace lx {
 
 constexpr int GEN_NT = 256;
 
-template <typename T> __device__ __forceinline__ void gsincos(T a, T* s, T* c);
-template <> __device__ __forceinline__ void gsincos<float>(float a, float* s, float* c) { sincosf(a, s, c); }
-template <> __device__ __forceinline__ void gsincos<double>(double a, double* s, double* c) { sincos(a, s, c); }
 
 // ia[t] = number of a-points among the first min(t*tile, n+k) merged elements
 // (the merge path of a before b on ties).  One warp per diagonal: each round
@@ -67,7 +64,7 @@ __device__ __forceinline__ void gen_bvalue(const GenArgs<T>& A, int64_t j, T (&v
     const int64_t row = A.pin ? (int64_t)A.pin[j] : j;
     const T dsc = A.D ? A.D[A.pD ? (int64_t)A.pD[j] : j] : T(1);
     T cs = T(1), sn = T(0);
-    if (PHASED) gsincos<T>(A.psi[A.ppsi ? (int64_t)A.ppsi[j] : j], &sn, &cs);
+    if (PHASED) psincos<T>(A.psi[A.ppsi ? (int64_t)A.ppsi[j] : j], &sn, &cs);
     const T* xr = A.x + row * A.ldx + A.col0;
 #pragma unroll
     for (int c = 0; c < NCOL; ++c) {
@@ -238,7 +235,7 @@ __device__ __forceinline__ void gen_tile(const GenArgs<T>& A, const TPWs<T, PHAS
         T* yr = A.y + row * A.ldy + A.col0;
         if (PHASED) {
             T sp, cp;
-            gsincos<T>(A.phi[A.pphi ? (int64_t)A.pphi[i] : i], &sp, &cp);
+            psincos<T>(A.phi[A.pphi ? (int64_t)A.pphi[i] : i], &sp, &cp);
 #pragma unroll
             for (int c = 0; c < NCOL; ++c)
                 if (c < A.ncol) yr[c] = cp * o[e][2 * c] + sp * o[e][2 * c + 1];
@@ -339,7 +336,7 @@ __global__ void __launch_bounds__(256) k_gen_headtail(GenArgs<T> A, TPWs<T, PHAS
                 T* yr = A.y + row * A.ldy + A.col0;
                 if (PHASED) {
                     T sp, cp;
-                    gsincos<T>(A.phi[A.pphi ? (int64_t)A.pphi[iu[u]] : iu[u]], &sp, &cp);
+                    psincos<T>(A.phi[A.pphi ? (int64_t)A.pphi[iu[u]] : iu[u]], &sp, &cp);
                     for (int q2 = 0; q2 < A.ncol; ++q2)
                         yr[q2] += fL * (cp * cL[2 * q2] + sp * cL[2 * q2 + 1]) +
                                   fR * (cp * cR[2 * q2] + sp * cR[2 * q2 + 1]);

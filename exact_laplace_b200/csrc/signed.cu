@@ -273,8 +273,6 @@ cudaError_t sgen_run(const T* sa, const int32_t* pa, int64_t n, const T* sb, con
 // sums above): P = F_{ub-1} exp(b_{ub-1} - a) + G_{ub} exp(a - b_{ub}),
 // S = F_{lb-1} exp(b_{lb-1} - a) - G_{ub} exp(a - b_{ub}).
 
-static __device__ __forceinline__ void pb_sincos(float t, float* sn, float* cs) { sincosf(t, sn, cs); }
-static __device__ __forceinline__ void pb_sincos(double t, double* sn, double* cs) { sincos(t, sn, cs); }
 
 // Policy of threepass.cuh: channels cos(ph) v and sin(ph) v (v and ph gathered
 // through perm), prefix F and suffix G written interleaved, [n][2], sorted order.
@@ -294,7 +292,7 @@ struct OneSidedPhasedTP {
     __device__ __forceinline__ void value(int64_t r, T (&vj)[C]) const {
         const int64_t o = perm ? (int64_t)perm[r] : r;
         T sn, cs;
-        pb_sincos(ph[o], &sn, &cs);
+        psincos(ph[o], &sn, &cs);
         const T x = v[o];
         vj[0] = cs * x;
         vj[1] = sn * x;
@@ -462,7 +460,7 @@ __global__ void __launch_bounds__(QCH) k_phased_query(const T* __restrict__ sq, 
         }
         const int64_t row = pq ? (int64_t)pq[r] : r;
         T sn, cs;
-        pb_sincos(th[row], &sn, &cs);
+        psincos(th[row], &sn, &cs);
         if (prod) prod[row] = cs * P0 + sn * P1;
         if (dph || dan) {
             const T wr = w[row];

@@ -22,9 +22,6 @@ namespace lx {
 
 constexpr int SYM_NT = 256;
 
-template <typename T> __device__ __forceinline__ void dsincos(T a, T* s, T* c);
-template <> __device__ __forceinline__ void dsincos<float>(float a, float* s, float* c) { sincosf(a, s, c); }
-template <> __device__ __forceinline__ void dsincos<double>(double a, double* s, double* c) { sincos(a, s, c); }
 
 // Load the chunk [r0, r0 + E) : anchors, channel values, and (phased) cos/sin.
 template <typename T, int NCOL, bool PHASED, int E>
@@ -56,7 +53,7 @@ __device__ __forceinline__ void sym_load(const SymArgs<T>& A, const int64_t r0, 
             const int64_t row = A.pin ? (int64_t)A.pin[r] : r;
             const int64_t ar = A.paux ? (int64_t)A.paux[r] : r;
             const T dsc = A.D ? A.D[ar] : T(1);
-            if (PHASED) dsincos<T>(A.phi[ar], &sph[i], &cph[i]);
+            if (PHASED) psincos<T>(A.phi[ar], &sph[i], &cph[i]);
             const T* xr = A.x + row * A.ldx + A.col0;
             T xv[NCOL];
             if (NCOL >= VN && (NCOL % VN) == 0 && A.ncol == NCOL && (A.ldx % VN) == 0 &&
@@ -276,7 +273,7 @@ struct SymTP {
     __device__ __forceinline__ void value(const T (&xe)[NIN], T (&vv)[C]) const {
         if constexpr (PHASED_) {
             T sp, cp;
-            dsincos<T>(xe[1], &sp, &cp);
+            psincos<T>(xe[1], &sp, &cp);
             vv[0] = cp * xe[0];
             vv[1] = sp * xe[0];
         } else {
@@ -286,7 +283,7 @@ struct SymTP {
     __device__ __forceinline__ void value_chunk(const T (&xe)[NIN], T (&vv)[C], Aux& a, int k) const {
         if constexpr (PHASED_) {
             T sp, cp;
-            dsincos<T>(xe[1], &sp, &cp);
+            psincos<T>(xe[1], &sp, &cp);
             a.cph[k] = cp;
             a.sph[k] = sp;
             vv[0] = cp * xe[0];
@@ -311,7 +308,7 @@ struct SymTP {
         const int64_t ar = A.paux ? (int64_t)A.paux[j] : j;
         const T dsc = A.D ? A.D[ar] : T(1);
         T sp = T(0), cp = T(1);
-        if (PHASED_) dsincos<T>(A.phi[ar], &sp, &cp);
+        if (PHASED_) psincos<T>(A.phi[ar], &sp, &cp);
         const T* xr = A.x + row * A.ldx + A.col0;
 #pragma unroll
         for (int c = 0; c < NCOL; ++c) {
