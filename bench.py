@@ -412,7 +412,7 @@ def run_ours(args):
         r["warm_ms"] = crow(timed_warm(fn, steps), bytes_per, hbm)["ms"]
         return r
 
-    fsteps = max(3, min(20, args.steps // 10))
+    fsteps = max(10, min(20, args.steps))  # calls per C2-C4 row (each well under a millisecond)
     try:
         if "c2" in wanted:
             n2 = 1 << 24

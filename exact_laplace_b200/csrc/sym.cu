@@ -12,7 +12,8 @@
 //   * several columns, phases or a scale: the wait-free three-kernel scheme of
 //     threepass.cuh with the SymTP policy below;
 //   * laplex_matvec_sym_noalloc: the three-phase reduce-then-scan below
-//     (k_sym_reduce, k_tile_carries, k_sym_final) with a fixed scratch array.
+//     (k_sym_reduce, the carry kernels of threepass.cuh, k_sym_final) with a
+//     fixed scratch array.
 #include <algorithm>
 
 #include "laplex_impl.h"
@@ -122,8 +123,7 @@ __device__ __forceinline__ void sym_store(const SymArgs<T>& A, const int64_t r0,
 }
 
 template <typename T, int NCOL, bool PHASED, int E, int NT>
-__global__ void __launch_bounds__(NT) k_sym_reduce(SymArgs<T> A, T* __restrict__ aggF,
-                                                   T* __restrict__ aggB) {
+__global__ void __launch_bounds__(NT) k_sym_reduce(SymArgs<T> A, TPWs<T, PHASED ? 2 * NCOL : NCOL> W) {
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
     __shared__ BlockScanSmem<T, C, NT> smf, smb;
     const int64_t r0 = (int64_t)blockIdx.x * (NT * E) + (int64_t)threadIdx.x * E;
@@ -135,80 +135,14 @@ __global__ void __launch_bounds__(NT) k_sym_reduce(SymArgs<T> A, T* __restrict__
     block_excl_fwd<T, C, NT>(s[E - 1], fV, hf, pe, pV, te, tV, smf);
     block_excl_bwd<T, C, NT>(s[0], bW, hb, nf, nW, tf, tW, smb);
     if (threadIdx.x == 0) {
+        W.tfirst[blockIdx.x] = tf;
+        W.tlast[blockIdx.x] = te;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            aggF[(int64_t)blockIdx.x * C + c] = tV[c];
-            aggB[(int64_t)blockIdx.x * C + c] = tW[c];
+            W.fagg[(int64_t)blockIdx.x * C + c] = tV[c];
+            W.bagg[(int64_t)blockIdx.x * C + c] = tW[c];
         }
-    }
-}
-
-// Carries into each tile from the tile totals (one block; segments per thread).
-// carF[t] = L at the element before tile t (anchor = last anchor of tile t-1);
-// carB[t] = U at the element after tile t (anchor = first anchor of tile t+1).
-template <typename T, int C, int NT>
-__global__ void __launch_bounds__(NT) k_tile_carries(const T* __restrict__ s, int64_t n, int64_t tile,
-                                                     int64_t ntiles, const T* __restrict__ aggF,
-                                                     const T* __restrict__ aggB, T* __restrict__ carF,
-                                                     T* __restrict__ carB, const uint32_t* gate) {
-    if (gate != nullptr && *gate == 0u) return;  // nothing to fix up
-    __shared__ BlockScanSmem<T, C, NT> smf, smb;
-    const int64_t per = (ntiles + NT - 1) / NT;
-    const int64_t t0 = min((int64_t)threadIdx.x * per, ntiles);
-    const int64_t t1 = min(t0 + per, ntiles);
-    auto eL = [&](int64_t t) { return s[min((t + 1) * tile, n) - 1]; };
-    auto eF = [&](int64_t t) { return s[min(t * tile, n - 1)]; };
-    const T pad = s[n - 1];
-    // forward
-    T ae = pad, aV[C];
-#pragma unroll
-    for (int c = 0; c < C; ++c) aV[c] = T(0);
-    for (int64_t t = t0; t < t1; ++t) {
-        const T e = eL(t);
-        const T d = (t == t0) ? T(0) : dexp<T>(ae - e);
-#pragma unroll
-        for (int c = 0; c < C; ++c) aV[c] = dfma<T>(d, aV[c], aggF[t * C + c]);
-        ae = e;
-    }
-    bool has;
-    T pe, pV[C], te, tV[C];
-    block_excl_fwd<T, C, NT>(ae, aV, has, pe, pV, te, tV, smf);
-    T ce = has ? pe : s[0], cv[C];
-#pragma unroll
-    for (int c = 0; c < C; ++c) cv[c] = has ? pV[c] : T(0);
-    for (int64_t t = t0; t < t1; ++t) {
-#pragma unroll
-        for (int c = 0; c < C; ++c) carF[t * C + c] = cv[c];
-        const T e = eL(t);
-        const T d = dexp<T>(ce - e);
-#pragma unroll
-        for (int c = 0; c < C; ++c) cv[c] = dfma<T>(d, cv[c], aggF[t * C + c]);
-        ce = e;
-    }
-    // backward
-    T bf = pad, bW[C];
-#pragma unroll
-    for (int c = 0; c < C; ++c) bW[c] = T(0);
-    for (int64_t t = t1 - 1; t >= t0; --t) {
-        const T f = eF(t);
-        const T d = (t == t1 - 1) ? T(0) : dexp<T>(f - bf);
-#pragma unroll
-        for (int c = 0; c < C; ++c) bW[c] = dfma<T>(d, bW[c], aggB[t * C + c]);
-        bf = f;
-    }
-    T nf, nW[C], tf, tW[C];
-    block_excl_bwd<T, C, NT>(bf, bW, has, nf, nW, tf, tW, smb);
-    T cf = has ? nf : pad, cw[C];
-#pragma unroll
-    for (int c = 0; c < C; ++c) cw[c] = has ? nW[c] : T(0);
-    for (int64_t t = t1 - 1; t >= t0; --t) {
-#pragma unroll
-        for (int c = 0; c < C; ++c) carB[t * C + c] = cw[c];
-        const T f = eF(t);
-        const T d = dexp<T>(f - cf);
-#pragma unroll
-        for (int c = 0; c < C; ++c) cw[c] = dfma<T>(d, cw[c], aggB[t * C + c]);
-        cf = f;
+        if (blockIdx.x == 0) *W.redo_count = 1u;  // every tile takes the carry kernels
     }
 }
 
@@ -362,13 +296,14 @@ size_t sym_ws_bytes(int64_t n, int64_t B, bool phased, int f64) {
 }
 
 template <typename T, int NCOL, bool PHASED, int E>
-static cudaError_t sym_launch(const SymArgs<T>& A, int64_t ntiles, T* aggF, T* aggB, T* carF,
-                              T* carB, cudaStream_t st) {
+static cudaError_t sym_launch(const SymArgs<T>& A, int64_t ntiles, TPWs<T, PHASED ? 2 * NCOL : NCOL> W,
+                              cudaStream_t st) {
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
-    k_sym_reduce<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, aggF, aggB);
-    k_tile_carries<T, C, 1024><<<1, 1024, 0, st>>>(A.s, A.n, (int64_t)SYM_NT * E, ntiles, aggF,
-                                                     aggB, carF, carB, nullptr);
-    k_sym_final<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, carF, carB);
+    const int64_t nb = (ntiles + TP_CARRY_BT - 1) / TP_CARRY_BT;
+    k_sym_reduce<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, W);
+    k_tp_carry_blocks<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles);
+    k_tp_carry_tiles<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles, nb);
+    k_sym_final<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, W.carF, W.carB);
     return cudaGetLastError();
 }
 
@@ -438,10 +373,14 @@ namespace lx {
 
 constexpr int64_t NOALLOC_TILE = (int64_t)SYM_NT * 16;           // elements per tile (fp32, B = 1)
 constexpr int64_t NOALLOC_MAX_TILES = (int64_t)1 << 18;          // n <= 2^30
-constexpr size_t NOALLOC_BYTES = 4 * NOALLOC_MAX_TILES * sizeof(float);  // 4 MiB
+constexpr int64_t NOALLOC_MAX_CBLK = NOALLOC_MAX_TILES / TP_CARRY_BT;  // carry blocks
+constexpr size_t NOALLOC_BYTES = 4 * NOALLOC_MAX_TILES * sizeof(float) + 4096;  // 4 MiB + 4 KiB
+static_assert(4 * NOALLOC_MAX_CBLK * sizeof(float) + sizeof(uint32_t) <= 4096, "carry-block records");
 
-// Four float arrays of NOALLOC_MAX_TILES entries (tile totals and tile carries).
-// Every call writes each entry it reads, so nothing here needs clearing.
+// Per tile: first and last anchor, forward and backward totals (the carry
+// kernels overwrite the totals with the carries into each tile, in place);
+// per carry block: its four totals; one gate word.  Every call writes each
+// entry it reads, so nothing here needs clearing.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_BYTES];
 
 constexpr int NOALLOC_MAX_DEVICES = 64;
@@ -518,10 +457,21 @@ extern "C" laplex_status laplex_matvec_sym_noalloc(const float* sorted, const in
         return LAPLEX_OK;
     }
     const int64_t ntiles = (n + NOALLOC_TILE - 1) / NOALLOC_TILE;
-    float* aggF = static_cast<float*>(scratch);
-    float* aggB = aggF + NOALLOC_MAX_TILES;
-    float* carF = aggB + NOALLOC_MAX_TILES;
-    float* carB = carF + NOALLOC_MAX_TILES;
+    float* base = static_cast<float*>(scratch);
+    TPWs<float, 1> W;
+    W.tfirst = base;
+    W.tlast = base + NOALLOC_MAX_TILES;
+    W.fagg = base + 2 * NOALLOC_MAX_TILES;
+    W.bagg = base + 3 * NOALLOC_MAX_TILES;
+    W.carF = W.fagg;  // each carry thread reads its tiles' totals before it writes their carries
+    W.carB = W.bagg;
+    W.bfe = base + 4 * NOALLOC_MAX_TILES;
+    W.bfv = W.bfe + NOALLOC_MAX_CBLK;
+    W.bbf = W.bfv + NOALLOC_MAX_CBLK;
+    W.bbv = W.bbf + NOALLOC_MAX_CBLK;
+    W.redo_count = reinterpret_cast<uint32_t*>(W.bbv + NOALLOC_MAX_CBLK);
+    W.st = nullptr;
+    W.redo = nullptr;
     SymArgs<float> A;
     A.s = sorted;
     A.n = n;
@@ -537,7 +487,7 @@ extern "C" laplex_status laplex_matvec_sym_noalloc(const float* sorted, const in
     A.col0 = 0;
     A.ncol = 1;
     A.status = nullptr;
-    e = sym_launch<float, 1, false, 16>(A, ntiles, aggF, aggB, carF, carB, (cudaStream_t)stream);
+    e = sym_launch<float, 1, false, 16>(A, ntiles, W, (cudaStream_t)stream);
     if (e != cudaSuccess) {
         set_last_error("laplex_matvec_sym_noalloc: %s", cudaGetErrorString(e));
         return LAPLEX_ECUDA;

@@ -445,8 +445,10 @@ __global__ void __launch_bounds__(P::NT, P::MINB) k_tp_ring(P p, TPWs<typename P
 
 // ------------------------------------------------------------------ pass 2
 // The records of a thread's TP_CARRY_PT consecutive tiles, loaded at once (the
-// loads are independent; a tile past the end repeats the last one and is
-// masked out by `valid`).
+// loads are independent; entries past the last tile are 0 and never used).
+// Only the thread's own tiles are read, so k_tp_carry_tiles may write the
+// carries over the totals (carF == fagg, carB == bagg), as the fixed-scratch
+// product does.
 template <typename T, int C>
 struct TPSeg {
     T tl[TP_CARRY_PT], tf[TP_CARRY_PT];
@@ -454,13 +456,14 @@ struct TPSeg {
     __device__ __forceinline__ void load(const TPWs<T, C>& W, int64_t t0, int64_t ntiles) {
 #pragma unroll
         for (int k = 0; k < TP_CARRY_PT; ++k) {
-            const int64_t t = min(t0 + k, ntiles - 1);
-            tl[k] = W.tlast[t];
-            tf[k] = W.tfirst[t];
+            const int64_t t = t0 + k;
+            const bool in = t < ntiles;  // only this thread's own tiles are read
+            tl[k] = in ? W.tlast[t] : T(0);
+            tf[k] = in ? W.tfirst[t] : T(0);
 #pragma unroll
             for (int c = 0; c < C; ++c) {
-                fa[k][c] = W.fagg[t * C + c];
-                ba[k][c] = W.bagg[t * C + c];
+                fa[k][c] = in ? W.fagg[t * C + c] : T(0);
+                ba[k][c] = in ? W.bagg[t * C + c] : T(0);
             }
         }
     }

@@ -363,8 +363,10 @@ laplex_status laplex_test_set_sort_wait(uint32_t polls, int force_expiry);
  * provide the workspace laplex_matvec_sym needs.
  *   sorted [n], perm [n]|NULL, x [n], y [n]: as in laplex_matvec_sym (fp32, B = 1).
  *   stream: as elsewhere.
- * Scratch: a fixed 4 MiB array compiled into the library as a __device__
- * variable; every GPU that loads the library holds it until the process exits.
+ * Scratch: a fixed array of 4 MiB + 4 KiB compiled into the library as a
+ * __device__ variable (per tile its edge anchors and totals, then the carries
+ * into it; per group of 2048 tiles its totals); every GPU that loads the
+ * library holds it until the process exits.
  * It bounds n to 2^30 (2^18 tiles of 4096 anchors); larger n returns
  * LAPLEX_EINVAL with a message.  The call allocates and frees nothing.
  * The first call on each device looks up the array's device address (with that
