@@ -405,6 +405,20 @@ def run_ours(args):
         previous call where they fit)."""
         return timed(fn, steps, 2) / steps
 
+    def graphed(fn):
+        """fn captured once into a CUDA graph (after an eager call on the
+        capture stream, which sizes its workspace); returns the replay."""
+        s_cap = torch.cuda.Stream(dev)
+        s_cap.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s_cap):
+            fn()
+        torch.cuda.current_stream(dev).wait_stream(s_cap)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s_cap):
+            fn()
+        return g
+
     def frow(fn, bytes_per, steps):
         """A row timed both with L2 flushed before every call (ms, frac) and
         warm (warm_ms); frac = algorithmic bytes / time / HBM peak."""
@@ -445,6 +459,10 @@ def run_ours(args):
             z3 = torch.empty_like(xs3)
             nn, kk = 1 << 22, 1 << 20
             rows["c3_general_Kx"] = frow(lambda: X.matvec_general(sa, sb, xs3, out=y3), 8 * nn + 8 * kk, fsteps)
+            # the same call replayed from a CUDA graph (no per-kernel launch from the host)
+            g3 = graphed(lambda: X.matvec_general(sa, sb, xs3, out=y3))
+            rows["c3_general_Kx_graph"] = frow(g3.replay, 8 * nn + 8 * kk, fsteps)
+            del g3
             rows["c3_general_KTw"] = frow(lambda: X.matvec_general(sa, sb, ws3, transpose=True, out=z3), 8 * nn + 8 * kk, fsteps)
             # anchor gradients of <w, K x> (sorted order): reads a, b, x, w; writes dx, da, db
             rows["c3_backward_general"] = frow(lambda: X.backward_general(sa, sb, xs3, ws3), 16 * nn + 16 * kk, fsteps)
@@ -467,6 +485,9 @@ def run_ours(args):
             vs = torch.from_numpy(v4).to(dev)[p4.long()].contiguous()
             y4 = torch.empty_like(vs)
             rows["c4_phased_Kv"] = frow(lambda: X.matvec_phased(s4, phis, vs, out=y4), 16 * n4, fsteps)
+            g4 = graphed(lambda: X.matvec_phased(s4, phis, vs, out=y4))
+            rows["c4_phased_Kv_graph"] = frow(g4.replay, 16 * n4, fsteps)
+            del g4
             rows["c4_gram_KTKv"] = frow(lambda: X.gram(s4, vs, phi=phis, out=y4), 32 * n4, fsteps)
             gs4 = torch.from_numpy(synth.normal(n4, seed=rank, stream="g")).to(dev)
             rows["c4_backward_phased"] = frow(lambda: X.backward_phased(s4, phis, vs, gs4), 28 * n4, fsteps)

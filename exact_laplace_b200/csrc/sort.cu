@@ -976,7 +976,7 @@ __global__ void __launch_bounds__(1024) k_place_group(const uint32_t* __restrict
                                                       const int64_t* __restrict__ group_lo, int64_t n,
                                                       V* __restrict__ dst) {
     constexpr int GS = 1 << GB;
-    extern __shared__ __align__(16) unsigned char dyn[];
+    extern __shared__ __align__(128) unsigned char dyn[];
     V* buf = reinterpret_cast<V*>(dyn);                       // [GS]
     uint32_t* wrote = reinterpret_cast<uint32_t*>(buf + GS);  // [GS / 32]
     const int64_t q = blockIdx.x;
@@ -1065,13 +1065,16 @@ cudaError_t permute_run(const V* src, const int32_t* idx, int64_t n, V* dst, voi
     // group boundaries of the ordered keys (with no pass: one group, all of idx)
     k_group_bounds<<<(unsigned)((ng + 1 + 255) / 256), 256, 0, st>>>(ksrc, n, GB, ng, P > 0 ? 1 : 0, group_lo);
     constexpr size_t smem = ((size_t)1 << GB) * sizeof(V) + ((size_t)1 << GB) / 8;
-    auto place = [&](auto kern) -> cudaError_t {
-        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto place = [&](auto kc) -> cudaError_t {
+        constexpr auto kern = decltype(kc)::value;
+        int per = 0;  // raises the kernel's shared-memory limit once per device (no per-call host state)
+        cudaError_t r = blocks_per_sm<kern>(dev, 1024, smem, &per);
         if (r != cudaSuccess) return r;
         kern<<<(unsigned)ng, 1024, smem, st>>>(ksrc, vsrc, group_lo, n, dst);
         return cudaGetLastError();
     };
-    return vio ? place(k_place_group<V, GB, true>) : place(k_place_group<V, GB, false>);
+    return vio ? place(std::integral_constant<decltype(&k_place_group<V, GB, true>), &k_place_group<V, GB, true>>{})
+               : place(std::integral_constant<decltype(&k_place_group<V, GB, false>), &k_place_group<V, GB, false>>{});
 }
 
 template cudaError_t permute_run<int32_t>(const int32_t*, const int32_t*, int64_t, int32_t*, void*, size_t,
