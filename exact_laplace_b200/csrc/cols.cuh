@@ -258,7 +258,8 @@ cudaError_t cols_launch(const T* s, int64_t n, const T* x, T* y, void* ws, size_
     if (e != cudaSuccess) return e;
     profile_before(st);
     k_cols<T, B, E, false><<<(unsigned)ntiles, COLS_NT, 0, st>>>(s, n, x, y, W);
-    k_tp_carry_blocks<T, B, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles);
+    // the per-block totals are read only when there is more than one carry block
+    if (nb > 1) k_tp_carry_blocks<T, B, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles);
     k_tp_carry_tiles<T, B, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles, nb);
     k_cols<T, B, E, true><<<(unsigned)ntiles, COLS_NT, 0, st>>>(s, n, x, y, W);
     profile_after(st);

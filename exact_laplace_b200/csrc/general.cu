@@ -399,7 +399,8 @@ static cudaError_t gen_launch(const GenArgs<T>& A, const GenPlan& p, void* wsbod
     profile_before(st);
     k_gen_local<T, NCOL, PHASED, E, GEN_NT, H><<<(unsigned)p.ntiles, GEN_NT, 0, st>>>(A, W, ia);
     profile_after(st);
-    k_tp_carry_blocks<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, p.ntiles);
+    // the per-block totals are read only when there is more than one carry block
+    if (nb > 1) k_tp_carry_blocks<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, p.ntiles);
     k_tp_carry_tiles<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, p.ntiles, nb);
     const int64_t htb = std::max<int64_t>(1, std::min<int64_t>(p.ntiles, (int64_t)sms * 8));
     k_gen_headtail<T, NCOL, PHASED><<<(unsigned)htb, 256, 0, st>>>(A, W, ia, p.tile, p.ntiles);

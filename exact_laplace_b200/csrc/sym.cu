@@ -301,7 +301,8 @@ static cudaError_t sym_launch(const SymArgs<T>& A, int64_t ntiles, TPWs<T, PHASE
     constexpr int C = PHASED ? 2 * NCOL : NCOL;
     const int64_t nb = (ntiles + TP_CARRY_BT - 1) / TP_CARRY_BT;
     k_sym_reduce<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, W);
-    k_tp_carry_blocks<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles);
+    // the per-block totals are read only when there is more than one carry block
+    if (nb > 1) k_tp_carry_blocks<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles);
     k_tp_carry_tiles<T, C, 0><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles, nb);
     k_sym_final<T, NCOL, PHASED, E, SYM_NT><<<(unsigned)ntiles, SYM_NT, 0, st>>>(A, W.carF, W.carB);
     return cudaGetLastError();

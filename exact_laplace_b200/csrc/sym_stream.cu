@@ -578,7 +578,8 @@ cudaError_t stream_run(const T* s, const T* x, T* y, const int32_t* pout, int64_
     else
         e = launch_tiles<k_tile_local<T, E, LT_NT, LT_STAGES, H, true, 0>>(dev, sms, smem_p, true, st, s, x, y, pout, n, ntiles, W, status);
     if (e != cudaSuccess) return e;
-    k_carry_blocks<T><<<(unsigned)nb, CARRY_NT, 0, st>>>(W, ntiles);
+    // the per-block totals are read only when there is more than one carry block
+    if (nb > 1) k_carry_blocks<T><<<(unsigned)nb, CARRY_NT, 0, st>>>(W, ntiles);
     k_carry_tiles<T><<<(unsigned)nb, CARRY_NT, 0, st>>>(W, ntiles, nb);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

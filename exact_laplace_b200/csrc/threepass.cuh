@@ -640,7 +640,8 @@ cudaError_t tp_finish(const P& p, TPWs<typename P::T, P::C> W, int64_t ntiles, i
     using T = typename P::T;
     constexpr int C = P::C, CT = P::CT;
     const int64_t nb = (ntiles + TP_CARRY_BT - 1) / TP_CARRY_BT;
-    k_tp_carry_blocks<T, C, CT><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles);
+    // the per-block totals are read only when there is more than one carry block
+    if (nb > 1) k_tp_carry_blocks<T, C, CT><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles);
     k_tp_carry_tiles<T, C, CT><<<(unsigned)nb, TP_CARRY_NT, 0, st>>>(W, ntiles, nb);
     const int64_t rb = std::max<int64_t>(1, std::min<int64_t>(ntiles, (int64_t)sms * 4));
     k_tp_redo<P><<<(unsigned)rb, P::NT, 0, st>>>(p, W, ntiles);
