@@ -188,14 +188,15 @@ def test_halo_carries(case, use_perm):
 @pytest.mark.parametrize("dtype", [np.float32, np.float64])
 @pytest.mark.parametrize("B", [2, 4, 8])
 def test_columns_dense_and_tied(B, dtype):
-    """Several columns in sorted order (the column-parallel kernels): carries
-    that cross every tile (10^5 anchors in one unit; all anchors equal) and a
-    size that leaves a ragged last tile."""
+    """Several columns (the column-parallel kernels), in sorted order and
+    through perm: carries that cross every tile (10^5 anchors in one unit; all
+    anchors equal) and a size that leaves a ragged last tile."""
     rng = np.random.default_rng(B)
     for n, a in ((100_003, rng.uniform(0.0, 1.0, 100_003)), (5_003, np.full(5_003, 2.5)),
                  (70_001, np.round(rng.uniform(0.0, 400.0, 70_001)))):
         a = a.astype(dtype)
         x = synth.normal(n * B, seed=n, stream="x", dtype=dtype).reshape(n, B)
         y_ref = O.sym(a, x)
-        assert_close(run_sym(a, x, use_perm=False), y_ref, O.norm_sym(a, x), dtype, f"n={n} B={B}",
-                     slack=O.far_mass(a, x))
+        for use_perm in (False, True):  # through perm: rows gathered once, the same kernels, rows scattered
+            assert_close(run_sym(a, x, use_perm=use_perm), y_ref, O.norm_sym(a, x), dtype,
+                         f"n={n} B={B} perm={use_perm}", slack=O.far_mass(a, x))
