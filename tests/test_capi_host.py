@@ -97,3 +97,51 @@ def test_argument_errors_return_before_any_launch(L):
     size = ctypes.c_size_t()
     assert L.laplex_workspace_size(1, 0, 0, 1, 0, ctypes.byref(size)) == 0
     assert L.laplex_matvec_sym(None, None, 0, None, None, 1, 0, P(256), size.value, None) == 0
+
+
+def test_carry_and_unsorted_argument_errors(L):
+    """laplex_sort_anchors_carry and laplex_matvec_sym_unsorted check their
+    arguments on the host and return before any launch."""
+    from exact_laplace_b200 import laplex as X
+    P = ctypes.c_void_p
+    size = ctypes.c_size_t()
+    assert L.laplex_workspace_size(X.OP_SORT_CARRY, 1000, 0, 1, 0, ctypes.byref(size)) == 0
+    big = size.value
+    # NULL values with n > 0
+    st = L.laplex_sort_anchors_carry(P(256), None, 1000, 0, P(512), P(768), P(1024), P(256), big, None)
+    assert st == X.EINVAL and b"x" in L.laplex_last_error()
+    # misaligned xs
+    st = L.laplex_sort_anchors_carry(P(256), P(512), 1000, 0, P(768), P(1024), P(1284), P(256), big, None)
+    assert st == X.EINVAL and b"aligned" in L.laplex_last_error()
+    # workspace too small
+    st = L.laplex_sort_anchors_carry(P(256), P(512), 1000, 0, P(768), P(1024), P(1280), P(256), 300, None)
+    assert st == X.EWORKSPACE
+    # n out of range
+    st = L.laplex_sort_anchors_carry(P(256), P(512), 1 << 31, 0, P(768), P(1024), P(1280), P(256), big, None)
+    assert st == X.EINVAL
+    assert L.laplex_workspace_size(X.OP_SYM_UNSORTED, 1000, 0, 1, 1, ctypes.byref(size)) == 0
+    big = size.value
+    # NULL perm output, bad dtype, small workspace
+    st = L.laplex_matvec_sym_unsorted(P(256), P(512), 1000, 1, P(768), P(1024), None, P(256), big, None)
+    assert st == X.EINVAL and b"perm" in L.laplex_last_error()
+    st = L.laplex_matvec_sym_unsorted(P(256), P(512), 1000, 5, P(768), P(1024), P(1280), P(256), big, None)
+    assert st == X.EINVAL
+    st = L.laplex_matvec_sym_unsorted(P(256), P(512), 1000, 1, P(768), P(1024), P(1280), P(256), 300, None)
+    assert st == X.EWORKSPACE
+    # n = 0: no pointers needed
+    assert L.laplex_workspace_size(X.OP_SYM_UNSORTED, 0, 0, 1, 0, ctypes.byref(size)) == 0
+    assert L.laplex_matvec_sym_unsorted(None, None, 0, 0, None, None, None, P(256), size.value, None) == 0
+    assert L.laplex_workspace_size(X.OP_SORT_CARRY, 0, 0, 1, 0, ctypes.byref(size)) == 0
+    assert L.laplex_sort_anchors_carry(None, None, 0, 0, None, None, None, P(256), size.value, None) == 0
+
+
+def test_workspace_of_new_ops_grows_with_n(L):
+    from exact_laplace_b200 import laplex as X
+    for op in (X.OP_SORT_CARRY, X.OP_SYM_UNSORTED):
+        for dt in (0, 1):
+            sizes = []
+            for n in (1, 1 << 10, 1 << 20, 1 << 26):
+                size = ctypes.c_size_t()
+                assert L.laplex_workspace_size(op, n, 0, 1, dt, ctypes.byref(size)) == 0
+                sizes.append(size.value)
+            assert sizes == sorted(sizes) and sizes[-1] >= (1 << 26) * 12
