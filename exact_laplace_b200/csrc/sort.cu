@@ -948,7 +948,9 @@ cudaError_t sort_carry_run(const float* a, const float* x, int64_t n, float* sor
 // whole-sector stores.  Entries of idx outside [0, n) are clamped to n, sort
 // last and are dropped; a position that no entry names is left untouched
 // (a bitmap of the written positions guards the store).
-constexpr int PERM_KPT = 16;
+// keys per thread of the permutation's digit passes: 24 with 4-byte elements
+// (the plain sort's shape), 16 with 8-byte ones (shared memory for two blocks per SM)
+template <typename V> struct PermKPT { static constexpr int v = sizeof(V) == 4 ? 24 : 16; };
 template <typename V> struct PermGB { static constexpr int v = sizeof(V) == 8 ? 13 : 14; };  // 64 KB of outputs
 
 // group_lo[q] = first position of the ordered keys whose group (index below
@@ -1015,7 +1017,8 @@ static int perm_passes(int64_t n) {
 size_t permute_ws_bytes(int64_t n, int vbytes) {
     const int P = vbytes == 8 ? perm_passes<int64_t>(n) : perm_passes<int32_t>(n);
     const int64_t ng = vbytes == 8 ? perm_groups<int64_t>(n) : perm_groups<int32_t>(n);
-    const int64_t ntiles = (n + (int64_t)SORT_NT * PERM_KPT - 1) / ((int64_t)SORT_NT * PERM_KPT);
+    const int64_t ptile = (int64_t)SORT_NT * (vbytes == 8 ? PermKPT<int64_t>::v : PermKPT<int32_t>::v);
+    const int64_t ntiles = (n + ptile - 1) / ptile;
     const int bufs = P == 0 ? 0 : (P == 1 ? 1 : 2);
     return bufs * (Carve::need((size_t)n, 4) + Carve::need((size_t)n, (size_t)vbytes)) + pass_ws_bytes(ntiles) +
            Carve::need((size_t)(ng + 2), 8);
@@ -1032,6 +1035,7 @@ cudaError_t permute_run(const V* src, const int32_t* idx, int64_t n, V* dst, voi
     const bool iota = src == nullptr;
     const int P = perm_passes<V>(n);
     const int64_t ng = perm_groups<V>(n);
+    constexpr int PERM_KPT = PermKPT<V>::v;
     const int64_t ntiles = (n + (int64_t)SORT_NT * PERM_KPT - 1) / ((int64_t)SORT_NT * PERM_KPT);
     Carve cv(ws, ws_bytes);
     uint32_t* tk[2] = {nullptr, nullptr};
