@@ -11,11 +11,13 @@ times in a row on different inputs, and checks every result against the fp64
 oracle (the sequential recurrences on the same seeded inputs) and against
 laplex_matvec_sym on the same inputs, with the tolerance of the other parity
 tests: max_i |y_i - y_ref_i| / (K0|x|)_i <= 1e-4, fp32 terms below FLT_MIN
-allowed to vanish (oracle.far_mass).  The cases reach the scratch's carry pass
-in every shape it takes: one tile per carry thread, two and four tiles per
-thread (n above 1024 and 4096 tiles of 4096 anchors), a run of equal anchors
-across a tile boundary, and carries that cross every tile (all anchors equal;
-10^6 anchors inside one unit).  The file sorts last so that a run stopping at
+allowed to vanish (oracle.far_mass).  The cases reach the carry kernels in
+every shape they take over the fixed scratch: one carry block (up to 2048
+tiles of 4096 anchors, the carries written over the tile totals in place) and
+several (4097 tiles: three blocks, with carries between blocks), threads with
+fewer than 8 tiles at the end, a run of equal anchors across a tile boundary,
+and carries that cross every tile (all anchors equal; 10^6 anchors inside one
+unit).  The file sorts last so that a run stopping at
 the first failure has run every other test before it; it also passes on its own.
 """
 import ctypes
@@ -31,7 +33,7 @@ from gpu_util import assert_close
 
 pytestmark = pytest.mark.gpu
 
-TILE = 4096  # anchors per tile of the scratch's carry pass
+TILE = 4096  # anchors per tile of the allocation-free product
 
 
 def _call_noalloc(s_d, p_d, x_d, y_d):
@@ -58,7 +60,7 @@ CASES = [
     ("U(0,5000), perm", lambda: synth.sym_uniform(300_001, 0.0, 5000.0, seed=300_001), True),
     ("U(-100,100), sorted order", lambda: synth.sym_uniform(2_000_003, -100.0, 100.0, seed=3), False),
     ("1465 tiles, equal run across a tile boundary, perm", lambda: _equal_run_across_tile(6_000_007), True),
-    ("4097 tiles, U(0,2^24), sorted order",
+    ("4097 tiles (three carry blocks), U(0,2^24), sorted order",
      lambda: synth.sym_uniform((1 << 24) + 43, 0.0, float(1 << 24), seed=11), False),
     ("all anchors equal, perm",
      lambda: (np.full(1_000_003, 3.25, dtype=np.float32), synth.normal(1_000_003, seed=5, stream="x")), True),
